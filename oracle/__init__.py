@@ -1,0 +1,215 @@
+"""ctypes loader for the oracle -- TEST INFRASTRUCTURE ONLY.
+
+The oracle is a plain single-threaded C++ definition of one GPT-2-style training step
+(gpt_oracle.cpp). Only the tests, `__graft_entry__.smoke()` and the benchmark's CPU-baseline
+leg import this package; the CUDA library and its Python binding never do.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gpt_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (-O2, IEEE semantics: no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
+            os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "gpt_oracle.h"))):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-fno-fast-math",
+                               "-ffp-contract=off", _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int), ("vocab_padded", ctypes.c_int),
+                ("n_layer", ctypes.c_int), ("n_head", ctypes.c_int), ("n_embd", ctypes.c_int),
+                ("max_T", ctypes.c_int), ("mlp_mult", ctypes.c_int),
+                ("window_left", ctypes.POINTER(ctypes.c_int)), ("ln_eps", ctypes.c_double)]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        L = _lib
+        L.oracle_num_params.restype = ctypes.c_size_t
+        L.oracle_num_params.argtypes = [P]
+        L.oracle_layout.restype = ctypes.c_int
+        L.oracle_layout.argtypes = [P, P, P, ctypes.c_int]
+        for suf, R in (("f64", ctypes.c_double), ("f32", ctypes.c_float)):
+            f = getattr(L, f"oracle_forward_{suf}")
+            f.restype = R
+            f.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, P]
+            f = getattr(L, f"oracle_forward_backward_{suf}")
+            f.restype = R
+            f.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, P, P]
+            f = getattr(L, f"oracle_grad_norm_{suf}")
+            f.restype = ctypes.c_double
+            f.argtypes = [ctypes.c_size_t, P]
+            f = getattr(L, f"oracle_adamw_{suf}")
+            f.restype = None
+            f.argtypes = [ctypes.c_size_t, P, P, P, P] + [R] * 5 + [ctypes.c_long, R]
+            f = getattr(L, f"oracle_train_step_{suf}")
+            f.restype = R
+            f.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int] + [R] * 6 + \
+                [ctypes.c_long, P]
+        L.oracle_layernorm_fwd_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                               P, P, P]
+        L.oracle_layernorm_bwd_f64.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int, P, P]
+        L.oracle_attention_fwd_f64.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, P]
+        L.oracle_attention_bwd_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, P]
+        L.oracle_gelu_f64.restype = ctypes.c_double
+        L.oracle_gelu_f64.argtypes = [ctypes.c_double]
+        L.oracle_gelu_grad_f64.restype = ctypes.c_double
+        L.oracle_gelu_grad_f64.argtypes = [ctypes.c_double]
+        L.oracle_cross_entropy_f64.restype = ctypes.c_double
+        L.oracle_cross_entropy_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """Holds one model shape; `dtype` selects the float or double instantiation."""
+
+    def __init__(self, vocab: int, vocab_padded: int, n_layer: int, n_head: int, n_embd: int,
+                 max_T: int, mlp_mult: int = 4, window_left: Optional[Sequence[int]] = None,
+                 ln_eps: float = 1e-5, dtype=np.float64):
+        self.lib = _load()
+        self.dtype = np.dtype(dtype)
+        self.suf = "f64" if self.dtype == np.float64 else "f32"
+        self._win = (ctypes.c_int * n_layer)(*(window_left if window_left else [-1] * n_layer))
+        self.cfg = _Cfg(vocab, vocab_padded, n_layer, n_head, n_embd, max_T, mlp_mult,
+                        ctypes.cast(self._win, ctypes.POINTER(ctypes.c_int)), ln_eps)
+        self.n = int(self.lib.oracle_num_params(ctypes.byref(self.cfg)))
+
+    @classmethod
+    def from_shape(cls, sh, dtype=np.float64, ln_eps: float = 1e-5):
+        return cls(sh.vocab, sh.vocab_padded, sh.n_layer, sh.n_head, sh.n_embd, sh.max_T,
+                   sh.mlp_mult, sh.windows(), ln_eps, dtype)
+
+    def layout(self) -> List[tuple]:
+        cap = 16 + 6 * self.cfg.n_layer
+        off = np.zeros(cap, np.int64)
+        num = np.zeros(cap, np.int64)
+        k = self.lib.oracle_layout(ctypes.byref(self.cfg), _ptr(off), _ptr(num), cap)
+        return [(int(off[i]), int(num[i])) for i in range(k)]
+
+    def _arr(self, a):
+        return np.ascontiguousarray(a, dtype=self.dtype)
+
+    def forward(self, params, tokens, targets, per_token=False):
+        p = self._arr(params)
+        tok = np.ascontiguousarray(tokens, np.int32)
+        tgt = np.ascontiguousarray(targets, np.int32)
+        B, T = tok.shape
+        ptl = np.zeros(B * T, self.dtype) if per_token else None
+        f = getattr(self.lib, f"oracle_forward_{self.suf}")
+        loss = f(ctypes.byref(self.cfg), _ptr(p), _ptr(tok), _ptr(tgt), B, T, _ptr(ptl))
+        return (loss, ptl.reshape(B, T)) if per_token else loss
+
+    def forward_backward(self, params, tokens, targets, per_token=False):
+        p = self._arr(params)
+        tok = np.ascontiguousarray(tokens, np.int32)
+        tgt = np.ascontiguousarray(targets, np.int32)
+        B, T = tok.shape
+        g = np.zeros(self.n, self.dtype)
+        ptl = np.zeros(B * T, self.dtype) if per_token else None
+        f = getattr(self.lib, f"oracle_forward_backward_{self.suf}")
+        loss = f(ctypes.byref(self.cfg), _ptr(p), _ptr(tok), _ptr(tgt), B, T, _ptr(g), _ptr(ptl))
+        return (loss, g, ptl.reshape(B, T)) if per_token else (loss, g)
+
+    def grad_norm(self, g) -> float:
+        g = self._arr(g)
+        return getattr(self.lib, f"oracle_grad_norm_{self.suf}")(g.size, _ptr(g))
+
+    def adamw(self, p, g, m, v, lr, wd, step, coef=1.0, beta1=0.9, beta2=0.95, eps=1e-8):
+        """In place on p, m, v (arrays of this oracle's dtype)."""
+        for a in (p, m, v):
+            assert a.dtype == self.dtype and a.flags.c_contiguous
+        g = self._arr(g)
+        getattr(self.lib, f"oracle_adamw_{self.suf}")(p.size, _ptr(p), _ptr(g), _ptr(m), _ptr(v),
+                                                       lr, wd, beta1, beta2, eps, step, coef)
+
+    def train_step(self, p, m, v, tokens, targets, lr, wd, clip, step, beta1=0.9, beta2=0.95,
+                   eps=1e-8):
+        """In place on p, m, v. Returns (loss, raw grads, unclipped grad norm)."""
+        for a in (p, m, v):
+            assert a.dtype == self.dtype and a.flags.c_contiguous
+        tok = np.ascontiguousarray(tokens, np.int32)
+        tgt = np.ascontiguousarray(targets, np.int32)
+        B, T = tok.shape
+        g = np.zeros(self.n, self.dtype)
+        gn = ctypes.c_double(0.0)
+        f = getattr(self.lib, f"oracle_train_step_{self.suf}")
+        loss = f(ctypes.byref(self.cfg), _ptr(p), _ptr(g), _ptr(m), _ptr(v), _ptr(tok), _ptr(tgt),
+                 B, T, lr, wd, clip, beta1, beta2, eps, step, ctypes.byref(gn))
+        return loss, g, gn.value
+
+    # -- single pieces (double) --
+    def layernorm_fwd(self, x, g, eps=1e-5):
+        x = np.ascontiguousarray(x, np.float64)
+        rows, C = x.shape
+        y = np.zeros_like(x)
+        mu = np.zeros(rows)
+        rs = np.zeros(rows)
+        self.lib.oracle_layernorm_fwd_f64(_ptr(x), _ptr(np.ascontiguousarray(g, np.float64)),
+                                          rows, C, eps, _ptr(y), _ptr(mu), _ptr(rs))
+        return y, mu, rs
+
+    def layernorm_bwd(self, x, g, mu, rs, dy):
+        x = np.ascontiguousarray(x, np.float64)
+        rows, C = x.shape
+        dx = np.zeros_like(x)
+        dg = np.zeros(C)
+        self.lib.oracle_layernorm_bwd_f64(_ptr(x), _ptr(np.ascontiguousarray(g, np.float64)),
+                                          _ptr(mu), _ptr(rs),
+                                          _ptr(np.ascontiguousarray(dy, np.float64)), rows, C,
+                                          _ptr(dx), _ptr(dg))
+        return dx, dg
+
+    def attention_fwd(self, qkv, H, window=-1):
+        qkv = np.ascontiguousarray(qkv, np.float64)
+        B, T, C3 = qkv.shape
+        o = np.zeros((B, T, C3 // 3))
+        self.lib.oracle_attention_fwd_f64(_ptr(qkv), B, T, C3 // 3, H, window, _ptr(o))
+        return o
+
+    def attention_bwd(self, qkv, dout, H, window=-1):
+        qkv = np.ascontiguousarray(qkv, np.float64)
+        B, T, C3 = qkv.shape
+        d = np.zeros_like(qkv)
+        self.lib.oracle_attention_bwd_f64(_ptr(qkv), _ptr(np.ascontiguousarray(dout, np.float64)),
+                                          B, T, C3 // 3, H, window, _ptr(d))
+        return d
+
+    def gelu(self, x: float) -> float:
+        return self.lib.oracle_gelu_f64(x)
+
+    def gelu_grad(self, x: float) -> float:
+        return self.lib.oracle_gelu_grad_f64(x)
+
+    def cross_entropy(self, logits, targets, V):
+        lg = np.ascontiguousarray(logits, np.float64)
+        rows, Vp = lg.shape
+        d = np.zeros_like(lg)
+        loss = self.lib.oracle_cross_entropy_f64(_ptr(lg), _ptr(np.ascontiguousarray(targets, np.int32)),
+                                                 rows, V, Vp, _ptr(d))
+        return loss, d
