@@ -1,0 +1,15 @@
+// tcgen05 / TMEM / TMA GEMM for sm_100a (bf16 operands, fp32 accumulation in TMEM).
+#pragma once
+#include "common.cuh"
+
+constexpr int TC_BM = 128;  // rows per CTA tile (TMEM lanes)
+constexpr int TC_BN = 256;  // columns per CTA tile (TMEM fp32 columns)
+constexpr int TC_BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
+
+struct TcGemm;
+cudaError_t tc_gemm_create(TcGemm **out);
+void tc_gemm_destroy(TcGemm *t);
+// True when the shape, strides and epilogue can run on the tensor-core path.
+bool tc_gemm_supported(const GemmDesc &d);
+// Enqueues the GEMM (and its split-K reduction, if any); adds its kernel count to *launches.
+cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches);

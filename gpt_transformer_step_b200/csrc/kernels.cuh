@@ -1,0 +1,65 @@
+// Launchers of the step's kernels. T is the activation type: float (validation mode) or
+// bf16. Every launcher enqueues on `st` and returns the launch status.
+#pragma once
+#include "common.cuh"
+
+// K1: x[m] = wte[tok[m]] + wpe[m % T]; flags ids outside [0, V) (tokens and targets).
+template <typename T>
+cudaError_t launch_embed_fwd(const int *tok, const int *tgt, const T *wte, const T *wpe, T *x,
+                             int M, int Tlen, int C, int V, DevScalars *sc, cudaStream_t st);
+
+// K13: dwpe[t] = sum_b dx[b,t] (rows t >= T zeroed); dwte[id] += sum over positions with
+// that id, in position order (deterministic). dwte already holds the lm_head part.
+struct EmbedBwdWs {
+  unsigned *keys;      // [M] sorted (id << 14 | m)
+  float *partial;      // [nwin][2][C]
+};
+template <typename T>
+cudaError_t launch_embed_bwd(const int *tok, const T *dx, float *dwte, float *dwpe, int M,
+                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st);
+
+// K2: y = (x - mean) * rstd * g, one warp per row.
+template <typename T>
+cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
+                                 int C, float eps, cudaStream_t st);
+
+// K12: dres += LN_backward(dy); dgamma partial sums per block -> dg (fp32) after reduce.
+template <typename T>
+cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
+                                 const T *dy, T *dres, float *dg_partial, float *dg, int M,
+                                 int C, cudaStream_t st);
+int layernorm_bwd_blocks(int M);
+
+// Cross-entropy: per-row lse and loss from the per-tile stats; mean loss into sc->loss.
+cudaError_t launch_ce_combine(const float *stats, const float *tgt_logit, float *lse,
+                              float *per_token, int M, int ntiles, DevScalars *sc,
+                              cudaStream_t st);
+
+// K14: sum of squares of g[0..n) (two-stage, fixed order) -> sc->norm, sc->coef.
+cudaError_t launch_grad_norm(const float *g, size_t n, double *partials, DevScalars *sc,
+                             cudaStream_t st);
+int grad_norm_blocks();
+
+// K15: AdamW with g <- coef*g; skipped when sc->nonfinite. shadow (bf16, may be NULL)
+// receives the rounded new params.
+cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, bf16 *shadow, size_t n,
+                         const DevScalars *sc, cudaStream_t st);
+
+// fp32 -> bf16 copy of the weights.
+cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st);
+
+// Attention (head h of q/k/v at columns h*hd of each third of qkv [M, 3C]).
+template <typename T>
+cudaError_t launch_attention_fwd(const T *qkv, T *o, float *lse, int B, int Tlen, int C, int H,
+                                 int window, cudaStream_t st);
+template <typename T>
+cudaError_t launch_attention_bwd(const T *qkv, const T *o, const T *dout, const float *lse,
+                                 float *Dbuf, T *dqkv, int B, int Tlen, int C, int H, int window,
+                                 cudaStream_t st);
+
+// GEMM on CUDA cores (fp32 validation mode and shapes the tensor-core path does not take).
+template <typename T>
+cudaError_t launch_gemm_simt(const GemmDesc &d, cudaStream_t st);
+// Ordered reduction of split-K partials through the (elementwise) epilogue.
+template <typename T>
+cudaError_t launch_splitk_reduce(const GemmDesc &d, cudaStream_t st);

@@ -1,0 +1,596 @@
+// Memory-bound kernels of the step: embedding (K1, K13), LayerNorm (K2, K12),
+// cross-entropy combine, global grad norm (K14), AdamW (K15). All reductions run in a fixed
+// order, so results are bitwise reproducible run to run.
+#include "kernels.cuh"
+
+namespace {
+
+// 16-byte vectors: 8 bf16 or 4 float.
+template <typename T> struct Vec;
+template <> struct Vec<float> { static constexpr int N = 4; typedef float4 type; };
+template <> struct Vec<bf16> { static constexpr int N = 8; typedef uint4 type; };
+
+template <typename T>
+__device__ __forceinline__ void load_vec(const T *p, float (&f)[Vec<T>::N]);
+template <>
+__device__ __forceinline__ void load_vec<float>(const float *p, float (&f)[4]) {
+  float4 v = *reinterpret_cast<const float4 *>(p);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load_vec<bf16>(const bf16 *p, float (&f)[8]) {
+  uint4 v = *reinterpret_cast<const uint4 *>(p);
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x; f[2 * i + 1] = t.y;
+  }
+}
+template <typename T>
+__device__ __forceinline__ void store_vec(T *p, const float (&f)[Vec<T>::N]);
+template <>
+__device__ __forceinline__ void store_vec<float>(float *p, const float (&f)[4]) {
+  *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+template <>
+__device__ __forceinline__ void store_vec<bf16>(bf16 *p, const float (&f)[8]) {
+  uint4 v;
+  __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  *reinterpret_cast<uint4 *>(p) = v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ------------------------------------------------------------------------------------------
+// K1 embedding forward
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void embed_fwd_kernel(const int *__restrict__ tok, const int *__restrict__ tgt,
+                                 const T *__restrict__ wte, const T *__restrict__ wpe,
+                                 T *__restrict__ x, int M, int Tlen, int C, int V,
+                                 DevScalars *sc) {
+  constexpr int VN = Vec<T>::N;
+  const int vpr = C / VN;  // vectors per row
+  long total = (long)M * vpr;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
+       i += (long)gridDim.x * blockDim.x) {
+    int m = (int)(i / vpr), c = (int)(i % vpr) * VN;
+    int id = tok[m];
+    if (c == 0) {
+      if (id < 0 || id >= V) atomicOr(&sc->err, GPT_DEVERR_BAD_TOKEN);
+      int t = tgt[m];
+      if (t < 0 || t >= V) atomicOr(&sc->err, GPT_DEVERR_BAD_TARGET);
+    }
+    if (id < 0 || id >= V) id = 0;
+    float a[VN], b[VN];
+    load_vec<T>(wte + (long)id * C + c, a);
+    load_vec<T>(wpe + (long)(m % Tlen) * C + c, b);
+#pragma unroll
+    for (int k = 0; k < VN; ++k) a[k] += b[k];
+    store_vec<T>(x + (long)m * C + c, a);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// K2 LayerNorm forward: one warp per row, the row kept in registers (two-pass variance).
+// ------------------------------------------------------------------------------------------
+constexpr int LN_MAXV = 8;  // vectors per lane: C <= 32*8*VN
+
+template <typename T>
+__global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
+                                     T *__restrict__ y, float *__restrict__ mean,
+                                     float *__restrict__ rstd, int M, int C, float eps) {
+  constexpr int VN = Vec<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= M) return;
+  const int nv = C / VN;
+  float v[LN_MAXV][VN];
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < LN_MAXV; ++j) {
+    int c = (lane + 32 * j) * VN;
+    if (lane + 32 * j < nv) {
+      load_vec<T>(x + (long)row * C + c, v[j]);
+#pragma unroll
+      for (int k = 0; k < VN; ++k) s += v[j][k];
+    }
+  }
+  const float mu = warp_sum(s) / (float)C;
+  float q = 0.f;
+#pragma unroll
+  for (int j = 0; j < LN_MAXV; ++j)
+    if (lane + 32 * j < nv) {
+#pragma unroll
+      for (int k = 0; k < VN; ++k) {
+        float d = v[j][k] - mu;
+        q += d * d;
+      }
+    }
+  const float var = warp_sum(q) / (float)C;
+  const float rs = 1.0f / sqrtf(var + eps);
+#pragma unroll
+  for (int j = 0; j < LN_MAXV; ++j) {
+    int c = (lane + 32 * j) * VN;
+    if (lane + 32 * j < nv) {
+      float gg[VN], o[VN];
+      load_vec<T>(g + c, gg);
+#pragma unroll
+      for (int k = 0; k < VN; ++k) o[k] = (v[j][k] - mu) * rs * gg[k];
+      store_vec<T>(y + (long)row * C + c, o);
+    }
+  }
+  if (lane == 0) {
+    mean[row] = mu;
+    rstd[row] = rs;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// K12 LayerNorm backward (+ residual-gradient add, + per-block dgamma partials)
+// ------------------------------------------------------------------------------------------
+constexpr int LNB_WARPS = 8;
+constexpr int LNB_MAX_BLOCKS = 296;
+
+template <typename T>
+__global__ void __launch_bounds__(LNB_WARPS * 32)
+layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
+                     const float *__restrict__ mean, const float *__restrict__ rstd,
+                     const T *__restrict__ dy, T *__restrict__ dres,
+                     float *__restrict__ dg_partial, int M, int C, int rows_per_block) {
+  constexpr int VN = Vec<T>::N;
+  extern __shared__ float sm_dg[];  // [LNB_WARPS][C]
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nv = C / VN;
+  float dgacc[LN_MAXV][VN];
+#pragma unroll
+  for (int j = 0; j < LN_MAXV; ++j)
+#pragma unroll
+    for (int k = 0; k < VN; ++k) dgacc[j][k] = 0.f;
+  const int r0 = blockIdx.x * rows_per_block;
+  const int r1 = min(M, r0 + rows_per_block);
+  for (int row = r0 + w; row < r1; row += LNB_WARPS) {
+    const float mu = mean[row], rs = rstd[row];
+    float xh[LN_MAXV][VN], dxh[LN_MAXV][VN];
+    float a = 0.f, b = 0.f;
+#pragma unroll
+    for (int j = 0; j < LN_MAXV; ++j) {
+      int c = (lane + 32 * j) * VN;
+      if (lane + 32 * j < nv) {
+        float xv[VN], dv[VN], gv[VN];
+        load_vec<T>(x + (long)row * C + c, xv);
+        load_vec<T>(dy + (long)row * C + c, dv);
+        load_vec<T>(g + c, gv);
+#pragma unroll
+        for (int k = 0; k < VN; ++k) {
+          xh[j][k] = (xv[k] - mu) * rs;
+          dxh[j][k] = dv[k] * gv[k];
+          a += dxh[j][k];
+          b += dxh[j][k] * xh[j][k];
+          dgacc[j][k] += dv[k] * xh[j][k];
+        }
+      }
+    }
+    a = warp_sum(a) / (float)C;
+    b = warp_sum(b) / (float)C;
+#pragma unroll
+    for (int j = 0; j < LN_MAXV; ++j) {
+      int c = (lane + 32 * j) * VN;
+      if (lane + 32 * j < nv) {
+        float r[VN];
+        load_vec<T>(dres + (long)row * C + c, r);
+#pragma unroll
+        for (int k = 0; k < VN; ++k) r[k] += rs * (dxh[j][k] - a - xh[j][k] * b);
+        store_vec<T>(dres + (long)row * C + c, r);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < LN_MAXV; ++j) {
+    int c = (lane + 32 * j) * VN;
+    if (lane + 32 * j < nv)
+#pragma unroll
+      for (int k = 0; k < VN; ++k) sm_dg[w * C + c + k] = dgacc[j][k];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float s = 0.f;
+    for (int ww = 0; ww < LNB_WARPS; ++ww) s += sm_dg[ww * C + c];
+    dg_partial[(long)blockIdx.x * C + c] = s;
+  }
+}
+
+__global__ void colsum_kernel(const float *__restrict__ partial, int nrows, int C,
+                              float *__restrict__ out) {
+  int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= C) return;
+  float s = 0.f;
+  for (int r = 0; r < nrows; ++r) s += partial[(long)r * C + c];
+  out[c] = s;
+}
+
+// ------------------------------------------------------------------------------------------
+// K13 embedding backward
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void dwpe_kernel(const T *__restrict__ dx, float *__restrict__ dwpe, int Bn,
+                            int Tlen, int maxT, int C) {
+  long total = (long)maxT * C;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
+       i += (long)gridDim.x * blockDim.x) {
+    int t = (int)(i / C), c = (int)(i % C);
+    float s = 0.f;
+    if (t < Tlen)
+      for (int b = 0; b < Bn; ++b) s += to_f(dx[((long)b * Tlen + t) * C + c]);
+    dwpe[i] = s;
+  }
+}
+
+// One CTA sorts the M keys (id << 14 | m) in shared memory with a bitonic network.
+constexpr int SORT_MAX = 16384;
+__global__ void __launch_bounds__(1024) sort_keys_kernel(const int *__restrict__ tok, int M,
+                                                         unsigned *__restrict__ keys_out) {
+  extern __shared__ unsigned sk[];
+  int n = 1;
+  while (n < M) n <<= 1;
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    sk[i] = i < M ? ((unsigned)tok[i] << 14) | (unsigned)i : 0xffffffffu;
+  __syncthreads();
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        int p = i ^ j;
+        if (p > i) {
+          unsigned a = sk[i], b = sk[p];
+          bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            sk[i] = b;
+            sk[p] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < M; i += blockDim.x) keys_out[i] = sk[i];
+}
+
+constexpr int EW = 32;  // sorted entries per window
+
+// Window w covers sorted entries [w*EW, (w+1)*EW). Runs of one id that lie wholly inside the
+// window are added to dwte here; a run that starts before the window goes to slot 0, a run
+// that continues past it (and did not start before) to slot 1, for the merge kernel.
+template <typename T>
+__global__ void embed_seg_kernel(const unsigned *__restrict__ keys, const T *__restrict__ dx,
+                                 float *__restrict__ dwte, float *__restrict__ partial, int M,
+                                 int C) {
+  const int w = blockIdx.x;
+  const int e0 = w * EW, e1 = min(M, e0 + EW);
+  __shared__ unsigned skey[EW];
+  if (threadIdx.x < EW) skey[threadIdx.x] = (e0 + (int)threadIdx.x < M) ? keys[e0 + threadIdx.x] : 0u;
+  __syncthreads();
+  const unsigned id_before = e0 > 0 ? (keys[e0 - 1] >> 14) : 0xffffffffu;
+  const unsigned id_after = e1 < M ? (keys[e1] >> 14) : 0xffffffffu;
+  int s = e0;
+  while (s < e1) {
+    const unsigned id = skey[s - e0] >> 14;
+    int e = s;
+    while (e < e1 && (skey[e - e0] >> 14) == id) ++e;
+    const bool before = (s == e0) && (id == id_before);
+    const bool after = (e == e1) && (id == id_after);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float acc = 0.f;
+      for (int k = s; k < e; ++k) {
+        int m = (int)(skey[k - e0] & 0x3fffu);
+        acc += to_f(dx[(long)m * C + c]);
+      }
+      if (!before && !after)
+        dwte[(long)id * C + c] += acc;
+      else
+        partial[((long)w * 2 + (before ? 0 : 1)) * C + c] = acc;
+    }
+    s = e;
+  }
+}
+
+// For each run that continues past window w (and started inside it): sum slot 1 of w and
+// slot 0 of the following windows while the run goes on, in window order.
+__global__ void embed_merge_kernel(const unsigned *__restrict__ keys,
+                                   const float *__restrict__ partial, float *__restrict__ dwte,
+                                   int M, int C, int nwin) {
+  const int w = blockIdx.x;
+  const int e0 = w * EW, e1 = min(M, e0 + EW);
+  if (e1 >= M) return;
+  const unsigned id = keys[e1 - 1] >> 14;
+  if ((keys[e1] >> 14) != id) return;  // does not continue
+  // the run must not have started before the window
+  int s = e1 - 1;
+  while (s > e0 && (keys[s - 1] >> 14) == id) --s;
+  if (s == e0 && e0 > 0 && (keys[e0 - 1] >> 14) == id) return;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float acc = partial[((long)w * 2 + 1) * C + c];
+    for (int ww = w + 1; ww < nwin; ++ww) {
+      int f0 = ww * EW;
+      if ((keys[f0] >> 14) != id) break;
+      acc += partial[((long)ww * 2 + 0) * C + c];
+      int f1 = min(M, f0 + EW);
+      if (f1 >= M || (keys[f1] >> 14) != id) break;  // run ends in this window
+      if ((keys[f1 - 1] >> 14) != id) break;
+    }
+    dwte[(long)id * C + c] += acc;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Cross-entropy combine and mean loss
+// ------------------------------------------------------------------------------------------
+__global__ void ce_combine_kernel(const float *__restrict__ stats,
+                                  const float *__restrict__ tgt_logit, float *__restrict__ lse,
+                                  float *__restrict__ per_token, int M, int ntiles) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= M) return;
+  const float *s = stats + (long)row * ntiles * 2;
+  float mx = -INFINITY;
+  for (int t = lane; t < ntiles; t += 32) mx = fmaxf(mx, s[2 * t]);
+  mx = warp_max(mx);
+  float sum = 0.f;
+  for (int t = lane; t < ntiles; t += 32) {
+    float m = s[2 * t];
+    if (m > -INFINITY) sum += s[2 * t + 1] * expf(m - mx);
+  }
+  sum = warp_sum(sum);
+  if (lane == 0) {
+    float l = mx + logf(sum);
+    lse[row] = l;
+    per_token[row] = l - tgt_logit[row];
+  }
+}
+
+__global__ void mean_loss_kernel(const float *__restrict__ per_token, int M, DevScalars *sc) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) s += (double)per_token[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh[w];
+    float loss = (float)(t / (double)M);
+    sc->loss = loss;
+    sc->nonfinite = isfinite(loss) ? 0 : 1;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// K14 global grad norm: fixed partition into GN_BLOCKS contiguous ranges, last-arriving
+// block sums the partials in index order.
+// ------------------------------------------------------------------------------------------
+constexpr int GN_BLOCKS = 592;
+constexpr int GN_THREADS = 512;
+
+__global__ void __launch_bounds__(GN_THREADS)
+grad_norm_kernel(const float *__restrict__ g, size_t n, double *__restrict__ partials,
+                 DevScalars *sc) {
+  __shared__ double sh[GN_THREADS / 32];
+  __shared__ bool last;
+  const size_t n4 = n / 4;
+  const size_t per = (n4 + gridDim.x - 1) / gridDim.x;
+  const size_t b0 = blockIdx.x * per, b1 = min(n4, b0 + per);
+  float s = 0.f;
+  const float4 *g4 = reinterpret_cast<const float4 *>(g);
+  for (size_t i = b0 + threadIdx.x; i < b1; i += blockDim.x) {
+    float4 v = g4[i];
+    s += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (blockIdx.x == gridDim.x - 1)  // tail elements
+    for (size_t i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) s += g[i] * g[i];
+  double d = (double)s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = d;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < GN_THREADS / 32; ++w) t += sh[w];
+    partials[blockIdx.x] = t;
+    __threadfence();
+    unsigned prev = atomicAdd(&sc->counter, 1u);
+    last = (prev == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    double t = 0.0;
+    for (int b = 0; b < (int)gridDim.x; ++b) t += ((volatile double *)partials)[b];
+    sc->sumsq = t;
+    float nrm = (float)sqrt(t);
+    sc->norm = nrm;
+    float coef = (float)((double)sc->clip / (sqrt(t) + 1e-6));
+    sc->coef = coef > 1.f ? 1.f : coef;
+    if (!isfinite(nrm)) sc->nonfinite = 1;
+    sc->counter = 0u;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// K15 AdamW (order of the nanochat fused step: decay, first moment, bias correction, update)
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void adamw_one(float &p, float g, float &m, float &v, float lr,
+                                          float wd, float b1, float b2, float eps, float bias1,
+                                          float bias2, float coef) {
+  g *= coef;
+  p = p * (1.f - lr * wd);
+  m = m + (1.f - b1) * (g - m);
+  v = b2 * v + (1.f - b2) * g * g;
+  float denom = sqrtf(v / bias2) + eps;
+  p = p - (lr / bias1) * m / denom;
+}
+
+__global__ void adamw_kernel(float *__restrict__ p, const float *__restrict__ g,
+                             float *__restrict__ m, float *__restrict__ v,
+                             bf16 *__restrict__ shadow, size_t n, const DevScalars *sc) {
+  if (sc->nonfinite) return;
+  const float lr = sc->lr, wd = sc->wd, b1 = sc->beta1, b2 = sc->beta2, eps = sc->eps;
+  const float bias1 = sc->bias1, bias2 = sc->bias2, coef = sc->coef;
+  const size_t n4 = n / 4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 P = reinterpret_cast<float4 *>(p)[i];
+    float4 G = reinterpret_cast<const float4 *>(g)[i];
+    float4 Mm = reinterpret_cast<float4 *>(m)[i];
+    float4 Vv = reinterpret_cast<float4 *>(v)[i];
+    adamw_one(P.x, G.x, Mm.x, Vv.x, lr, wd, b1, b2, eps, bias1, bias2, coef);
+    adamw_one(P.y, G.y, Mm.y, Vv.y, lr, wd, b1, b2, eps, bias1, bias2, coef);
+    adamw_one(P.z, G.z, Mm.z, Vv.z, lr, wd, b1, b2, eps, bias1, bias2, coef);
+    adamw_one(P.w, G.w, Mm.w, Vv.w, lr, wd, b1, b2, eps, bias1, bias2, coef);
+    reinterpret_cast<float4 *>(p)[i] = P;
+    reinterpret_cast<float4 *>(m)[i] = Mm;
+    reinterpret_cast<float4 *>(v)[i] = Vv;
+    if (shadow) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(P.x, P.y), hi = __floats2bfloat162_rn(P.z, P.w);
+      uint2 u;
+      u.x = *reinterpret_cast<unsigned *>(&lo);
+      u.y = *reinterpret_cast<unsigned *>(&hi);
+      reinterpret_cast<uint2 *>(shadow)[i] = u;
+    }
+  }
+  if (blockIdx.x == 0)
+    for (size_t i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) {
+      float pp = p[i], mm = m[i], vv = v[i];
+      adamw_one(pp, g[i], mm, vv, lr, wd, b1, b2, eps, bias1, bias2, coef);
+      p[i] = pp; m[i] = mm; v[i] = vv;
+      if (shadow) shadow[i] = __float2bfloat16_rn(pp);
+    }
+}
+
+__global__ void to_bf16_kernel(const float *__restrict__ p, bf16 *__restrict__ out, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(p[i]);
+}
+
+int grid_for(long work, int threads, int cap = 148 * 16) {
+  long b = (work + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > cap) b = cap;
+  return (int)b;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------
+template <typename T>
+cudaError_t launch_embed_fwd(const int *tok, const int *tgt, const T *wte, const T *wpe, T *x,
+                             int M, int Tlen, int C, int V, DevScalars *sc, cudaStream_t st) {
+  long work = (long)M * (C / Vec<T>::N);
+  embed_fwd_kernel<T><<<grid_for(work, 256), 256, 0, st>>>(tok, tgt, wte, wpe, x, M, Tlen, C, V, sc);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_embed_bwd(const int *tok, const T *dx, float *dwte, float *dwpe, int M,
+                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st) {
+  const int Bn = M / Tlen;
+  dwpe_kernel<T><<<grid_for((long)maxT * C, 256), 256, 0, st>>>(dx, dwpe, Bn, Tlen, maxT, C);
+  CUDA_TRY(cudaGetLastError());
+  int n = 1;
+  while (n < M) n <<= 1;
+  sort_keys_kernel<<<1, 1024, n * sizeof(unsigned), st>>>(tok, M, ws.keys);
+  CUDA_TRY(cudaGetLastError());
+  const int nwin = (M + EW - 1) / EW;
+  embed_seg_kernel<T><<<nwin, 256, 0, st>>>(ws.keys, dx, dwte, ws.partial, M, C);
+  CUDA_TRY(cudaGetLastError());
+  embed_merge_kernel<<<nwin, 256, 0, st>>>(ws.keys, ws.partial, dwte, M, C, nwin);
+  return cudaGetLastError();
+}
+
+cudaError_t embed_sort_smem_attr() {
+  return cudaFuncSetAttribute(sort_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SORT_MAX * sizeof(unsigned));
+}
+
+template <typename T>
+cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
+                                 int C, float eps, cudaStream_t st) {
+  const int warps = 8;
+  layernorm_fwd_kernel<T><<<(M + warps - 1) / warps, warps * 32, 0, st>>>(x, g, y, mean, rstd,
+                                                                          M, C, eps);
+  return cudaGetLastError();
+}
+
+int layernorm_bwd_blocks(int M) {
+  int b = (M + LNB_WARPS - 1) / LNB_WARPS;
+  return b < LNB_MAX_BLOCKS ? b : LNB_MAX_BLOCKS;
+}
+
+template <typename T>
+cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
+                                 const T *dy, T *dres, float *dg_partial, float *dg, int M,
+                                 int C, cudaStream_t st) {
+  const int nb = layernorm_bwd_blocks(M);
+  const int rpb = (M + nb - 1) / nb;
+  const size_t smem = (size_t)LNB_WARPS * C * sizeof(float);
+  layernorm_bwd_kernel<T><<<nb, LNB_WARPS * 32, smem, st>>>(x, g, mean, rstd, dy, dres,
+                                                            dg_partial, M, C, rpb);
+  CUDA_TRY(cudaGetLastError());
+  colsum_kernel<<<(C + 255) / 256, 256, 0, st>>>(dg_partial, nb, C, dg);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ce_combine(const float *stats, const float *tgt_logit, float *lse,
+                              float *per_token, int M, int ntiles, DevScalars *sc,
+                              cudaStream_t st) {
+  ce_combine_kernel<<<(M + 7) / 8, 256, 0, st>>>(stats, tgt_logit, lse, per_token, M, ntiles);
+  CUDA_TRY(cudaGetLastError());
+  mean_loss_kernel<<<1, 1024, 0, st>>>(per_token, M, sc);
+  return cudaGetLastError();
+}
+
+int grad_norm_blocks() { return GN_BLOCKS; }
+
+cudaError_t launch_grad_norm(const float *g, size_t n, double *partials, DevScalars *sc,
+                             cudaStream_t st) {
+  grad_norm_kernel<<<GN_BLOCKS, GN_THREADS, 0, st>>>(g, n, partials, sc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, bf16 *shadow, size_t n,
+                         const DevScalars *sc, cudaStream_t st) {
+  adamw_kernel<<<grid_for((long)(n / 4), 256, 148 * 8), 256, 0, st>>>(p, g, m, v, shadow, n, sc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st) {
+  to_bf16_kernel<<<grid_for((long)n, 256, 148 * 8), 256, 0, st>>>(p, out, n);
+  return cudaGetLastError();
+}
+
+#define INST(T)                                                                              \
+  template cudaError_t launch_embed_fwd<T>(const int *, const int *, const T *, const T *, T *, \
+                                           int, int, int, int, DevScalars *, cudaStream_t);    \
+  template cudaError_t launch_embed_bwd<T>(const int *, const T *, float *, float *, int, int,  \
+                                           int, int, EmbedBwdWs, cudaStream_t);                \
+  template cudaError_t launch_layernorm_fwd<T>(const T *, const T *, T *, float *, float *, int, \
+                                               int, float, cudaStream_t);                      \
+  template cudaError_t launch_layernorm_bwd<T>(const T *, const T *, const float *,             \
+                                               const float *, const T *, T *, float *, float *, \
+                                               int, int, cudaStream_t);
+INST(float)
+INST(bf16)

@@ -1,0 +1,721 @@
+// C ABI and step schedule of the GPT-2 training-step library.
+//
+// One gpt_train_step enqueues, on the caller's stream: token staging, the embedding, n_layer
+// forward blocks, final LayerNorm, lm_head cross-entropy statistics, the chunked lm_head
+// backward, the block backward in reverse, the embedding backward, the global grad norm
+// and AdamW. The whole sequence for one (B, T) and one set of buffers is captured once into
+// a CUDA graph and replayed; lr / wd / clip / step live in device memory (nanochat
+// architecture page, "AdamW Fused Step": hyper-parameters held as tensors so that a
+// compiled step is reused when lr changes). The only host synchronisation is the read-back
+// of the loss, the grad norm and the device error word at the end of the call.
+#include <cuda.h>
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/gpt_step.h"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+cudaError_t embed_sort_smem_attr();
+
+namespace {
+
+constexpr int ALIGN = 256;
+constexpr int SIMT_TILE_N = 64;
+
+struct Layer {
+  size_t ln1, wqkv, wap, ln2, wfc, wmp;
+};
+
+struct Acts {  // per-layer saved activations
+  void *x_in, *a, *qkv, *o, *x_mid, *c, *pre, *h;
+  float *lse, *mu1, *rs1, *mu2, *rs2;
+};
+
+struct GraphKey {
+  int B, T, train;
+  const void *p, *g, *m, *v, *ptl;
+  bool operator<(const GraphKey &o) const {
+    return std::tie(B, T, train, p, g, m, v, ptl) <
+           std::tie(o.B, o.T, o.train, o.p, o.g, o.m, o.v, o.ptl);
+  }
+};
+
+}  // namespace
+
+struct gpt_handle {
+  gpt_config cfg;
+  std::vector<int> windows;
+  int C, H, hd, mC, V, Vp, L, maxT, maxB, maxM;
+  bool use_bf16;
+  size_t nparams;
+  size_t off_wte, off_wpe, off_lnf;
+  std::vector<Layer> layer;
+  std::vector<gpt_tensor_desc> descs;
+  int device;
+  cudaStream_t stream;
+  // workspace
+  char *ws;
+  size_t ws_bytes;
+  DevScalars *sc;
+  DevScalars *sc_host;  // pinned
+  int *tok, *tgt;
+  std::vector<Acts> acts;
+  void *x_final, *yf;
+  float *muf, *rsf;
+  float *stats, *tgt_logit, *lse_ce, *per_token;
+  int ce_tile_n, ce_ntiles;
+  void *dS;
+  long ldS;
+  int chunk_rows;
+  void *dx, *dh, *dc, *dqkv, *dout, *dyf;
+  float *Dbuf, *dg_partial;
+  double *gn_partials;
+  float *splitk;
+  size_t splitk_elems;
+  unsigned *sort_keys;
+  float *emb_partial;
+  bf16 *shadow;
+  // state
+  long step;
+  float last_norm;
+  const float *shadow_src;
+  bool shadow_valid;
+  bool use_graphs;
+  struct Captured {
+    cudaGraphExec_t exec;
+    int launches;
+  };
+  std::map<GraphKey, Captured> graphs;
+  int launches;
+  std::string cuda_err;
+  // kernel timing
+  bool time_kernels;
+  std::vector<cudaEvent_t> ev;
+  std::vector<double> ev_flops;
+  int ev_used;
+  long long stat_launches;
+  double stat_ms, stat_flops;
+  TcGemm *tc;
+};
+
+namespace {
+
+size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
+
+int fail(gpt_handle *h, cudaError_t e) {
+  if (h) h->cuda_err = cudaGetErrorString(e);
+  return e == cudaErrorMemoryAllocation ? GPT_ERR_OOM : GPT_ERR_CUDA;
+}
+
+#define TRY(x)                                  \
+  do {                                          \
+    cudaError_t e__ = (x);                      \
+    if (e__ != cudaSuccess) return fail(h, e__); \
+  } while (0)
+
+bool misaligned(const void *p) { return ((uintptr_t)p & 15u) != 0; }
+
+bool is_device_ptr(const void *p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+// --------------------------------------------------------------------------------------
+// GEMM dispatch
+// --------------------------------------------------------------------------------------
+int choose_split(const gpt_handle *h, int M, int N, int K, int tm, int tn) {
+  long tiles = (long)((M + tm - 1) / tm) * ((N + tn - 1) / tn);
+  int s = 1;
+  while (tiles * s < 2 * 148 && K / (s * 2) >= 256) s *= 2;
+  while (s > 1 && (size_t)s * M * N > h->splitk_elems) s /= 2;
+  return s;
+}
+
+cudaError_t gemm(gpt_handle *h, GemmDesc d) {
+  if (d.M <= 0 || d.N <= 0) return cudaSuccess;
+  const double flops = 2.0 * d.M * d.N * d.K;
+  int k = -1;
+  if (h->time_kernels && h->ev_used + 2 <= (int)h->ev.size()) {
+    k = h->ev_used;
+    h->ev_used += 2;
+    h->ev_flops[k / 2] = flops;
+    cudaError_t e = cudaEventRecord(h->ev[k], h->stream);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e;
+  const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
+  if (!h->use_bf16) {
+    if (d.epi.kind == EPI_CE_STATS) {
+      d.epi.tile_n = SIMT_TILE_N;
+      d.epi.ntiles = (d.N + SIMT_TILE_N - 1) / SIMT_TILE_N;
+      h->ce_ntiles = d.epi.ntiles;
+    }
+    if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 64, 64) : 1;
+    d.partial = h->splitk;
+    e = launch_gemm_simt<float>(d, h->stream);
+  } else if (h->tc && tc_gemm_supported(d)) {
+    if (d.epi.kind == EPI_CE_STATS) {
+      d.epi.tile_n = TC_BN;
+      d.epi.ntiles = (d.N + TC_BN - 1) / TC_BN;
+      h->ce_ntiles = d.epi.ntiles;
+    }
+    if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 128, 256) : 1;
+    d.partial = h->splitk;
+    e = tc_gemm_launch(h->tc, d, h->stream, &h->launches);
+  } else {
+    if (d.epi.kind == EPI_CE_STATS) {
+      d.epi.tile_n = SIMT_TILE_N;
+      d.epi.ntiles = (d.N + SIMT_TILE_N - 1) / SIMT_TILE_N;
+      h->ce_ntiles = d.epi.ntiles;
+    }
+    if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 64, 64) : 1;
+    d.partial = h->splitk;
+    e = launch_gemm_simt<bf16>(d, h->stream);
+  }
+  h->launches += 1 + (d.split_k > 1 ? 1 : 0);
+  if (e != cudaSuccess) return e;
+  if (k >= 0) return cudaEventRecord(h->ev[k + 1], h->stream);
+  return cudaSuccess;
+}
+
+GemmDesc gdesc(int M, int N, int K, const void *A, long lda, int ak, const void *B, long ldb,
+               int bk) {
+  GemmDesc d;
+  memset(&d, 0, sizeof(d));
+  d.M = M; d.N = N; d.K = K;
+  d.A = A; d.lda = lda; d.a_kmajor = ak;
+  d.B = B; d.ldb = ldb; d.b_kmajor = bk;
+  d.split_k = 0;
+  return d;
+}
+
+// --------------------------------------------------------------------------------------
+// the step schedule
+// --------------------------------------------------------------------------------------
+template <typename T>
+cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *adam_m,
+                    float *adam_v, int B, int Tlen, bool train, float *per_token_out) {
+  cudaStream_t st = h->stream;
+  const int C = h->C, H = h->H, mC = h->mC, V = h->V, M = B * Tlen;
+  const T *W = h->use_bf16 ? (const T *)h->shadow : (const T *)params;
+  DevScalars *sc = h->sc;
+  int &nl = h->launches;
+  h->ev_used = 0;
+
+  // ---------------- forward ----------------
+  T *x0 = (T *)h->acts[0].x_in;
+  CUDA_TRY(launch_embed_fwd<T>(h->tok, h->tgt, W + h->off_wte, W + h->off_wpe, x0, M, Tlen, C,
+                               V, sc, st)); nl++;
+  for (int l = 0; l < h->L; ++l) {
+    Acts &A = h->acts[l];
+    const Layer &P = h->layer[l];
+    T *xnext = (T *)(l + 1 < h->L ? h->acts[l + 1].x_in : h->x_final);
+    CUDA_TRY(launch_layernorm_fwd<T>((T *)A.x_in, W + P.ln1, (T *)A.a, A.mu1, A.rs1, M, C,
+                                     h->cfg.ln_eps, st)); nl++;
+    GemmDesc d = gdesc(M, 3 * C, C, A.a, C, 1, W + P.wqkv, C, 1);
+    d.epi.kind = EPI_STORE; d.epi.out = A.qkv; d.epi.ldo = 3 * C;
+    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(launch_attention_fwd<T>((T *)A.qkv, (T *)A.o, A.lse, B, Tlen, C, H,
+                                     h->windows[l], st)); nl++;
+    d = gdesc(M, C, C, A.o, C, 1, W + P.wap, C, 1);
+    d.epi.kind = EPI_RESID; d.epi.out = A.x_mid; d.epi.ldo = C; d.epi.aux = A.x_in; d.epi.ld_aux = C;
+    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(launch_layernorm_fwd<T>((T *)A.x_mid, W + P.ln2, (T *)A.c, A.mu2, A.rs2, M, C,
+                                     h->cfg.ln_eps, st)); nl++;
+    d = gdesc(M, mC, C, A.c, C, 1, W + P.wfc, C, 1);
+    d.epi.kind = EPI_STORE_GELU; d.epi.out = A.pre; d.epi.ldo = mC; d.epi.out2 = A.h; d.epi.ldo2 = mC;
+    CUDA_TRY(gemm(h, d));
+    d = gdesc(M, C, mC, A.h, mC, 1, W + P.wmp, mC, 1);
+    d.epi.kind = EPI_RESID; d.epi.out = xnext; d.epi.ldo = C; d.epi.aux = A.x_mid; d.epi.ld_aux = C;
+    CUDA_TRY(gemm(h, d));
+  }
+  CUDA_TRY(launch_layernorm_fwd<T>((T *)h->x_final, W + h->off_lnf, (T *)h->yf, h->muf, h->rsf,
+                                   M, C, h->cfg.ln_eps, st)); nl++;
+  // lm_head statistics (the logits stay on chip)
+  {
+    GemmDesc d = gdesc(M, V, C, h->yf, C, 1, W + h->off_wte, C, 1);
+    d.split_k = 1;
+    Epi &e = d.epi;
+    e.kind = EPI_CE_STATS; e.targets = h->tgt; e.stats = h->stats; e.tgt_logit = h->tgt_logit;
+    e.V = V; e.row_offset = 0; e.sc = sc;
+    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(launch_ce_combine(h->stats, h->tgt_logit, h->lse_ce, h->per_token, M, h->ce_ntiles,
+                               sc, st)); nl += 2;
+  }
+  if (per_token_out) {
+    CUDA_TRY(cudaMemcpyAsync(per_token_out, h->per_token, sizeof(float) * M,
+                             cudaMemcpyDeviceToDevice, st));
+  }
+  if (!train) return cudaSuccess;
+
+  // ---------------- backward ----------------
+  float *G = grads;
+  CUDA_TRY(cudaMemsetAsync(G + h->off_wte, 0, sizeof(float) * (size_t)h->Vp * C, st));
+  for (int r0 = 0; r0 < M; r0 += h->chunk_rows) {
+    const int R = M - r0 < h->chunk_rows ? M - r0 : h->chunk_rows;
+    const T *yf_c = (const T *)h->yf + (size_t)r0 * C;
+    GemmDesc d = gdesc(R, V, C, yf_c, C, 1, W + h->off_wte, C, 1);
+    d.split_k = 1;
+    Epi &e = d.epi;
+    e.kind = EPI_CE_DS; e.out = h->dS; e.ldo = h->ldS; e.targets = h->tgt; e.lse = h->lse_ce;
+    e.V = V; e.row_offset = r0; e.sc = sc;
+    CUDA_TRY(gemm(h, d));
+    // dyf = dS . wte
+    d = gdesc(R, C, V, h->dS, h->ldS, 1, W + h->off_wte, C, 0);
+    d.epi.kind = EPI_STORE; d.epi.out = (T *)h->dyf + (size_t)r0 * C; d.epi.ldo = C;
+    CUDA_TRY(gemm(h, d));
+    // dwte += dS^T . yf
+    d = gdesc(V, C, R, h->dS, h->ldS, 0, yf_c, C, 0);
+    d.epi.kind = EPI_F32_ACCUM; d.epi.outf = G + h->off_wte; d.epi.ldf = C;
+    d.split_k = 1;
+    CUDA_TRY(gemm(h, d));
+  }
+  T *dx = (T *)h->dx;
+  CUDA_TRY(cudaMemsetAsync(dx, 0, sizeof(T) * (size_t)M * C, st));
+  CUDA_TRY(launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf,
+                                   dx, h->dg_partial, G + h->off_lnf, M, C, st)); nl += 2;
+  for (int l = h->L - 1; l >= 0; --l) {
+    Acts &A = h->acts[l];
+    const Layer &P = h->layer[l];
+    // MLP: x_out = x_mid + gelu(c Wfc^T) Wmp^T
+    GemmDesc d = gdesc(M, mC, C, dx, C, 1, W + P.wmp, mC, 0);
+    d.epi.kind = EPI_DGELU; d.epi.out = h->dh; d.epi.ldo = mC; d.epi.aux = A.pre; d.epi.ld_aux = mC;
+    CUDA_TRY(gemm(h, d));
+    d = gdesc(C, mC, M, dx, C, 0, A.h, mC, 0);
+    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wmp; d.epi.ldf = mC;
+    CUDA_TRY(gemm(h, d));
+    d = gdesc(M, C, mC, h->dh, mC, 1, W + P.wfc, C, 0);
+    d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
+    CUDA_TRY(gemm(h, d));
+    d = gdesc(mC, C, M, h->dh, mC, 0, A.c, C, 0);
+    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wfc; d.epi.ldf = C;
+    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx,
+                                     h->dg_partial, G + P.ln2, M, C, st)); nl += 2;
+    // attention: x_mid = x_in + attn(a) Wap^T
+    d = gdesc(M, C, C, dx, C, 1, W + P.wap, C, 0);
+    d.epi.kind = EPI_STORE; d.epi.out = h->dout; d.epi.ldo = C;
+    CUDA_TRY(gemm(h, d));
+    d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
+    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wap; d.epi.ldf = C;
+    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(launch_attention_bwd<T>((T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, h->Dbuf,
+                                     (T *)h->dqkv, B, Tlen, C, H, h->windows[l], st)); nl += 2;
+    d = gdesc(M, C, 3 * C, h->dqkv, 3 * C, 1, W + P.wqkv, C, 0);
+    d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
+    CUDA_TRY(gemm(h, d));
+    d = gdesc(3 * C, C, M, h->dqkv, 3 * C, 0, A.a, C, 0);
+    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
+    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
+                                     h->dg_partial, G + P.ln1, M, C, st)); nl += 2;
+  }
+  EmbedBwdWs ew{h->sort_keys, h->emb_partial};
+  CUDA_TRY(launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C,
+                               ew, st)); nl += 4;
+  // ---------------- clip + AdamW ----------------
+  CUDA_TRY(launch_grad_norm(G, h->nparams, h->gn_partials, sc, st)); nl++;
+  CUDA_TRY(launch_adamw((float *)params, G, adam_m, adam_v, h->use_bf16 ? h->shadow : nullptr,
+                        h->nparams, sc, st)); nl++;
+  return cudaSuccess;
+}
+
+cudaError_t run(gpt_handle *h, const float *params, float *grads, float *m, float *v, int B,
+                int Tlen, bool train, float *ptl) {
+  if (h->use_bf16) return enqueue<bf16>(h, params, grads, m, v, B, Tlen, train, ptl);
+  return enqueue<float>(h, params, grads, m, v, B, Tlen, train, ptl);
+}
+
+int check_common(gpt_handle *h, const void *params, const int *tokens, const int *targets, int B,
+                 int Tlen) {
+  if (!h || !params || !tokens || !targets) return GPT_ERR_INVALID_ARG;
+  if (B <= 0 || Tlen <= 0 || B > h->maxB || Tlen > h->maxT) return GPT_ERR_SHAPE;
+  if (misaligned(params)) return GPT_ERR_ALIGN;
+  return GPT_OK;
+}
+
+// Copies tokens/targets (host or device) into the workspace and the hyper-parameters into
+// device scalars.
+int stage_inputs(gpt_handle *h, const int *tokens, const int *targets, int M) {
+  const cudaMemcpyKind kt = is_device_ptr(tokens) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  const cudaMemcpyKind kg = is_device_ptr(targets) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  TRY(cudaMemcpyAsync(h->tok, tokens, sizeof(int) * M, kt, h->stream));
+  TRY(cudaMemcpyAsync(h->tgt, targets, sizeof(int) * M, kg, h->stream));
+  TRY(cudaMemcpyAsync(h->sc, h->sc_host, offsetof(DevScalars, sumsq), cudaMemcpyHostToDevice,
+                      h->stream));
+  // the device-written results of the previous call are cleared
+  TRY(cudaMemsetAsync((char *)h->sc + offsetof(DevScalars, loss), 0,
+                      offsetof(DevScalars, counter) - offsetof(DevScalars, loss), h->stream));
+  return GPT_OK;
+}
+
+int launch_step(gpt_handle *h, const float *params, float *grads, float *m, float *v, int B,
+                int Tlen, bool train, float *ptl) {
+  h->launches = 0;
+  const bool capture_ok = h->use_graphs && h->stream != nullptr && !h->time_kernels;
+  if (!capture_ok) {
+    TRY(run(h, params, grads, m, v, B, Tlen, train, ptl));
+    return GPT_OK;
+  }
+  GraphKey key{B, Tlen, train ? 1 : 0, params, grads, m, v, ptl};
+  auto it = h->graphs.find(key);
+  if (it == h->graphs.end()) {
+    cudaGraph_t g;
+    TRY(cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
+    cudaError_t e = run(h, params, grads, m, v, B, Tlen, train, ptl);
+    cudaError_t e2 = cudaStreamEndCapture(h->stream, &g);
+    if (e != cudaSuccess) return fail(h, e);
+    if (e2 != cudaSuccess) return fail(h, e2);
+    cudaGraphExec_t ex;
+    e = cudaGraphInstantiate(&ex, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return fail(h, e);
+    it = h->graphs.emplace(key, gpt_handle::Captured{ex, h->launches}).first;
+  }
+  h->launches = it->second.launches;
+  TRY(cudaGraphLaunch(it->second.exec, h->stream));
+  return GPT_OK;
+}
+
+int finish(gpt_handle *h, float *loss) {
+  TRY(cudaMemcpyAsync(h->sc_host, h->sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, h->stream));
+  TRY(cudaStreamSynchronize(h->stream));
+  if (loss) *loss = h->sc_host->loss;
+  if (h->time_kernels) {
+    for (int k = 0; k + 1 < h->ev_used; k += 2) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, h->ev[k], h->ev[k + 1]) == cudaSuccess) {
+        h->stat_ms += ms;
+        h->stat_flops += h->ev_flops[k / 2];
+        h->stat_launches++;
+      }
+    }
+  }
+  const unsigned err = h->sc_host->err;
+  if (err & GPT_DEVERR_TIMEOUT) return GPT_ERR_DEVICE_TIMEOUT;
+  if (err & (GPT_DEVERR_BAD_TOKEN | GPT_DEVERR_BAD_TARGET)) return GPT_ERR_BAD_TOKEN;
+  return GPT_OK;
+}
+
+void set_hyper(gpt_handle *h, int M, float lr, float wd, float clip, long t) {
+  DevScalars *s = h->sc_host;
+  s->lr = lr; s->wd = wd; s->clip = clip;
+  s->beta1 = h->cfg.beta1; s->beta2 = h->cfg.beta2; s->eps = h->cfg.adam_eps;
+  s->bias1 = (float)(1.0 - pow((double)h->cfg.beta1, (double)t));
+  s->bias2 = (float)(1.0 - pow((double)h->cfg.beta2, (double)t));
+  s->inv_M = (float)(1.0 / (double)M);
+  s->step = (int)t;
+}
+
+}  // namespace
+
+// ======================================================================================
+// C ABI
+// ======================================================================================
+extern "C" {
+
+const char *gpt_strerror(int s) {
+  switch (s) {
+    case GPT_OK: return "ok";
+    case GPT_ERR_INVALID_ARG: return "invalid argument";
+    case GPT_ERR_SHAPE: return "unsupported shape";
+    case GPT_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case GPT_ERR_OOM: return "out of device memory";
+    case GPT_ERR_CUDA: return "CUDA error";
+    case GPT_ERR_NONFINITE: return "non-finite loss or gradient norm; update skipped";
+    case GPT_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case GPT_ERR_BAD_TOKEN: return "token or target id out of range";
+    default: return "unknown status";
+  }
+}
+
+gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
+  int dummy;
+  if (!status) status = &dummy;
+  *status = GPT_ERR_INVALID_ARG;
+  if (!cfg) return nullptr;
+  const gpt_config c = *cfg;
+  if (c.precision != GPT_FP32 && c.precision != GPT_BF16) return nullptr;
+  if (c.vocab <= 0 || c.vocab_padded < c.vocab || c.n_layer <= 0 || c.n_head <= 0 ||
+      c.n_embd <= 0 || c.max_T <= 0 || c.max_B <= 0 || c.mlp_mult <= 0)
+    return nullptr;
+  if (!(c.ln_eps > 0.f) || !(c.beta1 >= 0.f && c.beta1 < 1.f) || !(c.beta2 >= 0.f && c.beta2 < 1.f) ||
+      !(c.adam_eps > 0.f))
+    return nullptr;
+  *status = GPT_ERR_SHAPE;
+  const int C = c.n_embd, H = c.n_head;
+  if (C % H) return nullptr;
+  const int hd = C / H;
+  if (hd != 32 && hd != 64 && hd != 128) return nullptr;
+  const bool bf = c.precision == GPT_BF16;
+  if (bf ? (C % 64 != 0) : (C % 4 != 0)) return nullptr;
+  if (C > (bf ? 2048 : 1024)) return nullptr;
+  if ((long)c.max_B * c.max_T > 16384) return nullptr;
+  if (c.vocab_padded > 131072) return nullptr;
+
+  gpt_handle *h = new gpt_handle();
+  h->cfg = c;
+  h->windows.assign(c.n_layer, -1);
+  if (c.window_left)
+    for (int l = 0; l < c.n_layer; ++l) h->windows[l] = c.window_left[l];
+  h->cfg.window_left = nullptr;
+  h->C = C; h->H = H; h->hd = hd; h->mC = c.mlp_mult * C; h->V = c.vocab; h->Vp = c.vocab_padded;
+  h->L = c.n_layer; h->maxT = c.max_T; h->maxB = c.max_B; h->maxM = c.max_B * c.max_T;
+  h->use_bf16 = bf;
+  h->stream = nullptr;
+  h->step = 0;
+  h->last_norm = NAN;
+  h->shadow_src = nullptr;
+  h->shadow_valid = false;
+  h->use_graphs = true;
+  h->time_kernels = false;
+  h->ev_used = 0;
+  h->stat_launches = 0; h->stat_ms = 0; h->stat_flops = 0;
+  h->tc = nullptr;
+  cudaGetDevice(&h->device);
+
+  // ---- parameter layout ----
+  size_t off = 0;
+  auto add = [&](const char *name, int nd, long long d0, long long d1) {
+    gpt_tensor_desc d;
+    memset(&d, 0, sizeof(d));
+    snprintf(d.name, sizeof(d.name), "%s", name);
+    d.offset = (long long)off; d.ndim = nd; d.shape[0] = d0; d.shape[1] = nd > 1 ? d1 : 0;
+    h->descs.push_back(d);
+    size_t n = (size_t)d0 * (nd > 1 ? (size_t)d1 : 1);
+    size_t o = off;
+    off += n;
+    return o;
+  };
+  char nm[32];
+  h->off_wte = add("wte", 2, h->Vp, C);
+  h->off_wpe = add("wpe", 2, h->maxT, C);
+  for (int l = 0; l < h->L; ++l) {
+    Layer P;
+    snprintf(nm, 32, "h%d.ln1.g", l); P.ln1 = add(nm, 1, C, 0);
+    snprintf(nm, 32, "h%d.w_qkv", l); P.wqkv = add(nm, 2, 3 * C, C);
+    snprintf(nm, 32, "h%d.w_attnproj", l); P.wap = add(nm, 2, C, C);
+    snprintf(nm, 32, "h%d.ln2.g", l); P.ln2 = add(nm, 1, C, 0);
+    snprintf(nm, 32, "h%d.w_fc", l); P.wfc = add(nm, 2, h->mC, C);
+    snprintf(nm, 32, "h%d.w_mlpproj", l); P.wmp = add(nm, 2, C, h->mC);
+    h->layer.push_back(P);
+  }
+  h->off_lnf = add("lnf.g", 1, C, 0);
+  h->nparams = off;
+
+  // ---- workspace ----
+  const size_t es = bf ? 2 : 4;
+  const size_t M = h->maxM;
+  h->ce_tile_n = SIMT_TILE_N;  // the stats buffer is sized for the narrowest column tile
+  h->ce_ntiles = (h->V + h->ce_tile_n - 1) / h->ce_tile_n;
+  h->chunk_rows = c.lmhead_chunk_rows > 0 ? c.lmhead_chunk_rows : 4096;
+  if (h->chunk_rows > (int)M) h->chunk_rows = (int)M;
+  h->ldS = (h->V + 7) / 8 * 8;
+  h->splitk_elems = (size_t)8 * ((size_t)h->mC * C > (size_t)M * C ? (size_t)h->mC * C : (size_t)M * C);
+
+  std::vector<std::pair<void **, size_t>> req;
+  auto need = [&](void **p, size_t bytes) { req.push_back({p, bytes}); };
+  h->acts.resize(h->L);
+  for (int l = 0; l < h->L; ++l) {
+    Acts &A = h->acts[l];
+    need(&A.x_in, M * C * es); need(&A.a, M * C * es); need(&A.qkv, M * 3 * C * es);
+    need(&A.o, M * C * es); need(&A.x_mid, M * C * es); need(&A.c, M * C * es);
+    need(&A.pre, M * h->mC * es); need(&A.h, M * h->mC * es);
+    need((void **)&A.lse, M * H * 4); need((void **)&A.mu1, M * 4); need((void **)&A.rs1, M * 4);
+    need((void **)&A.mu2, M * 4); need((void **)&A.rs2, M * 4);
+  }
+  need(&h->x_final, M * C * es); need(&h->yf, M * C * es);
+  need((void **)&h->muf, M * 4); need((void **)&h->rsf, M * 4);
+  need((void **)&h->stats, M * h->ce_ntiles * 8); need((void **)&h->tgt_logit, M * 4);
+  need((void **)&h->lse_ce, M * 4); need((void **)&h->per_token, M * 4);
+  need(&h->dS, (size_t)h->chunk_rows * h->ldS * es);
+  need(&h->dx, M * C * es); need(&h->dh, M * h->mC * es); need(&h->dc, M * C * es);
+  need(&h->dqkv, M * 3 * C * es); need(&h->dout, M * C * es); need(&h->dyf, M * C * es);
+  need((void **)&h->Dbuf, M * H * 4);
+  need((void **)&h->dg_partial, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
+  need((void **)&h->gn_partials, (size_t)grad_norm_blocks() * 8);
+  need((void **)&h->splitk, h->splitk_elems * 4);
+  need((void **)&h->sort_keys, M * 4);
+  need((void **)&h->emb_partial, ((M + 31) / 32) * 2 * (size_t)C * 4);
+  need((void **)&h->tok, M * 4); need((void **)&h->tgt, M * 4);
+  need((void **)&h->sc, sizeof(DevScalars));
+  if (bf) need((void **)&h->shadow, h->nparams * 2);
+  else h->shadow = nullptr;
+  size_t total = 0;
+  for (auto &r : req) total += align_up(r.second);
+  h->ws_bytes = total;
+  cudaError_t e = cudaMalloc(&h->ws, total);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *status = e == cudaErrorMemoryAllocation ? GPT_ERR_OOM : GPT_ERR_CUDA;
+    delete h;
+    return nullptr;
+  }
+  size_t o2 = 0;
+  for (auto &r : req) {
+    *r.first = h->ws + o2;
+    o2 += align_up(r.second);
+  }
+  *status = GPT_ERR_CUDA;
+  if (cudaMemset(h->ws, 0, total) != cudaSuccess || cudaMallocHost(&h->sc_host, sizeof(DevScalars)) != cudaSuccess ||
+      embed_sort_smem_attr() != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(h->ws);
+    delete h;
+    return nullptr;
+  }
+  memset(h->sc_host, 0, sizeof(DevScalars));
+  if (bf) {
+    if (tc_gemm_create(&h->tc) != cudaSuccess) {
+      cudaGetLastError();
+      h->tc = nullptr;
+    }
+  }
+  *status = GPT_OK;
+  return h;
+}
+
+void gpt_destroy(gpt_handle *h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  for (auto &kv : h->graphs) cudaGraphExecDestroy(kv.second.exec);
+  for (auto ev : h->ev) cudaEventDestroy(ev);
+  if (h->tc) tc_gemm_destroy(h->tc);
+  cudaFree(h->ws);
+  cudaFreeHost(h->sc_host);
+  delete h;
+}
+
+size_t gpt_num_params(const gpt_handle *h) { return h ? h->nparams : 0; }
+
+int gpt_param_layout(const gpt_handle *h, gpt_tensor_desc *out, int cap) {
+  if (!h || (cap > 0 && !out)) return GPT_ERR_INVALID_ARG;
+  for (int i = 0; i < (int)h->descs.size() && i < cap; ++i) out[i] = h->descs[i];
+  return (int)h->descs.size();
+}
+
+int gpt_set_stream(gpt_handle *h, void *s) {
+  if (!h) return GPT_ERR_INVALID_ARG;
+  h->stream = (cudaStream_t)s;
+  return GPT_OK;
+}
+
+int gpt_params_changed(gpt_handle *h) {
+  if (!h) return GPT_ERR_INVALID_ARG;
+  h->shadow_valid = false;
+  return GPT_OK;
+}
+
+int gpt_forward_loss(gpt_handle *h, const float *params, const int *tokens, const int *targets,
+                     int B, int T, float *loss, float *per_token_loss) {
+  int s = check_common(h, params, tokens, targets, B, T);
+  if (s) return s;
+  if (!loss) return GPT_ERR_INVALID_ARG;
+  cudaSetDevice(h->device);
+  const int M = B * T;
+  set_hyper(h, M, 0.f, 0.f, 1.f, h->step + 1);
+  if ((s = stage_inputs(h, tokens, targets, M))) return s;
+  if (h->use_bf16) {  // forward-only calls refresh the bf16 weights every time
+    TRY(launch_to_bf16(params, h->shadow, h->nparams, h->stream));
+    h->shadow_src = params;
+    h->shadow_valid = true;
+  }
+  h->launches = 0;
+  TRY(run(h, params, nullptr, nullptr, nullptr, B, T, false, per_token_loss));
+  s = finish(h, loss);
+  if (s) return s;
+  return isfinite(*loss) ? GPT_OK : GPT_ERR_NONFINITE;
+}
+
+int gpt_train_step(gpt_handle *h, float *params, float *grads, float *adam_m, float *adam_v,
+                   const int *tokens, const int *targets, int B, int T, float lr, float wd,
+                   float clip, float *loss) {
+  int s = check_common(h, params, tokens, targets, B, T);
+  if (s) return s;
+  if (!grads || !adam_m || !adam_v || !loss) return GPT_ERR_INVALID_ARG;
+  if (misaligned(grads) || misaligned(adam_m) || misaligned(adam_v)) return GPT_ERR_ALIGN;
+  if (!isfinite(lr) || !isfinite(wd) || !(clip > 0.f)) return GPT_ERR_INVALID_ARG;
+  cudaSetDevice(h->device);
+  const int M = B * T;
+  const long t = h->step + 1;
+  set_hyper(h, M, lr, wd, clip, t);
+  if ((s = stage_inputs(h, tokens, targets, M))) return s;
+  if (h->use_bf16 && (!h->shadow_valid || h->shadow_src != params)) {
+    TRY(launch_to_bf16(params, h->shadow, h->nparams, h->stream));
+    h->shadow_src = params;
+    h->shadow_valid = true;
+  }
+  if ((s = launch_step(h, params, grads, adam_m, adam_v, B, T, true, nullptr))) return s;
+  s = finish(h, loss);
+  h->last_norm = h->sc_host->norm;
+  if (s) return s;
+  if (h->sc_host->nonfinite) return GPT_ERR_NONFINITE;
+  h->step = t;
+  return GPT_OK;
+}
+
+int gpt_get_step(const gpt_handle *h, long *step) {
+  if (!h || !step) return GPT_ERR_INVALID_ARG;
+  *step = h->step;
+  return GPT_OK;
+}
+
+int gpt_set_step(gpt_handle *h, long step) {
+  if (!h || step < 0) return GPT_ERR_INVALID_ARG;
+  h->step = step;
+  h->shadow_valid = false;
+  return GPT_OK;
+}
+
+float gpt_last_grad_norm(const gpt_handle *h) { return h ? h->last_norm : NAN; }
+
+int gpt_set_option(gpt_handle *h, int option, long value) {
+  if (!h) return GPT_ERR_INVALID_ARG;
+  if (option == GPT_OPT_USE_GRAPHS) {
+    h->use_graphs = value != 0;
+    return GPT_OK;
+  }
+  if (option == GPT_OPT_TIME_KERNELS) {
+    h->time_kernels = value != 0;
+    if (h->time_kernels && h->ev.empty()) {
+      const int n = 2 * (16 * h->L + 64);
+      h->ev.resize(n);
+      h->ev_flops.assign(n / 2, 0.0);
+      for (int i = 0; i < n; ++i)
+        if (cudaEventCreate(&h->ev[i]) != cudaSuccess) return fail(h, cudaGetLastError());
+    }
+    return GPT_OK;
+  }
+  return GPT_ERR_INVALID_ARG;
+}
+
+int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
+                     double *flops, int reset) {
+  if (!h || kind != 0) return GPT_ERR_INVALID_ARG;
+  if (launches) *launches = h->stat_launches;
+  if (total_ms) *total_ms = h->stat_ms;
+  if (flops) *flops = h->stat_flops;
+  if (reset) {
+    h->stat_launches = 0;
+    h->stat_ms = 0;
+    h->stat_flops = 0;
+  }
+  return GPT_OK;
+}
+
+int gpt_last_launch_count(const gpt_handle *h) { return h ? h->launches : 0; }
+
+const char *gpt_last_cuda_error(const gpt_handle *h) { return h ? h->cuda_err.c_str() : ""; }
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+/* gpt_step.h -- C ABI of the B200 (sm_100a) GPT-2-style training-step library.
+ *
+ * One call runs one whole training step of a nanoGPT/GPT-2 decoder on one GPU: token +
+ * position embedding, n_layer pre-LayerNorm blocks (causal attention with an optional left
+ * window per layer, GELU(tanh) MLP), final LayerNorm, tied lm_head with mean softmax
+ * cross-entropy, the full backward pass, a global grad-norm clip and a fused AdamW update.
+ *
+ * What the operations follow (pages cited by title and section):
+ *   - model and config fields: nanoGPT README (intro: reproduces GPT-2 124M, loads OpenAI's
+ *     GPT-2 weights) and the Panthalia "Create a Plugin" page (GPTConfig: block_size,
+ *     vocab_size, n_layer, n_head, n_embd, dropout, bias=False);
+ *   - per-layer sliding window and the FLOPs count: nanochat architecture page,
+ *     "Modellarchitektur und FLOPs-Berechnung";
+ *   - loss: NiNo README, "Usage" (F.cross_entropy over the logits, mean reduction);
+ *   - clipping: llm.c summary ("Reimplementando el modelo GPT-2 ... con llm.c"),
+ *     "Proceso de entrenamiento";
+ *   - AdamW order and hyper-parameters held in device memory so a captured step replays
+ *     with a new lr: nanochat architecture page, "Optimierungsstrategien Muon und AdamW",
+ *     "AdamW Fused Step";
+ *   - the flat parameter vector: Panthalia page, "Components of the Example Plugin" (the
+ *     model adapter maps the model to and from a flattened tensor).
+ *
+ * Threading: a handle is not thread-safe; use one handle per host thread.
+ * Errors: every int-returning call returns GPT_OK (0) or a negative GPT_ERR_* code; no C++
+ * exception crosses this boundary. gpt_strerror() names a code.
+ */
+#ifndef GPT_STEP_H
+#define GPT_STEP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPT_OK                  0
+#define GPT_ERR_INVALID_ARG    -1  /* NULL handle/pointer, bad enum, bad hyper-parameter      */
+#define GPT_ERR_SHAPE          -2  /* config not supported, B > max_B, T > max_T, B*T = 0     */
+#define GPT_ERR_ALIGN          -3  /* a device pointer is not 16-byte aligned                 */
+#define GPT_ERR_OOM            -4  /* cudaMalloc of the workspace failed                      */
+#define GPT_ERR_CUDA           -5  /* a CUDA runtime/driver call failed (see gpt_last_cuda_error) */
+#define GPT_ERR_NONFINITE      -6  /* loss or grad norm is NaN/Inf: the update was skipped    */
+#define GPT_ERR_DEVICE_TIMEOUT -7  /* a bounded device-side wait expired                      */
+#define GPT_ERR_BAD_TOKEN      -8  /* a token id outside [0, vocab) or target outside [0, vocab) */
+
+#define GPT_FP32 0  /* validation mode: fp32 activations and fp32 GEMMs (CUDA cores)          */
+#define GPT_BF16 1  /* bf16 operands on tcgen05 tensor cores, fp32 accumulation/master state  */
+
+typedef struct {
+  int vocab;             /* V: ids 0..V-1 take part in the softmax                            */
+  int vocab_padded;      /* Vp >= V: rows of wte; rows >= V are outside the softmax            */
+  int n_layer, n_head, n_embd;
+  int max_T;             /* rows of wpe and the largest T a call may use                       */
+  int max_B;             /* largest B a call may use (sizes the workspace)                     */
+  int mlp_mult;          /* MLP hidden = mlp_mult * n_embd (4 for GPT-2)                      */
+  const int *window_left;/* n_layer entries (copied), or NULL for all -1. -1 = full causal;
+                            w >= 0 = query i attends keys j with i-w <= j <= i                 */
+  float ln_eps;          /* LayerNorm epsilon (1e-5)                                            */
+  float beta1, beta2;    /* AdamW betas (0.9, 0.95)                                             */
+  float adam_eps;        /* AdamW epsilon (1e-8)                                                */
+  int precision;         /* GPT_FP32 or GPT_BF16                                                */
+  int lmhead_chunk_rows; /* rows per lm_head backward chunk (0 = library default); the largest
+                            B*T*V-shaped buffer the step keeps is chunk_rows * Vp bf16          */
+} gpt_config;
+
+typedef struct {
+  char name[32];         /* e.g. "wte", "h3.w_fc", "lnf.g"                                     */
+  long long offset;      /* element offset into the flat fp32 vector                           */
+  int ndim;              /* 1 or 2                                                              */
+  long long shape[2];    /* row-major [out, in] for weights                                     */
+} gpt_tensor_desc;
+
+typedef struct gpt_handle gpt_handle;
+
+/* Validates cfg, computes the parameter layout, allocates the workspace (activations for
+ * max_B*max_T tokens, the bf16 weight shadow, device scalars) on the current CUDA device.
+ * Returns NULL and sets *status (if non-NULL) on failure. Supported shapes: n_embd % n_head
+ * == 0, head_dim in {32, 64, 128} (bf16: n_embd % 64 == 0, head_dim == 64),
+ * max_B * max_T <= 16384, vocab_padded <= 131072. */
+gpt_handle *gpt_create(const gpt_config *cfg, int *status);
+void gpt_destroy(gpt_handle *h);
+
+/* Number of fp32 elements in the flat params/grads/adam_m/adam_v vectors. */
+size_t gpt_num_params(const gpt_handle *h);
+
+/* Writes up to cap descriptors in flat order: wte [Vp,C], wpe [max_T,C], per layer
+ * (ln1.g [C], w_qkv [3C,C], w_attnproj [C,C], ln2.g [C], w_fc [mC,C], w_mlpproj [C,mC]),
+ * lnf.g [C]. Returns the number of tensors (6*n_layer + 3), or a negative code. */
+int gpt_param_layout(const gpt_handle *h, gpt_tensor_desc *out, int cap);
+
+/* All device work of later calls is enqueued on this cudaStream_t (NULL = legacy default). */
+int gpt_set_stream(gpt_handle *h, void *cuda_stream);
+
+/* Forward pass only. params: device fp32 [num_params], read only. tokens, targets: int32
+ * [B,T] row-major, device memory or host memory (host buffers are copied in; pinned host
+ * memory keeps the copy asynchronous). loss: host float, the mean cross-entropy.
+ * per_token_loss: NULL or device fp32 [B,T]. Blocks until the loss is on the host. */
+int gpt_forward_loss(gpt_handle *h, const float *params, const int *tokens, const int *targets,
+                     int B, int T, float *loss, float *per_token_loss);
+
+/* One training step with t = (current step) + 1:
+ *   forward -> loss; backward -> grads (RAW, unclipped, overwritten; every element written);
+ *   norm = ||grads||_2; coef = min(1, clip / (norm + 1e-6));
+ *   AdamW on coef*grads: p *= 1 - lr*wd; m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+ *   p -= (lr / (1-b1^t)) * m / (sqrt(v / (1-b2^t)) + eps).
+ * params, adam_m, adam_v: device fp32 [num_params], updated in place (caller-owned; adam_m
+ * and adam_v start zeroed). grads: device fp32 [num_params], written. tokens/targets as in
+ * gpt_forward_loss. loss: host float. Weight decay applies to every element.
+ * On GPT_ERR_NONFINITE, params/m/v are unchanged and the step counter does not advance. */
+int gpt_train_step(gpt_handle *h, float *params, float *grads, float *adam_m, float *adam_v,
+                   const int *tokens, const int *targets, int B, int T, float lr, float wd,
+                   float clip, float *loss);
+
+/* Step counter (number of completed AdamW updates); gpt_set_step is for resuming. */
+int gpt_get_step(const gpt_handle *h, long *step);
+int gpt_set_step(gpt_handle *h, long step);
+
+/* Unclipped global grad norm of the last gpt_train_step (NaN before the first). */
+float gpt_last_grad_norm(const gpt_handle *h);
+
+/* In bf16 mode the step keeps a bf16 copy of the weights that AdamW refreshes. Call this
+ * after changing params outside gpt_train_step (e.g. loading a checkpoint into the same
+ * buffer); a different params pointer is detected automatically. */
+int gpt_params_changed(gpt_handle *h);
+
+/* Options (gpt_set_option): capture each (B,T) step shape into a CUDA graph (default 1);
+ * record CUDA events around every GEMM launch for kernel timing (default 0). */
+#define GPT_OPT_USE_GRAPHS 1
+#define GPT_OPT_TIME_KERNELS 2
+int gpt_set_option(gpt_handle *h, int option, long value);
+
+/* Per kernel class accumulated by GPT_OPT_TIME_KERNELS since the last reset: launches,
+ * total milliseconds and algorithmic FLOPs. kind: 0 = tensor-core GEMMs (all of them).
+ * reset != 0 clears the counters after reading. */
+int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
+                     double *flops, int reset);
+
+/* Number of kernels the last gpt_train_step / gpt_forward_loss enqueued. */
+int gpt_last_launch_count(const gpt_handle *h);
+
+const char *gpt_strerror(int status);
+/* Text of the last CUDA error seen by this handle ("" if none). */
+const char *gpt_last_cuda_error(const gpt_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT_STEP_H */
