@@ -51,7 +51,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if bad:
         raise RuntimeError("nvcc failed")
     tmp = OUT + f".tmp{os.getpid()}"
-    subprocess.check_call([_nvcc(), *ARCH, "-shared", *objs, "-o", tmp, "-lcuda"])
+    subprocess.check_call([_nvcc(), *ARCH, "-shared", *objs, "-o", tmp])
     os.replace(tmp, OUT)
     return OUT
 

@@ -94,6 +94,7 @@ struct GemmDesc {
   Epi epi;
   int split_k;       // > 1: fp32 partials [split][M][N] then an ordered reduction
   float *partial;
+  unsigned *err;     // device error word (bounded-wait timeouts); NULL = &epi.sc->err
 };
 
 template <typename T>

@@ -1,6 +1,639 @@
+// bf16 GEMM on the 5th-generation tensor cores (sm_100a): tcgen05.mma with operands staged
+// in shared memory by TMA (128-byte swizzle) and fp32 accumulators in tensor memory (TMEM).
+//
+//   acc[m][n] = sum_k A[m][k] * B[n][k]
+//
+// A and B may each be K-major (k contiguous) or MN-major (m / n contiguous); the MMA reads
+// both layouts directly (instruction-descriptor transpose bits), so the weight-gradient and
+// data-gradient GEMMs of the backward pass need no transposed copies.
+//
+// Structure: persistent CTAs (one per SM), 6 warps.
+//   warp 0      TMA producer: fills a ring of STAGES shared-memory stages (A 128x64, B 256x64)
+//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x (128x256x16) MMAs per stage,
+//               tcgen05.commit frees the stage; a second commit marks the accumulator full
+//   warps 2..5  epilogue: tcgen05.ld of the 128x256 fp32 accumulator (one row per thread),
+//               the fused epilogue, global stores
+// The accumulator is double-buffered in TMEM (2 x 256 columns), so the epilogue of one tile
+// overlaps the MMAs of the next. Every mbarrier wait is bounded: after ~2 s it sets the
+// device error word and the CTA leaves through its normal teardown (TMEM is always freed).
+#include <cuda.h>
+
 #include "gemm_tc.cuh"
-struct TcGemm { int dummy; };
-cudaError_t tc_gemm_create(TcGemm **out) { *out = new TcGemm(); return cudaSuccess; }
+#include "kernels.cuh"
+
+namespace {
+
+constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr unsigned long long TIMEOUT_NS = 2000000000ull;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+enum TcEpi {
+  TE_STORE = 0, TE_STORE_GELU, TE_RESID, TE_DGELU, TE_F32_STORE, TE_F32_ACCUM, TE_CE_STATS,
+  TE_CE_DS, TE_PARTIAL
+};
+
+struct TcParams {
+  int M, N, K;
+  int num_mt, num_nt, splits, kblocks_per_split, total_kblocks;
+  int units;
+  int a_mn, b_mn;  // 1 = MN-major
+  uint32_t idesc;
+  Epi epi;
+  float *partial;
+  unsigned *err;
+};
+
+// ---------------------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the CTA is aborting or the wait exceeded TIMEOUT_NS.
+__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                       unsigned *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 127u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > TIMEOUT_NS) {
+        *abort_flag = 1;
+        atomicOr(err, GPT_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor (sm_100 format, version 1), 128-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // version
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// ---------------------------------------------------------------------------------------
+// epilogue helpers (one thread = one row, 32 consecutive columns per call)
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void st_bf16x32(bf16 *dst, const float (&v)[32]) {
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * q + 0], v[8 * q + 1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * q + 2], v[8 * q + 3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 4], v[8 * q + 5]);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * q + 6], v[8 * q + 7]);
+    u.x = *reinterpret_cast<uint32_t *>(&h0);
+    u.y = *reinterpret_cast<uint32_t *>(&h1);
+    u.z = *reinterpret_cast<uint32_t *>(&h2);
+    u.w = *reinterpret_cast<uint32_t *>(&h3);
+    d[q] = u;
+  }
+}
+__device__ __forceinline__ void ld_bf16x32(const bf16 *src, float (&v)[32]) {
+  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u = s[q];
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      v[8 * q + 2 * i] = f.x;
+      v[8 * q + 2 * i + 1] = f.y;
+    }
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epi_chunk(const TcParams &P, int row, int col0, int z,
+                                          float (&v)[32], float &ce_max, float &ce_sum) {
+  const Epi &e = P.epi;
+  const bool full = col0 + 32 <= P.N;
+  if (EPI == TE_CE_STATS) {
+    const int lim = min(P.N, e.V) - col0;  // valid columns in this chunk
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < lim) mx = fmaxf(mx, v[i]);
+    const float mnew = fmaxf(ce_max, mx);
+    if (mnew > -INFINITY) {
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < lim) s += __expf(v[i] - mnew);
+      ce_sum = ce_sum * __expf(ce_max - mnew) + s;
+      ce_max = mnew;
+    }
+    const int grow = e.row_offset + row;
+    const int t = e.targets[grow] - col0;
+    if (t >= 0 && t < 32 && t < lim) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i == t) e.tgt_logit[grow] = v[i];
+    }
+    return;
+  }
+  if (EPI == TE_CE_DS) {
+    const int grow = e.row_offset + row;
+    const float L = e.lse[grow];
+    const int t = e.targets[grow];
+    const float s = e.sc->inv_M;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = col0 + i;
+      float p = 0.f;
+      if (c < e.V) {
+        p = __expf(v[i] - L);
+        if (c == t) p -= 1.f;
+        p *= s;
+      }
+      v[i] = p;
+    }
+    bf16 *dst = (bf16 *)e.out + (long)row * e.ldo + col0;
+    if (full) {
+      st_bf16x32(dst, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < P.N) dst[i] = __float2bfloat16_rn(v[i]);
+    }
+    return;
+  }
+  if (EPI == TE_PARTIAL || EPI == TE_F32_STORE || EPI == TE_F32_ACCUM) {
+    float *dst = EPI == TE_PARTIAL ? P.partial + ((long)z * P.M + row) * P.N + col0
+                                   : e.outf + (long)row * e.ldf + col0;
+    if (EPI == TE_F32_ACCUM) {
+      if (full) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 o = reinterpret_cast<float4 *>(dst)[q];
+          o.x += v[4 * q]; o.y += v[4 * q + 1]; o.z += v[4 * q + 2]; o.w += v[4 * q + 3];
+          reinterpret_cast<float4 *>(dst)[q] = o;
+        }
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < P.N) dst[i] += v[i];
+      }
+    } else {
+      if (full && (EPI != TE_PARTIAL || (P.N & 3) == 0)) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          reinterpret_cast<float4 *>(dst)[q] =
+              make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < P.N) dst[i] = v[i];
+      }
+    }
+    return;
+  }
+  // activation (bf16) outputs
+  bf16 *dst = (bf16 *)e.out + (long)row * e.ldo + col0;
+  if (EPI == TE_RESID || EPI == TE_DGELU) {
+    const bf16 *aux = (const bf16 *)e.aux + (long)row * e.ld_aux + col0;
+    float a[32];
+    if (full) {
+      ld_bf16x32(aux, a);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = (col0 + i < P.N) ? __bfloat162float(aux[i]) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_f(a[i]);
+  }
+  if (full) {
+    st_bf16x32(dst, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col0 + i < P.N) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+  if (EPI == TE_STORE_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+    bf16 *d2 = (bf16 *)e.out2 + (long)row * e.ldo2 + col0;
+    if (full) {
+      st_bf16x32(d2, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < P.N) d2[i] = __float2bfloat16_rn(v[i]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------------------
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t *full_bar = (uint64_t *)(smem + STAGES * STAGE_BYTES);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *tfull_bar = empty_bar + STAGES;
+  uint64_t *tempty_bar = tfull_bar + 2;
+  uint32_t *tmem_holder = (uint32_t *)(tempty_bar + 2);
+  volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t issued = 0;  // bit s: stage s has been filled at least once; phase of last fill
+      uint32_t last_par = 0;
+      for (int u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
+        const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
+        const int m0 = mt * BM, n0 = nt * BN;
+        const int kb0 = z * P.kblocks_per_split;
+        const int kb1 = min(P.total_kblocks, kb0 + P.kblocks_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, P.err)) { ok = false; break; }
+          uint8_t *sA = smem + stage * STAGE_BYTES;
+          uint8_t *sB = sA + A_BYTES;
+          mbar_expect_tx(&full_bar[stage], STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (!P.a_mn) {
+            tma_load_2d(sA, &tmA, &full_bar[stage], k0, m0);
+          } else {
+            tma_load_2d(sA, &tmA, &full_bar[stage], m0, k0);
+            tma_load_2d(sA + A_BYTES / 2, &tmA, &full_bar[stage], m0 + 64, k0);
+          }
+          if (!P.b_mn) {
+            tma_load_2d(sB, &tmB, &full_bar[stage], k0, n0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sB + j * (B_BYTES / 4), &tmB, &full_bar[stage], n0 + 64 * j, k0);
+          }
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag) {
+        // leave no bulk copy in flight: wait (bounded) for the last fill of every stage
+        const uint64_t t0 = globaltimer();
+        for (int s2 = 0; s2 < STAGES; ++s2) {
+          if (!(issued >> s2 & 1u)) continue;
+          while (!mbar_try_wait(&full_bar[s2], (last_par >> s2) & 1u) &&
+                 globaltimer() - t0 < 200000000ull) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int i = 0;
+      // per-k16 start-address advance inside a stage
+      const uint32_t a_step = P.a_mn ? 2048u : 32u;
+      const uint32_t b_step = P.b_mn ? 2048u : 32u;
+      const uint32_t a_lbo = P.a_mn ? (uint32_t)(A_BYTES / 2) : 16u;
+      const uint32_t b_lbo = P.b_mn ? (uint32_t)(B_BYTES / 4) : 16u;
+      for (int u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++i) {
+        const int z = u / (P.num_mt * P.num_nt);
+        const int kb0 = z * P.kblocks_per_split;
+        const int kb1 = min(P.total_kblocks, kb0 + P.kblocks_per_split);
+        const int acc = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        if (!mbar_wait(&tempty_bar[acc], (use & 1u) ^ 1u, abort_flag, P.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, P.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = sdesc(sA + k * a_step, a_lbo, 1024u);
+            const uint64_t bd = sdesc(sB + k * b_step, b_lbo, 1024u);
+            umma_bf16(d_tmem, ad, bd, P.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int i = 0;
+    for (int u = blockIdx.x; u < P.units; u += gridDim.x, ++i) {
+      const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
+      const int acc = i & 1;
+      const uint32_t use = (uint32_t)(i >> 1);
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(&tfull_bar[acc], use & 1u, abort_flag, P.err) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      tc_fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float ce_max = -INFINITY, ce_sum = 0.f;
+      const int ncols = min(BN, P.N - nt * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        if (c * 32 >= ncols) break;  // uniform across the warp
+        float v[32];
+        tmem_ld32(tbase + (uint32_t)(c * 32), v);
+        if (row < P.M) epi_chunk<EPI>(P, row, nt * BN + c * 32, z, v, ce_max, ce_sum);
+      }
+      if (EPI == TE_CE_STATS && row < P.M) {
+        const Epi &e = P.epi;
+        float *st = e.stats + ((long)(e.row_offset + row) * e.ntiles + nt) * 2;
+        st[0] = ce_max;
+        st[1] = ce_sum;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// 2-D bf16 tensor map: inner dimension `inner` (contiguous), outer `outer`, row stride `ld`
+// elements, box {64, box_outer}, 128-byte swizzle.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up at run time so the library loads without libcuda.
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld, int box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)base, dims,
+                                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                      CU_TENSOR_MAP_SWIZZLE_128B,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_kind(const CUtensorMap &a, const CUtensorMap &b, const TcParams &P, int grid,
+                        cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  tc_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(a, b, P);
+  return cudaGetLastError();
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+struct TcGemm {
+  unsigned *err;
+};
+
+cudaError_t tc_gemm_create(TcGemm **out) {
+  *out = new TcGemm();
+  (*out)->err = nullptr;
+  return cudaSuccess;
+}
 void tc_gemm_destroy(TcGemm *t) { delete t; }
-bool tc_gemm_supported(const GemmDesc &) { return false; }
-cudaError_t tc_gemm_launch(TcGemm *, GemmDesc &, cudaStream_t, int *) { return cudaErrorNotSupported; }
+
+bool tc_gemm_supported(const GemmDesc &d) {
+  if (d.K <= 0 || d.M <= 0 || d.N <= 0) return false;
+  if ((d.lda & 7) || (d.ldb & 7)) return false;
+  if (!aligned16(d.A) || !aligned16(d.B)) return false;
+  const Epi &e = d.epi;
+  switch (e.kind) {
+    case EPI_STORE:
+    case EPI_CE_DS:
+      return (e.ldo & 7) == 0 && aligned16(e.out);
+    case EPI_STORE_GELU:
+      return (e.ldo & 7) == 0 && (e.ldo2 & 7) == 0 && aligned16(e.out) && aligned16(e.out2);
+    case EPI_RESID:
+    case EPI_DGELU:
+      return (e.ldo & 7) == 0 && (e.ld_aux & 7) == 0 && aligned16(e.out) && aligned16(e.aux);
+    case EPI_F32_STORE:
+    case EPI_F32_ACCUM:
+      return (e.ldf & 3) == 0 && aligned16(e.outf);
+    case EPI_CE_STATS:
+      return true;
+    default:
+      return false;
+  }
+}
+
+cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches) {
+  TcParams P;
+  memset(&P, 0, sizeof(P));
+  P.M = d.M; P.N = d.N; P.K = d.K;
+  P.num_mt = (d.M + BM - 1) / BM;
+  P.num_nt = (d.N + BN - 1) / BN;
+  P.total_kblocks = (d.K + BK - 1) / BK;
+  int S = d.split_k > 1 ? d.split_k : 1;
+  if (S > P.total_kblocks) S = P.total_kblocks;
+  P.kblocks_per_split = (P.total_kblocks + S - 1) / S;
+  S = (P.total_kblocks + P.kblocks_per_split - 1) / P.kblocks_per_split;  // no empty split
+  d.split_k = S;
+  P.splits = S;
+  P.units = P.num_mt * P.num_nt * S;
+  P.a_mn = d.a_kmajor ? 0 : 1;
+  P.b_mn = d.b_kmajor ? 0 : 1;
+  P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)P.a_mn << 15) |
+            ((uint32_t)P.b_mn << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  P.epi = d.epi;
+  P.partial = d.partial;
+  P.err = d.err ? d.err : (d.epi.sc ? (unsigned *)&d.epi.sc->err : t->err);
+  if (!P.err) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  bool ok = P.a_mn ? make_map(&ma, d.A, d.M, d.K, d.lda, 64)
+                   : make_map(&ma, d.A, d.K, d.M, d.lda, BM);
+  ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, 64)
+                     : make_map(&mb, d.B, d.K, d.N, d.ldb, BN));
+  if (!ok) return cudaErrorInvalidValue;
+  const int grid = P.units < num_sms() ? P.units : num_sms();
+  cudaError_t e;
+  if (S > 1) {
+    e = launch_kind<TE_PARTIAL>(ma, mb, P, grid, st);
+    if (e != cudaSuccess) return e;
+    return launch_splitk_reduce<bf16>(d, st);
+  }
+  switch (d.epi.kind) {
+    case EPI_STORE: e = launch_kind<TE_STORE>(ma, mb, P, grid, st); break;
+    case EPI_STORE_GELU: e = launch_kind<TE_STORE_GELU>(ma, mb, P, grid, st); break;
+    case EPI_RESID: e = launch_kind<TE_RESID>(ma, mb, P, grid, st); break;
+    case EPI_DGELU: e = launch_kind<TE_DGELU>(ma, mb, P, grid, st); break;
+    case EPI_F32_STORE: e = launch_kind<TE_F32_STORE>(ma, mb, P, grid, st); break;
+    case EPI_F32_ACCUM: e = launch_kind<TE_F32_ACCUM>(ma, mb, P, grid, st); break;
+    case EPI_CE_STATS: e = launch_kind<TE_CE_STATS>(ma, mb, P, grid, st); break;
+    case EPI_CE_DS: e = launch_kind<TE_CE_DS>(ma, mb, P, grid, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  (void)launches;
+  return e;
+}

@@ -1,0 +1,55 @@
+// Single-kernel entry points (include/gpt_kernels.h): the step's own kernels on caller
+// buffers, for tests and per-kernel timing.
+#include "../../include/gpt_kernels.h"
+#include "../../include/gpt_step.h"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+namespace {
+TcGemm *tc_instance() {
+  static TcGemm *t = nullptr;
+  if (!t) tc_gemm_create(&t);
+  return t;
+}
+}  // namespace
+
+extern "C" int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int a_kmajor,
+                              const void *B, long ldb, int b_kmajor, int epi, void *out, long ldo,
+                              void *out2, long ldo2, const void *aux, long ld_aux, float *outf,
+                              long ldf, int split_k, float *scratch, size_t scratch_floats,
+                              unsigned *dev_err, int path, void *stream) {
+  if (M < 0 || N < 0 || K < 0 || !A || !B || !dev_err) return GPT_ERR_INVALID_ARG;
+  if (epi < GPTK_EPI_STORE || epi > GPTK_EPI_F32_ACCUM) return GPT_ERR_INVALID_ARG;
+  const bool f32 = epi == GPTK_EPI_F32_STORE || epi == GPTK_EPI_F32_ACCUM;
+  if (f32 ? !outf : !out) return GPT_ERR_INVALID_ARG;
+  if ((epi == GPTK_EPI_STORE_GELU && !out2) ||
+      ((epi == GPTK_EPI_RESID || epi == GPTK_EPI_DGELU) && !aux))
+    return GPT_ERR_INVALID_ARG;
+  if (split_k < 1) split_k = 1;
+  if (split_k > 1 && (!f32 || !scratch || scratch_floats < (size_t)split_k * M * N))
+    return GPT_ERR_INVALID_ARG;
+  GemmDesc d;
+  memset(&d, 0, sizeof(d));
+  d.M = M; d.N = N; d.K = K;
+  d.A = A; d.lda = lda; d.a_kmajor = a_kmajor ? 1 : 0;
+  d.B = B; d.ldb = ldb; d.b_kmajor = b_kmajor ? 1 : 0;
+  d.epi.kind = epi;  // GPTK_EPI_* equal EPI_* for these six kinds
+  d.epi.out = out; d.epi.ldo = ldo; d.epi.out2 = out2; d.epi.ldo2 = ldo2;
+  d.epi.aux = aux; d.epi.ld_aux = ld_aux; d.epi.outf = outf; d.epi.ldf = ldf;
+  d.split_k = split_k;
+  d.partial = scratch;
+  d.err = dev_err;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (M == 0 || N == 0) return GPT_OK;
+  if (path == GPTK_PATH_TCGEN05) {
+    if (!tc_gemm_supported(d)) return GPT_ERR_ALIGN;
+    int n = 0;
+    e = tc_gemm_launch(tc_instance(), d, st, &n);
+  } else if (path == GPTK_PATH_SIMT) {
+    e = launch_gemm_simt<bf16>(d, st);
+  } else {
+    return GPT_ERR_INVALID_ARG;
+  }
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}

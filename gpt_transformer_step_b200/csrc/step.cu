@@ -144,6 +144,7 @@ int choose_split(const gpt_handle *h, int M, int N, int K, int tm, int tn) {
 
 cudaError_t gemm(gpt_handle *h, GemmDesc d) {
   if (d.M <= 0 || d.N <= 0) return cudaSuccess;
+  d.epi.sc = h->sc;  // device error word and 1/M for every epilogue
   const double flops = 2.0 * d.M * d.N * d.K;
   int k = -1;
   if (h->time_kernels && h->ev_used + 2 <= (int)h->ev.size()) {

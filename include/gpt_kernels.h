@@ -1,0 +1,50 @@
+/* gpt_kernels.h -- single-kernel entry points of the step library, for tests and per-kernel
+ * measurement. They run exactly the kernels gpt_train_step uses, on caller-owned device
+ * buffers, on the given cudaStream_t (NULL = legacy default stream), and do not
+ * synchronise. Status codes are those of gpt_step.h.
+ *
+ * Operation (the dense contractions of the GPT-2 block and tied lm_head; nanoGPT README,
+ * intro; llm.c summary, "Estructura del código", where these were library GEMMs):
+ *   acc[m][n] = sum_k A[m][k] * B[n][k]   (bf16 operands, fp32 accumulation)
+ *   A[m][k] = A[m*lda + k] if a_kmajor else A[k*lda + m]     (bf16, device)
+ *   B[n][k] = B[n*ldb + k] if b_kmajor else B[k*ldb + n]     (bf16, device)
+ * then epilogue `epi`:
+ *   GPTK_EPI_STORE      out[m*ldo+n]  = bf16(acc)
+ *   GPTK_EPI_STORE_GELU out[m*ldo+n]  = bf16(acc); out2[m*ldo2+n] = bf16(gelu_tanh(acc))
+ *   GPTK_EPI_RESID      out[m*ldo+n]  = bf16(aux[m*ld_aux+n] + acc)
+ *   GPTK_EPI_DGELU      out[m*ldo+n]  = bf16(acc * gelu_tanh'(aux[m*ld_aux+n]))
+ *   GPTK_EPI_F32_STORE  outf[m*ldf+n] = acc
+ *   GPTK_EPI_F32_ACCUM  outf[m*ldf+n] += acc
+ * split_k > 1 splits K into split_k ranges whose fp32 partials are summed in a fixed order
+ * (only for the two F32 epilogues; needs scratch of split_k*M*N floats, caller-owned).
+ * path: GPTK_PATH_TCGEN05 (tensor cores; needs lda, ldb, ldo... multiples of 8 elements and
+ * 16-byte aligned pointers, else GPT_ERR_ALIGN) or GPTK_PATH_SIMT (CUDA cores, any layout).
+ * dev_err: device unsigned word that receives GPT_DEVERR bits (bounded-wait timeout = 2).
+ */
+#ifndef GPT_KERNELS_H
+#define GPT_KERNELS_H
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPTK_EPI_STORE 0
+#define GPTK_EPI_STORE_GELU 1
+#define GPTK_EPI_RESID 2
+#define GPTK_EPI_DGELU 3
+#define GPTK_EPI_F32_STORE 4
+#define GPTK_EPI_F32_ACCUM 5
+#define GPTK_PATH_TCGEN05 0
+#define GPTK_PATH_SIMT 1
+
+int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int a_kmajor, const void *B,
+                   long ldb, int b_kmajor, int epi, void *out, long ldo, void *out2, long ldo2,
+                   const void *aux, long ld_aux, float *outf, long ldf, int split_k,
+                   float *scratch, size_t scratch_floats, unsigned *dev_err, int path,
+                   void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,96 @@
+"""The tcgen05 GEMM (and the CUDA-core GEMM) through the kernel-level C ABI vs torch.matmul
+in fp32 on the same bf16 operands: every operand layout, every epilogue, ragged tiles,
+split-K."""
+import ctypes
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+    from gpt_transformer_step_b200 import binding as gb
+    torch.backends.cuda.matmul.allow_tf32 = False
+    dev = torch.device("cuda", 0)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    return torch, gb, dev, err
+
+
+def _operand(torch, dev, rows, cols, kmajor, seed):
+    """Logical [rows, cols] (rows = M or N, cols = K) operand stored K-major or MN-major."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    x = torch.randn(rows, cols, generator=g).to(torch.bfloat16)
+    if kmajor:
+        stor = x.contiguous()
+        ld = cols
+    else:
+        stor = x.t().contiguous()  # [cols(K), rows]
+        ld = rows
+    return x.float().to(dev), stor.to(dev), ld
+
+
+def _gelu(torch, x):
+    return torch.nn.functional.gelu(x, approximate="tanh")
+
+
+CASES = [
+    # M, N, K, a_kmajor, b_kmajor, epi, split
+    (256, 512, 256, 1, 1, "store", 1),
+    (200, 300, 136, 1, 1, "store", 1),
+    (128, 256, 64, 1, 1, "store", 1),
+    (130, 260, 520, 0, 1, "store", 1),
+    (130, 260, 520, 1, 0, "store", 1),
+    (384, 768, 1024, 0, 0, "f32_store", 1),
+    (300, 200, 1000, 0, 0, "f32_store", 4),
+    (257, 129, 777 // 8 * 8, 1, 0, "f32_accum", 1),
+    (333, 700, 192, 1, 1, "store_gelu", 1),
+    (333, 700, 192, 1, 1, "resid", 1),
+    (333, 700, 192, 1, 0, "dgelu", 1),
+    (1024, 2304, 768, 1, 1, "store", 1),
+]
+
+
+@pytest.mark.parametrize("path", [0, 1])
+@pytest.mark.parametrize("M,N,K,ak,bk,epi,split", CASES)
+def test_gemm_vs_torch(env, path, M, N, K, ak, bk, epi, split):
+    torch, gb, dev, err = env
+    A, As, lda = _operand(torch, dev, M, K, ak, 1)
+    B, Bs, ldb = _operand(torch, dev, N, K, bk, 2)
+    ref = A @ B.t()
+    out = torch.zeros(M, N, dtype=torch.bfloat16, device=dev)
+    out2 = torch.zeros(M, N, dtype=torch.bfloat16, device=dev)
+    aux = (torch.randn(M, N, device=dev) * 0.5).to(torch.bfloat16)
+    outf = torch.randn(M, N, device=dev)
+    outf0 = outf.clone()
+    scratch = torch.zeros(max(1, split * M * N), device=dev)
+    err.zero_()
+    s = gb.gptk_gemm_bf16(M, N, K, As.data_ptr(), lda, ak, Bs.data_ptr(), ldb, bk, gb.GPTK_EPI[epi],
+                          out.data_ptr(), N, out2.data_ptr(), N, aux.data_ptr(), N,
+                          outf.data_ptr(), N, split, scratch.data_ptr(), scratch.numel(),
+                          err.data_ptr(), path, torch.cuda.current_stream().cuda_stream)
+    assert s == 0, gb.gpt_strerror(s)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    scale = ref.abs().max().item()
+    if epi == "store":
+        d = (out.float() - ref).abs().max().item()
+        assert d <= 1e-2 * scale, d
+    elif epi == "store_gelu":
+        assert (out.float() - ref).abs().max().item() <= 1e-2 * scale
+        g = _gelu(torch, ref)
+        assert (out2.float() - g).abs().max().item() <= 1e-2 * g.abs().max().item()
+    elif epi == "resid":
+        r = aux.float() + ref
+        assert (out.float() - r).abs().max().item() <= 1e-2 * r.abs().max().item()
+    elif epi == "dgelu":
+        x = aux.float().requires_grad_()
+        _gelu(torch, x).backward(ref)
+        r = x.grad
+        assert (out.float() - r).abs().max().item() <= 1e-2 * r.abs().max().item()
+    elif epi == "f32_store":
+        assert (outf - ref).abs().max().item() <= 1e-4 * scale
+    elif epi == "f32_accum":
+        assert (outf - (outf0 + ref)).abs().max().item() <= 1e-4 * scale
