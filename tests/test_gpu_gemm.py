@@ -19,16 +19,23 @@ def env():
     return torch, gb, dev, err
 
 
+def _pad8(n):
+    return (n + 7) // 8 * 8
+
+
 def _operand(torch, dev, rows, cols, kmajor, seed):
-    """Logical [rows, cols] (rows = M or N, cols = K) operand stored K-major or MN-major."""
+    """Logical [rows, cols] (rows = M or N, cols = K) operand stored K-major or MN-major,
+    with the leading dimension padded to a multiple of 8 elements (16 bytes)."""
     g = torch.Generator(device="cpu").manual_seed(seed)
     x = torch.randn(rows, cols, generator=g).to(torch.bfloat16)
     if kmajor:
-        stor = x.contiguous()
-        ld = cols
+        ld = _pad8(cols)
+        stor = torch.zeros(rows, ld, dtype=torch.bfloat16)
+        stor[:, :cols] = x
     else:
-        stor = x.t().contiguous()  # [cols(K), rows]
-        ld = rows
+        ld = _pad8(rows)
+        stor = torch.zeros(cols, ld, dtype=torch.bfloat16)
+        stor[:, :rows] = x.t()
     return x.float().to(dev), stor.to(dev), ld
 
 
@@ -60,19 +67,21 @@ def test_gemm_vs_torch(env, path, M, N, K, ak, bk, epi, split):
     A, As, lda = _operand(torch, dev, M, K, ak, 1)
     B, Bs, ldb = _operand(torch, dev, N, K, bk, 2)
     ref = A @ B.t()
-    out = torch.zeros(M, N, dtype=torch.bfloat16, device=dev)
-    out2 = torch.zeros(M, N, dtype=torch.bfloat16, device=dev)
-    aux = (torch.randn(M, N, device=dev) * 0.5).to(torch.bfloat16)
-    outf = torch.randn(M, N, device=dev)
-    outf0 = outf.clone()
+    ldo = _pad8(N)
+    out_s = torch.zeros(M, ldo, dtype=torch.bfloat16, device=dev)
+    out2_s = torch.zeros(M, ldo, dtype=torch.bfloat16, device=dev)
+    aux_s = (torch.randn(M, ldo, device=dev) * 0.5).to(torch.bfloat16)
+    outf_s = torch.randn(M, ldo, device=dev)
+    outf0 = outf_s[:, :N].clone()
     scratch = torch.zeros(max(1, split * M * N), device=dev)
     err.zero_()
     s = gb.gptk_gemm_bf16(M, N, K, As.data_ptr(), lda, ak, Bs.data_ptr(), ldb, bk, gb.GPTK_EPI[epi],
-                          out.data_ptr(), N, out2.data_ptr(), N, aux.data_ptr(), N,
-                          outf.data_ptr(), N, split, scratch.data_ptr(), scratch.numel(),
+                          out_s.data_ptr(), ldo, out2_s.data_ptr(), ldo, aux_s.data_ptr(), ldo,
+                          outf_s.data_ptr(), ldo, split, scratch.data_ptr(), scratch.numel(),
                           err.data_ptr(), path, torch.cuda.current_stream().cuda_stream)
     assert s == 0, gb.gpt_strerror(s)
     torch.cuda.synchronize()
+    out, out2, aux, outf = out_s[:, :N], out2_s[:, :N], aux_s[:, :N], outf_s[:, :N]
     assert int(err.item()) == 0
     scale = ref.abs().max().item()
     if epi == "store":
