@@ -35,7 +35,8 @@ EXPORTED = [
     "gpt_create", "gpt_destroy", "gpt_num_params", "gpt_param_layout", "gpt_set_stream",
     "gpt_forward_loss", "gpt_train_step", "gpt_get_step", "gpt_set_step", "gpt_last_grad_norm",
     "gpt_params_changed", "gpt_set_option", "gpt_kernel_stats", "gpt_last_launch_count",
-    "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16",
+    "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
+    "gptk_attention_bwd_bf16",
 ]
 
 
@@ -93,6 +94,10 @@ gpt_last_cuda_error = _sig("gpt_last_cuda_error", ctypes.c_char_p, [_P])
 _L = ctypes.c_long
 gptk_gemm_bf16 = _sig("gptk_gemm_bf16", _I, [_I, _I, _I, _P, _L, _I, _P, _L, _I, _I, _P, _L, _P, _L,
                                              _P, _L, _P, _L, _I, _P, ctypes.c_size_t, _P, _I, _P])
+gptk_attention_fwd_bf16 = _sig("gptk_attention_fwd_bf16", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _P,
+                                                               _I, _P])
+gptk_attention_bwd_bf16 = _sig("gptk_attention_bwd_bf16", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I,
+                                                               _I, _I, _P, _I, _P])
 GPTK_EPI = {"store": 0, "store_gelu": 1, "resid": 2, "dgelu": 3, "f32_store": 4, "f32_accum": 5}
 GPTK_PATH_TCGEN05 = 0
 GPTK_PATH_SIMT = 1

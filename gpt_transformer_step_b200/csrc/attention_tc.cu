@@ -1,0 +1,687 @@
+// Causal (optionally left-windowed) attention, head_dim 64, on the sm_100a tensor cores.
+//
+// Semantics (nanochat architecture page, "Modellarchitektur und FLOPs-Berechnung": causal
+// attention with a per-layer left window; reading: window w >= 0 admits keys i-w <= j <= i):
+//   s_ij = q_i . k_j / sqrt(64);  P = softmax_j(s) over admitted j;  o_i = sum_j P_ij v_j;
+//   lse_i = log sum_j exp(s_ij) (natural log) is kept for the backward pass.
+//
+// All three kernels use 128x128 tiles, TMA loads of 128x64 bf16 tiles (128-byte swizzle) from
+// the fused qkv buffer [B*T, 3C], tcgen05.mma with fp32 accumulators in TMEM, and 4 "row"
+// warps in which each thread owns one row of the 128x128 score tile:
+//   forward  (CTA = b, h, 128 queries): S = Q K^T -> TMEM; online softmax in the log2 domain
+//            with a conditional rescale of O (only when the running max grows by > 8);
+//            P (bf16) -> swizzled smem; O += P V in TMEM.
+//   dQ       (CTA = b, h, 128 queries): also writes D_i = dO_i . O_i. S = Q K^T, dP = dO V^T,
+//            dS = P o (dP - D) -> smem, dQ += dS K.
+//   dK / dV  (CTA = b, h, 128 keys):    S^T = K Q^T, dP^T = V dO^T, P^T and dS^T -> smem,
+//            dV += P^T dO, dK += dS^T Q.
+// No atomics: every output element is written by exactly one CTA, so results are bitwise
+// reproducible. Tiles entirely outside the causal/window band are skipped; edge tiles are
+// masked element by element. Every wait is bounded (device error word on timeout).
+#include "kernels.cuh"
+#include "tc_ptx.cuh"
+
+namespace {
+using namespace tc;
+
+constexpr int HD = 64;
+constexpr int TILE = 128;
+constexpr int TILE_BYTES = TILE * HD * 2;  // 16 KB: 128 rows x 64 bf16, K-major SW128
+constexpr int SQ_BYTES = TILE * TILE * 2;  // 32 KB: 128 x 128 bf16 (two 16 KB K-blocks)
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+struct AttnParams {
+  int B, T, C, H, window;
+  float scale_log2;  // log2(e) / sqrt(64)
+  float scale;       // 1 / sqrt(64)
+  bf16 *o;           // forward output [B*T, C]
+  float *lse;        // forward output [B, H, T]
+  const bf16 *O;     // backward inputs
+  const bf16 *dO;    // [B*T, C]
+  const float *lse_in;
+  float *Dbuf;       // [B, H, T]
+  bf16 *dqkv;        // [B*T, 3C]
+  unsigned *err;
+};
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TILE >> 4) << 24);
+}
+
+__device__ __forceinline__ bool admitted(int i, int j, int w) {
+  return j <= i && (w < 0 || j >= i - w);
+}
+
+// One warp-collective bounded wait: lane 0 polls, the result is broadcast.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned *err) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, err) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  return (uint8_t *)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+// A = 128 x K (K-major, SW128, K-blocks of 64 at stride 16 KB); B K-major N x 64 tile.
+// S[128 x N] (+)= A[:, 0:64] * B^T  with 4 MMAs of K = 16.
+__device__ __forceinline__ void mma_qk(uint32_t d, uint32_t sA, uint32_t sB, int n) {
+  const uint32_t id = idesc_bf16(n, 0, 0);
+#pragma unroll
+  for (int k = 0; k < HD / 16; ++k)
+    umma_bf16(d, sdesc(sA + 32 * k, 16, 1024), sdesc(sB + 32 * k, 16, 1024), id, k > 0 ? 1u : 0u);
+}
+// O[128 x 64] (+)= P[128 x 128] * V where P is K-major (two 16 KB K-blocks) and V is a
+// 128(k) x 64(n) tile stored with n contiguous (MN-major operand).
+__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t sP, uint32_t sV, bool accumulate) {
+  const uint32_t id = idesc_bf16(HD, 0, 1);
+#pragma unroll
+  for (int k = 0; k < TILE / 16; ++k) {
+    const uint32_t a = sP + (k >> 2) * 16384 + (k & 3) * 32;
+    const uint32_t b = sV + k * 2048;
+    umma_bf16(d, sdesc(a, 16, 1024), sdesc(b, 8192, 1024), id, (accumulate || k > 0) ? 1u : 0u);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// forward
+// ------------------------------------------------------------------------------------------
+enum { F_QFULL, F_KFULL, F_VFULL, F_KFREE, F_VFREE, F_SFULL, F_PFULL, F_OFULL, F_NBAR };
+constexpr int FWD_SMEM = 3 * TILE_BYTES + SQ_BYTES + 1024 + 256;
+
+__global__ void __launch_bounds__(192, 2)
+attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sQ = smem, *sK = smem + TILE_BYTES, *sV = smem + 2 * TILE_BYTES;
+  uint8_t *sP = smem + 3 * TILE_BYTES;
+  uint64_t *bar = (uint64_t *)(smem + 3 * TILE_BYTES + SQ_BYTES);
+  uint32_t *tmem_holder = (uint32_t *)(bar + F_NBAR);
+  volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = P.B * P.H, nqt = (P.T + TILE - 1) / TILE;
+  const int qt = nqt - 1 - (int)blockIdx.x / BH;  // heaviest (last) query tiles first
+  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
+  const int q0 = qt * TILE, row0 = b * P.T, w = P.window;
+  const int kt0 = (w >= 0 ? max(0, q0 - w) : 0) / TILE;
+  const int kt1 = (min(P.T, q0 + TILE) + TILE - 1) / TILE;
+  const int n = kt1 - kt0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < F_NBAR; ++i) mbar_init(&bar[i], i == F_PFULL ? 4 : 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;  // S: columns [0,128), O: [128,192)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bar[F_QFULL], TILE_BYTES);
+      tma_load_2d(sQ, &tmQKV, &bar[F_QFULL], h * HD, row0 + q0);
+      for (int j = 0; j < n; ++j) {
+        const int k0 = (kt0 + j) * TILE;
+        if (j > 0 && !mbar_wait(&bar[F_KFREE], (j - 1) & 1, abort_flag, P.err)) break;
+        mbar_expect_tx(&bar[F_KFULL], TILE_BYTES);
+        tma_load_2d(sK, &tmQKV, &bar[F_KFULL], P.C + h * HD, row0 + k0);
+        if (j > 0 && !mbar_wait(&bar[F_VFREE], (j - 1) & 1, abort_flag, P.err)) break;
+        mbar_expect_tx(&bar[F_VFULL], TILE_BYTES);
+        tma_load_2d(sV, &tmQKV, &bar[F_VFULL], 2 * P.C + h * HD, row0 + k0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) &&
+                mbar_wait(&bar[F_KFULL], 0, abort_flag, P.err);
+      if (ok) {
+        tc_fence_after();
+        mma_qk(tmem, aQ, aK, TILE);
+        umma_commit(&bar[F_SFULL]);
+        umma_commit(&bar[F_KFREE]);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait(&bar[F_PFULL], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
+        if (j + 1 < n) {
+          if (!mbar_wait(&bar[F_KFULL], (j + 1) & 1, abort_flag, P.err)) break;
+          tc_fence_after();
+          mma_qk(tmem, aQ, aK, TILE);
+          umma_commit(&bar[F_SFULL]);
+          umma_commit(&bar[F_KFREE]);
+        }
+        if (!mbar_wait(&bar[F_VFULL], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
+        mma_pv(tmem + 128, aP, aV, j > 0);
+        umma_commit(&bar[F_OFULL]);
+        umma_commit(&bar[F_VFREE]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3, r = q * 32 + lane, qi = q0 + r;
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tO = tS + 128;
+    float m2 = -INFINITY, l = 0.f;
+    bool have = false, ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int k0 = (kt0 + j) * TILE;
+      if (!warp_wait(&bar[F_SFULL], j & 1, abort_flag, P.err)) { ok = false; break; }
+      tc_fence_after();
+      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tS + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool a = interior || admitted(qi, k0 + c * 32 + i, w);
+          if (a) mt = fmaxf(mt, v[i] * P.scale_log2);
+        }
+      }
+      float mnew = m2;
+      bool resc = false;
+      if (mt > -INFINITY) {
+        if (!have) mnew = mt;
+        else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
+      }
+      if (j > 0) {
+        if (!warp_wait(&bar[F_OFULL], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? ex2(m2 - mnew) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          tmem_ld32(tO + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= f;
+          tmem_st32(tO + c * 32, v);
+        }
+        l *= f;
+      }
+      m2 = mnew;
+      if (mt > -INFINITY) have = true;
+      float ls = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tS + c * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p0 = 0.f, p1 = 0.f;
+          if (have && (interior || admitted(qi, k0 + c * 32 + i, w))) p0 = ex2(v[i] * P.scale_log2 - m2);
+          if (have && (interior || admitted(qi, k0 + c * 32 + i + 1, w))) p1 = ex2(v[i + 1] * P.scale_log2 - m2);
+          ls += p0 + p1;
+          pk[i >> 1] = pack_bf16(p0, p1);
+        }
+        uint8_t *blk = sP + (c >> 1) * 16384;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          st_sw128_chunk(blk, r, (c & 1) * 4 + t,
+                         make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
+      }
+      l += ls;
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[F_PFULL]);
+    }
+    if (ok && warp_wait(&bar[F_OFULL], (n - 1) & 1, abort_flag, P.err)) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint32_t pk[32];
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        tmem_ld32(tO + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * inv, v[i + 1] * inv);
+      }
+      if (qi < P.T) {
+        uint4 *dst = reinterpret_cast<uint4 *>(P.o + (size_t)(row0 + qi) * P.C + h * HD);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        P.lse[((size_t)b * P.H + h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// backward: dQ (+ D)
+// ------------------------------------------------------------------------------------------
+enum { Q_QDO, Q_KV0, Q_KV1, Q_FREE0, Q_FREE1, Q_SDP, Q_DS, Q_MM2, Q_NBAR };
+constexpr int DQ_SMEM = 6 * TILE_BYTES + SQ_BYTES + 1024 + 256;
+
+__global__ void __launch_bounds__(192, 1)
+attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+               const AttnParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sQ = smem, *sdO = smem + TILE_BYTES;
+  uint8_t *sK0 = smem + 2 * TILE_BYTES;  // stage s: K at 2+2s, V at 3+2s
+  uint8_t *sdS = smem + 6 * TILE_BYTES;
+  uint64_t *bar = (uint64_t *)(smem + 6 * TILE_BYTES + SQ_BYTES);
+  uint32_t *tmem_holder = (uint32_t *)(bar + Q_NBAR);
+  volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = P.B * P.H, nqt = (P.T + TILE - 1) / TILE;
+  const int qt = nqt - 1 - (int)blockIdx.x / BH;
+  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
+  const int q0 = qt * TILE, row0 = b * P.T, w = P.window;
+  const int kt0 = (w >= 0 ? max(0, q0 - w) : 0) / TILE;
+  const int kt1 = (min(P.T, q0 + TILE) + TILE - 1) / TILE;
+  const int n = kt1 - kt0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Q_NBAR; ++i) mbar_init(&bar[i], i == Q_DS ? 4 : 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;  // S [0,128), dP [128,256), dQ [256,320)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bar[Q_QDO], 2 * TILE_BYTES);
+      tma_load_2d(sQ, &tmQKV, &bar[Q_QDO], h * HD, row0 + q0);
+      tma_load_2d(sdO, &tmDO, &bar[Q_QDO], h * HD, row0 + q0);
+      for (int j = 0; j < n; ++j) {
+        const int s = j & 1, k0 = (kt0 + j) * TILE;
+        if (j >= 2 && !mbar_wait(&bar[Q_FREE0 + s], ((j >> 1) - 1) & 1, abort_flag, P.err)) break;
+        uint8_t *sK = sK0 + s * 2 * TILE_BYTES;
+        mbar_expect_tx(&bar[Q_KV0 + s], 2 * TILE_BYTES);
+        tma_load_2d(sK, &tmQKV, &bar[Q_KV0 + s], P.C + h * HD, row0 + k0);
+        tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[Q_KV0 + s], 2 * P.C + h * HD, row0 + k0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), adS = smem_u32(sdS);
+      auto issue_sdp = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&bar[Q_KV0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sK0 + s * 2 * TILE_BYTES), aV = aK + TILE_BYTES;
+        mma_qk(tmem, aQ, aK, TILE);
+        mma_qk(tmem + 128, adO, aV, TILE);
+        umma_commit(&bar[Q_SDP]);
+        return true;
+      };
+      bool ok = mbar_wait(&bar[Q_QDO], 0, abort_flag, P.err) && issue_sdp(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait(&bar[Q_DS], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
+        if (j + 1 < n && !issue_sdp(j + 1)) break;
+        const uint32_t aK = smem_u32(sK0 + (j & 1) * 2 * TILE_BYTES);
+        mma_pv(tmem + 256, adS, aK, j > 0);  // dQ += dS K  (K tile as the MN-major operand)
+        umma_commit(&bar[Q_MM2]);
+        umma_commit(&bar[Q_FREE0 + (j & 1)]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3, r = q * 32 + lane, qi = q0 + r;
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tdP = tS + 128, tdQ = tS + 256;
+    // D_i = dO_i . O_i (written for the dK/dV pass) and the saved lse in the log2 domain
+    float D = 0.f, lse2 = 0.f;
+    if (qi < P.T) {
+      const size_t off = (size_t)(row0 + qi) * P.C + h * HD;
+      const uint4 *go = reinterpret_cast<const uint4 *>(P.O + off);
+      const uint4 *gd = reinterpret_cast<const uint4 *>(P.dO + off);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        uint4 a = go[t], c = gd[t];
+        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&c);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
+          D += fa.x * fc.x + fa.y * fc.y;
+        }
+      }
+      const size_t li = ((size_t)b * P.H + h) * P.T + qi;
+      P.Dbuf[li] = D;
+      lse2 = P.lse_in[li] * LOG2E;
+    }
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int k0 = (kt0 + j) * TILE;
+      if (!warp_wait(&bar[Q_SDP], j & 1, abort_flag, P.err)) { ok = false; break; }
+      tc_fence_after();
+      if (j > 0) {
+        if (!warp_wait(&bar[Q_MM2], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        tc_fence_after();
+      }
+      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32], dp[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tdP + c * 32, dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float d0 = 0.f, d1 = 0.f;
+          if (qi < P.T && (interior || admitted(qi, k0 + c * 32 + i, w)))
+            d0 = ex2(sv[i] * P.scale_log2 - lse2) * (dp[i] - D);
+          if (qi < P.T && (interior || admitted(qi, k0 + c * 32 + i + 1, w)))
+            d1 = ex2(sv[i + 1] * P.scale_log2 - lse2) * (dp[i + 1] - D);
+          pk[i >> 1] = pack_bf16(d0, d1);
+        }
+        uint8_t *blk = sdS + (c >> 1) * 16384;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          st_sw128_chunk(blk, r, (c & 1) * 4 + t,
+                         make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[Q_DS]);
+    }
+    if (ok && warp_wait(&bar[Q_MM2], (n - 1) & 1, abort_flag, P.err)) {
+      tc_fence_after();
+      uint32_t pk[32];
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        tmem_ld32(tdQ + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * P.scale, v[i + 1] * P.scale);
+      }
+      if (qi < P.T) {
+        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + qi) * 3 * P.C + h * HD);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// backward: dK, dV
+// ------------------------------------------------------------------------------------------
+enum { K_KV, K_QDO0, K_QDO1, K_FREE0, K_FREE1, K_SDP, K_PS, K_MM2, K_NBAR };
+constexpr int DKV_SMEM = 6 * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * TILE * 4 + 256;
+
+__global__ void __launch_bounds__(192, 1)
+attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+                const AttnParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sK = smem, *sV = smem + TILE_BYTES;
+  uint8_t *sQ0 = smem + 2 * TILE_BYTES;  // stage s: Q at 2+2s, dO at 3+2s
+  uint8_t *sPT = smem + 6 * TILE_BYTES, *sdST = sPT + SQ_BYTES;
+  float *s_lse = (float *)(sdST + SQ_BYTES), *s_D = s_lse + TILE;
+  uint64_t *bar = (uint64_t *)(s_D + TILE);
+  uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
+  volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = P.B * P.H;
+  const int kt = (int)blockIdx.x / BH;  // low key tiles see the most queries: first
+  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
+  const int k0 = kt * TILE, row0 = b * P.T, w = P.window;
+  const int qhi = w >= 0 ? min(P.T - 1, k0 + TILE - 1 + w) : P.T - 1;
+  const int qt0 = kt, n = qhi / TILE + 1 - qt0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < K_NBAR; ++i) mbar_init(&bar[i], i == K_PS ? 4 : 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;  // S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bar[K_KV], 2 * TILE_BYTES);
+      tma_load_2d(sK, &tmQKV, &bar[K_KV], P.C + h * HD, row0 + k0);
+      tma_load_2d(sV, &tmQKV, &bar[K_KV], 2 * P.C + h * HD, row0 + k0);
+      for (int j = 0; j < n; ++j) {
+        const int s = j & 1, qq0 = (qt0 + j) * TILE;
+        if (j >= 2 && !mbar_wait(&bar[K_FREE0 + s], ((j >> 1) - 1) & 1, abort_flag, P.err)) break;
+        uint8_t *sQ = sQ0 + s * 2 * TILE_BYTES;
+        mbar_expect_tx(&bar[K_QDO0 + s], 2 * TILE_BYTES);
+        tma_load_2d(sQ, &tmQKV, &bar[K_QDO0 + s], h * HD, row0 + qq0);
+        tma_load_2d(sQ + TILE_BYTES, &tmDO, &bar[K_QDO0 + s], h * HD, row0 + qq0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPT = smem_u32(sPT), adST = smem_u32(sdST);
+      auto issue_sdp = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&bar[K_QDO0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ0 + s * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
+        mma_qk(tmem, aK, aQ, TILE);         // S^T  = K Q^T
+        mma_qk(tmem + 128, aV, adO, TILE);  // dP^T = V dO^T
+        umma_commit(&bar[K_SDP]);
+        return true;
+      };
+      bool ok = mbar_wait(&bar[K_KV], 0, abort_flag, P.err) && issue_sdp(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait(&bar[K_PS], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
+        if (j + 1 < n && !issue_sdp(j + 1)) break;
+        const uint32_t aQ = smem_u32(sQ0 + (j & 1) * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
+        mma_pv(tmem + 256, aPT, adO, j > 0);   // dV += P^T dO
+        mma_pv(tmem + 320, adST, aQ, j > 0);   // dK += dS^T Q
+        umma_commit(&bar[K_MM2]);
+        umma_commit(&bar[K_FREE0 + (j & 1)]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3, r = q * 32 + lane, ki = k0 + r;
+    const int t = threadIdx.x - 64;  // 0..127 among the row warps
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tdP = tS + 128;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int qq0 = (qt0 + j) * TILE;
+      // this query tile's lse (log2 domain) and D, shared by all row threads
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      {
+        const int qi = qq0 + t;
+        const size_t li = ((size_t)b * P.H + h) * P.T + qi;
+        s_lse[t] = qi < P.T ? P.lse_in[li] * LOG2E : 0.f;
+        s_D[t] = qi < P.T ? P.Dbuf[li] : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // after an abort every row warp still passes both named barriers of each iteration
+      if (ok) ok = warp_wait(&bar[K_SDP], j & 1, abort_flag, P.err);
+      if (ok && j > 0) ok = warp_wait(&bar[K_MM2], (j - 1) & 1, abort_flag, P.err);
+      if (!ok) continue;
+      tc_fence_after();
+      const bool interior = (k0 + TILE - 1 <= qq0) && (w < 0 || k0 >= qq0 + TILE - 1 - w) &&
+                            (qq0 + TILE <= P.T);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32], dp[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tdP + c * 32, dp);
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+          const int qa = qq0 + c * 32 + i;
+          if (interior || (qa < P.T && admitted(qa, ki, w))) {
+            p0 = ex2(sv[i] * P.scale_log2 - s_lse[c * 32 + i]);
+            d0 = p0 * (dp[i] - s_D[c * 32 + i]);
+          }
+          if (interior || (qa + 1 < P.T && admitted(qa + 1, ki, w))) {
+            p1 = ex2(sv[i + 1] * P.scale_log2 - s_lse[c * 32 + i + 1]);
+            d1 = p1 * (dp[i + 1] - s_D[c * 32 + i + 1]);
+          }
+          pp[i >> 1] = pack_bf16(p0, p1);
+          pd[i >> 1] = pack_bf16(d0, d1);
+        }
+        const int blk = (c >> 1) * 16384;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          st_sw128_chunk(sPT + blk, r, (c & 1) * 4 + u,
+                         make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]));
+          st_sw128_chunk(sdST + blk, r, (c & 1) * 4 + u,
+                         make_uint4(pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]));
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[K_PS]);
+    }
+    if (ok && warp_wait(&bar[K_MM2], (n - 1) & 1, abort_flag, P.err)) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int part = 0; part < 2; ++part) {  // 0: dV, 1: dK (times the softmax scale)
+        const float f = part ? P.scale : 1.f;
+        uint32_t pk[32];
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          tmem_ld32(tS + 256 + part * 64 + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * f, v[i + 1] * f);
+        }
+        if (ki < P.T) {
+          const int col = (part ? P.C : 2 * P.C) + h * HD;
+          uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + ki) * 3 * P.C + col);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// [rows, cols] bf16 matrix with row stride ld elements; box 64 columns x 128 rows, SW128.
+bool map_rows(CUtensorMap *m, const void *base, long cols, long rows, long ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64u, 128u};
+  cuuint32_t es[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+AttnParams make_params(int B, int T, int C, int H, int window, unsigned *err) {
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = B; p.T = T; p.C = C; p.H = H; p.window = window;
+  p.scale = 1.0f / sqrtf((float)HD);
+  p.scale_log2 = p.scale * LOG2E;
+  p.err = err;
+  return p;
+}
+
+bool smem_attrs_set = false;
+cudaError_t set_attrs() {
+  if (smem_attrs_set) return cudaSuccess;
+  CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, FWD_SMEM));
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM));
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM));
+  smem_attrs_set = true;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+bool attention_tc_supported(int C, int H) { return C / H == HD && C % H == 0 && (C % 8) == 0; }
+
+cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B, int T, int C,
+                                    int H, int window, unsigned *err, cudaStream_t st) {
+  CUDA_TRY(set_attrs());
+  CUtensorMap m;
+  if (!map_rows(&m, qkv, 3L * C, (long)B * T, 3L * C)) return cudaErrorInvalidValue;
+  AttnParams p = make_params(B, T, C, H, window, err);
+  p.o = o;
+  p.lse = lse;
+  const int nqt = (T + TILE - 1) / TILE;
+  attn_fwd_tc<<<B * H * nqt, 192, FWD_SMEM, st>>>(m, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
+                                    const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
+                                    int C, int H, int window, unsigned *err, cudaStream_t st) {
+  CUDA_TRY(set_attrs());
+  CUtensorMap mq, md;
+  if (!map_rows(&mq, qkv, 3L * C, (long)B * T, 3L * C) ||
+      !map_rows(&md, dout, (long)C, (long)B * T, (long)C))
+    return cudaErrorInvalidValue;
+  AttnParams p = make_params(B, T, C, H, window, err);
+  p.O = o;
+  p.dO = dout;
+  p.lse_in = lse;
+  p.Dbuf = Dbuf;
+  p.dqkv = dqkv;
+  const int nt = (T + TILE - 1) / TILE;
+  attn_bwd_dq_tc<<<B * H * nt, 192, DQ_SMEM, st>>>(mq, md, p);
+  CUDA_TRY(cudaGetLastError());
+  attn_bwd_dkv_tc<<<B * H * nt, 192, DKV_SMEM, st>>>(mq, md, p);
+  return cudaGetLastError();
+}

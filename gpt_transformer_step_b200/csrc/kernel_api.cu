@@ -53,3 +53,42 @@ extern "C" int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int 
   }
   return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }
+
+extern "C" int gptk_attention_fwd_bf16(const void *qkv, void *o, float *lse, int B, int T, int C,
+                                       int H, int window, unsigned *dev_err, int path,
+                                       void *stream) {
+  if (!qkv || !o || !lse || !dev_err || B <= 0 || T <= 0 || H <= 0 || C % H) return GPT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (path == GPTK_PATH_TCGEN05) {
+    if (!attention_tc_supported(C, H)) return GPT_ERR_SHAPE;
+    e = launch_attention_fwd_tc((const bf16 *)qkv, (bf16 *)o, lse, B, T, C, H, window, dev_err, st);
+  } else if (path == GPTK_PATH_SIMT) {
+    e = launch_attention_fwd<bf16>((const bf16 *)qkv, (bf16 *)o, lse, B, T, C, H, window, st);
+  } else {
+    return GPT_ERR_INVALID_ARG;
+  }
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
+extern "C" int gptk_attention_bwd_bf16(const void *qkv, const void *o, const void *dout,
+                                       const float *lse, float *Dbuf, void *dqkv, int B, int T,
+                                       int C, int H, int window, unsigned *dev_err, int path,
+                                       void *stream) {
+  if (!qkv || !o || !dout || !lse || !Dbuf || !dqkv || !dev_err || B <= 0 || T <= 0 || H <= 0 ||
+      C % H)
+    return GPT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (path == GPTK_PATH_TCGEN05) {
+    if (!attention_tc_supported(C, H)) return GPT_ERR_SHAPE;
+    e = launch_attention_bwd_tc((const bf16 *)qkv, (const bf16 *)o, (const bf16 *)dout, lse, Dbuf,
+                                (bf16 *)dqkv, B, T, C, H, window, dev_err, st);
+  } else if (path == GPTK_PATH_SIMT) {
+    e = launch_attention_bwd<bf16>((const bf16 *)qkv, (const bf16 *)o, (const bf16 *)dout, lse,
+                                   Dbuf, (bf16 *)dqkv, B, T, C, H, window, st);
+  } else {
+    return GPT_ERR_INVALID_ARG;
+  }
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}

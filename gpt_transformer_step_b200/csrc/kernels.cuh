@@ -57,6 +57,15 @@ cudaError_t launch_attention_bwd(const T *qkv, const T *o, const T *dout, const 
                                  float *Dbuf, T *dqkv, int B, int Tlen, int C, int H, int window,
                                  cudaStream_t st);
 
+// Attention on the tensor cores (head_dim 64, bf16): forward, and backward (dQ pass that also
+// writes D = rowsum(dO o O), then the dK/dV pass). err: device error word.
+bool attention_tc_supported(int C, int H);
+cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B, int T, int C,
+                                    int H, int window, unsigned *err, cudaStream_t st);
+cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
+                                    const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
+                                    int C, int H, int window, unsigned *err, cudaStream_t st);
+
 // GEMM on CUDA cores (fp32 validation mode and shapes the tensor-core path does not take).
 template <typename T>
 cudaError_t launch_gemm_simt(const GemmDesc &d, cudaStream_t st);

@@ -201,6 +201,34 @@ GemmDesc gdesc(int M, int N, int K, const void *A, long lda, int ak, const void 
   return d;
 }
 
+// Attention: tensor-core kernels for bf16 with head_dim 64, CUDA-core kernels otherwise.
+template <typename T>
+cudaError_t attention_fwd(gpt_handle *h, const T *qkv, T *o, float *lse, int B, int Tlen, int w) {
+  return launch_attention_fwd<T>(qkv, o, lse, B, Tlen, h->C, h->H, w, h->stream);
+}
+template <>
+cudaError_t attention_fwd<bf16>(gpt_handle *h, const bf16 *qkv, bf16 *o, float *lse, int B,
+                                int Tlen, int w) {
+  if (attention_tc_supported(h->C, h->H))
+    return launch_attention_fwd_tc(qkv, o, lse, B, Tlen, h->C, h->H, w, &h->sc->err, h->stream);
+  return launch_attention_fwd<bf16>(qkv, o, lse, B, Tlen, h->C, h->H, w, h->stream);
+}
+template <typename T>
+cudaError_t attention_bwd(gpt_handle *h, const T *qkv, const T *o, const T *dout,
+                          const float *lse, T *dqkv, int B, int Tlen, int w) {
+  return launch_attention_bwd<T>(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
+                                 h->stream);
+}
+template <>
+cudaError_t attention_bwd<bf16>(gpt_handle *h, const bf16 *qkv, const bf16 *o, const bf16 *dout,
+                                const float *lse, bf16 *dqkv, int B, int Tlen, int w) {
+  if (attention_tc_supported(h->C, h->H))
+    return launch_attention_bwd_tc(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
+                                   &h->sc->err, h->stream);
+  return launch_attention_bwd<bf16>(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
+                                    h->stream);
+}
+
 // --------------------------------------------------------------------------------------
 // the step schedule
 // --------------------------------------------------------------------------------------
@@ -227,8 +255,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     GemmDesc d = gdesc(M, 3 * C, C, A.a, C, 1, W + P.wqkv, C, 1);
     d.epi.kind = EPI_STORE; d.epi.out = A.qkv; d.epi.ldo = 3 * C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(launch_attention_fwd<T>((T *)A.qkv, (T *)A.o, A.lse, B, Tlen, C, H,
-                                     h->windows[l], st)); nl++;
+    CUDA_TRY(attention_fwd<T>(h, (T *)A.qkv, (T *)A.o, A.lse, B, Tlen, h->windows[l])); nl++;
     d = gdesc(M, C, C, A.o, C, 1, W + P.wap, C, 1);
     d.epi.kind = EPI_RESID; d.epi.out = A.x_mid; d.epi.ldo = C; d.epi.aux = A.x_in; d.epi.ld_aux = C;
     CUDA_TRY(gemm(h, d));
@@ -311,8 +338,8 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
     d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wap; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(launch_attention_bwd<T>((T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, h->Dbuf,
-                                     (T *)h->dqkv, B, Tlen, C, H, h->windows[l], st)); nl += 2;
+    CUDA_TRY(attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B,
+                              Tlen, h->windows[l])); nl += 2;
     d = gdesc(M, C, 3 * C, h->dqkv, 3 * C, 1, W + P.wqkv, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));

@@ -44,6 +44,19 @@ int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int a_kmajor, c
                    float *scratch, size_t scratch_floats, unsigned *dev_err, int path,
                    void *stream);
 
+/* Causal attention with an optional left window (window < 0: full causal; w >= 0: query i
+ * attends keys i-w..i), per head h of qkv [B*T, 3C] (q | k | v, head h at columns h*hd of
+ * each third), nanochat architecture page, "Modellarchitektur und FLOPs-Berechnung".
+ * forward:  o [B*T, C] bf16, lse [B, H, T] fp32 (natural-log log-sum-exp of the scaled scores).
+ * backward: dqkv [B*T, 3C] bf16 from dout [B*T, C] and the forward's o and lse; Dbuf [B, H, T]
+ *           fp32 scratch (receives rowsum(dout * o)).
+ * GPTK_PATH_TCGEN05 needs head_dim 64; GPTK_PATH_SIMT takes head_dim 32, 64 or 128. */
+int gptk_attention_fwd_bf16(const void *qkv, void *o, float *lse, int B, int T, int C, int H,
+                            int window, unsigned *dev_err, int path, void *stream);
+int gptk_attention_bwd_bf16(const void *qkv, const void *o, const void *dout, const float *lse,
+                            float *Dbuf, void *dqkv, int B, int T, int C, int H, int window,
+                            unsigned *dev_err, int path, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
