@@ -72,9 +72,15 @@ def test_attention_vs_sdpa(env, path, B, T, H, w):
     ro, rlse, rdq = _ref(torch, qkv, B, T, C, H, w, dout)
     assert (o.float() - ro).abs().max().item() <= 2e-2 * ro.abs().max().item()
     assert (lse - rlse).abs().max().item() <= 2e-3 * max(1.0, rlse.abs().max().item())
+    dv_scale = rdq[:, 2 * C:].abs().max().item()
     for part in range(3):
         a = dq.float()[:, part * C:(part + 1) * C]
         r = rdq[:, part * C:(part + 1) * C]
+        if r.abs().max().item() <= 1e-3 * dv_scale:
+            # window 0: each query sees only itself, so dS = P(dP - D) = 0 and dq = dk = 0
+            # exactly; both sides hold rounding noise only
+            assert a.abs().max().item() <= 1e-2 * dv_scale, part
+            continue
         cos = torch.nn.functional.cosine_similarity(a.flatten(), r.flatten(), dim=0).item()
         assert cos >= 0.999, (part, cos)
         assert (a - r).abs().max().item() <= 5e-2 * r.abs().max().item(), part
