@@ -1,0 +1,119 @@
+"""Per-kernel timing of the step's GEMM and attention kernels at the GPT-2 124M shapes
+(B=16, T=1024, C=768, H=12), through the kernel-level C ABI (include/gpt_kernels.h).
+
+    python -m gpt_transformer_step_b200.kernel_bench [--case NAME ...] [--reps N] [--path tc|simt]
+
+Each case runs `warmup` untimed launches, then `reps` launches timed with CUDA events on the
+launching stream; prints one JSON line per case with ms per launch and TFLOP/s (algorithmic
+FLOPs: 2*M*N*K per GEMM; 4*hd per admitted score forward, 10*hd backward).
+Also the workload for small ncu captures of a single kernel (few hundred MB on the device).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+B, T, C, H = 16, 1024, 768, 12
+M = B * T
+
+# name: (M, N, K, a_kmajor, b_kmajor, epilogue, split)
+GEMMS = {
+    "gemm_qkv": (M, 3 * C, C, 1, 1, "store", 1),
+    "gemm_attnproj": (M, C, C, 1, 1, "resid", 1),
+    "gemm_fc": (M, 4 * C, C, 1, 1, "store_gelu", 1),
+    "gemm_mlpproj": (M, C, 4 * C, 1, 1, "resid", 1),
+    "gemm_dgrad_mlpproj": (M, 4 * C, C, 1, 0, "dgelu", 1),
+    "gemm_dgrad_fc": (M, C, 4 * C, 1, 0, "store", 1),
+    "gemm_wgrad_fc": (4 * C, C, M, 0, 0, "f32_store", 2),
+    "gemm_wgrad_qkv": (3 * C, C, M, 0, 0, "f32_store", 2),
+    "gemm_lmhead": (M, 50304, C, 1, 1, "store", 1),
+}
+ATTN = ("attn_fwd", "attn_bwd")
+
+
+def causal_scores(Bn, Tn, Hn, w=-1):
+    s = 0
+    for i in range(Tn):
+        lo = 0 if w < 0 else max(0, i - w)
+        s += i - lo + 1
+    return s * Bn * Hn
+
+
+def main():
+    import torch
+
+    from gpt_transformer_step_b200 import binding as gb
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", nargs="*", default=list(GEMMS) + list(ATTN))
+    ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--path", default="tc", choices=["tc", "simt"])
+    args = ap.parse_args()
+    path = gb.GPTK_PATH_TCGEN05 if args.path == "tc" else gb.GPTK_PATH_SIMT
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    for name in args.case:
+        with torch.cuda.stream(stream):
+            s = stream.cuda_stream
+            if name in GEMMS:
+                m, n, k, ak, bk, epi, split = GEMMS[name]
+                A = torch.randn(m * k, device=dev).to(torch.bfloat16)
+                Bm = torch.randn(n * k, device=dev).to(torch.bfloat16)
+                lda = k if ak else m
+                ldb = k if bk else n
+                f32 = epi.startswith("f32")
+                out = torch.empty(1 if f32 else m * n, dtype=torch.bfloat16, device=dev)
+                out2 = torch.empty(m * n if epi == "store_gelu" else 1, dtype=torch.bfloat16, device=dev)
+                aux = torch.randn(m * n if epi in ("resid", "dgelu") else 1, device=dev).to(torch.bfloat16)
+                outf = torch.empty(m * n if f32 else 1, device=dev)
+                scratch = torch.empty(max(1, split * m * n) if split > 1 else 1, device=dev)
+
+                def run():
+                    rc = gb.gptk_gemm_bf16(m, n, k, A.data_ptr(), lda, ak, Bm.data_ptr(), ldb, bk,
+                                           gb.GPTK_EPI[epi], out.data_ptr(), n, out2.data_ptr(), n,
+                                           aux.data_ptr(), n, outf.data_ptr(), n, split,
+                                           scratch.data_ptr(), scratch.numel(), err.data_ptr(),
+                                           path, s)
+                    assert rc == 0, rc
+                flops = 2.0 * m * n * k
+            else:
+                qkv = torch.randn(M, 3 * C, device=dev).to(torch.bfloat16)
+                o = torch.empty(M, C, dtype=torch.bfloat16, device=dev)
+                lse = torch.empty(B, H, T, device=dev)
+                dout = torch.randn(M, C, device=dev).to(torch.bfloat16)
+                D = torch.empty(B, H, T, device=dev)
+                dq = torch.empty(M, 3 * C, dtype=torch.bfloat16, device=dev)
+                gb.gptk_attention_fwd_bf16(qkv.data_ptr(), o.data_ptr(), lse.data_ptr(), B, T, C,
+                                           H, -1, err.data_ptr(), path, s)
+                hd = C // H
+                sc = causal_scores(B, T, H)
+                if name == "attn_fwd":
+                    def run():
+                        rc = gb.gptk_attention_fwd_bf16(qkv.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                                        B, T, C, H, -1, err.data_ptr(), path, s)
+                        assert rc == 0, rc
+                    flops = 4.0 * hd * sc
+                else:
+                    def run():
+                        rc = gb.gptk_attention_bwd_bf16(qkv.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                                        lse.data_ptr(), D.data_ptr(), dq.data_ptr(),
+                                                        B, T, C, H, -1, err.data_ptr(), path, s)
+                        assert rc == 0, rc
+                    flops = 10.0 * hd * sc
+            for _ in range(args.warmup):
+                run()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.reps):
+                run()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.reps
+        print(json.dumps({"case": name, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                          "err": int(err.item())}), flush=True)
+
+
+if __name__ == "__main__":
+    main()
