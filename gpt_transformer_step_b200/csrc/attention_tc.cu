@@ -175,18 +175,36 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
       const int k0 = (kt0 + j) * TILE;
       if (!warp_wait(&bar[F_SFULL], j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
-      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-      float mt = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tS + c * 32, v);
+      // the whole 128-key score row of this thread, one wait for the four loads
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32_nw(tS, s0);
+      tmem_ld32_nw(tS + 32, s1);
+      tmem_ld32_nw(tS + 64, s2);
+      tmem_ld32_nw(tS + 96, s3);
+      tmem_wait_ld32(s0);
+      reg_fence32(s1);
+      reg_fence32(s2);
+      reg_fence32(s3);
+      float sv[128];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool a = interior || admitted(qi, k0 + c * 32 + i, w);
-          if (a) mt = fmaxf(mt, v[i] * P.scale_log2);
-        }
+      for (int i = 0; i < 32; ++i) {
+        sv[i] = __uint_as_float(s0[i]);
+        sv[32 + i] = __uint_as_float(s1[i]);
+        sv[64 + i] = __uint_as_float(s2[i]);
+        sv[96 + i] = __uint_as_float(s3[i]);
       }
+      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+      if (!interior) {
+        // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= i <= hi
+        const int hi = qi - k0;
+        const int lo = w >= 0 ? qi - w - k0 : -1;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sv[i] = (i <= hi && i >= lo) ? sv[i] : -INFINITY;
+      }
+      float mx = sv[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+      const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
       float mnew = m2;
       bool resc = false;
       if (mt > -INFINITY) {
@@ -211,17 +229,15 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
       }
       m2 = mnew;
       if (mt > -INFINITY) have = true;
+      const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
       float ls = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tS + c * 32, v);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (have && (interior || admitted(qi, k0 + c * 32 + i, w))) p0 = ex2(v[i] * P.scale_log2 - m2);
-          if (have && (interior || admitted(qi, k0 + c * 32 + i + 1, w))) p1 = ex2(v[i + 1] * P.scale_log2 - m2);
+          const float p0 = ex2(fmaf(sv[c * 32 + i], P.scale_log2, -mu));
+          const float p1 = ex2(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
           ls += p0 + p1;
           pk[i >> 1] = pack_bf16(p0, p1);
         }
@@ -376,19 +392,25 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         tc_fence_after();
       }
       const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+      const int hi = qi < P.T ? qi - k0 : -1;  // admitted keys: lo <= i <= hi
+      const int lo = w >= 0 ? qi - w - k0 : -1;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
-        float sv[32], dp[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tdP + c * 32, dp);
+        uint32_t sr[32], dr[32];
+        tmem_ld32_nw(tS + c * 32, sr);
+        tmem_ld32_nw(tdP + c * 32, dr);
+        tmem_wait_ld32(sr);
+        reg_fence32(dr);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float d0 = 0.f, d1 = 0.f;
-          if (qi < P.T && (interior || admitted(qi, k0 + c * 32 + i, w)))
-            d0 = ex2(sv[i] * P.scale_log2 - lse2) * (dp[i] - D);
-          if (qi < P.T && (interior || admitted(qi, k0 + c * 32 + i + 1, w)))
-            d1 = ex2(sv[i + 1] * P.scale_log2 - lse2) * (dp[i + 1] - D);
+          float d0 = ex2(fmaf(__uint_as_float(sr[i]), P.scale_log2, -lse2)) * (__uint_as_float(dr[i]) - D);
+          float d1 = ex2(fmaf(__uint_as_float(sr[i + 1]), P.scale_log2, -lse2)) * (__uint_as_float(dr[i + 1]) - D);
+          if (!interior) {
+            const int ii = c * 32 + i;
+            d0 = (ii <= hi && ii >= lo) ? d0 : 0.f;
+            d1 = (ii + 1 <= hi && ii + 1 >= lo) ? d1 : 0.f;
+          }
           pk[i >> 1] = pack_bf16(d0, d1);
         }
         uint8_t *blk = sdS + (c >> 1) * 16384;
@@ -529,24 +551,28 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       tc_fence_after();
       const bool interior = (k0 + TILE - 1 <= qq0) && (w < 0 || k0 >= qq0 + TILE - 1 - w) &&
                             (qq0 + TILE <= P.T);
+      // queries admitted for key ki: ki <= q <= ki + w, q < T  ->  lo <= i <= hi
+      const int lo = ki - qq0;
+      const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
-        float sv[32], dp[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tdP + c * 32, dp);
+        uint32_t sr[32], dr[32];
+        tmem_ld32_nw(tS + c * 32, sr);
+        tmem_ld32_nw(tdP + c * 32, dr);
+        tmem_wait_ld32(sr);
+        reg_fence32(dr);
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-          const int qa = qq0 + c * 32 + i;
-          if (interior || (qa < P.T && admitted(qa, ki, w))) {
-            p0 = ex2(sv[i] * P.scale_log2 - s_lse[c * 32 + i]);
-            d0 = p0 * (dp[i] - s_D[c * 32 + i]);
+          const int ii = c * 32 + i;
+          float p0 = ex2(fmaf(__uint_as_float(sr[i]), P.scale_log2, -s_lse[ii]));
+          float p1 = ex2(fmaf(__uint_as_float(sr[i + 1]), P.scale_log2, -s_lse[ii + 1]));
+          if (!interior) {
+            p0 = (ii <= hi && ii >= lo) ? p0 : 0.f;
+            p1 = (ii + 1 <= hi && ii + 1 >= lo) ? p1 : 0.f;
           }
-          if (interior || (qa + 1 < P.T && admitted(qa + 1, ki, w))) {
-            p1 = ex2(sv[i + 1] * P.scale_log2 - s_lse[c * 32 + i + 1]);
-            d1 = p1 * (dp[i + 1] - s_D[c * 32 + i + 1]);
-          }
+          const float d0 = p0 * (__uint_as_float(dr[i]) - s_D[ii]);
+          const float d1 = p1 * (__uint_as_float(dr[i + 1]) - s_D[ii + 1]);
           pp[i >> 1] = pack_bf16(p0, p1);
           pd[i >> 1] = pack_bf16(d0, d1);
         }

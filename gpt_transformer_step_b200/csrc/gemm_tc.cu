@@ -30,7 +30,9 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
 constexpr int TMEM_COLS = 512;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
@@ -179,7 +181,7 @@ __device__ __forceinline__ void epi_chunk(const TcParams &P, int row, int col0, 
       for (int i = 0; i < 32; ++i) a[i] = (col0 + i < P.N) ? __bfloat162float(aux[i]) : 0.f;
     }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_f(a[i]);
+    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_fast(a[i]);
   }
   if (full) {
     st_bf16x32(dst, v);
@@ -190,7 +192,7 @@ __device__ __forceinline__ void epi_chunk(const TcParams &P, int row, int col0, 
   }
   if (EPI == TE_STORE_GELU) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+    for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i]);
     bf16 *d2 = (bf16 *)e.out2 + (long)row * e.ldo2 + col0;
     if (full) {
       st_bf16x32(d2, v);
@@ -226,7 +228,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 4);
+      mbar_init(&tempty_bar[a], EPI_WARPS);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -335,7 +337,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     __syncwarp();
   } else {
     // ------------------------------ epilogue ------------------------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // 8 warps: warp w reads TMEM lane quarter (w % 4) and columns [half*128, half*128+128)
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     int i = 0;
     for (int u = blockIdx.x; u < P.units; u += gridDim.x, ++i) {
       const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
@@ -347,19 +351,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!okw) break;
       tc_fence_after();
       const int row = mt * BM + q * 32 + lane;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int c0 = half * EPI_COLS;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0);
       float ce_max = -INFINITY, ce_sum = 0.f;
-      const int ncols = min(BN, P.N - nt * BN);
+      const int ncols = min(BN, P.N - nt * BN) - c0;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < EPI_COLS / 32; ++c) {
         if (c * 32 >= ncols) break;  // uniform across the warp
         float v[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), v);
-        if (row < P.M) epi_chunk<EPI>(P, row, nt * BN + c * 32, z, v, ce_max, ce_sum);
+        if (row < P.M) epi_chunk<EPI>(P, row, nt * BN + c0 + c * 32, z, v, ce_max, ce_sum);
       }
-      if (EPI == TE_CE_STATS && row < P.M) {
+      if (EPI == TE_CE_STATS && row < P.M && ncols > 0) {
         const Epi &e = P.epi;
-        float *st = e.stats + ((long)(e.row_offset + row) * e.ntiles + nt) * 2;
+        float *st = e.stats + ((long)(e.row_offset + row) * e.ntiles + nt * 2 + half) * 2;
         st[0] = ce_max;
         st[1] = ce_sum;
       }

@@ -167,8 +167,8 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
     e = launch_gemm_simt<float>(d, h->stream);
   } else if (h->tc && tc_gemm_supported(d)) {
     if (d.epi.kind == EPI_CE_STATS) {
-      d.epi.tile_n = TC_BN;
-      d.epi.ntiles = (d.N + TC_BN - 1) / TC_BN;
+      d.epi.tile_n = TC_CE_TILE;
+      d.epi.ntiles = (d.N + TC_CE_TILE - 1) / TC_CE_TILE;
       h->ce_ntiles = d.epi.ntiles;
     }
     if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 128, 256) : 1;
