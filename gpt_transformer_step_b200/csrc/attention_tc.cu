@@ -711,3 +711,49 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
   attn_bwd_dkv_tc<<<B * H * nt, 192, DKV_SMEM, st>>>(mq, md, p);
   return cudaGetLastError();
 }
+
+// ------------------------------------------------------------------------------------------
+// Attention backward that allocates nothing.
+//
+// For callers that cannot call cudaMalloc (for example code running inside a memory pool
+// or an allocator hook that must not re-enter the allocator, or a host that only owns the
+// tensors it passes in): the backward's per-row scratch D = rowsum(dO * O) lives in this
+// file-scope device array instead of a caller buffer. Every GPU that loads the library
+// keeps NOALLOC_D_MAX floats (4 MiB) of it until the process exits. The kernels below write
+// D for every row before reading it, so nothing has to be cleared between calls. All calls
+// on a device share the array: calls that overlap on the GPU (different streams, no
+// ordering) race on it.
+// ------------------------------------------------------------------------------------------
+constexpr size_t NOALLOC_D_MAX = 1u << 20;  // B * n_head * T rows
+static __device__ __align__(256) float g_noalloc_D[NOALLOC_D_MAX];
+
+namespace {
+constexpr int NOALLOC_MAX_DEVICES = 64;
+float *g_noalloc_D_addr[NOALLOC_MAX_DEVICES];  // device address per device ordinal
+
+// Device address of g_noalloc_D on the current device; looked up once per device. In host
+// code the symbol itself is only a host-side stand-in, never a device address.
+cudaError_t noalloc_D_address(float **out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
+  if (!g_noalloc_D_addr[dev]) {
+    void *ptr = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_D));
+    g_noalloc_D_addr[dev] = (float *)ptr;
+  }
+  *out = g_noalloc_D_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+size_t attention_bwd_noalloc_max_rows() { return NOALLOC_D_MAX; }
+
+cudaError_t launch_attention_bwd_tc_noalloc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
+                                            const float *lse, bf16 *dqkv, int B, int T, int C,
+                                            int H, int window, unsigned *err, cudaStream_t st) {
+  if ((size_t)B * H * T > NOALLOC_D_MAX) return cudaErrorInvalidValue;
+  float *D = nullptr;
+  CUDA_TRY(noalloc_D_address(&D));
+  return launch_attention_bwd_tc(qkv, o, dout, lse, D, dqkv, B, T, C, H, window, err, st);
+}

@@ -92,3 +92,18 @@ extern "C" int gptk_attention_bwd_bf16(const void *qkv, const void *o, const voi
   }
   return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }
+
+// Attention backward without any allocation: see include/gpt_kernels.h.
+extern "C" int gptk_attention_bwd_bf16_noalloc(const void *qkv, const void *o, const void *dout,
+                                               const float *lse, void *dqkv, int B, int T, int C,
+                                               int H, int window, unsigned *dev_err,
+                                               void *stream) {
+  if (!qkv || !o || !dout || !lse || !dqkv || !dev_err || B <= 0 || T <= 0 || H <= 0 || C % H)
+    return GPT_ERR_INVALID_ARG;
+  if (!attention_tc_supported(C, H)) return GPT_ERR_SHAPE;
+  if ((size_t)B * H * T > attention_bwd_noalloc_max_rows()) return GPT_ERR_SHAPE;
+  cudaError_t e = launch_attention_bwd_tc_noalloc((const bf16 *)qkv, (const bf16 *)o,
+                                                  (const bf16 *)dout, lse, (bf16 *)dqkv, B, T, C,
+                                                  H, window, dev_err, (cudaStream_t)stream);
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}

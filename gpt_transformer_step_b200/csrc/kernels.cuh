@@ -66,6 +66,13 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
                                     const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
                                     int C, int H, int window, unsigned *err, cudaStream_t st);
 
+// The same backward with its D scratch in a file-scope device array (no allocation); rejects
+// B*H*T > attention_bwd_noalloc_max_rows() with cudaErrorInvalidValue.
+size_t attention_bwd_noalloc_max_rows();
+cudaError_t launch_attention_bwd_tc_noalloc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
+                                            const float *lse, bf16 *dqkv, int B, int T, int C,
+                                            int H, int window, unsigned *err, cudaStream_t st);
+
 // GEMM on CUDA cores (fp32 validation mode and shapes the tensor-core path does not take).
 template <typename T>
 cudaError_t launch_gemm_simt(const GemmDesc &d, cudaStream_t st);

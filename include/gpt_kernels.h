@@ -57,6 +57,21 @@ int gptk_attention_bwd_bf16(const void *qkv, const void *o, const void *dout, co
                             float *Dbuf, void *dqkv, int B, int T, int C, int H, int window,
                             unsigned *dev_err, int path, void *stream);
 
+/* Attention backward that allocates nothing (no counterpart in the pages: it exists for
+ * callers that cannot call cudaMalloc, such as code running inside an allocator hook or a
+ * memory pool that must not re-enter the allocator). Same arguments and results as
+ * gptk_attention_bwd_bf16 on the tensor-core path, minus the Dbuf scratch: the per-row
+ * scratch D = rowsum(dout * o) lives in a static device array of 2^20 floats (4 MiB) that
+ * every GPU loading this library holds until the process exits.
+ * Limits: head_dim 64; B * H * T <= 1048576, else GPT_ERR_SHAPE (nothing is launched).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture. All calls on one device share the array:
+ * calls that overlap on the GPU (unordered streams) race on it. Nothing in it needs clearing
+ * between calls: every row of D is written before it is read. Calls no allocating routine. */
+int gptk_attention_bwd_bf16_noalloc(const void *qkv, const void *o, const void *dout,
+                                    const float *lse, void *dqkv, int B, int T, int C, int H,
+                                    int window, unsigned *dev_err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
