@@ -88,7 +88,9 @@ __global__ void embed_fwd_kernel(const int *__restrict__ tok, const int *__restr
 // ------------------------------------------------------------------------------------------
 constexpr int LN_MAXV = 8;  // vectors per lane: C <= 32*8*VN
 
-template <typename T>
+// NV = 16-byte vectors per lane (ceil(C / (32*VN))), a compile-time bound on the row slice
+// each lane keeps in registers.
+template <typename T, int NV>
 __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
                                      T *__restrict__ y, float *__restrict__ mean,
                                      float *__restrict__ rstd, int M, int C, float eps) {
@@ -97,10 +99,10 @@ __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restric
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
   const int nv = C / VN;
-  float v[LN_MAXV][VN];
+  float v[NV][VN];
   float s = 0.f;
 #pragma unroll
-  for (int j = 0; j < LN_MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     int c = (lane + 32 * j) * VN;
     if (lane + 32 * j < nv) {
       load_vec<T>(x + (long)row * C + c, v[j]);
@@ -111,7 +113,7 @@ __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restric
   const float mu = warp_sum(s) / (float)C;
   float q = 0.f;
 #pragma unroll
-  for (int j = 0; j < LN_MAXV; ++j)
+  for (int j = 0; j < NV; ++j)
     if (lane + 32 * j < nv) {
 #pragma unroll
       for (int k = 0; k < VN; ++k) {
@@ -122,7 +124,7 @@ __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restric
   const float var = warp_sum(q) / (float)C;
   const float rs = 1.0f / sqrtf(var + eps);
 #pragma unroll
-  for (int j = 0; j < LN_MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     int c = (lane + 32 * j) * VN;
     if (lane + 32 * j < nv) {
       float gg[VN], o[VN];
@@ -142,9 +144,9 @@ __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restric
 // K12 LayerNorm backward (+ residual-gradient add, + per-block dgamma partials)
 // ------------------------------------------------------------------------------------------
 constexpr int LNB_WARPS = 8;
-constexpr int LNB_MAX_BLOCKS = 296;
+constexpr int LNB_MAX_BLOCKS = 592;
 
-template <typename T>
+template <typename T, int NV>
 __global__ void __launch_bounds__(LNB_WARPS * 32)
 layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
                      const float *__restrict__ mean, const float *__restrict__ rstd,
@@ -154,25 +156,26 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
   extern __shared__ float sm_dg[];  // [LNB_WARPS][C]
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nv = C / VN;
-  float dgacc[LN_MAXV][VN];
+  float dgacc[NV][VN];
 #pragma unroll
-  for (int j = 0; j < LN_MAXV; ++j)
+  for (int j = 0; j < NV; ++j)
 #pragma unroll
     for (int k = 0; k < VN; ++k) dgacc[j][k] = 0.f;
   const int r0 = blockIdx.x * rows_per_block;
   const int r1 = min(M, r0 + rows_per_block);
   for (int row = r0 + w; row < r1; row += LNB_WARPS) {
     const float mu = mean[row], rs = rstd[row];
-    float xh[LN_MAXV][VN], dxh[LN_MAXV][VN];
+    float xh[NV][VN], dxh[NV][VN], rv[NV][VN];
     float a = 0.f, b = 0.f;
 #pragma unroll
-    for (int j = 0; j < LN_MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       int c = (lane + 32 * j) * VN;
       if (lane + 32 * j < nv) {
         float xv[VN], dv[VN], gv[VN];
         load_vec<T>(x + (long)row * C + c, xv);
         load_vec<T>(dy + (long)row * C + c, dv);
         load_vec<T>(g + c, gv);
+        load_vec<T>(dres + (long)row * C + c, rv[j]);  // issued with the others
 #pragma unroll
         for (int k = 0; k < VN; ++k) {
           xh[j][k] = (xv[k] - mu) * rs;
@@ -186,19 +189,18 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
     a = warp_sum(a) / (float)C;
     b = warp_sum(b) / (float)C;
 #pragma unroll
-    for (int j = 0; j < LN_MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       int c = (lane + 32 * j) * VN;
       if (lane + 32 * j < nv) {
         float r[VN];
-        load_vec<T>(dres + (long)row * C + c, r);
 #pragma unroll
-        for (int k = 0; k < VN; ++k) r[k] += rs * (dxh[j][k] - a - xh[j][k] * b);
+        for (int k = 0; k < VN; ++k) r[k] = rv[j][k] + rs * (dxh[j][k] - a - xh[j][k] * b);
         store_vec<T>(dres + (long)row * C + c, r);
       }
     }
   }
 #pragma unroll
-  for (int j = 0; j < LN_MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     int c = (lane + 32 * j) * VN;
     if (lane + 32 * j < nv)
 #pragma unroll
@@ -212,13 +214,24 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
   }
 }
 
-__global__ void colsum_kernel(const float *__restrict__ partial, int nrows, int C,
-                              float *__restrict__ out) {
-  int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= C) return;
+// out[c] = sum_r partial[r][c]: block = 32 columns x 8 row groups; each thread sums rows
+// g, g+8, ... in order, then the 8 group sums are added in group order (deterministic).
+__global__ void __launch_bounds__(256) colsum_kernel(const float *__restrict__ partial, int nrows,
+                                                     int C, float *__restrict__ out) {
+  __shared__ float sh[8][33];
+  const int cx = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + cx;
   float s = 0.f;
-  for (int r = 0; r < nrows; ++r) s += partial[(long)r * C + c];
-  out[c] = s;
+  if (c < C)
+    for (int r = g; r < nrows; r += 8) s += partial[(long)r * C + c];
+  sh[g][cx] = s;
+  __syncthreads();
+  if (g == 0 && c < C) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t += sh[i][cx];
+    out[c] = t;
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -526,12 +539,30 @@ cudaError_t embed_sort_smem_attr() {
                               SORT_MAX * sizeof(unsigned));
 }
 
+#define LN_DISPATCH(NVV, CALL)                    \
+  switch (NVV) {                                  \
+    case 1: CALL(1); break;                       \
+    case 2: CALL(2); break;                       \
+    case 3: CALL(3); break;                       \
+    case 4: CALL(4); break;                       \
+    case 5: case 6: CALL(6); break;               \
+    default: CALL(8); break;                      \
+  }
+
+template <typename T>
+int ln_nv(int C) {
+  const int per = 32 * Vec<T>::N;
+  return (C + per - 1) / per;
+}
+
 template <typename T>
 cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
                                  int C, float eps, cudaStream_t st) {
   const int warps = 8;
-  layernorm_fwd_kernel<T><<<(M + warps - 1) / warps, warps * 32, 0, st>>>(x, g, y, mean, rstd,
-                                                                          M, C, eps);
+  const int grid = (M + warps - 1) / warps;
+#define LNF(NVC) layernorm_fwd_kernel<T, NVC><<<grid, warps * 32, 0, st>>>(x, g, y, mean, rstd, M, C, eps)
+  LN_DISPATCH(ln_nv<T>(C), LNF)
+#undef LNF
   return cudaGetLastError();
 }
 
@@ -547,10 +578,13 @@ cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, cons
   const int nb = layernorm_bwd_blocks(M);
   const int rpb = (M + nb - 1) / nb;
   const size_t smem = (size_t)LNB_WARPS * C * sizeof(float);
-  layernorm_bwd_kernel<T><<<nb, LNB_WARPS * 32, smem, st>>>(x, g, mean, rstd, dy, dres,
-                                                            dg_partial, M, C, rpb);
+#define LNB(NVC)                                                                              \
+  layernorm_bwd_kernel<T, NVC><<<nb, LNB_WARPS * 32, smem, st>>>(x, g, mean, rstd, dy, dres, \
+                                                                 dg_partial, M, C, rpb)
+  LN_DISPATCH(ln_nv<T>(C), LNB)
+#undef LNB
   CUDA_TRY(cudaGetLastError());
-  colsum_kernel<<<(C + 255) / 256, 256, 0, st>>>(dg_partial, nb, C, dg);
+  colsum_kernel<<<(C + 31) / 32, 256, 0, st>>>(dg_partial, nb, C, dg);
   return cudaGetLastError();
 }
 

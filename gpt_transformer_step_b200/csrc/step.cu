@@ -156,6 +156,7 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
   }
   cudaError_t e;
   const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
+  const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
   if (!h->use_bf16) {
     if (d.epi.kind == EPI_CE_STATS) {
       d.epi.tile_n = SIMT_TILE_N;
@@ -171,7 +172,12 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
       d.epi.ntiles = (d.N + TC_CE_TILE - 1) / TC_CE_TILE;
       h->ce_ntiles = d.epi.ntiles;
     }
-    if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 128, 256) : 1;
+    // weight gradients (fp32 out) and any elementwise epilogue whose tile grid leaves SMs
+    // idle split K; the fp32 partials are reduced in a fixed order
+    if (d.split_k == 0) {
+      const long tiles = (long)((d.M + TC_BM - 1) / TC_BM) * ((d.N + TC_BN - 1) / TC_BN);
+      d.split_k = (f32out || (elementwise && tiles < 148)) ? choose_split(h, d.M, d.N, d.K, TC_BM, TC_BN) : 1;
+    }
     d.partial = h->splitk;
     e = tc_gemm_launch(h->tc, d, h->stream, &h->launches);
   } else {
@@ -547,7 +553,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   const size_t M = h->maxM;
   h->ce_tile_n = SIMT_TILE_N;  // the stats buffer is sized for the narrowest column tile
   h->ce_ntiles = (h->V + h->ce_tile_n - 1) / h->ce_tile_n;
-  h->chunk_rows = c.lmhead_chunk_rows > 0 ? c.lmhead_chunk_rows : 4096;
+  h->chunk_rows = c.lmhead_chunk_rows > 0 ? c.lmhead_chunk_rows : 8192;
   if (h->chunk_rows > (int)M) h->chunk_rows = (int)M;
   h->ldS = (h->V + 7) / 8 * 8;
   h->splitk_elems = (size_t)8 * ((size_t)h->mC * C > (size_t)M * C ? (size_t)h->mC * C : (size_t)M * C);
