@@ -85,6 +85,17 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest value over all ranks (the slowest replica's time); identity for world 1."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def oracle_sample_step(wl, T_sample: int, seed: int = 0):
     """One oracle training step (float instantiation, one thread) on B=1 x T_sample tokens of
     the workload's model. Returns (seconds, tokens)."""
@@ -181,11 +192,7 @@ def run_ours(args, wl, rank, world, local_rank):
             e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1) / n
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
         return ms, losses
 
     st.set_stream(stream.cuda_stream)

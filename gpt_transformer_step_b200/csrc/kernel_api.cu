@@ -4,6 +4,7 @@
 #include "../../include/gpt_step.h"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace {
 TcGemm *tc_instance() {
@@ -106,4 +107,34 @@ extern "C" int gptk_attention_bwd_bf16_noalloc(const void *qkv, const void *o, c
                                                   (const bf16 *)dout, lse, (bf16 *)dqkv, B, T, C,
                                                   H, window, dev_err, (cudaStream_t)stream);
   return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
+namespace {
+// Waits, with the library's bounded wait, on an mbarrier that nothing ever arrives on. The
+// wait gives up after timeout_ns, sets the timeout bit in the device error word and the
+// kernel returns: the context stays usable.
+__global__ void wait_selftest_kernel(unsigned long long timeout_ns, unsigned *err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    abort_flag = 0;
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_try_wait(&bar, 0)) {
+    if (tc::globaltimer() - t0 > timeout_ns) {
+      atomicOr(err, GPT_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+}  // namespace
+
+extern "C" int gptk_selftest_bounded_wait(unsigned timeout_us, unsigned *dev_err, void *stream) {
+  if (!dev_err || timeout_us == 0 || timeout_us > 2000000u) return GPT_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(1000ull * timeout_us, dev_err);
+  return cudaGetLastError() == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }

@@ -57,6 +57,12 @@ int gptk_attention_bwd_bf16(const void *qkv, const void *o, const void *dout, co
                             float *Dbuf, void *dqkv, int B, int T, int C, int H, int window,
                             unsigned *dev_err, int path, void *stream);
 
+/* Failure-detection self test: launches one CTA that waits on an mbarrier nothing arrives
+ * on, with the bounded wait every kernel of the step uses for its barriers; after timeout_us
+ * (1 .. 2,000,000) it gives up, ORs GPT_DEVERR_TIMEOUT (2) into *dev_err and returns, leaving
+ * the CUDA context usable. Does not synchronise. */
+int gptk_selftest_bounded_wait(unsigned timeout_us, unsigned *dev_err, void *stream);
+
 /* Attention backward that allocates nothing (no counterpart in the pages: it exists for
  * callers that cannot call cudaMalloc, such as code running inside an allocator hook or a
  * memory pool that must not re-enter the allocator). Same arguments and results as
