@@ -7,12 +7,16 @@
 // both layouts directly (instruction-descriptor transpose bits), so the weight-gradient and
 // data-gradient GEMMs of the backward pass need no transposed copies.
 //
-// Structure: persistent CTAs (one per SM), 6 warps.
-//   warp 0      TMA producer: fills a ring of STAGES shared-memory stages (A 128x64, B 256x64)
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x (128x256x16) MMAs per stage,
+// Structure: persistent CTAs (one per SM), 10 warps.
+//   warp 0      TMA producer: fills a ring of shared-memory stages (A 128x64, B 256x64 or,
+//               for CTA pairs, this CTA's 128x64 half of B)
+//   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K = 16 per stage
+//               (128x256 per CTA, or 256x256 per CTA pair with cta_group::2);
 //               tcgen05.commit frees the stage; a second commit marks the accumulator full
-//   warps 2..5  epilogue: tcgen05.ld of the 128x256 fp32 accumulator (one row per thread),
-//               the fused epilogue, global stores
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (one row per thread, two warps
+//               per TMEM lane quarter, 128 columns each), the fused epilogue, global stores
+// Tiles of 256 rows run on CTA pairs whenever they fill the machine (the pair halves each
+// SM's shared-memory traffic per MMA); small-M GEMMs keep single-CTA 128-row tiles.
 // The accumulator is double-buffered in TMEM (2 x 256 columns), so the epilogue of one tile
 // overlaps the MMAs of the next. Every mbarrier wait is bounded: after ~2 s it sets the
 // device error word and the CTA leaves through its normal teardown (TMEM is always freed).
@@ -26,15 +30,11 @@ namespace {
 using namespace tc;
 
 constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK;
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 enum TcEpi {
   TE_STORE = 0, TE_STORE_GELU, TE_RESID, TE_DGELU, TE_F32_STORE, TE_F32_ACCUM, TE_CE_STATS,
@@ -207,86 +207,190 @@ __device__ __forceinline__ void epi_chunk(const TcParams &P, int row, int col0, 
 // ---------------------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------------------
-template <int EPI>
+// CG = 1: one CTA per 128x256 tile. CG = 2: a cluster of two CTAs per 256x256 tile; each CTA
+// TMA-loads its own 128 rows of A and 128 rows (N) of B into its own shared memory, the
+// leader (cluster rank 0) issues tcgen05.mma.cta_group::2, which reads both CTAs' stages and
+// writes rows 0-127 to the leader's TMEM and rows 128-255 to the peer's. Both CTAs' TMA
+// loads complete on the leader's stage barrier; the leader's commits arrive on both CTAs'
+// barriers (commit multicast); the peer's epilogue releases the accumulator with a remote
+// arrive on the leader's barrier. No TMA load uses cluster multicast.
+template <int CG>
+struct TcCfg {
+  static constexpr int B_ROWS = BN / CG;                 // rows of B each CTA loads
+  static constexpr int B_CTA_BYTES = B_ROWS * BK * 2;    // 32 KB / 16 KB
+  static constexpr int STAGE = A_BYTES + B_CTA_BYTES;    // 48 KB / 32 KB
+  static constexpr int NSTAGE = CG == 1 ? 4 : 6;
+  static constexpr int SMEM = NSTAGE * STAGE + 1024 + 256;
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory location in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx_addr(uint32_t addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes)
+               : "memory");
+}
+// TMA tile load whose completion is counted on mbarrier `mbar_cluster` (a shared::cluster
+// address, possibly in the peer CTA of the pair).
+template <int CG>
+__device__ __forceinline__ void tma_load_pair(void *dst, const CUtensorMap *map,
+                                              uint32_t mbar_cluster, int c0, int c1) {
+  if (CG == 2)
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+  else
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+template <int CG>
+__device__ __forceinline__ void umma_issue(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  if (CG == 2)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    umma_bf16(d_tmem, adesc, bdesc, idesc, accumulate);
+}
+// Arrive on `bar` (same offset) in every CTA of the pair once all prior MMAs complete.
+template <int CG>
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+  if (CG == 2)
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+  else
+    umma_commit(bar);
+}
+
+template <int EPI, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcParams P) {
+  using Cf = TcCfg<CG>;
+  constexpr int NS = Cf::NSTAGE;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t *full_bar = (uint64_t *)(smem + STAGES * STAGE_BYTES);
-  uint64_t *empty_bar = full_bar + STAGES;
-  uint64_t *tfull_bar = empty_bar + STAGES;
+  uint64_t *full_bar = (uint64_t *)(smem + NS * Cf::STAGE);
+  uint64_t *empty_bar = full_bar + NS;
+  uint64_t *tfull_bar = empty_bar + NS;
   uint64_t *tempty_bar = tfull_bar + 2;
   uint32_t *tmem_holder = (uint32_t *)(tempty_bar + 2);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int unit0 = CG == 2 ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int ustride = CG == 2 ? (int)nclusters_x() : (int)gridDim.x;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], EPI_WARPS);
+      mbar_init(&tempty_bar[a], EPI_WARPS * CG);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_holder)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (CG == 2) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_holder)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      tmem_alloc(tmem_holder, TMEM_COLS);
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
-    // ------------------------------ TMA producer ------------------------------
+    // ------------------------------ TMA producer (each CTA) ------------------------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      uint32_t issued = 0;  // bit s: stage s has been filled at least once; phase of last fill
-      uint32_t last_par = 0;
-      for (int u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
+      uint32_t issued = 0, last_par = 0;
+      for (int u = unit0; u < P.units && ok; u += ustride) {
         const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
-        const int m0 = mt * BM, n0 = nt * BN;
+        const int m0 = mt * BM * CG + (int)rank * BM;
+        const int n0 = nt * BN + (int)rank * Cf::B_ROWS;
         const int kb0 = z * P.kblocks_per_split;
         const int kb1 = min(P.total_kblocks, kb0 + P.kblocks_per_split);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, P.err)) { ok = false; break; }
-          uint8_t *sA = smem + stage * STAGE_BYTES;
+          uint8_t *sA = smem + stage * Cf::STAGE;
           uint8_t *sB = sA + A_BYTES;
-          mbar_expect_tx(&full_bar[stage], STAGE_BYTES);
+          const uint32_t fb = smem_u32(&full_bar[stage]);
+          const uint32_t fbl = CG == 2 ? mapa_shared(fb, 0) : fb;  // the leader's barrier
+          if (rank == 0) mbar_expect_tx_addr(fb, Cf::STAGE * CG);
           const int k0 = kb * BK;
           if (!P.a_mn) {
-            tma_load_2d(sA, &tmA, &full_bar[stage], k0, m0);
+            tma_load_pair<CG>(sA, &tmA, fbl, k0, m0);
           } else {
-            tma_load_2d(sA, &tmA, &full_bar[stage], m0, k0);
-            tma_load_2d(sA + A_BYTES / 2, &tmA, &full_bar[stage], m0 + 64, k0);
+            tma_load_pair<CG>(sA, &tmA, fbl, m0, k0);
+            tma_load_pair<CG>(sA + A_BYTES / 2, &tmA, fbl, m0 + 64, k0);
           }
           if (!P.b_mn) {
-            tma_load_2d(sB, &tmB, &full_bar[stage], k0, n0);
+            tma_load_pair<CG>(sB, &tmB, fbl, k0, n0);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sB + j * (B_BYTES / 4), &tmB, &full_bar[stage], n0 + 64 * j, k0);
+            for (int j = 0; j < Cf::B_ROWS / 64; ++j)
+              tma_load_pair<CG>(sB + j * 8192, &tmB, fbl, n0 + 64 * j, k0);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == NS) { stage = 0; phase ^= 1u; }
         }
       }
-      if (*abort_flag) {
+      if (*abort_flag && rank == 0) {
         // leave no bulk copy in flight: wait (bounded) for the last fill of every stage
         const uint64_t t0 = globaltimer();
-        for (int s2 = 0; s2 < STAGES; ++s2) {
+        for (int s2 = 0; s2 < NS; ++s2) {
           if (!(issued >> s2 & 1u)) continue;
           while (!mbar_try_wait(&full_bar[s2], (last_par >> s2) & 1u) &&
                  globaltimer() - t0 < 200000000ull) {
@@ -296,18 +400,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    // ------------------------------ MMA issuer (leader CTA) ------------------------------
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int i = 0;
-      // per-k16 start-address advance inside a stage
       const uint32_t a_step = P.a_mn ? 2048u : 32u;
       const uint32_t b_step = P.b_mn ? 2048u : 32u;
-      const uint32_t a_lbo = P.a_mn ? (uint32_t)(A_BYTES / 2) : 16u;
-      const uint32_t b_lbo = P.b_mn ? (uint32_t)(B_BYTES / 4) : 16u;
-      for (int u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++i) {
+      const uint32_t a_lbo = P.a_mn ? 8192u : 16u;
+      const uint32_t b_lbo = P.b_mn ? 8192u : 16u;
+      for (int u = unit0; u < P.units && ok; u += ustride, ++i) {
         const int z = u / (P.num_mt * P.num_nt);
         const int kb0 = z * P.kblocks_per_split;
         const int kb1 = min(P.total_kblocks, kb0 + P.kblocks_per_split);
@@ -319,29 +422,29 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, P.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sA = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sA = smem_u32(smem + stage * Cf::STAGE);
           const uint32_t sB = sA + A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = sdesc(sA + k * a_step, a_lbo, 1024u);
             const uint64_t bd = sdesc(sB + k * b_step, b_lbo, 1024u);
-            umma_bf16(d_tmem, ad, bd, P.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            umma_issue<CG>(d_tmem, ad, bd, P.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(&empty_bar[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          umma_commit_pair<CG>(&empty_bar[stage]);
+          if (++stage == NS) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull_bar[acc]);
+        umma_commit_pair<CG>(&tfull_bar[acc]);
       }
     }
     __syncwarp();
   } else {
-    // ------------------------------ epilogue ------------------------------
+    // ------------------------------ epilogue (each CTA) ------------------------------
     // 8 warps: warp w reads TMEM lane quarter (w % 4) and columns [half*128, half*128+128)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     int i = 0;
-    for (int u = blockIdx.x; u < P.units; u += gridDim.x, ++i) {
+    for (int u = unit0; u < P.units; u += ustride, ++i) {
       const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
       const int acc = i & 1;
       const uint32_t use = (uint32_t)(i >> 1);
@@ -350,7 +453,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
       tc_fence_after();
-      const int row = mt * BM + q * 32 + lane;
+      const int row = mt * BM * CG + (int)rank * BM + q * 32 + lane;
       const int c0 = half * EPI_COLS;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0);
       float ce_max = -INFINITY, ce_sum = 0.f;
@@ -370,16 +473,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      if (lane == 0) {
+        if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[acc]), 0));
+        else mbar_arrive(&tempty_bar[acc]);
+      }
     }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync_all(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(TMEM_COLS)
-                 : "memory");
+    if (CG == 2)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(TMEM_COLS)
+                   : "memory");
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -433,18 +542,48 @@ bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld,
   return r == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, int CG>
 cudaError_t launch_kind(const CUtensorMap &a, const CUtensorMap &b, const TcParams &P, int grid,
                         cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI, CG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcCfg<CG>::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  tc_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(a, b, P);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = TcCfg<CG>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CG;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<EPI, CG>, a, b, P);
+}
+
+template <int CG>
+cudaError_t launch_epi(int kind, bool split, const CUtensorMap &ma, const CUtensorMap &mb,
+                       const TcParams &P, int grid, cudaStream_t st) {
+  if (split) return launch_kind<TE_PARTIAL, CG>(ma, mb, P, grid, st);
+  switch (kind) {
+    case EPI_STORE: return launch_kind<TE_STORE, CG>(ma, mb, P, grid, st);
+    case EPI_STORE_GELU: return launch_kind<TE_STORE_GELU, CG>(ma, mb, P, grid, st);
+    case EPI_RESID: return launch_kind<TE_RESID, CG>(ma, mb, P, grid, st);
+    case EPI_DGELU: return launch_kind<TE_DGELU, CG>(ma, mb, P, grid, st);
+    case EPI_F32_STORE: return launch_kind<TE_F32_STORE, CG>(ma, mb, P, grid, st);
+    case EPI_F32_ACCUM: return launch_kind<TE_F32_ACCUM, CG>(ma, mb, P, grid, st);
+    case EPI_CE_STATS: return launch_kind<TE_CE_STATS, CG>(ma, mb, P, grid, st);
+    case EPI_CE_DS: return launch_kind<TE_CE_DS, CG>(ma, mb, P, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -453,13 +592,16 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 struct TcGemm {
   unsigned *err;
+  size_t splitk_capacity;  // floats available at GemmDesc::partial
 };
 
 cudaError_t tc_gemm_create(TcGemm **out) {
   *out = new TcGemm();
   (*out)->err = nullptr;
+  (*out)->splitk_capacity = 0;
   return cudaSuccess;
 }
+void tc_gemm_set_splitk_capacity(TcGemm *t, size_t floats) { t->splitk_capacity = floats; }
 void tc_gemm_destroy(TcGemm *t) { delete t; }
 
 bool tc_gemm_supported(const GemmDesc &d) {
@@ -487,51 +629,60 @@ bool tc_gemm_supported(const GemmDesc &d) {
 }
 
 cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches) {
+  (void)launches;
   TcParams P;
   memset(&P, 0, sizeof(P));
+  const int sms = num_sms();
+  // CTA pairs (256-row tiles) whenever they fill the machine; single CTAs otherwise
+  const int nt = (d.N + BN - 1) / BN;
+  const int CG = ((long)((d.M + 2 * BM - 1) / (2 * BM)) * nt >= sms / 2) ? 2 : 1;
   P.M = d.M; P.N = d.N; P.K = d.K;
-  P.num_mt = (d.M + BM - 1) / BM;
-  P.num_nt = (d.N + BN - 1) / BN;
+  P.num_mt = (d.M + BM * CG - 1) / (BM * CG);
+  P.num_nt = nt;
   P.total_kblocks = (d.K + BK - 1) / BK;
-  int S = d.split_k > 1 ? d.split_k : 1;
+  int S = d.split_k;
+  if (S <= 0) {  // automatic: split K while the tile grid leaves SMs idle
+    const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
+    const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
+    const long tiles = (long)P.num_mt * P.num_nt;
+    S = 1;
+    if (f32out || (elementwise && tiles * CG < sms))
+      while (tiles * S * CG < 2L * sms && P.total_kblocks / (S * 2) >= 4 &&
+             (size_t)S * 2 * d.M * d.N <= t->splitk_capacity && d.partial)
+        S *= 2;
+  }
   if (S > P.total_kblocks) S = P.total_kblocks;
   P.kblocks_per_split = (P.total_kblocks + S - 1) / S;
   S = (P.total_kblocks + P.kblocks_per_split - 1) / P.kblocks_per_split;  // no empty split
+  if (S > 1 && (!d.partial || (size_t)S * d.M * d.N > t->splitk_capacity)) return cudaErrorInvalidValue;
   d.split_k = S;
   P.splits = S;
   P.units = P.num_mt * P.num_nt * S;
   P.a_mn = d.a_kmajor ? 0 : 1;
   P.b_mn = d.b_kmajor ? 0 : 1;
   P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)P.a_mn << 15) |
-            ((uint32_t)P.b_mn << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            ((uint32_t)P.b_mn << 16) | ((uint32_t)(BN >> 3) << 17) |
+            ((uint32_t)((BM * CG) >> 4) << 24);
   P.epi = d.epi;
   P.partial = d.partial;
   P.err = d.err ? d.err : (d.epi.sc ? (unsigned *)&d.epi.sc->err : t->err);
   if (!P.err) return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
+  const int b_rows = BN / CG;
   bool ok = P.a_mn ? make_map(&ma, d.A, d.M, d.K, d.lda, 64)
                    : make_map(&ma, d.A, d.K, d.M, d.lda, BM);
   ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, 64)
-                     : make_map(&mb, d.B, d.K, d.N, d.ldb, BN));
+                     : make_map(&mb, d.B, d.K, d.N, d.ldb, b_rows));
   if (!ok) return cudaErrorInvalidValue;
-  const int grid = P.units < num_sms() ? P.units : num_sms();
   cudaError_t e;
-  if (S > 1) {
-    e = launch_kind<TE_PARTIAL>(ma, mb, P, grid, st);
-    if (e != cudaSuccess) return e;
-    return launch_splitk_reduce<bf16>(d, st);
+  if (CG == 2) {
+    const int clusters = P.units < sms / 2 ? P.units : sms / 2;
+    e = launch_epi<2>(d.epi.kind, S > 1, ma, mb, P, 2 * clusters, st);
+  } else {
+    const int grid = P.units < sms ? P.units : sms;
+    e = launch_epi<1>(d.epi.kind, S > 1, ma, mb, P, grid, st);
   }
-  switch (d.epi.kind) {
-    case EPI_STORE: e = launch_kind<TE_STORE>(ma, mb, P, grid, st); break;
-    case EPI_STORE_GELU: e = launch_kind<TE_STORE_GELU>(ma, mb, P, grid, st); break;
-    case EPI_RESID: e = launch_kind<TE_RESID>(ma, mb, P, grid, st); break;
-    case EPI_DGELU: e = launch_kind<TE_DGELU>(ma, mb, P, grid, st); break;
-    case EPI_F32_STORE: e = launch_kind<TE_F32_STORE>(ma, mb, P, grid, st); break;
-    case EPI_F32_ACCUM: e = launch_kind<TE_F32_ACCUM>(ma, mb, P, grid, st); break;
-    case EPI_CE_STATS: e = launch_kind<TE_CE_STATS>(ma, mb, P, grid, st); break;
-    case EPI_CE_DS: e = launch_kind<TE_CE_DS>(ma, mb, P, grid, st); break;
-    default: return cudaErrorInvalidValue;
-  }
-  (void)launches;
-  return e;
+  if (e != cudaSuccess) return e;
+  if (S > 1) return launch_splitk_reduce<bf16>(d, st);
+  return cudaSuccess;
 }

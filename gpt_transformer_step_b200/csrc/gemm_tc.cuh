@@ -10,7 +10,10 @@ constexpr int TC_CE_TILE = TC_BN / 2;  // column width of one cross-entropy stat
 struct TcGemm;
 cudaError_t tc_gemm_create(TcGemm **out);
 void tc_gemm_destroy(TcGemm *t);
+// Floats available for split-K partials at GemmDesc::partial (0: never split).
+void tc_gemm_set_splitk_capacity(TcGemm *t, size_t floats);
 // True when the shape, strides and epilogue can run on the tensor-core path.
 bool tc_gemm_supported(const GemmDesc &d);
-// Enqueues the GEMM (and its split-K reduction, if any); adds its kernel count to *launches.
+// Enqueues the GEMM (and its split-K reduction, if any). d.split_k <= 0 lets the launcher
+// choose the split (only for elementwise epilogues); the chosen value is written back.
 cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches);

@@ -46,6 +46,7 @@ extern "C" int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int 
   if (path == GPTK_PATH_TCGEN05) {
     if (!tc_gemm_supported(d)) return GPT_ERR_ALIGN;
     int n = 0;
+    tc_gemm_set_splitk_capacity(tc_instance(), scratch ? scratch_floats : 0);
     e = tc_gemm_launch(tc_instance(), d, st, &n);
   } else if (path == GPTK_PATH_SIMT) {
     e = launch_gemm_simt<bf16>(d, st);

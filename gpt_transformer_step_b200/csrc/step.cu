@@ -172,12 +172,7 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
       d.epi.ntiles = (d.N + TC_CE_TILE - 1) / TC_CE_TILE;
       h->ce_ntiles = d.epi.ntiles;
     }
-    // weight gradients (fp32 out) and any elementwise epilogue whose tile grid leaves SMs
-    // idle split K; the fp32 partials are reduced in a fixed order
-    if (d.split_k == 0) {
-      const long tiles = (long)((d.M + TC_BM - 1) / TC_BM) * ((d.N + TC_BN - 1) / TC_BN);
-      d.split_k = (f32out || (elementwise && tiles < 148)) ? choose_split(h, d.M, d.N, d.K, TC_BM, TC_BN) : 1;
-    }
+    // the launcher picks the CTA group and, for elementwise epilogues, the K split
     d.partial = h->splitk;
     e = tc_gemm_launch(h->tc, d, h->stream, &h->launches);
   } else {
@@ -614,6 +609,8 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
     if (tc_gemm_create(&h->tc) != cudaSuccess) {
       cudaGetLastError();
       h->tc = nullptr;
+    } else {
+      tc_gemm_set_splitk_capacity(h->tc, h->splitk_elems);
     }
   }
   *status = GPT_OK;

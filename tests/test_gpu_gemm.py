@@ -57,6 +57,14 @@ CASES = [
     (333, 700, 192, 1, 1, "resid", 1),
     (333, 700, 192, 1, 0, "dgelu", 1),
     (1024, 2304, 768, 1, 1, "store", 1),
+    # large enough for 256-row tiles on CTA pairs
+    (4096, 2304, 768, 1, 1, "store", 1),
+    (4000, 3000, 520, 1, 0, "store", 1),
+    (4100, 2600, 264, 0, 1, "dgelu", 1),
+    (4096, 4096, 256, 0, 0, "f32_store", 1),
+    (3900, 4000, 640, 1, 1, "store_gelu", 1),
+    (4096, 3072, 512, 1, 1, "resid", 1),
+    (4096, 3000, 1024, 0, 0, "f32_accum", 1),
 ]
 
 
