@@ -219,8 +219,9 @@ struct TcCfg {
   static constexpr int B_ROWS = BN / CG;                 // rows of B each CTA loads
   static constexpr int B_CTA_BYTES = B_ROWS * BK * 2;    // 32 KB / 16 KB
   static constexpr int STAGE = A_BYTES + B_CTA_BYTES;    // 48 KB / 32 KB
-  static constexpr int NSTAGE = CG == 1 ? 4 : 6;
-  static constexpr int SMEM = NSTAGE * STAGE + 1024 + 256;
+  static constexpr int NSTAGE = CG == 1 ? 4 : 5;
+  static constexpr int WARP_STAGE = CG == 1 ? 4096 : 8192;  // epilogue staging per warp
+  static constexpr int SMEM = NSTAGE * STAGE + EPI_WARPS * WARP_STAGE + 1024 + 256;
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -300,15 +301,102 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
     umma_commit(bar);
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   (uint64_t)map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1,
+                                             int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   (uint64_t)map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, const void *src, int c0,
+                                                  int c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          (uint64_t)map),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Epilogue math for one 32-column chunk of one row (everything but the store): v holds the
+// fp32 accumulators on entry and the values to store on exit; v2 the second output (GELU).
+template <int EPI>
+__device__ __forceinline__ void epi_math(const TcParams &P, int row, int col0, float (&v)[32],
+                                         float (&v2)[32]) {
+  const Epi &e = P.epi;
+  if (EPI == TE_CE_DS) {
+    const int grow = e.row_offset + row;
+    const bool ok = row < P.M;
+    const float L = ok ? e.lse[grow] : 0.f;
+    const int t = ok ? e.targets[grow] : -1;
+    const float s = e.sc->inv_M;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = col0 + i;
+      float p = 0.f;
+      if (c < e.V) {
+        p = __expf(v[i] - L);
+        if (c == t) p -= 1.f;
+        p *= s;
+      }
+      v[i] = p;
+    }
+  } else if (EPI == TE_RESID || EPI == TE_DGELU) {
+    float a[32];
+    if (row < P.M && col0 + 32 <= P.N) {
+      ld_bf16x32((const bf16 *)e.aux + (long)row * e.ld_aux + col0, a);
+    } else {
+      const bf16 *aux = (const bf16 *)e.aux + (long)row * e.ld_aux + col0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = (row < P.M && col0 + i < P.N) ? __bfloat162float(aux[i]) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_fast(a[i]);
+  } else if (EPI == TE_STORE_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v2[i] = gelu_fast(v[i]);
+  }
+}
+
+// Writes row `r` (this lane) of a 32x32 chunk into a staging slot laid out for a TMA store:
+// bf16 rows of 64 bytes with the 64-byte swizzle, fp32 rows of 128 bytes with the 128-byte one.
+__device__ __forceinline__ void stage_bf16_row(uint8_t *slot, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 u = make_uint4(pack_bf16(v[8 * c], v[8 * c + 1]), pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                         pack_bf16(v[8 * c + 4], v[8 * c + 5]), pack_bf16(v[8 * c + 6], v[8 * c + 7]));
+    *reinterpret_cast<uint4 *>(slot + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) = u;
+  }
+}
+__device__ __forceinline__ void stage_f32_row(uint8_t *slot, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<float4 *>(slot + r * 128 + ((c ^ (r & 7)) << 4)) =
+        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
 template <int EPI, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                const TcParams P) {
   using Cf = TcCfg<CG>;
   constexpr int NS = Cf::NSTAGE;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t *full_bar = (uint64_t *)(smem + NS * Cf::STAGE);
+  uint8_t *epi_stage = smem + NS * Cf::STAGE;  // EPI_WARPS x WARP_STAGE bytes
+  uint64_t *full_bar = (uint64_t *)(epi_stage + EPI_WARPS * Cf::WARP_STAGE);
   uint64_t *empty_bar = full_bar + NS;
   uint64_t *tfull_bar = empty_bar + NS;
   uint64_t *tempty_bar = tfull_bar + 2;
@@ -443,6 +531,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // 8 warps: warp w reads TMEM lane quarter (w % 4) and columns [half*128, half*128+128)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
+    constexpr int OUT_BYTES = (EPI == TE_F32_STORE || EPI == TE_F32_ACCUM || EPI == TE_PARTIAL) ? 4 : 2;
+    constexpr int SLOT_BYTES = 32 * 32 * OUT_BYTES;
+    constexpr int NOUT = EPI == TE_STORE_GELU ? 2 : 1;
+    constexpr int CHUNK_SLOTS = Cf::WARP_STAGE / (SLOT_BYTES * NOUT) >= 4 ? 4
+                              : Cf::WARP_STAGE / (SLOT_BYTES * NOUT);
+    static_assert(CHUNK_SLOTS >= 1, "epilogue staging too small");
+    uint8_t *wstage = epi_stage + (warp - 2) * Cf::WARP_STAGE;
+    int chunk_seq = 0;
     int i = 0;
     for (int u = unit0; u < P.units; u += ustride, ++i) {
       const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
@@ -453,7 +549,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
       tc_fence_after();
-      const int row = mt * BM * CG + (int)rank * BM + q * 32 + lane;
+      const int row0 = mt * BM * CG + (int)rank * BM + q * 32;  // this warp's 32 rows
+      const int row = row0 + lane;
       const int c0 = half * EPI_COLS;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0);
       float ce_max = -INFINITY, ce_sum = 0.f;
@@ -463,7 +560,34 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (c * 32 >= ncols) break;  // uniform across the warp
         float v[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), v);
-        if (row < P.M) epi_chunk<EPI>(P, row, nt * BN + c0 + c * 32, z, v, ce_max, ce_sum);
+        const int col0 = nt * BN + c0 + c * 32;
+        if (EPI == TE_CE_STATS) {
+          if (row < P.M) epi_chunk<EPI>(P, row, col0, z, v, ce_max, ce_sum);
+          continue;
+        }
+        float v2[32];
+        epi_math<EPI>(P, row, col0, v, v2);
+        // staging slot of this chunk (round robin); wait until its previous store has read it
+        if (lane == 0) {
+          if (CHUNK_SLOTS == 1) bulk_wait_read<0>();
+          else if (CHUNK_SLOTS == 2) bulk_wait_read<1>();
+          else bulk_wait_read<3>();
+        }
+        __syncwarp();
+        uint8_t *slot = wstage + (chunk_seq % CHUNK_SLOTS) * SLOT_BYTES * NOUT;
+        if (OUT_BYTES == 4) stage_f32_row(slot, lane, v);
+        else stage_bf16_row(slot, lane, v);
+        if (NOUT == 2) stage_bf16_row(slot + SLOT_BYTES, lane, v2);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (EPI == TE_PARTIAL) tma_store_3d(&tmO, slot, col0, row0, z);
+          else if (EPI == TE_F32_ACCUM) tma_reduce_add_2d(&tmO, slot, col0, row0);
+          else tma_store_2d(&tmO, slot, col0, row0);
+          if (NOUT == 2) tma_store_2d(&tmO2, slot + SLOT_BYTES, col0, row0);
+          bulk_commit();
+        }
+        ++chunk_seq;
       }
       if (EPI == TE_CE_STATS && row < P.M && ncols > 0) {
         const Epi &e = P.epi;
@@ -478,6 +602,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         else mbar_arrive(&tempty_bar[acc]);
       }
     }
+    if (lane == 0) bulk_wait_all();  // every TMA store of this warp has completed
+    __syncwarp();
   }
   tc_fence_before();
   if (CG == 2) cluster_sync_all(); else __syncthreads();
@@ -527,6 +653,25 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Output tensor map for the TMA-store epilogue: [rows, cols] (plus `depth` planes of
+// `plane` elements for split-K partials), box 32 x 32, bf16 with the 64-byte swizzle or fp32
+// with the 128-byte swizzle.
+bool make_out_map(CUtensorMap *m, const void *base, bool f32, long cols, long rows, long ld,
+                  long depth = 1, long plane = 0) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)depth};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * es, (cuuint64_t)plane * es};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+             depth > 1 ? 3 : 2, (void *)base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld, int box_outer) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -543,8 +688,8 @@ bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld,
 }
 
 template <int EPI, int CG>
-cudaError_t launch_kind(const CUtensorMap &a, const CUtensorMap &b, const TcParams &P, int grid,
-                        cudaStream_t st) {
+cudaError_t launch_kind(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &o,
+                        const CUtensorMap &o2, const TcParams &P, int grid, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI, CG>,
@@ -566,24 +711,27 @@ cudaError_t launch_kind(const CUtensorMap &a, const CUtensorMap &b, const TcPara
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<EPI, CG>, a, b, P);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<EPI, CG>, a, b, o, o2, P);
 }
 
 template <int CG>
 cudaError_t launch_epi(int kind, bool split, const CUtensorMap &ma, const CUtensorMap &mb,
-                       const TcParams &P, int grid, cudaStream_t st) {
-  if (split) return launch_kind<TE_PARTIAL, CG>(ma, mb, P, grid, st);
+                       const CUtensorMap &mo, const CUtensorMap &mo2, const TcParams &P, int grid,
+                       cudaStream_t st) {
+#define TC_L(K) launch_kind<K, CG>(ma, mb, mo, mo2, P, grid, st)
+  if (split) return TC_L(TE_PARTIAL);
   switch (kind) {
-    case EPI_STORE: return launch_kind<TE_STORE, CG>(ma, mb, P, grid, st);
-    case EPI_STORE_GELU: return launch_kind<TE_STORE_GELU, CG>(ma, mb, P, grid, st);
-    case EPI_RESID: return launch_kind<TE_RESID, CG>(ma, mb, P, grid, st);
-    case EPI_DGELU: return launch_kind<TE_DGELU, CG>(ma, mb, P, grid, st);
-    case EPI_F32_STORE: return launch_kind<TE_F32_STORE, CG>(ma, mb, P, grid, st);
-    case EPI_F32_ACCUM: return launch_kind<TE_F32_ACCUM, CG>(ma, mb, P, grid, st);
-    case EPI_CE_STATS: return launch_kind<TE_CE_STATS, CG>(ma, mb, P, grid, st);
-    case EPI_CE_DS: return launch_kind<TE_CE_DS, CG>(ma, mb, P, grid, st);
+    case EPI_STORE: return TC_L(TE_STORE);
+    case EPI_STORE_GELU: return TC_L(TE_STORE_GELU);
+    case EPI_RESID: return TC_L(TE_RESID);
+    case EPI_DGELU: return TC_L(TE_DGELU);
+    case EPI_F32_STORE: return TC_L(TE_F32_STORE);
+    case EPI_F32_ACCUM: return TC_L(TE_F32_ACCUM);
+    case EPI_CE_STATS: return TC_L(TE_CE_STATS);
+    case EPI_CE_DS: return TC_L(TE_CE_DS);
     default: return cudaErrorInvalidValue;
   }
+#undef TC_L
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -674,13 +822,37 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, 64)
                      : make_map(&mb, d.B, d.K, d.N, d.ldb, b_rows));
   if (!ok) return cudaErrorInvalidValue;
+  // output maps of the TMA-store epilogue (rows and columns past M, N are clipped by TMA)
+  CUtensorMap mo, mo2;
+  memset(&mo, 0, sizeof(mo));
+  memset(&mo2, 0, sizeof(mo2));
+  const Epi &e0 = d.epi;
+  if (S > 1) {
+    ok = make_out_map(&mo, d.partial, true, d.N, d.M, d.N, S, (long)d.M * d.N);
+  } else {
+    switch (e0.kind) {
+      case EPI_STORE: case EPI_RESID: case EPI_DGELU: case EPI_CE_DS:
+        ok = make_out_map(&mo, e0.out, false, d.N, d.M, e0.ldo);
+        break;
+      case EPI_STORE_GELU:
+        ok = make_out_map(&mo, e0.out, false, d.N, d.M, e0.ldo) &&
+             make_out_map(&mo2, e0.out2, false, d.N, d.M, e0.ldo2);
+        break;
+      case EPI_F32_STORE: case EPI_F32_ACCUM:
+        ok = make_out_map(&mo, e0.outf, true, d.N, d.M, e0.ldf);
+        break;
+      default:
+        break;
+    }
+  }
+  if (!ok) return cudaErrorInvalidValue;
   cudaError_t e;
   if (CG == 2) {
     const int clusters = P.units < sms / 2 ? P.units : sms / 2;
-    e = launch_epi<2>(d.epi.kind, S > 1, ma, mb, P, 2 * clusters, st);
+    e = launch_epi<2>(d.epi.kind, S > 1, ma, mb, mo, mo2, P, 2 * clusters, st);
   } else {
     const int grid = P.units < sms ? P.units : sms;
-    e = launch_epi<1>(d.epi.kind, S > 1, ma, mb, P, grid, st);
+    e = launch_epi<1>(d.epi.kind, S > 1, ma, mb, mo, mo2, P, grid, st);
   }
   if (e != cudaSuccess) return e;
   if (S > 1) return launch_splitk_reduce<bf16>(d, st);
