@@ -281,12 +281,37 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 }
 
 // ------------------------------------------------------------------------------------------
+// backward kernels: 10 warps. warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..9 "row" warps:
+// warp w owns TMEM lane quarter (w % 4) and column half ch = (w - 2) / 4 (64 of the 128
+// columns of the S / dP tiles), so every row of a tile is shared by two warps. A row warp
+// loads its S and dP columns into registers, releases the accumulators at once (the MMA warp
+// then computes the next tile's S and dP while the row warps do the math), and writes its
+// bf16 results into its 64-column K-block of the smem operand tile.
+// ------------------------------------------------------------------------------------------
+constexpr int BWD_THREADS = 320;
+constexpr int ROW_WARPS = 8;
+
+// 64 consecutive columns (two TMEM loads of 32) of S and dP for this thread's row.
+__device__ __forceinline__ void ld_s_dp64(uint32_t tS, uint32_t tdP, uint32_t (&s0)[32],
+                                          uint32_t (&s1)[32], uint32_t (&d0)[32],
+                                          uint32_t (&d1)[32]) {
+  tmem_ld32_nw(tS, s0);
+  tmem_ld32_nw(tS + 32, s1);
+  tmem_ld32_nw(tdP, d0);
+  tmem_ld32_nw(tdP + 32, d1);
+  tmem_wait_ld32(s0);
+  reg_fence32(s1);
+  reg_fence32(d0);
+  reg_fence32(d1);
+}
+
+// ------------------------------------------------------------------------------------------
 // backward: dQ (+ D)
 // ------------------------------------------------------------------------------------------
-enum { Q_QDO, Q_KV0, Q_KV1, Q_FREE0, Q_FREE1, Q_SDP, Q_DS, Q_MM2, Q_NBAR };
+enum { Q_QDO, Q_KV0, Q_KV1, Q_FREE0, Q_FREE1, Q_SDP, Q_SDPFREE, Q_DS, Q_MM2, Q_NBAR };
 constexpr int DQ_SMEM = 6 * TILE_BYTES + SQ_BYTES + 1024 + 256;
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -308,7 +333,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
   const int n = kt1 - kt0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < Q_NBAR; ++i) mbar_init(&bar[i], i == Q_DS ? 4 : 1);
+    for (int i = 0; i < Q_NBAR; ++i)
+      mbar_init(&bar[i], (i == Q_DS || i == Q_SDPFREE) ? ROW_WARPS : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -348,9 +374,11 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       };
       bool ok = mbar_wait(&bar[Q_QDO], 0, abort_flag, P.err) && issue_sdp(0);
       for (int j = 0; ok && j < n; ++j) {
-        if (!mbar_wait(&bar[Q_DS], j & 1, abort_flag, P.err)) break;
+        if (!mbar_wait(&bar[Q_SDPFREE], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
         if (j + 1 < n && !issue_sdp(j + 1)) break;
+        if (!mbar_wait(&bar[Q_DS], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
         const uint32_t aK = smem_u32(sK0 + (j & 1) * 2 * TILE_BYTES);
         mma_pv(tmem + 256, adS, aK, j > 0);  // dQ += dS K  (K tile as the MN-major operand)
         umma_commit(&bar[Q_MM2]);
@@ -359,8 +387,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, r = q * 32 + lane, qi = q0 + r;
-    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tdP = tS + 128, tdQ = tS + 256;
+    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane, qi = q0 + r;
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     // D_i = dO_i . O_i (written for the dK/dV pass) and the saved lse in the log2 domain
     float D = 0.f, lse2 = 0.f;
     if (qi < P.T) {
@@ -369,9 +397,9 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       const uint4 *gd = reinterpret_cast<const uint4 *>(P.dO + off);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        uint4 a = go[t], c = gd[t];
-        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
-        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&c);
+        uint4 av = go[t], cv = gd[t];
+        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&av);
+        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
@@ -379,7 +407,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         }
       }
       const size_t li = ((size_t)b * P.H + h) * P.T + qi;
-      P.Dbuf[li] = D;
+      if (ch == 0) P.Dbuf[li] = D;
       lse2 = P.lse_in[li] * LOG2E;
     }
     bool ok = true;
@@ -387,38 +415,36 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       const int k0 = (kt0 + j) * TILE;
       if (!warp_wait(&bar[Q_SDP], j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      ld_s_dp64(tS, tdP, s0, s1, d0, d1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[Q_SDPFREE]);  // S / dP may be overwritten now
+      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+      const int hi = qi < P.T ? qi - k0 - ch * 64 : -1;  // admitted local columns: lo..hi
+      const int lo = w >= 0 ? qi - w - k0 - ch * 64 : -1;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float sa = __uint_as_float(i < 32 ? s0[i] : s1[i - 32]);
+        const float sb = __uint_as_float(i < 32 ? s0[i + 1] : s1[i - 31]);
+        const float da = __uint_as_float(i < 32 ? d0[i] : d1[i - 32]);
+        const float db = __uint_as_float(i < 32 ? d0[i + 1] : d1[i - 31]);
+        float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
+        float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
+        if (!interior) {
+          x0 = (i <= hi && i >= lo) ? x0 : 0.f;
+          x1 = (i + 1 <= hi && i + 1 >= lo) ? x1 : 0.f;
+        }
+        pk[i >> 1] = pack_bf16(x0, x1);
+      }
       if (j > 0) {
         if (!warp_wait(&bar[Q_MM2], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
       }
-      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-      const int hi = qi < P.T ? qi - k0 : -1;  // admitted keys: lo <= i <= hi
-      const int lo = w >= 0 ? qi - w - k0 : -1;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32_nw(tS + c * 32, sr);
-        tmem_ld32_nw(tdP + c * 32, dr);
-        tmem_wait_ld32(sr);
-        reg_fence32(dr);
-        uint32_t pk[16];
+      uint8_t *blk = sdS + ch * 16384;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float d0 = ex2(fmaf(__uint_as_float(sr[i]), P.scale_log2, -lse2)) * (__uint_as_float(dr[i]) - D);
-          float d1 = ex2(fmaf(__uint_as_float(sr[i + 1]), P.scale_log2, -lse2)) * (__uint_as_float(dr[i + 1]) - D);
-          if (!interior) {
-            const int ii = c * 32 + i;
-            d0 = (ii <= hi && ii >= lo) ? d0 : 0.f;
-            d1 = (ii + 1 <= hi && ii + 1 >= lo) ? d1 : 0.f;
-          }
-          pk[i >> 1] = pack_bf16(d0, d1);
-        }
-        uint8_t *blk = sdS + (c >> 1) * 16384;
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          st_sw128_chunk(blk, r, (c & 1) * 4 + t,
-                         make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
-      }
+      for (int t = 0; t < 8; ++t)
+        st_sw128_chunk(blk, r, t, make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -426,18 +452,16 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     }
     if (ok && warp_wait(&bar[Q_MM2], (n - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
-      uint32_t pk[32];
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        float v[32];
-        tmem_ld32(tdQ + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * P.scale, v[i + 1] * P.scale);
-      }
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 32, v);  // dQ columns ch*32..
       if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + qi) * 3 * P.C + h * HD);
+        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + qi) * 3 * P.C + h * HD + ch * 32);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        for (int t = 0; t < 4; ++t)
+          dst[t] = make_uint4(pack_bf16(v[8 * t] * P.scale, v[8 * t + 1] * P.scale),
+                              pack_bf16(v[8 * t + 2] * P.scale, v[8 * t + 3] * P.scale),
+                              pack_bf16(v[8 * t + 4] * P.scale, v[8 * t + 5] * P.scale),
+                              pack_bf16(v[8 * t + 6] * P.scale, v[8 * t + 7] * P.scale));
       }
     }
   }
@@ -452,10 +476,10 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // ------------------------------------------------------------------------------------------
 // backward: dK, dV
 // ------------------------------------------------------------------------------------------
-enum { K_KV, K_QDO0, K_QDO1, K_FREE0, K_FREE1, K_SDP, K_PS, K_MM2, K_NBAR };
-constexpr int DKV_SMEM = 6 * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * TILE * 4 + 256;
+enum { K_KV, K_QDO0, K_QDO1, K_FREE0, K_FREE1, K_SDP, K_SDPFREE, K_PS, K_MM2, K_NBAR };
+constexpr int DKV_SMEM = 6 * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __maxnreg__(200)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                 const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -463,8 +487,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   uint8_t *sK = smem, *sV = smem + TILE_BYTES;
   uint8_t *sQ0 = smem + 2 * TILE_BYTES;  // stage s: Q at 2+2s, dO at 3+2s
   uint8_t *sPT = smem + 6 * TILE_BYTES, *sdST = sPT + SQ_BYTES;
-  float *s_lse = (float *)(sdST + SQ_BYTES), *s_D = s_lse + TILE;
-  uint64_t *bar = (uint64_t *)(s_D + TILE);
+  float *s_lsd = (float *)(sdST + SQ_BYTES);  // [2 buffers][lse 128 | D 128]
+  uint64_t *bar = (uint64_t *)(s_lsd + 2 * 2 * TILE);
   uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
 
@@ -477,7 +501,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   const int qt0 = kt, n = qhi / TILE + 1 - qt0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < K_NBAR; ++i) mbar_init(&bar[i], i == K_PS ? 4 : 1);
+    for (int i = 0; i < K_NBAR; ++i)
+      mbar_init(&bar[i], (i == K_PS || i == K_SDPFREE) ? ROW_WARPS : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -517,9 +542,11 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       };
       bool ok = mbar_wait(&bar[K_KV], 0, abort_flag, P.err) && issue_sdp(0);
       for (int j = 0; ok && j < n; ++j) {
-        if (!mbar_wait(&bar[K_PS], j & 1, abort_flag, P.err)) break;
+        if (!mbar_wait(&bar[K_SDPFREE], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
         if (j + 1 < n && !issue_sdp(j + 1)) break;
+        if (!mbar_wait(&bar[K_PS], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
         const uint32_t aQ = smem_u32(sQ0 + (j & 1) * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
         mma_pv(tmem + 256, aPT, adO, j > 0);   // dV += P^T dO
         mma_pv(tmem + 320, adST, aQ, j > 0);   // dK += dS^T Q
@@ -529,61 +556,69 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, r = q * 32 + lane, ki = k0 + r;
-    const int t = threadIdx.x - 64;  // 0..127 among the row warps
-    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tdP = tS + 128;
+    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane, ki = k0 + r;
+    const int t = threadIdx.x - 64;  // 0..255 among the row warps
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int qq0 = (qt0 + j) * TILE;
-      // this query tile's lse (log2 domain) and D, shared by all row threads
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // this query tile's lse (log2 domain) and D, into buffer j & 1; one barrier per tile
+      // (the other buffer may still be read by a warp finishing the previous tile)
+      float *lsd = s_lsd + (j & 1) * 2 * TILE;
       {
-        const int qi = qq0 + t;
+        const int qi = qq0 + (t & 127);
         const size_t li = ((size_t)b * P.H + h) * P.T + qi;
-        s_lse[t] = qi < P.T ? P.lse_in[li] * LOG2E : 0.f;
-        s_D[t] = qi < P.T ? P.Dbuf[li] : 0.f;
+        if (t < 128) lsd[t] = qi < P.T ? P.lse_in[li] * LOG2E : 0.f;
+        else lsd[t] = qi < P.T ? P.Dbuf[li] : 0.f;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      // after an abort every row warp still passes both named barriers of each iteration
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      // after an abort every row warp still passes the named barrier of each tile
       if (ok) ok = warp_wait(&bar[K_SDP], j & 1, abort_flag, P.err);
-      if (ok && j > 0) ok = warp_wait(&bar[K_MM2], (j - 1) & 1, abort_flag, P.err);
       if (!ok) continue;
       tc_fence_after();
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      ld_s_dp64(tS, tdP, s0, s1, d0, d1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[K_SDPFREE]);
       const bool interior = (k0 + TILE - 1 <= qq0) && (w < 0 || k0 >= qq0 + TILE - 1 - w) &&
                             (qq0 + TILE <= P.T);
-      // queries admitted for key ki: ki <= q <= ki + w, q < T  ->  lo <= i <= hi
-      const int lo = ki - qq0;
-      const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32_nw(tS + c * 32, sr);
-        tmem_ld32_nw(tdP + c * 32, dr);
-        tmem_wait_ld32(sr);
-        reg_fence32(dr);
-        uint32_t pp[16], pd[16];
+      // queries admitted for key ki: ki <= q <= ki + w, q < T  ->  local columns lo..hi
+      const int lo = ki - qq0 - ch * 64;
+      const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0 - ch * 64;
+      const float4 *L4 = reinterpret_cast<const float4 *>(lsd + ch * 64);
+      const float4 *D4 = reinterpret_cast<const float4 *>(lsd + TILE + ch * 64);
+      if (j > 0) {  // P^T / dS^T smem is free once the previous tile's dV / dK MMAs are done
+        ok = warp_wait(&bar[K_MM2], (j - 1) & 1, abort_flag, P.err);
+        if (!ok) continue;
+      }
+      const int blk = ch * 16384;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int ii = c * 32 + i;
-          float p0 = ex2(fmaf(__uint_as_float(sr[i]), P.scale_log2, -s_lse[ii]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[i + 1]), P.scale_log2, -s_lse[ii + 1]));
-          if (!interior) {
-            p0 = (ii <= hi && ii >= lo) ? p0 : 0.f;
-            p1 = (ii + 1 <= hi && ii + 1 >= lo) ? p1 : 0.f;
+      for (int u = 0; u < 8; ++u) {  // 8 columns -> one 16-byte chunk of P^T and of dS^T
+        uint32_t pp[4], pd[4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int i = 8 * u + 4 * hh;
+          const float4 L = L4[i >> 2], Dv = D4[i >> 2];
+          const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+          float pr[4], dr[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int ii = i + e;
+            const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
+            const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
+            float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
+            if (!interior) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
+            pr[e] = pv;
+            dr[e] = pv * (dpv - dv[e]);
           }
-          const float d0 = p0 * (__uint_as_float(dr[i]) - s_D[ii]);
-          const float d1 = p1 * (__uint_as_float(dr[i + 1]) - s_D[ii + 1]);
-          pp[i >> 1] = pack_bf16(p0, p1);
-          pd[i >> 1] = pack_bf16(d0, d1);
+          pp[2 * hh] = pack_bf16(pr[0], pr[1]);
+          pp[2 * hh + 1] = pack_bf16(pr[2], pr[3]);
+          pd[2 * hh] = pack_bf16(dr[0], dr[1]);
+          pd[2 * hh + 1] = pack_bf16(dr[2], dr[3]);
         }
-        const int blk = (c >> 1) * 16384;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          st_sw128_chunk(sPT + blk, r, (c & 1) * 4 + u,
-                         make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]));
-          st_sw128_chunk(sdST + blk, r, (c & 1) * 4 + u,
-                         make_uint4(pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]));
-        }
+        st_sw128_chunk(sPT + blk, r, u, make_uint4(pp[0], pp[1], pp[2], pp[3]));
+        st_sw128_chunk(sdST + blk, r, u, make_uint4(pd[0], pd[1], pd[2], pd[3]));
       }
       fence_async_smem();
       tc_fence_before();
@@ -592,23 +627,21 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     }
     if (ok && warp_wait(&bar[K_MM2], (n - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
+      // column half 0 writes dV, half 1 writes dK (times the softmax scale)
+      const float f = ch ? P.scale : 1.f;
+      uint32_t pk[32];
 #pragma unroll 1
-      for (int part = 0; part < 2; ++part) {  // 0: dV, 1: dK (times the softmax scale)
-        const float f = part ? P.scale : 1.f;
-        uint32_t pk[32];
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          tmem_ld32(tS + 256 + part * 64 + c * 32, v);
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 64 + c * 32, v);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * f, v[i + 1] * f);
-        }
-        if (ki < P.T) {
-          const int col = (part ? P.C : 2 * P.C) + h * HD;
-          uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + ki) * 3 * P.C + col);
+        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * f, v[i + 1] * f);
+      }
+      if (ki < P.T) {
+        const int col = (ch ? P.C : 2 * P.C) + h * HD;
+        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + ki) * 3 * P.C + col);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
+        for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
     }
   }
@@ -706,9 +739,9 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
   p.Dbuf = Dbuf;
   p.dqkv = dqkv;
   const int nt = (T + TILE - 1) / TILE;
-  attn_bwd_dq_tc<<<B * H * nt, 192, DQ_SMEM, st>>>(mq, md, p);
+  attn_bwd_dq_tc<<<B * H * nt, BWD_THREADS, DQ_SMEM, st>>>(mq, md, p);
   CUDA_TRY(cudaGetLastError());
-  attn_bwd_dkv_tc<<<B * H * nt, 192, DKV_SMEM, st>>>(mq, md, p);
+  attn_bwd_dkv_tc<<<B * H * nt, BWD_THREADS, DKV_SMEM, st>>>(mq, md, p);
   return cudaGetLastError();
 }
 
