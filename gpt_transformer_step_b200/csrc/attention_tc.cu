@@ -479,7 +479,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 enum { K_KV, K_QDO0, K_QDO1, K_FREE0, K_FREE1, K_SDP, K_SDPFREE, K_PS, K_MM2, K_NBAR };
 constexpr int DKV_SMEM = 6 * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                 const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
