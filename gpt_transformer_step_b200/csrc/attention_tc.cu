@@ -308,8 +308,10 @@ __device__ __forceinline__ void ld_s_dp64(uint32_t tS, uint32_t tdP, uint32_t (&
 // ------------------------------------------------------------------------------------------
 // backward: dQ (+ D)
 // ------------------------------------------------------------------------------------------
-enum { Q_QDO, Q_KV0, Q_KV1, Q_FREE0, Q_FREE1, Q_SDP, Q_SDPFREE, Q_DS, Q_MM2, Q_NBAR };
-constexpr int DQ_SMEM = 6 * TILE_BYTES + SQ_BYTES + 1024 + 256;
+constexpr int DQ_STAGES = 4;  // K/V tiles in flight (the TMA latency spans ~2 tiles)
+enum { Q_QDO, Q_KV0, Q_FREE0 = Q_KV0 + DQ_STAGES, Q_SDP = Q_FREE0 + DQ_STAGES, Q_SDPFREE, Q_DS,
+       Q_MM2, Q_NBAR };
+constexpr int DQ_SMEM = (2 + 2 * DQ_STAGES) * TILE_BYTES + SQ_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
@@ -318,8 +320,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sQ = smem, *sdO = smem + TILE_BYTES;
   uint8_t *sK0 = smem + 2 * TILE_BYTES;  // stage s: K at 2+2s, V at 3+2s
-  uint8_t *sdS = smem + 6 * TILE_BYTES;
-  uint64_t *bar = (uint64_t *)(smem + 6 * TILE_BYTES + SQ_BYTES);
+  uint8_t *sdS = smem + (2 + 2 * DQ_STAGES) * TILE_BYTES;
+  uint64_t *bar = (uint64_t *)(sdS + SQ_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + Q_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
 
@@ -350,8 +352,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       tma_load_2d(sQ, &tmQKV, &bar[Q_QDO], h * HD, row0 + q0);
       tma_load_2d(sdO, &tmDO, &bar[Q_QDO], h * HD, row0 + q0);
       for (int j = 0; j < n; ++j) {
-        const int s = j & 1, k0 = (kt0 + j) * TILE;
-        if (j >= 2 && !mbar_wait(&bar[Q_FREE0 + s], ((j >> 1) - 1) & 1, abort_flag, P.err)) break;
+        const int s = j % DQ_STAGES, use = j / DQ_STAGES, k0 = (kt0 + j) * TILE;
+        if (use > 0 && !mbar_wait(&bar[Q_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
         uint8_t *sK = sK0 + s * 2 * TILE_BYTES;
         mbar_expect_tx(&bar[Q_KV0 + s], 2 * TILE_BYTES);
         tma_load_2d(sK, &tmQKV, &bar[Q_KV0 + s], P.C + h * HD, row0 + k0);
@@ -363,8 +365,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     if (lane == 0) {
       const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), adS = smem_u32(sdS);
       auto issue_sdp = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&bar[Q_KV0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
+        const int s = j % DQ_STAGES;
+        if (!mbar_wait(&bar[Q_KV0 + s], (j / DQ_STAGES) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
         const uint32_t aK = smem_u32(sK0 + s * 2 * TILE_BYTES), aV = aK + TILE_BYTES;
         mma_qk(tmem, aQ, aK, TILE);
@@ -379,10 +381,10 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         if (j + 1 < n && !issue_sdp(j + 1)) break;
         if (!mbar_wait(&bar[Q_DS], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        const uint32_t aK = smem_u32(sK0 + (j & 1) * 2 * TILE_BYTES);
+        const uint32_t aK = smem_u32(sK0 + (j % DQ_STAGES) * 2 * TILE_BYTES);
         mma_pv(tmem + 256, adS, aK, j > 0);  // dQ += dS K  (K tile as the MN-major operand)
         umma_commit(&bar[Q_MM2]);
-        umma_commit(&bar[Q_FREE0 + (j & 1)]);
+        umma_commit(&bar[Q_FREE0 + (j % DQ_STAGES)]);
       }
     }
     __syncwarp();
@@ -476,8 +478,10 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // ------------------------------------------------------------------------------------------
 // backward: dK, dV
 // ------------------------------------------------------------------------------------------
-enum { K_KV, K_QDO0, K_QDO1, K_FREE0, K_FREE1, K_SDP, K_SDPFREE, K_PS, K_MM2, K_NBAR };
-constexpr int DKV_SMEM = 6 * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
+constexpr int DKV_STAGES = 3;  // Q/dO tiles in flight
+enum { K_KV, K_QDO0, K_FREE0 = K_QDO0 + DKV_STAGES, K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE,
+       K_PS, K_MM2, K_NBAR };
+constexpr int DKV_SMEM = (2 + 2 * DKV_STAGES) * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
@@ -486,7 +490,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sK = smem, *sV = smem + TILE_BYTES;
   uint8_t *sQ0 = smem + 2 * TILE_BYTES;  // stage s: Q at 2+2s, dO at 3+2s
-  uint8_t *sPT = smem + 6 * TILE_BYTES, *sdST = sPT + SQ_BYTES;
+  uint8_t *sPT = smem + (2 + 2 * DKV_STAGES) * TILE_BYTES, *sdST = sPT + SQ_BYTES;
   float *s_lsd = (float *)(sdST + SQ_BYTES);  // [2 buffers][lse 128 | D 128]
   uint64_t *bar = (uint64_t *)(s_lsd + 2 * 2 * TILE);
   uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
@@ -518,8 +522,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       tma_load_2d(sK, &tmQKV, &bar[K_KV], P.C + h * HD, row0 + k0);
       tma_load_2d(sV, &tmQKV, &bar[K_KV], 2 * P.C + h * HD, row0 + k0);
       for (int j = 0; j < n; ++j) {
-        const int s = j & 1, qq0 = (qt0 + j) * TILE;
-        if (j >= 2 && !mbar_wait(&bar[K_FREE0 + s], ((j >> 1) - 1) & 1, abort_flag, P.err)) break;
+        const int s = j % DKV_STAGES, use = j / DKV_STAGES, qq0 = (qt0 + j) * TILE;
+        if (use > 0 && !mbar_wait(&bar[K_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
         uint8_t *sQ = sQ0 + s * 2 * TILE_BYTES;
         mbar_expect_tx(&bar[K_QDO0 + s], 2 * TILE_BYTES);
         tma_load_2d(sQ, &tmQKV, &bar[K_QDO0 + s], h * HD, row0 + qq0);
@@ -531,8 +535,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPT = smem_u32(sPT), adST = smem_u32(sdST);
       auto issue_sdp = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&bar[K_QDO0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
+        const int s = j % DKV_STAGES;
+        if (!mbar_wait(&bar[K_QDO0 + s], (j / DKV_STAGES) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
         const uint32_t aQ = smem_u32(sQ0 + s * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
         mma_qk(tmem, aK, aQ, TILE);         // S^T  = K Q^T
@@ -547,11 +551,11 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         if (j + 1 < n && !issue_sdp(j + 1)) break;
         if (!mbar_wait(&bar[K_PS], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ0 + (j & 1) * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
+        const uint32_t aQ = smem_u32(sQ0 + (j % DKV_STAGES) * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
         mma_pv(tmem + 256, aPT, adO, j > 0);   // dV += P^T dO
         mma_pv(tmem + 320, adST, aQ, j > 0);   // dK += dS^T Q
         umma_commit(&bar[K_MM2]);
-        umma_commit(&bar[K_FREE0 + (j & 1)]);
+        umma_commit(&bar[K_FREE0 + (j % DKV_STAGES)]);
       }
     }
     __syncwarp();
