@@ -70,19 +70,22 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 // S[128 x N] (+)= A[:, 0:64] * B^T  with 4 MMAs of K = 16.
 __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t sA, uint32_t sB, int n) {
   const uint32_t id = idesc_bf16(n, 0, 0);
+  const uint64_t a0 = sdesc(sA, 16, 1024), b0 = sdesc(sB, 16, 1024);
 #pragma unroll
   for (int k = 0; k < HD / 16; ++k)
-    umma_bf16(d, sdesc(sA + 32 * k, 16, 1024), sdesc(sB + 32 * k, 16, 1024), id, k > 0 ? 1u : 0u);
+    umma_bf16(d, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), id, k > 0 ? 1u : 0u);  // +32 B
 }
 // O[128 x 64] (+)= P[128 x 128] * V where P is K-major (two 16 KB K-blocks) and V is a
 // 128(k) x 64(n) tile stored with n contiguous (MN-major operand).
 __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t sP, uint32_t sV, bool accumulate) {
   const uint32_t id = idesc_bf16(HD, 0, 1);
+  const uint64_t a0 = sdesc(sP, 16, 1024), b0 = sdesc(sV, 8192, 1024);
 #pragma unroll
   for (int k = 0; k < TILE / 16; ++k) {
-    const uint32_t a = sP + (k >> 2) * 16384 + (k & 3) * 32;
-    const uint32_t b = sV + k * 2048;
-    umma_bf16(d, sdesc(a, 16, 1024), sdesc(b, 8192, 1024), id, (accumulate || k > 0) ? 1u : 0u);
+    const uint32_t ao = (k >> 2) * 16384 + (k & 3) * 32;  // byte offsets of this K step
+    const uint32_t bo = k * 2048;
+    umma_bf16(d, a0 + (uint64_t)(ao >> 4), b0 + (uint64_t)(bo >> 4), id,
+              (accumulate || k > 0) ? 1u : 0u);
   }
 }
 

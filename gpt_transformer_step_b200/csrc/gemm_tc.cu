@@ -511,13 +511,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, P.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sA = smem_u32(smem + stage * Cf::STAGE);
-          const uint32_t sB = sA + A_BYTES;
+          const uint64_t ad0 = sdesc(sA, a_lbo, 1024u), bd0 = sdesc(sA + A_BYTES, b_lbo, 1024u);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = sdesc(sA + k * a_step, a_lbo, 1024u);
-            const uint64_t bd = sdesc(sB + k * b_step, b_lbo, 1024u);
-            umma_issue<CG>(d_tmem, ad, bd, P.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            umma_issue<CG>(d_tmem, ad0 + (uint64_t)((k * a_step) >> 4),
+                           bd0 + (uint64_t)((k * b_step) >> 4), P.idesc,
+                           (kb > kb0 || k > 0) ? 1u : 0u);
           umma_commit_pair<CG>(&empty_bar[stage]);
           if (++stage == NS) { stage = 0; phase ^= 1u; }
         }

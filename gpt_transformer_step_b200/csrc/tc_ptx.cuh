@@ -104,7 +104,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor (sm_100 format, version 1), 128-byte swizzle.
+// Shared-memory matrix descriptor (sm_100 format, version 1), 128-byte swizzle. The start
+// address occupies the low 14 bits (address >> 4; shared addresses are < 256 KB), so a
+// descriptor for a later K step of the same tile is this value plus (byte offset >> 4): one
+// add, no carry into the next field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
