@@ -40,10 +40,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false when the CTA is aborting or the wait exceeded TIMEOUT_NS.
-static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                       unsigned *err) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait: false when the CTA is aborting or the wait exceeded TIMEOUT_NS. The first
+// probe is inlined (a satisfied wait costs a few cycles); only the polling loop is a call.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity,
+                                                   volatile int *abort_flag, unsigned *err) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -56,6 +56,11 @@ static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, vo
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, err);
 }
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
                                             int c0, int c1) {
