@@ -794,7 +794,7 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
     const long tiles = (long)P.num_mt * P.num_nt;
     S = 1;
     if (f32out || (elementwise && tiles * CG < sms))
-      while (tiles * S * CG < 2L * sms && P.total_kblocks / (S * 2) >= 4 &&
+      while (tiles * S * CG < (long)sms && P.total_kblocks / (S * 2) >= 4 &&
              (size_t)S * 2 * d.M * d.N <= t->splitk_capacity && d.partial)
         S *= 2;
   }
