@@ -37,7 +37,6 @@ EXPORTED = [
     "gpt_params_changed", "gpt_set_option", "gpt_kernel_stats", "gpt_last_launch_count",
     "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
     "gptk_attention_bwd_bf16", "gptk_attention_bwd_bf16_noalloc", "gptk_selftest_bounded_wait",
-    "gptk_selftest_exp2_poly",
 ]
 
 
@@ -102,7 +101,6 @@ gptk_attention_bwd_bf16 = _sig("gptk_attention_bwd_bf16", _I, [_P, _P, _P, _P, _
 gptk_attention_bwd_bf16_noalloc = _sig("gptk_attention_bwd_bf16_noalloc", _I,
                                        [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P])
 gptk_selftest_bounded_wait = _sig("gptk_selftest_bounded_wait", _I, [ctypes.c_uint, _P, _P])
-gptk_selftest_exp2_poly = _sig("gptk_selftest_exp2_poly", _I, [_P, _P, _I, _P])
 GPTK_EPI = {"store": 0, "store_gelu": 1, "resid": 2, "dgelu": 3, "f32_store": 4, "f32_accum": 5}
 GPTK_PATH_TCGEN05 = 0
 GPTK_PATH_SIMT = 1

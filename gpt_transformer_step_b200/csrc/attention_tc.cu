@@ -240,7 +240,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const float p0 = ex2(fmaf(sv[c * 32 + i], P.scale_log2, -mu));
-          const float p1 = ex2_poly(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
+          const float p1 = ex2(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
           ls += p0 + p1;
           pk[i >> 1] = pack_bf16(p0, p1);
         }
@@ -436,7 +436,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         const float da = __uint_as_float(i < 32 ? d0[i] : d1[i - 32]);
         const float db = __uint_as_float(i < 32 ? d0[i + 1] : d1[i - 31]);
         float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
-        float x1 = ex2_poly(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
+        float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
         if (!interior) {
           x0 = (i <= hi && i >= lo) ? x0 : 0.f;
           x1 = (i + 1 <= hi && i + 1 >= lo) ? x1 : 0.f;
@@ -614,8 +614,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
             const int ii = i + e;
             const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
             const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
-            const float xa = fmaf(sv, P.scale_log2, -lv[e]);
-            float pv = (e & 1) ? ex2_poly(xa) : ex2(xa);
+            float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
             if (!interior) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
             pr[e] = pv;
             dr[e] = pv * (dpv - dv[e]);

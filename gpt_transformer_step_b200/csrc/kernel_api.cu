@@ -140,16 +140,3 @@ extern "C" int gptk_selftest_bounded_wait(unsigned timeout_us, unsigned *dev_err
   return cudaGetLastError() == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }
 
-namespace {
-__global__ void exp2_selftest_kernel(const float *x, float *y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = tc::ex2_poly(x[i]);
-}
-}  // namespace
-
-extern "C" int gptk_selftest_exp2_poly(const float *x, float *y, int n, void *stream) {
-  if (!x || !y || n < 0) return GPT_ERR_INVALID_ARG;
-  if (n == 0) return GPT_OK;
-  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
-  return cudaGetLastError() == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
-}

@@ -192,21 +192,6 @@ __device__ __forceinline__ void mbar_fence_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// 2^x on the FMA pipe, to share the exponentials of a softmax tile between the MUFU unit and
-// the FMA units: 2^x = 2^floor(x) * q(x - floor(x)), q a degree-3 polynomial fitted to 2^f on
-// [0, 1) by relative-error minimax (Lawson's iteratively reweighted least squares; max
-// relative error 8.3e-5 = 2^-13.5, well below bf16 resolution). 2^floor(x) is added into the
-// exponent field. Inputs below -125 (masked scores are -inf) give exactly 0.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float fl = floorf(xc);
-  const float f = xc - fl;
-  float q = fmaf(0.07808296382427216f, f, 0.22612518072128296f);
-  q = fmaf(q, f, 0.695733368396759f);
-  q = fmaf(q, f, 0.9999415278434753f);
-  const float r = __int_as_float(__float_as_int(q) + ((int)fl << 23));
-  return x < -125.f ? 0.f : r;
-}
 // 2^x with the PTX approximate base-2 exponential instruction.
 __device__ __forceinline__ float ex2(float x) {
   float y;

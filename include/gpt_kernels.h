@@ -63,11 +63,6 @@ int gptk_attention_bwd_bf16(const void *qkv, const void *o, const void *dout, co
  * the CUDA context usable. Does not synchronise. */
 int gptk_selftest_bounded_wait(unsigned timeout_us, unsigned *dev_err, void *stream);
 
-/* Self test of the attention kernels' FMA-pipe exponential: y[i] = 2^x[i] for device fp32
- * arrays of n elements (degree-3 minimax polynomial on the fractional part, exponent add;
- * relative error <= 1e-4; inputs below -125 give 0). Does not synchronise. */
-int gptk_selftest_exp2_poly(const float *x, float *y, int n, void *stream);
-
 /* Attention backward that allocates nothing (no counterpart in the pages: it exists for
  * callers that cannot call cudaMalloc, such as code running inside an allocator hook or a
  * memory pool that must not re-enter the allocator). Same arguments and results as

@@ -122,20 +122,3 @@ def test_bounded_wait_times_out_and_context_survives():
     x = torch.arange(10, device="cuda").sum().item()  # the context still works
     assert x == 45
 
-
-def test_fma_pipe_exp2_against_exp2():
-    """The attention kernels' polynomial 2^x vs torch.exp2 (fp64): relative error <= 1e-4
-    over the range softmax uses; exactly 0 below -125 (masked scores)."""
-    import torch
-    from gpt_transformer_step_b200 import binding as gb
-    x = torch.cat([torch.linspace(-125.0, 8.0, 200001), torch.tensor([-126.0, -1e30, float("-inf"), 0.0, -1.0, 7.999])])
-    xd = x.float().cuda()
-    y = torch.empty_like(xd)
-    assert gb.gptk_selftest_exp2_poly(xd.data_ptr(), y.data_ptr(), xd.numel(),
-                                      torch.cuda.current_stream().cuda_stream) == 0
-    torch.cuda.synchronize()
-    ref = torch.exp2(xd.double())
-    ok = xd >= -125.0
-    rel = ((y.double()[ok] - ref[ok]).abs() / ref[ok]).max().item()
-    assert rel <= 1e-4, rel
-    assert torch.all(y[~ok] == 0)
