@@ -284,25 +284,28 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 }
 
 // ------------------------------------------------------------------------------------------
-// backward kernels: 18 warps. warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..17 "row" warps:
-// warp w owns TMEM lane quarter (w % 4) and column quarter cq = (w - 2) / 4 (32 of the 128
-// columns of the S / dP tiles), so every row of a tile is shared by four warps (enough
-// warps per SM sub-partition to hide the exponential and TMEM latencies). A row warp loads
-// its S and dP columns into registers, releases the accumulators at once (the MMA warp then
-// computes the next tile's S and dP while the row warps do the math), and writes its bf16
-// results into its 32 columns of the smem operand tile.
+// backward kernels: 10 warps. warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..9 "row" warps:
+// warp w owns TMEM lane quarter (w % 4) and column half ch = (w - 2) / 4 (64 of the 128
+// columns of the S / dP tiles), so every row of a tile is shared by two warps. A row warp
+// loads its S and dP columns into registers, releases the accumulators at once (the MMA warp
+// then computes the next tile's S and dP while the row warps do the math), and writes its
+// bf16 results into its 64-column K-block of the smem operand tile.
 // ------------------------------------------------------------------------------------------
-constexpr int ROW_WARPS = 16;                  // 4 per TMEM lane quarter
-constexpr int BWD_THREADS = 64 + 32 * ROW_WARPS;
-constexpr int RW_COLS = TILE / (ROW_WARPS / 4);  // 32 columns per row warp
+constexpr int BWD_THREADS = 320;
+constexpr int ROW_WARPS = 8;
 
-// 32 consecutive columns of S and of dP for this thread's row (two loads, one wait).
-__device__ __forceinline__ void ld_s_dp32(uint32_t tS, uint32_t tdP, uint32_t (&s0)[32],
-                                          uint32_t (&d0)[32]) {
+// 64 consecutive columns (two TMEM loads of 32) of S and dP for this thread's row.
+__device__ __forceinline__ void ld_s_dp64(uint32_t tS, uint32_t tdP, uint32_t (&s0)[32],
+                                          uint32_t (&s1)[32], uint32_t (&d0)[32],
+                                          uint32_t (&d1)[32]) {
   tmem_ld32_nw(tS, s0);
+  tmem_ld32_nw(tS + 32, s1);
   tmem_ld32_nw(tdP, d0);
+  tmem_ld32_nw(tdP + 32, d1);
   tmem_wait_ld32(s0);
+  reg_fence32(s1);
   reg_fence32(d0);
+  reg_fence32(d1);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -389,8 +392,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, cq = (warp - 2) >> 2, r = q * 32 + lane, qi = q0 + r;
-    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + cq * RW_COLS, tdP = tS + 128;
+    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane, qi = q0 + r;
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     // D_i = dO_i . O_i (written for the dK/dV pass) and the saved lse in the log2 domain
     float D = 0.f, lse2 = 0.f;
     if (qi < P.T) {
@@ -409,7 +412,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         }
       }
       const size_t li = ((size_t)b * P.H + h) * P.T + qi;
-      if (cq == 0) P.Dbuf[li] = D;
+      if (ch == 0) P.Dbuf[li] = D;
       lse2 = P.lse_in[li] * LOG2E;
     }
     bool ok = true;
@@ -417,19 +420,23 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       const int k0 = (kt0 + j) * TILE;
       if (!warp_wait(&bar[Q_SDP], j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
-      uint32_t s0[32], d0[32];
-      ld_s_dp32(tS, tdP, s0, d0);
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      ld_s_dp64(tS, tdP, s0, s1, d0, d1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[Q_SDPFREE]);  // S / dP may be overwritten now
       const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-      const int hi = qi < P.T ? qi - k0 - cq * RW_COLS : -1;  // admitted local columns: lo..hi
-      const int lo = w >= 0 ? qi - w - k0 - cq * RW_COLS : -1;
-      uint32_t pk[16];
+      const int hi = qi < P.T ? qi - k0 - ch * 64 : -1;  // admitted local columns: lo..hi
+      const int lo = w >= 0 ? qi - w - k0 - ch * 64 : -1;
+      uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float x0 = ex2(fmaf(__uint_as_float(s0[i]), P.scale_log2, -lse2)) * (__uint_as_float(d0[i]) - D);
-        float x1 = ex2(fmaf(__uint_as_float(s0[i + 1]), P.scale_log2, -lse2)) * (__uint_as_float(d0[i + 1]) - D);
+      for (int i = 0; i < 64; i += 2) {
+        const float sa = __uint_as_float(i < 32 ? s0[i] : s1[i - 32]);
+        const float sb = __uint_as_float(i < 32 ? s0[i + 1] : s1[i - 31]);
+        const float da = __uint_as_float(i < 32 ? d0[i] : d1[i - 32]);
+        const float db = __uint_as_float(i < 32 ? d0[i + 1] : d1[i - 31]);
+        float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
+        float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
         if (!interior) {
           x0 = (i <= hi && i >= lo) ? x0 : 0.f;
           x1 = (i + 1 <= hi && i + 1 >= lo) ? x1 : 0.f;
@@ -439,21 +446,21 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       if (j > 0) {
         if (!warp_wait(&bar[Q_MM2], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
       }
-      uint8_t *blk = sdS + (cq >> 1) * 16384;
+      uint8_t *blk = sdS + ch * 16384;
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
-        st_sw128_chunk(blk, r, (cq & 1) * 4 + t, make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
+      for (int t = 0; t < 8; ++t)
+        st_sw128_chunk(blk, r, t, make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[Q_DS]);
     }
-    if (ok && cq < 2 && warp_wait(&bar[Q_MM2], (n - 1) & 1, abort_flag, P.err)) {
+    if (ok && warp_wait(&bar[Q_MM2], (n - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
       float v[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + cq * 32, v);  // dQ columns cq*32..
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 32, v);  // dQ columns ch*32..
       if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + qi) * 3 * P.C + h * HD + cq * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + qi) * 3 * P.C + h * HD + ch * 32);
 #pragma unroll
         for (int t = 0; t < 4; ++t)
           dst[t] = make_uint4(pack_bf16(v[8 * t] * P.scale, v[8 * t + 1] * P.scale),
@@ -556,45 +563,45 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, cq = (warp - 2) >> 2, r = q * 32 + lane, ki = k0 + r;
-    const int t = threadIdx.x - 64;  // 0..511 among the row warps
-    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + cq * RW_COLS, tdP = tS + 128;
+    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane, ki = k0 + r;
+    const int t = threadIdx.x - 64;  // 0..255 among the row warps
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int qq0 = (qt0 + j) * TILE;
       // this query tile's lse (log2 domain) and D, into buffer j & 1; one barrier per tile
       // (the other buffer may still be read by a warp finishing the previous tile)
       float *lsd = s_lsd + (j & 1) * 2 * TILE;
-      if (t < 2 * TILE) {
-        const int qi = qq0 + (t & (TILE - 1));
+      {
+        const int qi = qq0 + (t & 127);
         const size_t li = ((size_t)b * P.H + h) * P.T + qi;
-        if (t < TILE) lsd[t] = qi < P.T ? P.lse_in[li] * LOG2E : 0.f;
+        if (t < 128) lsd[t] = qi < P.T ? P.lse_in[li] * LOG2E : 0.f;
         else lsd[t] = qi < P.T ? P.Dbuf[li] : 0.f;
       }
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * ROW_WARPS) : "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       // after an abort every row warp still passes the named barrier of each tile
       if (ok) ok = warp_wait(&bar[K_SDP], j & 1, abort_flag, P.err);
       if (!ok) continue;
       tc_fence_after();
-      uint32_t s0[32], d0[32];
-      ld_s_dp32(tS, tdP, s0, d0);
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      ld_s_dp64(tS, tdP, s0, s1, d0, d1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[K_SDPFREE]);
       const bool interior = (k0 + TILE - 1 <= qq0) && (w < 0 || k0 >= qq0 + TILE - 1 - w) &&
                             (qq0 + TILE <= P.T);
       // queries admitted for key ki: ki <= q <= ki + w, q < T  ->  local columns lo..hi
-      const int lo = ki - qq0 - cq * RW_COLS;
-      const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0 - cq * RW_COLS;
-      const float4 *L4 = reinterpret_cast<const float4 *>(lsd + cq * RW_COLS);
-      const float4 *D4 = reinterpret_cast<const float4 *>(lsd + TILE + cq * RW_COLS);
+      const int lo = ki - qq0 - ch * 64;
+      const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0 - ch * 64;
+      const float4 *L4 = reinterpret_cast<const float4 *>(lsd + ch * 64);
+      const float4 *D4 = reinterpret_cast<const float4 *>(lsd + TILE + ch * 64);
       if (j > 0) {  // P^T / dS^T smem is free once the previous tile's dV / dK MMAs are done
         ok = warp_wait(&bar[K_MM2], (j - 1) & 1, abort_flag, P.err);
         if (!ok) continue;
       }
-      uint8_t *pt = sPT + (cq >> 1) * 16384, *dt = sdST + (cq >> 1) * 16384;
+      const int blk = ch * 16384;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // 8 columns -> one 16-byte chunk of P^T and of dS^T
+      for (int u = 0; u < 8; ++u) {  // 8 columns -> one 16-byte chunk of P^T and of dS^T
         uint32_t pp[4], pd[4];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -605,19 +612,20 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int ii = i + e;
-            float pv = ex2(fmaf(__uint_as_float(s0[ii]), P.scale_log2, -lv[e]));
+            const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
+            const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
+            float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
             if (!interior) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
             pr[e] = pv;
-            dr[e] = pv * (__uint_as_float(d0[ii]) - dv[e]);
+            dr[e] = pv * (dpv - dv[e]);
           }
           pp[2 * hh] = pack_bf16(pr[0], pr[1]);
           pp[2 * hh + 1] = pack_bf16(pr[2], pr[3]);
           pd[2 * hh] = pack_bf16(dr[0], dr[1]);
           pd[2 * hh + 1] = pack_bf16(dr[2], dr[3]);
         }
-        const int chunk = (cq & 1) * 4 + u;
-        st_sw128_chunk(pt, r, chunk, make_uint4(pp[0], pp[1], pp[2], pp[3]));
-        st_sw128_chunk(dt, r, chunk, make_uint4(pd[0], pd[1], pd[2], pd[3]));
+        st_sw128_chunk(sPT + blk, r, u, make_uint4(pp[0], pp[1], pp[2], pp[3]));
+        st_sw128_chunk(sdST + blk, r, u, make_uint4(pd[0], pd[1], pd[2], pd[3]));
       }
       fence_async_smem();
       tc_fence_before();
@@ -626,18 +634,21 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     }
     if (ok && warp_wait(&bar[K_MM2], (n - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
-      // column quarters 0, 1 write the two halves of dV, quarters 2, 3 those of dK (times the
-      // softmax scale); TMEM columns 256 + 32 * cq
-      const float f = cq >= 2 ? P.scale : 1.f;
-      float v[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + cq * 32, v);
+      // column half 0 writes dV, half 1 writes dK (times the softmax scale)
+      const float f = ch ? P.scale : 1.f;
+      uint32_t pk[32];
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 64 + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * f, v[i + 1] * f);
+      }
       if (ki < P.T) {
-        const int col = (cq >= 2 ? P.C : 2 * P.C) + h * HD + (cq & 1) * 32;
+        const int col = (ch ? P.C : 2 * P.C) + h * HD;
         uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + ki) * 3 * P.C + col);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          dst[u] = make_uint4(pack_bf16(v[8 * u] * f, v[8 * u + 1] * f), pack_bf16(v[8 * u + 2] * f, v[8 * u + 3] * f),
-                              pack_bf16(v[8 * u + 4] * f, v[8 * u + 5] * f), pack_bf16(v[8 * u + 6] * f, v[8 * u + 7] * f));
+        for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
     }
   }
