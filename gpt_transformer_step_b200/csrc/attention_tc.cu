@@ -27,7 +27,6 @@ using namespace tc;
 constexpr int HD = 64;
 constexpr int TILE = 128;
 constexpr int TILE_BYTES = TILE * HD * 2;  // 16 KB: 128 rows x 64 bf16, K-major SW128
-constexpr int SQ_BYTES = TILE * TILE * 2;  // 32 KB: 128 x 128 bf16 (two 16 KB K-blocks)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -48,10 +47,6 @@ struct AttnParams {
 __host__ __device__ constexpr uint32_t idesc_bf16(int n, int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TILE >> 4) << 24);
-}
-
-__device__ __forceinline__ bool admitted(int i, int j, int w) {
-  return j <= i && (w < 0 || j >= i - w);
 }
 
 // One warp-collective bounded wait: lane 0 polls, the result is broadcast.
@@ -75,33 +70,34 @@ __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t sA, uint32_t sB, int
   for (int k = 0; k < HD / 16; ++k)
     umma_bf16(d, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), id, k > 0 ? 1u : 0u);  // +32 B
 }
-// O[128 x 64] (+)= P[128 x 128] * V where P is K-major (two 16 KB K-blocks) and V is a
-// 128(k) x 64(n) tile stored with n contiguous (MN-major operand).
-__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t sP, uint32_t sV, bool accumulate) {
+// O[128 x 64] (+)= A[128 x 128] * V with A in TMEM (64 columns of packed bf16 pairs, the
+// tcgen05 "A from tensor memory" form) and V the 128(k) x 64(n) MN-major smem tile.
+__device__ __forceinline__ void mma_pv_ts(uint32_t d, uint32_t a_tmem, uint32_t sV, bool accumulate) {
   const uint32_t id = idesc_bf16(HD, 0, 1);
-  const uint64_t a0 = sdesc(sP, 16, 1024), b0 = sdesc(sV, 8192, 1024);
+  const uint64_t b0 = sdesc(sV, 8192, 1024);
 #pragma unroll
-  for (int k = 0; k < TILE / 16; ++k) {
-    const uint32_t ao = (k >> 2) * 16384 + (k & 3) * 32;  // byte offsets of this K step
-    const uint32_t bo = k * 2048;
-    umma_bf16(d, a0 + (uint64_t)(ao >> 4), b0 + (uint64_t)(bo >> 4), id,
-              (accumulate || k > 0) ? 1u : 0u);
-  }
+  for (int k = 0; k < TILE / 16; ++k)  // K = 16 per MMA: 8 TMEM columns of A, 16 rows of V
+    umma_bf16_ts(d, a_tmem + 8 * k, b0 + (uint64_t)((k * 2048) >> 4), id,
+                 (accumulate || k > 0) ? 1u : 0u);
+}
+
+// Packs 32 fp32 values into 16 bf16 pairs and stores them to 16 TMEM columns.
+__device__ __forceinline__ void st_tmem_bf16x32(uint32_t taddr, const uint32_t (&pk)[16]) {
+  tmem_st16_nw(taddr, pk);
 }
 
 // ------------------------------------------------------------------------------------------
 // forward
 // ------------------------------------------------------------------------------------------
 enum { F_QFULL, F_KFULL, F_VFULL, F_KFREE, F_VFREE, F_SFULL, F_PFULL, F_OFULL, F_NBAR };
-constexpr int FWD_SMEM = 3 * TILE_BYTES + SQ_BYTES + 1024 + 256;
+constexpr int FWD_SMEM = 3 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sQ = smem, *sK = smem + TILE_BYTES, *sV = smem + 2 * TILE_BYTES;
-  uint8_t *sP = smem + 3 * TILE_BYTES;
-  uint64_t *bar = (uint64_t *)(smem + 3 * TILE_BYTES + SQ_BYTES);
+  uint64_t *bar = (uint64_t *)(smem + 3 * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + F_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
 
@@ -123,7 +119,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;  // S: columns [0,128), O: [128,192)
+  const uint32_t tmem = *tmem_holder;  // S: columns [0,128), O: [128,192), P (bf16): [192,256)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -142,7 +138,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) &&
                 mbar_wait(&bar[F_KFULL], 0, abort_flag, P.err);
       if (ok) {
@@ -163,7 +159,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
         }
         if (!mbar_wait(&bar[F_VFULL], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        mma_pv(tmem + 128, aP, aV, j > 0);
+        mma_pv_ts(tmem + 128, tmem + 192, aV, j > 0);
         umma_commit(&bar[F_OFULL]);
         umma_commit(&bar[F_VFREE]);
       }
@@ -171,7 +167,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
     __syncwarp();
   } else {
     const int q = warp & 3, r = q * 32 + lane, qi = q0 + r;
-    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tO = tS + 128;
+    const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tO = tS + 128, tP = tS + 192;
     float m2 = -INFINITY, l = 0.f;
     bool have = false, ok = true;
     for (int j = 0; j < n; ++j) {
@@ -244,14 +240,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
           ls += p0 + p1;
           pk[i >> 1] = pack_bf16(p0, p1);
         }
-        uint8_t *blk = sP + (c >> 1) * 16384;
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          st_sw128_chunk(blk, r, (c & 1) * 4 + t,
-                         make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
+        st_tmem_bf16x32(tP + c * 16, pk);
       }
       l += ls;
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[F_PFULL]);
@@ -314,7 +306,7 @@ __device__ __forceinline__ void ld_s_dp64(uint32_t tS, uint32_t tdP, uint32_t (&
 constexpr int DQ_STAGES = 4;  // K/V tiles in flight (the TMA latency spans ~2 tiles)
 enum { Q_QDO, Q_KV0, Q_FREE0 = Q_KV0 + DQ_STAGES, Q_SDP = Q_FREE0 + DQ_STAGES, Q_SDPFREE, Q_DS,
        Q_MM2, Q_NBAR };
-constexpr int DQ_SMEM = (2 + 2 * DQ_STAGES) * TILE_BYTES + SQ_BYTES + 1024 + 256;
+constexpr int DQ_SMEM = (2 + 2 * DQ_STAGES) * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
@@ -323,8 +315,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sQ = smem, *sdO = smem + TILE_BYTES;
   uint8_t *sK0 = smem + 2 * TILE_BYTES;  // stage s: K at 2+2s, V at 3+2s
-  uint8_t *sdS = smem + (2 + 2 * DQ_STAGES) * TILE_BYTES;
-  uint64_t *bar = (uint64_t *)(sdS + SQ_BYTES);
+  uint64_t *bar = (uint64_t *)(smem + (2 + 2 * DQ_STAGES) * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + Q_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
 
@@ -347,7 +338,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;  // S [0,128), dP [128,256), dQ [256,320)
+  const uint32_t tmem = *tmem_holder;  // S [0,128), dP [128,256), dQ [256,320), dS [320,384)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -366,7 +357,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), adS = smem_u32(sdS);
+      const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO);
       auto issue_sdp = [&](int j) -> bool {
         const int s = j % DQ_STAGES;
         if (!mbar_wait(&bar[Q_KV0 + s], (j / DQ_STAGES) & 1, abort_flag, P.err)) return false;
@@ -385,7 +376,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         if (!mbar_wait(&bar[Q_DS], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
         const uint32_t aK = smem_u32(sK0 + (j % DQ_STAGES) * 2 * TILE_BYTES);
-        mma_pv(tmem + 256, adS, aK, j > 0);  // dQ += dS K  (K tile as the MN-major operand)
+        mma_pv_ts(tmem + 256, tmem + 320, aK, j > 0);  // dQ += dS K (dS in TMEM, K tile MN-major)
         umma_commit(&bar[Q_MM2]);
         umma_commit(&bar[Q_FREE0 + (j % DQ_STAGES)]);
       }
@@ -446,11 +437,15 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       if (j > 0) {
         if (!warp_wait(&bar[Q_MM2], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
       }
-      uint8_t *blk = sdS + ch * 16384;
+      {
+        const uint32_t tdS = tmem + ((uint32_t)(q * 32) << 16) + 320 + ch * 32;
+        uint32_t lo16[16], hi16[16];
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
-        st_sw128_chunk(blk, r, t, make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]));
-      fence_async_smem();
+        for (int t = 0; t < 16; ++t) { lo16[t] = pk[t]; hi16[t] = pk[16 + t]; }
+        tmem_st16_nw(tdS, lo16);
+        tmem_st16_nw(tdS + 16, hi16);
+        tmem_wait_st();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[Q_DS]);
@@ -481,10 +476,10 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // ------------------------------------------------------------------------------------------
 // backward: dK, dV
 // ------------------------------------------------------------------------------------------
-constexpr int DKV_STAGES = 3;  // Q/dO tiles in flight
+constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight
 enum { K_KV, K_QDO0, K_FREE0 = K_QDO0 + DKV_STAGES, K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE,
        K_PS, K_MM2, K_NBAR };
-constexpr int DKV_SMEM = (2 + 2 * DKV_STAGES) * TILE_BYTES + 2 * SQ_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
+constexpr int DKV_SMEM = (2 + 2 * DKV_STAGES) * TILE_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
@@ -493,8 +488,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sK = smem, *sV = smem + TILE_BYTES;
   uint8_t *sQ0 = smem + 2 * TILE_BYTES;  // stage s: Q at 2+2s, dO at 3+2s
-  uint8_t *sPT = smem + (2 + 2 * DKV_STAGES) * TILE_BYTES, *sdST = sPT + SQ_BYTES;
-  float *s_lsd = (float *)(sdST + SQ_BYTES);  // [2 buffers][lse 128 | D 128]
+  float *s_lsd = (float *)(smem + (2 + 2 * DKV_STAGES) * TILE_BYTES);  // [2][lse 128 | D 128]
   uint64_t *bar = (uint64_t *)(s_lsd + 2 * 2 * TILE);
   uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
@@ -517,7 +511,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;  // S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384)
+  // S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384), P^T [384,448), dS^T [448,512)
+  const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -536,7 +531,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPT = smem_u32(sPT), adST = smem_u32(sdST);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
       auto issue_sdp = [&](int j) -> bool {
         const int s = j % DKV_STAGES;
         if (!mbar_wait(&bar[K_QDO0 + s], (j / DKV_STAGES) & 1, abort_flag, P.err)) return false;
@@ -555,8 +550,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         if (!mbar_wait(&bar[K_PS], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
         const uint32_t aQ = smem_u32(sQ0 + (j % DKV_STAGES) * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
-        mma_pv(tmem + 256, aPT, adO, j > 0);   // dV += P^T dO
-        mma_pv(tmem + 320, adST, aQ, j > 0);   // dK += dS^T Q
+        mma_pv_ts(tmem + 256, tmem + 384, adO, j > 0);  // dV += P^T dO   (P^T in TMEM)
+        mma_pv_ts(tmem + 320, tmem + 448, aQ, j > 0);   // dK += dS^T Q  (dS^T in TMEM)
         umma_commit(&bar[K_MM2]);
         umma_commit(&bar[K_FREE0 + (j % DKV_STAGES)]);
       }
@@ -599,35 +594,39 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         ok = warp_wait(&bar[K_MM2], (j - 1) & 1, abort_flag, P.err);
         if (!ok) continue;
       }
-      const int blk = ch * 16384;
+      const uint32_t tPT = tmem + ((uint32_t)(q * 32) << 16) + 384 + ch * 32, tdST = tPT + 64;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // 8 columns -> one 16-byte chunk of P^T and of dS^T
-        uint32_t pp[4], pd[4];
+      for (int half = 0; half < 2; ++half) {  // 32 columns -> 16 packed TMEM columns each
+        uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int i = 8 * u + 4 * hh;
-          const float4 L = L4[i >> 2], Dv = D4[i >> 2];
-          const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
-          float pr[4], dr[4];
+        for (int u = 0; u < 4; ++u) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int ii = i + e;
-            const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
-            const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
-            float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
-            if (!interior) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
-            pr[e] = pv;
-            dr[e] = pv * (dpv - dv[e]);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int i = 32 * half + 8 * u + 4 * hh;
+            const float4 L = L4[i >> 2], Dv = D4[i >> 2];
+            const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+            float pr[4], dr[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int ii = i + e;
+              const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
+              const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
+              float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
+              if (!interior) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
+              pr[e] = pv;
+              dr[e] = pv * (dpv - dv[e]);
+            }
+            const int o = 4 * u + 2 * hh;
+            pp[o] = pack_bf16(pr[0], pr[1]);
+            pp[o + 1] = pack_bf16(pr[2], pr[3]);
+            pd[o] = pack_bf16(dr[0], dr[1]);
+            pd[o + 1] = pack_bf16(dr[2], dr[3]);
           }
-          pp[2 * hh] = pack_bf16(pr[0], pr[1]);
-          pp[2 * hh + 1] = pack_bf16(pr[2], pr[3]);
-          pd[2 * hh] = pack_bf16(dr[0], dr[1]);
-          pd[2 * hh + 1] = pack_bf16(dr[2], dr[3]);
         }
-        st_sw128_chunk(sPT + blk, r, u, make_uint4(pp[0], pp[1], pp[2], pp[3]));
-        st_sw128_chunk(sdST + blk, r, u, make_uint4(pd[0], pd[1], pd[2], pd[3]));
+        tmem_st16_nw(tPT + 16 * half, pp);
+        tmem_st16_nw(tdST + 16 * half, pd);
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[K_PS]);
