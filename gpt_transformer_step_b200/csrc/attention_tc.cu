@@ -89,15 +89,17 @@ __device__ __forceinline__ void st_tmem_bf16x32(uint32_t taddr, const uint32_t (
 // ------------------------------------------------------------------------------------------
 // forward
 // ------------------------------------------------------------------------------------------
-enum { F_QFULL, F_KFULL, F_VFULL, F_KFREE, F_VFREE, F_SFULL, F_PFULL, F_OFULL, F_NBAR };
-constexpr int FWD_SMEM = 3 * TILE_BYTES + 1024 + 256;
+// K/V tiles in two stages; the softmax warps release S as soon as it is in registers, so the
+// next tile's S = Q K^T runs on the tensor core while they compute P.
+enum { F_QFULL, F_KV0, F_KV1, F_FREE0, F_FREE1, F_SFULL, F_SFREE, F_PFULL, F_OFULL, F_NBAR };
+constexpr int FWD_SMEM = 5 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ = smem, *sK = smem + TILE_BYTES, *sV = smem + 2 * TILE_BYTES;
-  uint64_t *bar = (uint64_t *)(smem + 3 * TILE_BYTES);
+  uint8_t *sQ = smem, *sKV0 = smem + TILE_BYTES;  // stage s: K at 1+2s, V at 2+2s
+  uint64_t *bar = (uint64_t *)(smem + 5 * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + F_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
 
@@ -111,7 +113,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   const int n = kt1 - kt0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < F_NBAR; ++i) mbar_init(&bar[i], i == F_PFULL ? 4 : 1);
+    for (int i = 0; i < F_NBAR; ++i) mbar_init(&bar[i], (i == F_PFULL || i == F_SFREE) ? 4 : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -126,42 +128,36 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
       mbar_expect_tx(&bar[F_QFULL], TILE_BYTES);
       tma_load_2d(sQ, &tmQKV, &bar[F_QFULL], h * HD, row0 + q0);
       for (int j = 0; j < n; ++j) {
-        const int k0 = (kt0 + j) * TILE;
-        if (j > 0 && !mbar_wait(&bar[F_KFREE], (j - 1) & 1, abort_flag, P.err)) break;
-        mbar_expect_tx(&bar[F_KFULL], TILE_BYTES);
-        tma_load_2d(sK, &tmQKV, &bar[F_KFULL], P.C + h * HD, row0 + k0);
-        if (j > 0 && !mbar_wait(&bar[F_VFREE], (j - 1) & 1, abort_flag, P.err)) break;
-        mbar_expect_tx(&bar[F_VFULL], TILE_BYTES);
-        tma_load_2d(sV, &tmQKV, &bar[F_VFULL], 2 * P.C + h * HD, row0 + k0);
+        const int s = j & 1, k0 = (kt0 + j) * TILE;
+        if (j >= 2 && !mbar_wait(&bar[F_FREE0 + s], ((j >> 1) - 1) & 1, abort_flag, P.err)) break;
+        uint8_t *sK = sKV0 + s * 2 * TILE_BYTES;
+        mbar_expect_tx(&bar[F_KV0 + s], 2 * TILE_BYTES);
+        tma_load_2d(sK, &tmQKV, &bar[F_KV0 + s], P.C + h * HD, row0 + k0);
+        tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[F_KV0 + s], 2 * P.C + h * HD, row0 + k0);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) &&
-                mbar_wait(&bar[F_KFULL], 0, abort_flag, P.err);
-      if (ok) {
+      const uint32_t aQ = smem_u32(sQ), aKV0 = smem_u32(sKV0);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&bar[F_KV0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        mma_qk(tmem, aQ, aK, TILE);
+        mma_qk(tmem, aQ, aKV0 + s * 2 * TILE_BYTES, TILE);
         umma_commit(&bar[F_SFULL]);
-        umma_commit(&bar[F_KFREE]);
-      }
+        return true;
+      };
+      bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) && issue_s(0);
       for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait(&bar[F_SFREE], j & 1, abort_flag, P.err)) break;  // S_j is in registers
+        tc_fence_after();
+        if (j + 1 < n && !issue_s(j + 1)) break;
         if (!mbar_wait(&bar[F_PFULL], j & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        if (j + 1 < n) {
-          if (!mbar_wait(&bar[F_KFULL], (j + 1) & 1, abort_flag, P.err)) break;
-          tc_fence_after();
-          mma_qk(tmem, aQ, aK, TILE);
-          umma_commit(&bar[F_SFULL]);
-          umma_commit(&bar[F_KFREE]);
-        }
-        if (!mbar_wait(&bar[F_VFULL], j & 1, abort_flag, P.err)) break;
-        tc_fence_after();
-        mma_pv_ts(tmem + 128, tmem + 192, aV, j > 0);
+        mma_pv_ts(tmem + 128, tmem + 192, aKV0 + (j & 1) * 2 * TILE_BYTES + TILE_BYTES, j > 0);
         umma_commit(&bar[F_OFULL]);
-        umma_commit(&bar[F_VFREE]);
+        umma_commit(&bar[F_FREE0 + (j & 1)]);  // K_j and V_j are no longer read
       }
     }
     __syncwarp();
@@ -184,6 +180,9 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
       reg_fence32(s1);
       reg_fence32(s2);
       reg_fence32(s3);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
       float sv[128];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
