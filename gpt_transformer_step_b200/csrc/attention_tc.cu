@@ -89,16 +89,18 @@ __device__ __forceinline__ void st_tmem_bf16x32(uint32_t taddr, const uint32_t (
 // ------------------------------------------------------------------------------------------
 // forward
 // ------------------------------------------------------------------------------------------
-// K/V tiles in two stages; the softmax warps release S as soon as it is in registers, so the
+// K and V tiles in separate two-stage rings (a K stage frees as soon as its S MMA is done, a V
+// stage after its P.V MMA); the softmax warps release S as soon as it is in registers, so the
 // next tile's S = Q K^T runs on the tensor core while they compute P.
-enum { F_QFULL, F_KV0, F_KV1, F_FREE0, F_FREE1, F_SFULL, F_SFREE, F_PFULL, F_OFULL, F_NBAR };
+enum { F_QFULL, F_K0, F_K1, F_V0, F_V1, F_KFREE0, F_KFREE1, F_VFREE0, F_VFREE1, F_SFULL, F_SFREE,
+       F_PFULL, F_OFULL, F_NBAR };
 constexpr int FWD_SMEM = 5 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ = smem, *sKV0 = smem + TILE_BYTES;  // stage s: K at 1+2s, V at 2+2s
+  uint8_t *sQ = smem, *sK0 = smem + TILE_BYTES, *sV0 = smem + 3 * TILE_BYTES;  // 2 stages each
   uint64_t *bar = (uint64_t *)(smem + 5 * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + F_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
@@ -128,24 +130,26 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
       mbar_expect_tx(&bar[F_QFULL], TILE_BYTES);
       tma_load_2d(sQ, &tmQKV, &bar[F_QFULL], h * HD, row0 + q0);
       for (int j = 0; j < n; ++j) {
-        const int s = j & 1, k0 = (kt0 + j) * TILE;
-        if (j >= 2 && !mbar_wait(&bar[F_FREE0 + s], ((j >> 1) - 1) & 1, abort_flag, P.err)) break;
-        uint8_t *sK = sKV0 + s * 2 * TILE_BYTES;
-        mbar_expect_tx(&bar[F_KV0 + s], 2 * TILE_BYTES);
-        tma_load_2d(sK, &tmQKV, &bar[F_KV0 + s], P.C + h * HD, row0 + k0);
-        tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[F_KV0 + s], 2 * P.C + h * HD, row0 + k0);
+        const int s = j & 1, use = j >> 1, k0 = (kt0 + j) * TILE;
+        if (use > 0 && !mbar_wait(&bar[F_KFREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
+        mbar_expect_tx(&bar[F_K0 + s], TILE_BYTES);
+        tma_load_2d(sK0 + s * TILE_BYTES, &tmQKV, &bar[F_K0 + s], P.C + h * HD, row0 + k0);
+        if (use > 0 && !mbar_wait(&bar[F_VFREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
+        mbar_expect_tx(&bar[F_V0 + s], TILE_BYTES);
+        tma_load_2d(sV0 + s * TILE_BYTES, &tmQKV, &bar[F_V0 + s], 2 * P.C + h * HD, row0 + k0);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aKV0 = smem_u32(sKV0);
+      const uint32_t aQ = smem_u32(sQ), aK0 = smem_u32(sK0), aV0 = smem_u32(sV0);
       auto issue_s = [&](int j) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(&bar[F_KV0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
+        if (!mbar_wait(&bar[F_K0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        mma_qk(tmem, aQ, aKV0 + s * 2 * TILE_BYTES, TILE);
+        mma_qk(tmem, aQ, aK0 + s * TILE_BYTES, TILE);
         umma_commit(&bar[F_SFULL]);
+        umma_commit(&bar[F_KFREE0 + s]);  // K_j is no longer read
         return true;
       };
       bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) && issue_s(0);
@@ -154,10 +158,11 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
         tc_fence_after();
         if (j + 1 < n && !issue_s(j + 1)) break;
         if (!mbar_wait(&bar[F_PFULL], j & 1, abort_flag, P.err)) break;
+        if (!mbar_wait(&bar[F_V0 + (j & 1)], (j >> 1) & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        mma_pv_ts(tmem + 128, tmem + 192, aKV0 + (j & 1) * 2 * TILE_BYTES + TILE_BYTES, j > 0);
+        mma_pv_ts(tmem + 128, tmem + 192, aV0 + (j & 1) * TILE_BYTES, j > 0);
         umma_commit(&bar[F_OFULL]);
-        umma_commit(&bar[F_FREE0 + (j & 1)]);  // K_j and V_j are no longer read
+        umma_commit(&bar[F_VFREE0 + (j & 1)]);  // V_j is no longer read
       }
     }
     __syncwarp();
