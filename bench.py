@@ -28,6 +28,11 @@ NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+
+# DRAM bytes (read + write) per tcgen05 GEMM launch, mean over all GEMM launches of the step,
+# from the ncu launch list in profiles/step_gpt2_124m_launch_list.md (same kernel version).
+GEMM_DRAM_BYTES_PER_LAUNCH = {"gpt2_124m_bf16": 204.06e6}
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -244,7 +249,10 @@ def run_ours(args, wl, rank, world, local_rank):
                 "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 128},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMMs (all launches, flop-weighted)",
                      "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": (achieved / peak_t) if achieved else None, "traffic": None,
+                     "frac": (achieved / peak_t) if achieved else None,
+                     "traffic": GEMM_DRAM_BYTES_PER_LAUNCH.get(wl.name),
+                     "traffic_unit": "bytes per GEMM launch (ncu dram__bytes_read.sum + "
+                                     "dram__bytes_write.sum, mean over one step's launches)",
                      "peak_kind": f"{pk_kind} sustained bf16", "launches_timed": n_l,
                      "gemm_ms_per_step": gemm_ms / max(1, max(2, args.steps // 4))},
         "clocks": clocks,

@@ -780,23 +780,32 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   TcParams P;
   memset(&P, 0, sizeof(P));
   const int sms = num_sms();
-  // CTA pairs (256-row tiles) whenever they fill the machine; single CTAs otherwise
+  // CTA pairs (256-row tiles) whenever they fill the machine, directly or with a K split of
+  // at most 16 (weight gradients: small output, long K); single CTAs otherwise
   const int nt = (d.N + BN - 1) / BN;
-  const int CG = ((long)((d.M + 2 * BM - 1) / (2 * BM)) * nt >= sms / 2) ? 2 : 1;
+  const long kblocks = (d.K + BK - 1) / BK;
+  const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
+  const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
+  const bool can_split = d.split_k <= 0 && (f32out || elementwise) && d.partial;
+  auto split_for = [&](long tiles, int cg) {
+    int s = 1;
+    while (tiles * s * cg < (long)sms && kblocks / (s * 2) >= 4 && s < 16 &&
+           (size_t)s * 2 * d.M * d.N <= t->splitk_capacity)
+      s *= 2;
+    return s;
+  };
+  const long tiles2 = (long)((d.M + 2 * BM - 1) / (2 * BM)) * nt;
+  int CG = 1;
+  if (tiles2 * 2 >= sms) CG = 2;
+  else if (can_split && tiles2 * 2 * split_for(tiles2, 2) >= sms) CG = 2;
   P.M = d.M; P.N = d.N; P.K = d.K;
   P.num_mt = (d.M + BM * CG - 1) / (BM * CG);
   P.num_nt = nt;
-  P.total_kblocks = (d.K + BK - 1) / BK;
+  P.total_kblocks = (int)kblocks;
   int S = d.split_k;
   if (S <= 0) {  // automatic: split K while the tile grid leaves SMs idle
-    const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
-    const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
     const long tiles = (long)P.num_mt * P.num_nt;
-    S = 1;
-    if (f32out || (elementwise && tiles * CG < sms))
-      while (tiles * S * CG < (long)sms && P.total_kblocks / (S * 2) >= 4 &&
-             (size_t)S * 2 * d.M * d.N <= t->splitk_capacity && d.partial)
-        S *= 2;
+    S = (f32out || (elementwise && tiles * CG < sms)) && d.partial ? split_for(tiles, CG) : 1;
   }
   if (S > P.total_kblocks) S = P.total_kblocks;
   P.kblocks_per_split = (P.total_kblocks + S - 1) / S;

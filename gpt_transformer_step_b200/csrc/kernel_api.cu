@@ -26,7 +26,7 @@ extern "C" int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int 
   if ((epi == GPTK_EPI_STORE_GELU && !out2) ||
       ((epi == GPTK_EPI_RESID || epi == GPTK_EPI_DGELU) && !aux))
     return GPT_ERR_INVALID_ARG;
-  if (split_k < 1) split_k = 1;
+  if (split_k < 0 || (split_k == 0 && path != GPTK_PATH_TCGEN05)) split_k = 1;
   if (split_k > 1 && (!f32 || !scratch || scratch_floats < (size_t)split_k * M * N))
     return GPT_ERR_INVALID_ARG;
   GemmDesc d;

@@ -16,7 +16,7 @@ import json
 B, T, C, H = 16, 1024, 768, 12
 M = B * T
 
-# name: (M, N, K, a_kmajor, b_kmajor, epilogue, split)
+# name: (M, N, K, a_kmajor, b_kmajor, epilogue, split); split 0 = the launcher's choice
 GEMMS = {
     "gemm_qkv": (M, 3 * C, C, 1, 1, "store", 1),
     "gemm_attnproj": (M, C, C, 1, 1, "resid", 1),
@@ -24,8 +24,10 @@ GEMMS = {
     "gemm_mlpproj": (M, C, 4 * C, 1, 1, "resid", 1),
     "gemm_dgrad_mlpproj": (M, 4 * C, C, 1, 0, "dgelu", 1),
     "gemm_dgrad_fc": (M, C, 4 * C, 1, 0, "store", 1),
-    "gemm_wgrad_fc": (4 * C, C, M, 0, 0, "f32_store", 2),
-    "gemm_wgrad_qkv": (3 * C, C, M, 0, 0, "f32_store", 2),
+    "gemm_wgrad_fc": (4 * C, C, M, 0, 0, "f32_store", 0),
+    "gemm_wgrad_qkv": (3 * C, C, M, 0, 0, "f32_store", 0),
+    "gemm_wgrad_attnproj": (C, C, M, 0, 0, "f32_store", 0),
+    "gemm_wgrad_mlpproj": (C, 4 * C, M, 0, 0, "f32_store", 0),
     "gemm_lmhead": (M, 50304, C, 1, 1, "store", 1),
 }
 ATTN = ("attn_fwd", "attn_bwd")
@@ -67,7 +69,8 @@ def main():
                 out2 = torch.empty(m * n if epi == "store_gelu" else 1, dtype=torch.bfloat16, device=dev)
                 aux = torch.randn(m * n if epi in ("resid", "dgelu") else 1, device=dev).to(torch.bfloat16)
                 outf = torch.empty(m * n if f32 else 1, device=dev)
-                scratch = torch.empty(max(1, split * m * n) if split > 1 else 1, device=dev)
+                scratch = torch.empty(16 * m * n if split == 0 else (split * m * n if split > 1 else 1),
+                                      device=dev)
 
                 def run():
                     rc = gb.gptk_gemm_bf16(m, n, k, A.data_ptr(), lda, ak, Bm.data_ptr(), ldb, bk,

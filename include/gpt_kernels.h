@@ -17,6 +17,8 @@
  *   GPTK_EPI_F32_ACCUM  outf[m*ldf+n] += acc
  * split_k > 1 splits K into split_k ranges whose fp32 partials are summed in a fixed order
  * (only for the two F32 epilogues; needs scratch of split_k*M*N floats, caller-owned).
+ * split_k = 0 on the tensor-core path lets the launcher choose the CTA group and a split of at
+ * most 16 that fits in scratch_floats (no split without scratch); on the SIMT path 0 means 1.
  * path: GPTK_PATH_TCGEN05 (tensor cores; needs lda, ldb, ldo... multiples of 8 elements and
  * 16-byte aligned pointers, else GPT_ERR_ALIGN) or GPTK_PATH_SIMT (CUDA cores, any layout).
  * dev_err: device unsigned word that receives GPT_DEVERR bits (bounded-wait timeout = 2).

@@ -65,6 +65,11 @@ CASES = [
     (3900, 4000, 640, 1, 1, "store_gelu", 1),
     (4096, 3072, 512, 1, 1, "resid", 1),
     (4096, 3000, 1024, 0, 0, "f32_accum", 1),
+    # split 0: the launcher picks CTA pairs plus a K split (the weight-gradient shapes)
+    (768, 768, 4096, 0, 0, "f32_store", 0),
+    (3072, 768, 16384, 0, 0, "f32_store", 0),
+    (700, 600, 4000, 0, 0, "f32_accum", 0),
+    (768, 3072, 8192, 0, 0, "f32_accum", 0),
 ]
 
 
@@ -81,7 +86,7 @@ def test_gemm_vs_torch(env, path, M, N, K, ak, bk, epi, split):
     aux_s = (torch.randn(M, ldo, device=dev) * 0.5).to(torch.bfloat16)
     outf_s = torch.randn(M, ldo, device=dev)
     outf0 = outf_s[:, :N].clone()
-    scratch = torch.zeros(max(1, split * M * N), device=dev)
+    scratch = torch.zeros(max(1, (split or 16) * M * N), device=dev)
     err.zero_()
     s = gb.gptk_gemm_bf16(M, N, K, As.data_ptr(), lda, ak, Bs.data_ptr(), ldb, bk, gb.GPTK_EPI[epi],
                           out_s.data_ptr(), ldo, out2_s.data_ptr(), ldo, aux_s.data_ptr(), ldo,
