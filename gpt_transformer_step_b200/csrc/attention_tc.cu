@@ -87,32 +87,90 @@ __device__ __forceinline__ void st_tmem_bf16x32(uint32_t taddr, const uint32_t (
 }
 
 // ------------------------------------------------------------------------------------------
-// forward
+// persistent schedule
 // ------------------------------------------------------------------------------------------
-// K and V tiles in separate two-stage rings (a K stage frees as soon as its S MMA is done, a V
-// stage after its P.V MMA); the softmax warps release S as soon as it is in registers, so the
-// next tile's S = Q K^T runs on the tensor core while they compute P.
-enum { F_QFULL, F_K0, F_K1, F_V0, F_V1, F_KFREE0, F_KFREE1, F_VFREE0, F_VFREE1, F_SFULL, F_SFREE,
-       F_PFULL, F_OFULL, F_NBAR };
-constexpr int FWD_SMEM = 5 * TILE_BYTES + 1024 + 256;
+// All three kernels are persistent: a CTA loops over work items (one 128-row tile of one
+// (batch, head)) numbered heavy-first, taking item r*G + c in even rounds r and
+// r*G + G-1-c in odd rounds (G CTAs, this is CTA c), so heavy and light items pair up. Every
+// warp role walks the same sequence, and the loads of the next item overlap the last tiles of
+// the current one. Each output element is still written by exactly one item.
+__device__ __forceinline__ int item_index(int r) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  return r * G + ((r & 1) ? G - 1 - c : c);
+}
+
+// A query tile of one (batch, head) and the key tiles it sees.
+struct QTile { int q0, b, h, kt0, n; };
+__device__ __forceinline__ bool query_item(const AttnParams &P, int r, QTile &it) {
+  const int BH = P.B * P.H, nqt = (P.T + TILE - 1) / TILE;
+  const int u = item_index(r);
+  if (u >= nqt * BH) return false;
+  const int bh = u % BH;
+  it.q0 = (nqt - 1 - u / BH) * TILE;  // the last query tiles see the most keys: first
+  it.b = bh / P.H;
+  it.h = bh % P.H;
+  const int w = P.window;
+  it.kt0 = (w >= 0 ? max(0, it.q0 - w) : 0) / TILE;
+  it.n = (min(P.T, it.q0 + TILE) + TILE - 1) / TILE - it.kt0;
+  return true;
+}
+struct QCursor {  // (item, key tile) walk of this CTA
+  QTile it;
+  int i, j;
+  bool valid;
+  __device__ __forceinline__ void start(const AttnParams &P) { i = 0; j = 0; valid = query_item(P, 0, it); }
+  __device__ __forceinline__ void next(const AttnParams &P) {
+    if (++j == it.n) { j = 0; ++i; valid = query_item(P, i, it); }
+  }
+};
+
+// A key tile of one (batch, head) and the query tiles that see it.
+struct KTile { int k0, b, h, qt0, n; };
+__device__ __forceinline__ bool key_item(const AttnParams &P, int r, KTile &it) {
+  const int BH = P.B * P.H, nkt = (P.T + TILE - 1) / TILE;
+  const int u = item_index(r);
+  if (u >= nkt * BH) return false;
+  const int bh = u % BH, kt = u / BH;  // the first key tiles are seen by the most queries
+  it.k0 = kt * TILE;
+  it.b = bh / P.H;
+  it.h = bh % P.H;
+  it.qt0 = kt;
+  const int w = P.window;
+  const int qhi = w >= 0 ? min(P.T - 1, it.k0 + TILE - 1 + w) : P.T - 1;
+  it.n = qhi / TILE + 1 - kt;
+  return true;
+}
+struct KCursor {  // (item, query tile) walk of this CTA
+  KTile it;
+  int i, j;
+  bool valid;
+  __device__ __forceinline__ void start(const AttnParams &P) { i = 0; j = 0; valid = key_item(P, 0, it); }
+  __device__ __forceinline__ void next(const AttnParams &P) {
+    if (++j == it.n) { j = 0; ++i; valid = key_item(P, i, it); }
+  }
+};
+
+// ------------------------------------------------------------------------------------------
+// forward (two CTAs per SM)
+// ------------------------------------------------------------------------------------------
+// Q double-buffered (the next item's Q loads during the current item); K and V in separate
+// two-stage rings, the producer running one K tile ahead of V (the next S = Q K^T is issued
+// before the current P.V); a K stage frees as soon as its S MMA is done, a V stage after its
+// P.V MMA. The softmax warps release S as soon as it is in registers, so the next tile's S
+// runs on the tensor core while they compute P.
+enum { F_Q0, F_QFREE0 = F_Q0 + 2, F_K0 = F_QFREE0 + 2, F_V0 = F_K0 + 2, F_KFREE0 = F_V0 + 2,
+       F_VFREE0 = F_KFREE0 + 2, F_SFULL = F_VFREE0 + 2, F_SFREE, F_PFULL, F_OFULL, F_NBAR };
+constexpr int FWD_SMEM = 6 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ = smem, *sK0 = smem + TILE_BYTES, *sV0 = smem + 3 * TILE_BYTES;  // 2 stages each
-  uint64_t *bar = (uint64_t *)(smem + 5 * TILE_BYTES);
+  uint8_t *sQ0 = smem, *sK0 = smem + 2 * TILE_BYTES, *sV0 = smem + 4 * TILE_BYTES;  // 2 each
+  uint64_t *bar = (uint64_t *)(smem + 6 * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + F_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = P.B * P.H, nqt = (P.T + TILE - 1) / TILE;
-  const int qt = nqt - 1 - (int)blockIdx.x / BH;  // heaviest (last) query tiles first
-  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
-  const int q0 = qt * TILE, row0 = b * P.T, w = P.window;
-  const int kt0 = (w >= 0 ? max(0, q0 - w) : 0) / TILE;
-  const int kt1 = (min(P.T, q0 + TILE) + TILE - 1) / TILE;
-  const int n = kt1 - kt0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < F_NBAR; ++i) mbar_init(&bar[i], (i == F_PFULL || i == F_SFREE) ? 4 : 1);
@@ -127,132 +185,176 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(&bar[F_QFULL], TILE_BYTES);
-      tma_load_2d(sQ, &tmQKV, &bar[F_QFULL], h * HD, row0 + q0);
-      for (int j = 0; j < n; ++j) {
-        const int s = j & 1, use = j >> 1, k0 = (kt0 + j) * TILE;
-        if (use > 0 && !mbar_wait(&bar[F_KFREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
+      QCursor kc, vc;
+      kc.start(P);
+      vc.start(P);
+      int gk = 0, gv = 0;
+      auto load_k = [&]() -> bool {  // (the item's Q first) and the next K tile
+        const int row0 = kc.it.b * P.T;
+        if (kc.j == 0) {
+          const int qb = kc.i & 1;
+          if (kc.i >= 2 && !mbar_wait(&bar[F_QFREE0 + qb], ((kc.i >> 1) - 1) & 1, abort_flag, P.err))
+            return false;
+          mbar_expect_tx(&bar[F_Q0 + qb], TILE_BYTES);
+          tma_load_2d(sQ0 + qb * TILE_BYTES, &tmQKV, &bar[F_Q0 + qb], kc.it.h * HD, row0 + kc.it.q0);
+        }
+        const int s = gk & 1, use = gk >> 1;
+        if (use > 0 && !mbar_wait(&bar[F_KFREE0 + s], (use - 1) & 1, abort_flag, P.err)) return false;
         mbar_expect_tx(&bar[F_K0 + s], TILE_BYTES);
-        tma_load_2d(sK0 + s * TILE_BYTES, &tmQKV, &bar[F_K0 + s], P.C + h * HD, row0 + k0);
+        tma_load_2d(sK0 + s * TILE_BYTES, &tmQKV, &bar[F_K0 + s], P.C + kc.it.h * HD,
+                    row0 + (kc.it.kt0 + kc.j) * TILE);
+        kc.next(P);
+        ++gk;
+        return true;
+      };
+      bool ok = !kc.valid || load_k();
+      while (ok && vc.valid) {
+        if (kc.valid && !load_k()) break;  // K of tile g+1 before V of tile g
+        const int s = gv & 1, use = gv >> 1;
         if (use > 0 && !mbar_wait(&bar[F_VFREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
         mbar_expect_tx(&bar[F_V0 + s], TILE_BYTES);
-        tma_load_2d(sV0 + s * TILE_BYTES, &tmQKV, &bar[F_V0 + s], 2 * P.C + h * HD, row0 + k0);
+        tma_load_2d(sV0 + s * TILE_BYTES, &tmQKV, &bar[F_V0 + s], 2 * P.C + vc.it.h * HD,
+                    vc.it.b * P.T + (vc.it.kt0 + vc.j) * TILE);
+        vc.next(P);
+        ++gv;
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aK0 = smem_u32(sK0), aV0 = smem_u32(sV0);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&bar[F_K0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
+      const uint32_t aQ0 = smem_u32(sQ0), aK0 = smem_u32(sK0), aV0 = smem_u32(sV0);
+      QCursor sc, pc;
+      sc.start(P);
+      pc.start(P);
+      int gs = 0;
+      auto issue_s = [&]() -> bool {  // S = Q K^T of the next tile in the walk
+        const int qb = sc.i & 1, s = gs & 1;
+        if (sc.j == 0 && !mbar_wait(&bar[F_Q0 + qb], (sc.i >> 1) & 1, abort_flag, P.err)) return false;
+        if (!mbar_wait(&bar[F_K0 + s], (gs >> 1) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        mma_qk(tmem, aQ, aK0 + s * TILE_BYTES, TILE);
+        mma_qk(tmem, aQ0 + qb * TILE_BYTES, aK0 + s * TILE_BYTES, TILE);
         umma_commit(&bar[F_SFULL]);
-        umma_commit(&bar[F_KFREE0 + s]);  // K_j is no longer read
+        umma_commit(&bar[F_KFREE0 + s]);  // K is no longer read
+        if (sc.j + 1 == sc.it.n) umma_commit(&bar[F_QFREE0 + qb]);  // nor this item's Q
+        sc.next(P);
+        ++gs;
         return true;
       };
-      bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) && issue_s(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (!mbar_wait(&bar[F_SFREE], j & 1, abort_flag, P.err)) break;  // S_j is in registers
+      bool ok = !sc.valid || issue_s();
+      for (int g = 0; ok && pc.valid; ++g, pc.next(P)) {
+        if (!mbar_wait(&bar[F_SFREE], g & 1, abort_flag, P.err)) break;  // S_g is in registers
         tc_fence_after();
-        if (j + 1 < n && !issue_s(j + 1)) break;
-        if (!mbar_wait(&bar[F_PFULL], j & 1, abort_flag, P.err)) break;
-        if (!mbar_wait(&bar[F_V0 + (j & 1)], (j >> 1) & 1, abort_flag, P.err)) break;
+        if (sc.valid && !issue_s()) break;
+        if (!mbar_wait(&bar[F_PFULL], g & 1, abort_flag, P.err)) break;
+        if (!mbar_wait(&bar[F_V0 + (g & 1)], (g >> 1) & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        mma_pv_ts(tmem + 128, tmem + 192, aV0 + (j & 1) * TILE_BYTES, j > 0);
+        mma_pv_ts(tmem + 128, tmem + 192, aV0 + (g & 1) * TILE_BYTES, pc.j > 0);
         umma_commit(&bar[F_OFULL]);
-        umma_commit(&bar[F_VFREE0 + (j & 1)]);  // V_j is no longer read
+        umma_commit(&bar[F_VFREE0 + (g & 1)]);  // V is no longer read
       }
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, r = q * 32 + lane, qi = q0 + r;
+    const int q = warp & 3, r = q * 32 + lane;
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tO = tS + 128, tP = tS + 192;
-    float m2 = -INFINITY, l = 0.f;
-    bool have = false, ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int k0 = (kt0 + j) * TILE;
-      if (!warp_wait(&bar[F_SFULL], j & 1, abort_flag, P.err)) { ok = false; break; }
-      tc_fence_after();
-      // the whole 128-key score row of this thread, one wait for the four loads
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32_nw(tS, s0);
-      tmem_ld32_nw(tS + 32, s1);
-      tmem_ld32_nw(tS + 64, s2);
-      tmem_ld32_nw(tS + 96, s3);
-      tmem_wait_ld32(s0);
-      reg_fence32(s1);
-      reg_fence32(s2);
-      reg_fence32(s3);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
-      float sv[128];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        sv[i] = __uint_as_float(s0[i]);
-        sv[32 + i] = __uint_as_float(s1[i]);
-        sv[64 + i] = __uint_as_float(s2[i]);
-        sv[96 + i] = __uint_as_float(s3[i]);
-      }
-      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-      if (!interior) {
-        // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= i <= hi
-        const int hi = qi - k0;
-        const int lo = w >= 0 ? qi - w - k0 : -1;
-#pragma unroll
-        for (int i = 0; i < 128; ++i) sv[i] = (i <= hi && i >= lo) ? sv[i] : -INFINITY;
-      }
-      float mx = sv[0];
-#pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-      const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
-      float mnew = m2;
-      bool resc = false;
-      if (mt > -INFINITY) {
-        if (!have) mnew = mt;
-        else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
-      }
-      if (j > 0) {
-        if (!warp_wait(&bar[F_OFULL], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+    const int w = P.window;
+    int g = 0;
+    bool ok = true;
+    QTile it;
+    for (int i = 0; ok && query_item(P, i, it); ++i) {
+      const int q0 = it.q0, qi = q0 + r, row0 = it.b * P.T;
+      float m2 = -INFINITY, l = 0.f;
+      bool have = false;
+      for (int j = 0; j < it.n; ++j, ++g) {
+        const int k0 = (it.kt0 + j) * TILE;
+        if (!warp_wait(&bar[F_SFULL], g & 1, abort_flag, P.err)) { ok = false; break; }
         tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        const float f = resc ? ex2(m2 - mnew) : 1.f;
+        // the whole 128-key score row of this thread, one wait for the four loads
+        uint32_t s0[32], s1[32], s2[32], s3[32];
+        tmem_ld32_nw(tS, s0);
+        tmem_ld32_nw(tS + 32, s1);
+        tmem_ld32_nw(tS + 64, s2);
+        tmem_ld32_nw(tS + 96, s3);
+        tmem_wait_ld32(s0);
+        reg_fence32(s1);
+        reg_fence32(s2);
+        reg_fence32(s3);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
+        float sv[128];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          sv[k] = __uint_as_float(s0[k]);
+          sv[32 + k] = __uint_as_float(s1[k]);
+          sv[64 + k] = __uint_as_float(s2[k]);
+          sv[96 + k] = __uint_as_float(s3[k]);
+        }
+        const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+        if (!interior) {
+          // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= k <= hi
+          const int hi = qi - k0;
+          const int lo = w >= 0 ? qi - w - k0 : -1;
+#pragma unroll
+          for (int k = 0; k < 128; ++k) sv[k] = (k <= hi && k >= lo) ? sv[k] : -INFINITY;
+        }
+        // row max as a tree of independent chains
+        float mx4[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx4[c] = sv[c];
+#pragma unroll
+        for (int k = 8; k < 128; ++k) mx4[k & 7] = fmaxf(mx4[k & 7], sv[k]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])),
+                               fmaxf(fmaxf(mx4[4], mx4[5]), fmaxf(mx4[6], mx4[7])));
+        const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
+        float mnew = m2;
+        bool resc = false;
+        if (mt > -INFINITY) {
+          if (!have) mnew = mt;
+          else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
+        }
+        // O and P are free once the previous tile's P.V is done (for j == 0 the previous
+        // item's epilogue waited for it)
+        if (j > 0) {
+          if (!warp_wait(&bar[F_OFULL], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          const float f = resc ? ex2(m2 - mnew) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          tmem_ld32(tO + c * 32, v);
+          for (int c = 0; c < 2; ++c) {
+            float v[32];
+            tmem_ld32(tO + c * 32, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= f;
-          tmem_st32(tO + c * 32, v);
+            for (int k = 0; k < 32; ++k) v[k] *= f;
+            tmem_st32(tO + c * 32, v);
+          }
+          l *= f;
         }
-        l *= f;
-      }
-      m2 = mnew;
-      if (mt > -INFINITY) have = true;
-      const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
-      float ls = 0.f;
+        m2 = mnew;
+        if (mt > -INFINITY) have = true;
+        const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
+        float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2(fmaf(sv[c * 32 + i], P.scale_log2, -mu));
-          const float p1 = ex2(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
-          ls += p0 + p1;
-          pk[i >> 1] = pack_bf16(p0, p1);
+          for (int k = 0; k < 32; k += 2) {
+            const float p0 = ex2(fmaf(sv[c * 32 + k], P.scale_log2, -mu));
+            const float p1 = ex2(fmaf(sv[c * 32 + k + 1], P.scale_log2, -mu));
+            ls0 += p0;
+            ls1 += p1;
+            pk[k >> 1] = pack_bf16(p0, p1);
+          }
+          st_tmem_bf16x32(tP + c * 16, pk);
         }
-        st_tmem_bf16x32(tP + c * 16, pk);
+        l += ls0 + ls1;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[F_PFULL]);
       }
-      l += ls;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[F_PFULL]);
-    }
-    if (ok && warp_wait(&bar[F_OFULL], (n - 1) & 1, abort_flag, P.err)) {
+      if (!ok || !warp_wait(&bar[F_OFULL], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint32_t pk[32];
@@ -261,13 +363,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
         float v[32];
         tmem_ld32(tO + c * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * inv, v[i + 1] * inv);
+        for (int k = 0; k < 32; k += 2) pk[c * 16 + (k >> 1)] = pack_bf16(v[k] * inv, v[k + 1] * inv);
       }
       if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.o + (size_t)(row0 + qi) * P.C + h * HD);
+        uint4 *dst = reinterpret_cast<uint4 *>(P.o + (size_t)(row0 + qi) * P.C + it.h * HD);
 #pragma unroll
         for (int t = 0; t < 8; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-        P.lse[((size_t)b * P.H + h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
+        P.lse[((size_t)it.b * P.H + it.h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
       }
     }
   }
@@ -280,12 +382,14 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 }
 
 // ------------------------------------------------------------------------------------------
-// backward kernels: 10 warps. warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..9 "row" warps:
-// warp w owns TMEM lane quarter (w % 4) and column half ch = (w - 2) / 4 (64 of the 128
-// columns of the S / dP tiles), so every row of a tile is shared by two warps. A row warp
-// loads its S and dP columns into registers, releases the accumulators at once (the MMA warp
-// then computes the next tile's S and dP while the row warps do the math), and writes its
-// bf16 results into its 64-column K-block of the smem operand tile.
+// backward kernels (one CTA per SM): 10 warps. warp 0 TMA, warp 1 TMEM + MMA issue, warps
+// 2..9 "row" warps: warp w owns TMEM lane quarter (w % 4) and column half ch = (w - 2) / 4
+// (64 of the 128 columns of the S / dP tiles), so every row of a tile is shared by two warps.
+// A row warp loads its S and dP columns into registers, releases the accumulators at once
+// (the MMA warp then computes the next tile's S and dP while the row warps do the math), and
+// writes its bf16 results into tensor memory as the A operand of the next MMAs. An item's
+// accumulators are read out before the row warps release the next item's first tile, so the
+// next item's accumulating MMAs never overwrite them early.
 // ------------------------------------------------------------------------------------------
 constexpr int BWD_THREADS = 320;
 constexpr int ROW_WARPS = 8;
@@ -307,34 +411,33 @@ __device__ __forceinline__ void ld_s_dp64(uint32_t tS, uint32_t tdP, uint32_t (&
 // ------------------------------------------------------------------------------------------
 // backward: dQ (+ D)
 // ------------------------------------------------------------------------------------------
-constexpr int DQ_STAGES = 4;  // K/V tiles in flight (the TMA latency spans ~2 tiles)
-enum { Q_QDO, Q_KV0, Q_FREE0 = Q_KV0 + DQ_STAGES, Q_SDP = Q_FREE0 + DQ_STAGES, Q_SDPFREE, Q_DS,
-       Q_MM2, Q_NBAR };
-constexpr int DQ_SMEM = (2 + 2 * DQ_STAGES) * TILE_BYTES + 1024 + 256;
+// Per item: Q, dO and O of the query tile (double-buffered); D_i = dO_i . O_i from the smem
+// tiles; then for every key tile S = Q K^T, dP = dO V^T, dS = P o (dP - D), dQ += dS K.
+constexpr int DQ_STAGES = 4;  // K/V tiles in flight
+enum { Q_QDO0, Q_QFREE0 = Q_QDO0 + 2, Q_KV0 = Q_QFREE0 + 2, Q_FREE0 = Q_KV0 + DQ_STAGES,
+       Q_SDP = Q_FREE0 + DQ_STAGES, Q_SDPFREE, Q_DS, Q_MM2, Q_NBAR };
+constexpr int DQ_QBUF = 3 * TILE_BYTES;  // Q | dO | O
+constexpr int DQ_SMEM = (2 * 3 + 2 * DQ_STAGES) * TILE_BYTES + 1024 + 256;
+static_assert(DQ_SMEM <= 232448, "dQ kernel shared memory");
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-               const AttnParams P) {
+               const __grid_constant__ CUtensorMap tmO, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ = smem, *sdO = smem + TILE_BYTES;
-  uint8_t *sK0 = smem + 2 * TILE_BYTES;  // stage s: K at 2+2s, V at 3+2s
-  uint64_t *bar = (uint64_t *)(smem + (2 + 2 * DQ_STAGES) * TILE_BYTES);
+  uint8_t *sK0 = smem + 2 * DQ_QBUF;  // stage s: K at 2s, V at 2s+1 (in tiles)
+  uint64_t *bar = (uint64_t *)(smem + (2 * 3 + 2 * DQ_STAGES) * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + Q_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = P.B * P.H, nqt = (P.T + TILE - 1) / TILE;
-  const int qt = nqt - 1 - (int)blockIdx.x / BH;
-  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
-  const int q0 = qt * TILE, row0 = b * P.T, w = P.window;
-  const int kt0 = (w >= 0 ? max(0, q0 - w) : 0) / TILE;
-  const int kt1 = (min(P.T, q0 + TILE) + TILE - 1) / TILE;
-  const int n = kt1 - kt0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < Q_NBAR; ++i)
-      mbar_init(&bar[i], (i == Q_DS || i == Q_SDPFREE) ? ROW_WARPS : 1);
+    for (int i = 0; i < Q_NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == Q_DS || i == Q_SDPFREE) cnt = ROW_WARPS;
+      if (i == Q_QFREE0 || i == Q_QFREE0 + 1) cnt = 1 + ROW_WARPS;  // last S/dP MMA + D reads
+      mbar_init(&bar[i], cnt);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -346,120 +449,153 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(&bar[Q_QDO], 2 * TILE_BYTES);
-      tma_load_2d(sQ, &tmQKV, &bar[Q_QDO], h * HD, row0 + q0);
-      tma_load_2d(sdO, &tmDO, &bar[Q_QDO], h * HD, row0 + q0);
-      for (int j = 0; j < n; ++j) {
-        const int s = j % DQ_STAGES, use = j / DQ_STAGES, k0 = (kt0 + j) * TILE;
-        if (use > 0 && !mbar_wait(&bar[Q_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
-        uint8_t *sK = sK0 + s * 2 * TILE_BYTES;
-        mbar_expect_tx(&bar[Q_KV0 + s], 2 * TILE_BYTES);
-        tma_load_2d(sK, &tmQKV, &bar[Q_KV0 + s], P.C + h * HD, row0 + k0);
-        tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[Q_KV0 + s], 2 * P.C + h * HD, row0 + k0);
+      QTile it;
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; ok && query_item(P, i, it); ++i) {
+        const int qb = i & 1, row0 = it.b * P.T;
+        if (i >= 2 && !mbar_wait(&bar[Q_QFREE0 + qb], ((i >> 1) - 1) & 1, abort_flag, P.err)) break;
+        uint8_t *sQ = smem + qb * DQ_QBUF;
+        mbar_expect_tx(&bar[Q_QDO0 + qb], 3 * TILE_BYTES);
+        tma_load_2d(sQ, &tmQKV, &bar[Q_QDO0 + qb], it.h * HD, row0 + it.q0);
+        tma_load_2d(sQ + TILE_BYTES, &tmDO, &bar[Q_QDO0 + qb], it.h * HD, row0 + it.q0);
+        tma_load_2d(sQ + 2 * TILE_BYTES, &tmO, &bar[Q_QDO0 + qb], it.h * HD, row0 + it.q0);
+        for (int j = 0; j < it.n; ++j, ++g) {
+          const int s = g % DQ_STAGES, use = g / DQ_STAGES, k0 = (it.kt0 + j) * TILE;
+          if (use > 0 && !mbar_wait(&bar[Q_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+          uint8_t *sK = sK0 + s * 2 * TILE_BYTES;
+          mbar_expect_tx(&bar[Q_KV0 + s], 2 * TILE_BYTES);
+          tma_load_2d(sK, &tmQKV, &bar[Q_KV0 + s], P.C + it.h * HD, row0 + k0);
+          tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[Q_KV0 + s], 2 * P.C + it.h * HD, row0 + k0);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO);
-      auto issue_sdp = [&](int j) -> bool {
-        const int s = j % DQ_STAGES;
-        if (!mbar_wait(&bar[Q_KV0 + s], (j / DQ_STAGES) & 1, abort_flag, P.err)) return false;
+      const uint32_t aQ0 = smem_u32(smem), aK0 = smem_u32(sK0);
+      QCursor sc, mc;
+      sc.start(P);
+      mc.start(P);
+      int gs = 0;
+      auto issue_sdp = [&]() -> bool {  // S and dP of the next tile in the walk
+        const int qb = sc.i & 1, s = gs % DQ_STAGES;
+        if (sc.j == 0 && !mbar_wait(&bar[Q_QDO0 + qb], (sc.i >> 1) & 1, abort_flag, P.err)) return false;
+        if (!mbar_wait(&bar[Q_KV0 + s], (gs / DQ_STAGES) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        const uint32_t aK = smem_u32(sK0 + s * 2 * TILE_BYTES), aV = aK + TILE_BYTES;
+        const uint32_t aQ = aQ0 + qb * DQ_QBUF, adO = aQ + TILE_BYTES;
+        const uint32_t aK = aK0 + s * 2 * TILE_BYTES, aV = aK + TILE_BYTES;
         mma_qk(tmem, aQ, aK, TILE);
         mma_qk(tmem + 128, adO, aV, TILE);
         umma_commit(&bar[Q_SDP]);
+        if (sc.j + 1 == sc.it.n) umma_commit(&bar[Q_QFREE0 + qb]);  // Q / dO no longer read
+        sc.next(P);
+        ++gs;
         return true;
       };
-      bool ok = mbar_wait(&bar[Q_QDO], 0, abort_flag, P.err) && issue_sdp(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (!mbar_wait(&bar[Q_SDPFREE], j & 1, abort_flag, P.err)) break;
+      bool ok = !sc.valid || issue_sdp();
+      for (int g = 0; ok && mc.valid; ++g, mc.next(P)) {
+        if (!mbar_wait(&bar[Q_SDPFREE], g & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        if (j + 1 < n && !issue_sdp(j + 1)) break;
-        if (!mbar_wait(&bar[Q_DS], j & 1, abort_flag, P.err)) break;
+        if (sc.valid && !issue_sdp()) break;
+        if (!mbar_wait(&bar[Q_DS], g & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        const uint32_t aK = smem_u32(sK0 + (j % DQ_STAGES) * 2 * TILE_BYTES);
-        mma_pv_ts(tmem + 256, tmem + 320, aK, j > 0);  // dQ += dS K (dS in TMEM, K tile MN-major)
+        const uint32_t aK = aK0 + (g % DQ_STAGES) * 2 * TILE_BYTES;
+        mma_pv_ts(tmem + 256, tmem + 320, aK, mc.j > 0);  // dQ += dS K (dS in TMEM, K MN-major)
         umma_commit(&bar[Q_MM2]);
-        umma_commit(&bar[Q_FREE0 + (j % DQ_STAGES)]);
+        umma_commit(&bar[Q_FREE0 + (g % DQ_STAGES)]);
       }
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane, qi = q0 + r;
+    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane;
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
-    // D_i = dO_i . O_i (written for the dK/dV pass) and the saved lse in the log2 domain
-    float D = 0.f, lse2 = 0.f;
-    if (qi < P.T) {
-      const size_t off = (size_t)(row0 + qi) * P.C + h * HD;
-      const uint4 *go = reinterpret_cast<const uint4 *>(P.O + off);
-      const uint4 *gd = reinterpret_cast<const uint4 *>(P.dO + off);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        uint4 av = go[t], cv = gd[t];
-        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&av);
-        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
-          D += fa.x * fc.x + fa.y * fc.y;
-        }
-      }
-      const size_t li = ((size_t)b * P.H + h) * P.T + qi;
-      if (ch == 0) P.Dbuf[li] = D;
-      lse2 = P.lse_in[li] * LOG2E;
-    }
+    const int w = P.window;
+    auto lse_of = [&](const QTile &t) -> float {
+      const int qi = t.q0 + r;
+      return qi < P.T ? P.lse_in[((size_t)t.b * P.H + t.h) * P.T + qi] : 0.f;
+    };
+    int g = 0;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int k0 = (kt0 + j) * TILE;
-      if (!warp_wait(&bar[Q_SDP], j & 1, abort_flag, P.err)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      ld_s_dp64(tS, tdP, s0, s1, d0, d1);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[Q_SDPFREE]);  // S / dP may be overwritten now
-      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-      const int hi = qi < P.T ? qi - k0 - ch * 64 : -1;  // admitted local columns: lo..hi
-      const int lo = w >= 0 ? qi - w - k0 - ch * 64 : -1;
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const float sa = __uint_as_float(i < 32 ? s0[i] : s1[i - 32]);
-        const float sb = __uint_as_float(i < 32 ? s0[i + 1] : s1[i - 31]);
-        const float da = __uint_as_float(i < 32 ? d0[i] : d1[i - 32]);
-        const float db = __uint_as_float(i < 32 ? d0[i + 1] : d1[i - 31]);
-        float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
-        float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
-        if (!interior) {
-          x0 = (i <= hi && i >= lo) ? x0 : 0.f;
-          x1 = (i + 1 <= hi && i + 1 >= lo) ? x1 : 0.f;
-        }
-        pk[i >> 1] = pack_bf16(x0, x1);
-      }
-      if (j > 0) {
-        if (!warp_wait(&bar[Q_MM2], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-      }
+    QTile it, nx;
+    bool have_it = query_item(P, 0, it);
+    float lse_cur = have_it ? lse_of(it) : 0.f;
+    for (int i = 0; ok && have_it; ++i) {
+      const bool have_nx = query_item(P, i + 1, nx);
+      const float lse_nx = have_nx ? lse_of(nx) : 0.f;  // in flight during this item
+      const int qb = i & 1, q0 = it.q0, qi = q0 + r;
+      if (!warp_wait(&bar[Q_QDO0 + qb], (i >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      // D_i = dO_i . O_i (also written for the dK/dV pass) from the swizzled smem tiles
+      float D = 0.f;
       {
-        const uint32_t tdS = tmem + ((uint32_t)(q * 32) << 16) + 320 + ch * 32;
-        uint32_t lo16[16], hi16[16];
+        const uint8_t *sdO = smem + qb * DQ_QBUF + TILE_BYTES, *sO = sdO + TILE_BYTES;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) { lo16[t] = pk[t]; hi16[t] = pk[16 + t]; }
-        tmem_st16_nw(tdS, lo16);
-        tmem_st16_nw(tdS + 16, hi16);
-        tmem_wait_st();
+        for (int c = 0; c < 8; ++c) {
+          const int off = r * 128 + ((c ^ (r & 7)) << 4);
+          const uint4 av = *reinterpret_cast<const uint4 *>(sO + off);
+          const uint4 cv = *reinterpret_cast<const uint4 *>(sdO + off);
+          const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&av);
+          const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
+            D += fa.x * fc.x + fa.y * fc.y;
+          }
+        }
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[Q_DS]);
-    }
-    if (ok && warp_wait(&bar[Q_MM2], (n - 1) & 1, abort_flag, P.err)) {
+      if (lane == 0) mbar_arrive(&bar[Q_QFREE0 + qb]);
+      if (ch == 0 && qi < P.T) P.Dbuf[((size_t)it.b * P.H + it.h) * P.T + qi] = D;
+      const float lse2 = lse_cur * LOG2E;
+      for (int j = 0; j < it.n; ++j, ++g) {
+        const int k0 = (it.kt0 + j) * TILE;
+        if (!warp_wait(&bar[Q_SDP], g & 1, abort_flag, P.err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t s0[32], s1[32], d0[32], d1[32];
+        ld_s_dp64(tS, tdP, s0, s1, d0, d1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[Q_SDPFREE]);  // S / dP may be overwritten now
+        const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+        const int hi = qi < P.T ? qi - k0 - ch * 64 : -1;  // admitted local columns: lo..hi
+        const int lo = w >= 0 ? qi - w - k0 - ch * 64 : -1;
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float sa = __uint_as_float(k < 32 ? s0[k] : s1[k - 32]);
+          const float sb = __uint_as_float(k < 32 ? s0[k + 1] : s1[k - 31]);
+          const float da = __uint_as_float(k < 32 ? d0[k] : d1[k - 32]);
+          const float db = __uint_as_float(k < 32 ? d0[k + 1] : d1[k - 31]);
+          float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
+          float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
+          if (!interior) {
+            x0 = (k <= hi && k >= lo) ? x0 : 0.f;
+            x1 = (k + 1 <= hi && k + 1 >= lo) ? x1 : 0.f;
+          }
+          pk[k >> 1] = pack_bf16(x0, x1);
+        }
+        // dS is free once the previous dQ MMA is done (for j == 0 the epilogue waited)
+        if (j > 0 && !warp_wait(&bar[Q_MM2], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        {
+          const uint32_t tdS = tmem + ((uint32_t)(q * 32) << 16) + 320 + ch * 32;
+          uint32_t lo16[16], hi16[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) { lo16[t] = pk[t]; hi16[t] = pk[16 + t]; }
+          tmem_st16_nw(tdS, lo16);
+          tmem_st16_nw(tdS + 16, hi16);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[Q_DS]);
+      }
+      if (!ok || !warp_wait(&bar[Q_MM2], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
       float v[32];
       tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 32, v);  // dQ columns ch*32..
       if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + qi) * 3 * P.C + h * HD + ch * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(it.b * P.T + qi) * 3 * P.C +
+                                               it.h * HD + ch * 32);
 #pragma unroll
         for (int t = 0; t < 4; ++t)
           dst[t] = make_uint4(pack_bf16(v[8 * t] * P.scale, v[8 * t + 1] * P.scale),
@@ -467,6 +603,9 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                               pack_bf16(v[8 * t + 4] * P.scale, v[8 * t + 5] * P.scale),
                               pack_bf16(v[8 * t + 6] * P.scale, v[8 * t + 7] * P.scale));
       }
+      it = nx;
+      have_it = have_nx;
+      lse_cur = lse_nx;
     }
   }
   tc_fence_before();
@@ -480,30 +619,27 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // ------------------------------------------------------------------------------------------
 // backward: dK, dV
 // ------------------------------------------------------------------------------------------
+// Per item: K and V of the key tile (double-buffered); then for every query tile that sees it
+// S^T = K Q^T, dP^T = V dO^T, P^T and dS^T -> TMEM, dV += P^T dO, dK += dS^T Q. The lse and
+// D of the next query tile are fetched from global memory one tile ahead.
 constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight
-enum { K_KV, K_QDO0, K_FREE0 = K_QDO0 + DKV_STAGES, K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE,
-       K_PS, K_MM2, K_NBAR };
-constexpr int DKV_SMEM = (2 + 2 * DKV_STAGES) * TILE_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
+enum { K_KV0, K_KVFREE0 = K_KV0 + 2, K_QDO0 = K_KVFREE0 + 2, K_FREE0 = K_QDO0 + DKV_STAGES,
+       K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE, K_PS, K_MM2, K_NBAR };
+constexpr int DKV_SMEM = (4 + 2 * DKV_STAGES) * TILE_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
+static_assert(DKV_SMEM <= 232448, "dK/dV kernel shared memory");
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                 const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sK = smem, *sV = smem + TILE_BYTES;
-  uint8_t *sQ0 = smem + 2 * TILE_BYTES;  // stage s: Q at 2+2s, dO at 3+2s
-  float *s_lsd = (float *)(smem + (2 + 2 * DKV_STAGES) * TILE_BYTES);  // [2][lse 128 | D 128]
+  uint8_t *sKV0 = smem;                  // buffer b: K at 2b, V at 2b+1 (in tiles)
+  uint8_t *sQ0 = smem + 4 * TILE_BYTES;  // stage s: Q at 2s, dO at 2s+1
+  float *s_lsd = (float *)(smem + (4 + 2 * DKV_STAGES) * TILE_BYTES);  // [2][lse 128 | D 128]
   uint64_t *bar = (uint64_t *)(s_lsd + 2 * 2 * TILE);
   uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = P.B * P.H;
-  const int kt = (int)blockIdx.x / BH;  // low key tiles see the most queries: first
-  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
-  const int k0 = kt * TILE, row0 = b * P.T, w = P.window;
-  const int qhi = w >= 0 ? min(P.T - 1, k0 + TILE - 1 + w) : P.T - 1;
-  const int qt0 = kt, n = qhi / TILE + 1 - qt0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < K_NBAR; ++i)
@@ -520,66 +656,94 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(&bar[K_KV], 2 * TILE_BYTES);
-      tma_load_2d(sK, &tmQKV, &bar[K_KV], P.C + h * HD, row0 + k0);
-      tma_load_2d(sV, &tmQKV, &bar[K_KV], 2 * P.C + h * HD, row0 + k0);
-      for (int j = 0; j < n; ++j) {
-        const int s = j % DKV_STAGES, use = j / DKV_STAGES, qq0 = (qt0 + j) * TILE;
-        if (use > 0 && !mbar_wait(&bar[K_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
-        uint8_t *sQ = sQ0 + s * 2 * TILE_BYTES;
-        mbar_expect_tx(&bar[K_QDO0 + s], 2 * TILE_BYTES);
-        tma_load_2d(sQ, &tmQKV, &bar[K_QDO0 + s], h * HD, row0 + qq0);
-        tma_load_2d(sQ + TILE_BYTES, &tmDO, &bar[K_QDO0 + s], h * HD, row0 + qq0);
+      KTile it;
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; ok && key_item(P, i, it); ++i) {
+        const int kb = i & 1, row0 = it.b * P.T;
+        if (i >= 2 && !mbar_wait(&bar[K_KVFREE0 + kb], ((i >> 1) - 1) & 1, abort_flag, P.err)) break;
+        uint8_t *sK = sKV0 + kb * 2 * TILE_BYTES;
+        mbar_expect_tx(&bar[K_KV0 + kb], 2 * TILE_BYTES);
+        tma_load_2d(sK, &tmQKV, &bar[K_KV0 + kb], P.C + it.h * HD, row0 + it.k0);
+        tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[K_KV0 + kb], 2 * P.C + it.h * HD, row0 + it.k0);
+        for (int j = 0; j < it.n; ++j, ++g) {
+          const int s = g % DKV_STAGES, use = g / DKV_STAGES, qq0 = (it.qt0 + j) * TILE;
+          if (use > 0 && !mbar_wait(&bar[K_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+          uint8_t *sQ = sQ0 + s * 2 * TILE_BYTES;
+          mbar_expect_tx(&bar[K_QDO0 + s], 2 * TILE_BYTES);
+          tma_load_2d(sQ, &tmQKV, &bar[K_QDO0 + s], it.h * HD, row0 + qq0);
+          tma_load_2d(sQ + TILE_BYTES, &tmDO, &bar[K_QDO0 + s], it.h * HD, row0 + qq0);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-      auto issue_sdp = [&](int j) -> bool {
-        const int s = j % DKV_STAGES;
-        if (!mbar_wait(&bar[K_QDO0 + s], (j / DKV_STAGES) & 1, abort_flag, P.err)) return false;
+      const uint32_t aKV0 = smem_u32(sKV0), aQ0 = smem_u32(sQ0);
+      KCursor sc, mc;
+      sc.start(P);
+      mc.start(P);
+      int gs = 0;
+      auto issue_sdp = [&]() -> bool {  // S^T and dP^T of the next tile in the walk
+        const int kb = sc.i & 1, s = gs % DKV_STAGES;
+        if (sc.j == 0 && !mbar_wait(&bar[K_KV0 + kb], (sc.i >> 1) & 1, abort_flag, P.err)) return false;
+        if (!mbar_wait(&bar[K_QDO0 + s], (gs / DKV_STAGES) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ0 + s * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
+        const uint32_t aK = aKV0 + kb * 2 * TILE_BYTES, aV = aK + TILE_BYTES;
+        const uint32_t aQ = aQ0 + s * 2 * TILE_BYTES, adO = aQ + TILE_BYTES;
         mma_qk(tmem, aK, aQ, TILE);         // S^T  = K Q^T
         mma_qk(tmem + 128, aV, adO, TILE);  // dP^T = V dO^T
         umma_commit(&bar[K_SDP]);
+        if (sc.j + 1 == sc.it.n) umma_commit(&bar[K_KVFREE0 + kb]);  // K / V no longer read
+        sc.next(P);
+        ++gs;
         return true;
       };
-      bool ok = mbar_wait(&bar[K_KV], 0, abort_flag, P.err) && issue_sdp(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (!mbar_wait(&bar[K_SDPFREE], j & 1, abort_flag, P.err)) break;
+      bool ok = !sc.valid || issue_sdp();
+      for (int g = 0; ok && mc.valid; ++g, mc.next(P)) {
+        if (!mbar_wait(&bar[K_SDPFREE], g & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        if (j + 1 < n && !issue_sdp(j + 1)) break;
-        if (!mbar_wait(&bar[K_PS], j & 1, abort_flag, P.err)) break;
+        if (sc.valid && !issue_sdp()) break;
+        if (!mbar_wait(&bar[K_PS], g & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ0 + (j % DKV_STAGES) * 2 * TILE_BYTES), adO = aQ + TILE_BYTES;
-        mma_pv_ts(tmem + 256, tmem + 384, adO, j > 0);  // dV += P^T dO   (P^T in TMEM)
-        mma_pv_ts(tmem + 320, tmem + 448, aQ, j > 0);   // dK += dS^T Q  (dS^T in TMEM)
+        const uint32_t aQ = aQ0 + (g % DKV_STAGES) * 2 * TILE_BYTES, adO = aQ + TILE_BYTES;
+        mma_pv_ts(tmem + 256, tmem + 384, adO, mc.j > 0);  // dV += P^T dO   (P^T in TMEM)
+        mma_pv_ts(tmem + 320, tmem + 448, aQ, mc.j > 0);   // dK += dS^T Q  (dS^T in TMEM)
         umma_commit(&bar[K_MM2]);
-        umma_commit(&bar[K_FREE0 + (j % DKV_STAGES)]);
+        umma_commit(&bar[K_FREE0 + (g % DKV_STAGES)]);
       }
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane, ki = k0 + r;
+    const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane;
     const int t = threadIdx.x - 64;  // 0..255 among the row warps
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
+    const int w = P.window;
+    // this thread's share of a query tile's (lse | D): t < 128 lse (log2 domain), else D
+    auto fetch = [&](const KTile &k, int j) -> float {
+      const int qi = (k.qt0 + j) * TILE + (t & 127);
+      if (qi >= P.T) return 0.f;
+      const size_t li = ((size_t)k.b * P.H + k.h) * P.T + qi;
+      return t < 128 ? P.lse_in[li] * LOG2E : P.Dbuf[li];
+    };
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int qq0 = (qt0 + j) * TILE;
-      // this query tile's lse (log2 domain) and D, into buffer j & 1; one barrier per tile
-      // (the other buffer may still be read by a warp finishing the previous tile)
-      float *lsd = s_lsd + (j & 1) * 2 * TILE;
-      {
-        const int qi = qq0 + (t & 127);
-        const size_t li = ((size_t)b * P.H + h) * P.T + qi;
-        if (t < 128) lsd[t] = qi < P.T ? P.lse_in[li] * LOG2E : 0.f;
-        else lsd[t] = qi < P.T ? P.Dbuf[li] : 0.f;
-      }
+    KCursor cur;
+    cur.start(P);
+    float pre = cur.valid ? fetch(cur.it, 0) : 0.f;
+    for (int g = 0; cur.valid; ++g) {
+      const KTile it = cur.it;
+      const int j = cur.j, k0 = it.k0, ki = k0 + r, qq0 = (it.qt0 + j) * TILE;
+      // this query tile's lse and D, into buffer g & 1; one barrier per tile (the other
+      // buffer may still be read by a warp finishing the previous tile)
+      float *lsd = s_lsd + (g & 1) * 2 * TILE;
+      lsd[t] = pre;
       asm volatile("bar.sync 1, 256;" ::: "memory");
+      KCursor nx = cur;
+      nx.next(P);
+      pre = nx.valid ? fetch(nx.it, nx.j) : 0.f;  // in flight during this tile
+      cur = nx;
       // after an abort every row warp still passes the named barrier of each tile
-      if (ok) ok = warp_wait(&bar[K_SDP], j & 1, abort_flag, P.err);
+      if (ok) ok = warp_wait(&bar[K_SDP], g & 1, abort_flag, P.err);
       if (!ok) continue;
       tc_fence_after();
       uint32_t s0[32], s1[32], d0[32], d1[32];
@@ -594,8 +758,10 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0 - ch * 64;
       const float4 *L4 = reinterpret_cast<const float4 *>(lsd + ch * 64);
       const float4 *D4 = reinterpret_cast<const float4 *>(lsd + TILE + ch * 64);
-      if (j > 0) {  // P^T / dS^T smem is free once the previous tile's dV / dK MMAs are done
-        ok = warp_wait(&bar[K_MM2], (j - 1) & 1, abort_flag, P.err);
+      // P^T / dS^T are free once the previous dV / dK MMAs are done (for j == 0 the
+      // previous item's epilogue waited for them)
+      if (j > 0) {
+        ok = warp_wait(&bar[K_MM2], (g - 1) & 1, abort_flag, P.err);
         if (!ok) continue;
       }
       const uint32_t tPT = tmem + ((uint32_t)(q * 32) << 16) + 384 + ch * 32, tdST = tPT + 64;
@@ -634,10 +800,12 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[K_PS]);
-    }
-    if (ok && warp_wait(&bar[K_MM2], (n - 1) & 1, abort_flag, P.err)) {
+      if (j + 1 < it.n) continue;
+      // the item's last query tile: dV / dK out (column half 0 writes dV, half 1 writes dK
+      // times the softmax scale)
+      ok = warp_wait(&bar[K_MM2], g & 1, abort_flag, P.err);
+      if (!ok) continue;
       tc_fence_after();
-      // column half 0 writes dV, half 1 writes dK (times the softmax scale)
       const float f = ch ? P.scale : 1.f;
       uint32_t pk[32];
 #pragma unroll 1
@@ -645,11 +813,11 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 64 + c * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * f, v[i + 1] * f);
+        for (int k = 0; k < 32; k += 2) pk[c * 16 + (k >> 1)] = pack_bf16(v[k] * f, v[k + 1] * f);
       }
       if (ki < P.T) {
-        const int col = (ch ? P.C : 2 * P.C) + h * HD;
-        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(row0 + ki) * 3 * P.C + col);
+        const int col = (ch ? P.C : 2 * P.C) + it.h * HD;
+        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(it.b * P.T + ki) * 3 * P.C + col);
 #pragma unroll
         for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
@@ -662,7 +830,6 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     tmem_dealloc(tmem, 512);
   }
 }
-
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -707,6 +874,17 @@ AttnParams make_params(int B, int T, int C, int H, int window, unsigned *err) {
   return p;
 }
 
+int attn_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 bool smem_attrs_set = false;
 cudaError_t set_attrs() {
   if (smem_attrs_set) return cudaSuccess;
@@ -729,8 +907,9 @@ cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B,
   AttnParams p = make_params(B, T, C, H, window, err);
   p.o = o;
   p.lse = lse;
-  const int nqt = (T + TILE - 1) / TILE;
-  attn_fwd_tc<<<B * H * nqt, 192, FWD_SMEM, st>>>(m, p);
+  const int items = B * H * ((T + TILE - 1) / TILE);
+  const int grid = items < 2 * attn_sms() ? items : 2 * attn_sms();  // two CTAs per SM
+  attn_fwd_tc<<<grid, 192, FWD_SMEM, st>>>(m, p);
   return cudaGetLastError();
 }
 
@@ -738,9 +917,10 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
                                     const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
                                     int C, int H, int window, unsigned *err, cudaStream_t st) {
   CUDA_TRY(set_attrs());
-  CUtensorMap mq, md;
+  CUtensorMap mq, md, mo;
   if (!map_rows(&mq, qkv, 3L * C, (long)B * T, 3L * C) ||
-      !map_rows(&md, dout, (long)C, (long)B * T, (long)C))
+      !map_rows(&md, dout, (long)C, (long)B * T, (long)C) ||
+      !map_rows(&mo, o, (long)C, (long)B * T, (long)C))
     return cudaErrorInvalidValue;
   AttnParams p = make_params(B, T, C, H, window, err);
   p.O = o;
@@ -748,10 +928,11 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
   p.lse_in = lse;
   p.Dbuf = Dbuf;
   p.dqkv = dqkv;
-  const int nt = (T + TILE - 1) / TILE;
-  attn_bwd_dq_tc<<<B * H * nt, BWD_THREADS, DQ_SMEM, st>>>(mq, md, p);
+  const int items = B * H * ((T + TILE - 1) / TILE);
+  const int grid = items < attn_sms() ? items : attn_sms();  // one CTA per SM
+  attn_bwd_dq_tc<<<grid, BWD_THREADS, DQ_SMEM, st>>>(mq, md, mo, p);
   CUDA_TRY(cudaGetLastError());
-  attn_bwd_dkv_tc<<<B * H * nt, BWD_THREADS, DKV_SMEM, st>>>(mq, md, p);
+  attn_bwd_dkv_tc<<<grid, BWD_THREADS, DKV_SMEM, st>>>(mq, md, p);
   return cudaGetLastError();
 }
 
