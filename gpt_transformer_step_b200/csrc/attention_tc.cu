@@ -6,16 +6,16 @@
 //   lse_i = log sum_j exp(s_ij) (natural log) is kept for the backward pass.
 //
 // All three kernels use 128x128 tiles, TMA loads of 128x64 bf16 tiles (128-byte swizzle) from
-// the fused qkv buffer [B*T, 3C], tcgen05.mma with fp32 accumulators in TMEM, and 4 "row"
-// warps in which each thread owns one row of the 128x128 score tile:
-//   forward  (CTA = b, h, 128 queries): S = Q K^T -> TMEM; online softmax in the log2 domain
-//            with a conditional rescale of O (only when the running max grows by > 8);
-//            P (bf16) -> swizzled smem; O += P V in TMEM.
-//   dQ       (CTA = b, h, 128 queries): also writes D_i = dO_i . O_i. S = Q K^T, dP = dO V^T,
-//            dS = P o (dP - D) -> smem, dQ += dS K.
-//   dK / dV  (CTA = b, h, 128 keys):    S^T = K Q^T, dP^T = V dO^T, P^T and dS^T -> smem,
-//            dV += P^T dO, dK += dS^T Q.
-// No atomics: every output element is written by exactly one CTA, so results are bitwise
+// the fused qkv buffer [B*T, 3C], tcgen05.mma with fp32 accumulators in TMEM, and "row" warps
+// in which each thread owns one row (or half a row) of the 128x128 score tile:
+//   forward  (CTA = b, h, 128 queries; two CTAs per SM): S = Q K^T -> TMEM; online softmax in
+//            the log2 domain with a conditional rescale of O (only when the running max grows
+//            by > 8); P (bf16) -> TMEM; O += P V with P read from TMEM.
+//   dQ       (persistent; item = b, h, 128 queries): D_i = dO_i . O_i (also written out),
+//            S = Q K^T, dP = dO V^T, dS = P o (dP - D) -> TMEM, dQ += dS K.
+//   dK / dV  (persistent; item = b, h, 128 keys): S^T = K Q^T, dP^T = V dO^T, P^T and dS^T ->
+//            TMEM, dV += P^T dO, dK += dS^T Q.
+// No atomics: every output element is written by exactly one work item, so results are bitwise
 // reproducible. Tiles entirely outside the causal/window band are skipped; edge tiles are
 // masked element by element. Every wait is bounded (device error word on timeout).
 #include "kernels.cuh"
@@ -89,7 +89,7 @@ __device__ __forceinline__ void st_tmem_bf16x32(uint32_t taddr, const uint32_t (
 // ------------------------------------------------------------------------------------------
 // persistent schedule
 // ------------------------------------------------------------------------------------------
-// All three kernels are persistent: a CTA loops over work items (one 128-row tile of one
+// The two backward kernels are persistent: a CTA loops over work items (one 128-row tile of one
 // (batch, head)) numbered heavy-first, taking item r*G + c in even rounds r and
 // r*G + G-1-c in odd rounds (G CTAs, this is CTA c), so heavy and light items pair up. Every
 // warp role walks the same sequence, and the loads of the next item overlap the last tiles of
@@ -151,26 +151,32 @@ struct KCursor {  // (item, query tile) walk of this CTA
 };
 
 // ------------------------------------------------------------------------------------------
-// forward (two CTAs per SM)
+// forward
 // ------------------------------------------------------------------------------------------
-// Q double-buffered (the next item's Q loads during the current item); K and V in separate
-// two-stage rings, the producer running one K tile ahead of V (the next S = Q K^T is issued
-// before the current P.V); a K stage frees as soon as its S MMA is done, a V stage after its
-// P.V MMA. The softmax warps release S as soon as it is in registers, so the next tile's S
-// runs on the tensor core while they compute P.
-enum { F_Q0, F_QFREE0 = F_Q0 + 2, F_K0 = F_QFREE0 + 2, F_V0 = F_K0 + 2, F_KFREE0 = F_V0 + 2,
-       F_VFREE0 = F_KFREE0 + 2, F_SFULL = F_VFREE0 + 2, F_SFREE, F_PFULL, F_OFULL, F_NBAR };
-constexpr int FWD_SMEM = 6 * TILE_BYTES + 1024 + 256;
+// K and V tiles in separate two-stage rings (a K stage frees as soon as its S MMA is done, a V
+// stage after its P.V MMA); the softmax warps release S as soon as it is in registers, so the
+// next tile's S = Q K^T runs on the tensor core while they compute P.
+enum { F_QFULL, F_K0, F_K1, F_V0, F_V1, F_KFREE0, F_KFREE1, F_VFREE0, F_VFREE1, F_SFULL, F_SFREE,
+       F_PFULL, F_OFULL, F_NBAR };
+constexpr int FWD_SMEM = 5 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ0 = smem, *sK0 = smem + 2 * TILE_BYTES, *sV0 = smem + 4 * TILE_BYTES;  // 2 each
-  uint64_t *bar = (uint64_t *)(smem + 6 * TILE_BYTES);
+  uint8_t *sQ = smem, *sK0 = smem + TILE_BYTES, *sV0 = smem + 3 * TILE_BYTES;  // 2 stages each
+  uint64_t *bar = (uint64_t *)(smem + 5 * TILE_BYTES);
   uint32_t *tmem_holder = (uint32_t *)(bar + F_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = P.B * P.H, nqt = (P.T + TILE - 1) / TILE;
+  const int qt = nqt - 1 - (int)blockIdx.x / BH;  // heaviest (last) query tiles first
+  const int bh = (int)blockIdx.x % BH, b = bh / P.H, h = bh % P.H;
+  const int q0 = qt * TILE, row0 = b * P.T, w = P.window;
+  const int kt0 = (w >= 0 ? max(0, q0 - w) : 0) / TILE;
+  const int kt1 = (min(P.T, q0 + TILE) + TILE - 1) / TILE;
+  const int n = kt1 - kt0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < F_NBAR; ++i) mbar_init(&bar[i], (i == F_PFULL || i == F_SFREE) ? 4 : 1);
@@ -185,176 +191,132 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 
   if (warp == 0) {
     if (lane == 0) {
-      QCursor kc, vc;
-      kc.start(P);
-      vc.start(P);
-      int gk = 0, gv = 0;
-      auto load_k = [&]() -> bool {  // (the item's Q first) and the next K tile
-        const int row0 = kc.it.b * P.T;
-        if (kc.j == 0) {
-          const int qb = kc.i & 1;
-          if (kc.i >= 2 && !mbar_wait(&bar[F_QFREE0 + qb], ((kc.i >> 1) - 1) & 1, abort_flag, P.err))
-            return false;
-          mbar_expect_tx(&bar[F_Q0 + qb], TILE_BYTES);
-          tma_load_2d(sQ0 + qb * TILE_BYTES, &tmQKV, &bar[F_Q0 + qb], kc.it.h * HD, row0 + kc.it.q0);
-        }
-        const int s = gk & 1, use = gk >> 1;
-        if (use > 0 && !mbar_wait(&bar[F_KFREE0 + s], (use - 1) & 1, abort_flag, P.err)) return false;
+      mbar_expect_tx(&bar[F_QFULL], TILE_BYTES);
+      tma_load_2d(sQ, &tmQKV, &bar[F_QFULL], h * HD, row0 + q0);
+      for (int j = 0; j < n; ++j) {
+        const int s = j & 1, use = j >> 1, k0 = (kt0 + j) * TILE;
+        if (use > 0 && !mbar_wait(&bar[F_KFREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
         mbar_expect_tx(&bar[F_K0 + s], TILE_BYTES);
-        tma_load_2d(sK0 + s * TILE_BYTES, &tmQKV, &bar[F_K0 + s], P.C + kc.it.h * HD,
-                    row0 + (kc.it.kt0 + kc.j) * TILE);
-        kc.next(P);
-        ++gk;
-        return true;
-      };
-      bool ok = !kc.valid || load_k();
-      while (ok && vc.valid) {
-        if (kc.valid && !load_k()) break;  // K of tile g+1 before V of tile g
-        const int s = gv & 1, use = gv >> 1;
+        tma_load_2d(sK0 + s * TILE_BYTES, &tmQKV, &bar[F_K0 + s], P.C + h * HD, row0 + k0);
         if (use > 0 && !mbar_wait(&bar[F_VFREE0 + s], (use - 1) & 1, abort_flag, P.err)) break;
         mbar_expect_tx(&bar[F_V0 + s], TILE_BYTES);
-        tma_load_2d(sV0 + s * TILE_BYTES, &tmQKV, &bar[F_V0 + s], 2 * P.C + vc.it.h * HD,
-                    vc.it.b * P.T + (vc.it.kt0 + vc.j) * TILE);
-        vc.next(P);
-        ++gv;
+        tma_load_2d(sV0 + s * TILE_BYTES, &tmQKV, &bar[F_V0 + s], 2 * P.C + h * HD, row0 + k0);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t aQ0 = smem_u32(sQ0), aK0 = smem_u32(sK0), aV0 = smem_u32(sV0);
-      QCursor sc, pc;
-      sc.start(P);
-      pc.start(P);
-      int gs = 0;
-      auto issue_s = [&]() -> bool {  // S = Q K^T of the next tile in the walk
-        const int qb = sc.i & 1, s = gs & 1;
-        if (sc.j == 0 && !mbar_wait(&bar[F_Q0 + qb], (sc.i >> 1) & 1, abort_flag, P.err)) return false;
-        if (!mbar_wait(&bar[F_K0 + s], (gs >> 1) & 1, abort_flag, P.err)) return false;
+      const uint32_t aQ = smem_u32(sQ), aK0 = smem_u32(sK0), aV0 = smem_u32(sV0);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&bar[F_K0 + s], (j >> 1) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        mma_qk(tmem, aQ0 + qb * TILE_BYTES, aK0 + s * TILE_BYTES, TILE);
+        mma_qk(tmem, aQ, aK0 + s * TILE_BYTES, TILE);
         umma_commit(&bar[F_SFULL]);
-        umma_commit(&bar[F_KFREE0 + s]);  // K is no longer read
-        if (sc.j + 1 == sc.it.n) umma_commit(&bar[F_QFREE0 + qb]);  // nor this item's Q
-        sc.next(P);
-        ++gs;
+        umma_commit(&bar[F_KFREE0 + s]);  // K_j is no longer read
         return true;
       };
-      bool ok = !sc.valid || issue_s();
-      for (int g = 0; ok && pc.valid; ++g, pc.next(P)) {
-        if (!mbar_wait(&bar[F_SFREE], g & 1, abort_flag, P.err)) break;  // S_g is in registers
+      bool ok = mbar_wait(&bar[F_QFULL], 0, abort_flag, P.err) && issue_s(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait(&bar[F_SFREE], j & 1, abort_flag, P.err)) break;  // S_j is in registers
         tc_fence_after();
-        if (sc.valid && !issue_s()) break;
-        if (!mbar_wait(&bar[F_PFULL], g & 1, abort_flag, P.err)) break;
-        if (!mbar_wait(&bar[F_V0 + (g & 1)], (g >> 1) & 1, abort_flag, P.err)) break;
+        if (j + 1 < n && !issue_s(j + 1)) break;
+        if (!mbar_wait(&bar[F_PFULL], j & 1, abort_flag, P.err)) break;
+        if (!mbar_wait(&bar[F_V0 + (j & 1)], (j >> 1) & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        mma_pv_ts(tmem + 128, tmem + 192, aV0 + (g & 1) * TILE_BYTES, pc.j > 0);
+        mma_pv_ts(tmem + 128, tmem + 192, aV0 + (j & 1) * TILE_BYTES, j > 0);
         umma_commit(&bar[F_OFULL]);
-        umma_commit(&bar[F_VFREE0 + (g & 1)]);  // V is no longer read
+        umma_commit(&bar[F_VFREE0 + (j & 1)]);  // V_j is no longer read
       }
     }
     __syncwarp();
   } else {
-    const int q = warp & 3, r = q * 32 + lane;
+    const int q = warp & 3, r = q * 32 + lane, qi = q0 + r;
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tO = tS + 128, tP = tS + 192;
-    const int w = P.window;
-    int g = 0;
-    bool ok = true;
-    QTile it;
-    for (int i = 0; ok && query_item(P, i, it); ++i) {
-      const int q0 = it.q0, qi = q0 + r, row0 = it.b * P.T;
-      float m2 = -INFINITY, l = 0.f;
-      bool have = false;
-      for (int j = 0; j < it.n; ++j, ++g) {
-        const int k0 = (it.kt0 + j) * TILE;
-        if (!warp_wait(&bar[F_SFULL], g & 1, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
-        // the whole 128-key score row of this thread, one wait for the four loads
-        uint32_t s0[32], s1[32], s2[32], s3[32];
-        tmem_ld32_nw(tS, s0);
-        tmem_ld32_nw(tS + 32, s1);
-        tmem_ld32_nw(tS + 64, s2);
-        tmem_ld32_nw(tS + 96, s3);
-        tmem_wait_ld32(s0);
-        reg_fence32(s1);
-        reg_fence32(s2);
-        reg_fence32(s3);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
-        float sv[128];
+    float m2 = -INFINITY, l = 0.f;
+    bool have = false, ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int k0 = (kt0 + j) * TILE;
+      if (!warp_wait(&bar[F_SFULL], j & 1, abort_flag, P.err)) { ok = false; break; }
+      tc_fence_after();
+      // the whole 128-key score row of this thread, one wait for the four loads
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32_nw(tS, s0);
+      tmem_ld32_nw(tS + 32, s1);
+      tmem_ld32_nw(tS + 64, s2);
+      tmem_ld32_nw(tS + 96, s3);
+      tmem_wait_ld32(s0);
+      reg_fence32(s1);
+      reg_fence32(s2);
+      reg_fence32(s3);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
+      float sv[128];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          sv[k] = __uint_as_float(s0[k]);
-          sv[32 + k] = __uint_as_float(s1[k]);
-          sv[64 + k] = __uint_as_float(s2[k]);
-          sv[96 + k] = __uint_as_float(s3[k]);
-        }
-        const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-        if (!interior) {
-          // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= k <= hi
-          const int hi = qi - k0;
-          const int lo = w >= 0 ? qi - w - k0 : -1;
-#pragma unroll
-          for (int k = 0; k < 128; ++k) sv[k] = (k <= hi && k >= lo) ? sv[k] : -INFINITY;
-        }
-        // row max as a tree of independent chains
-        float mx4[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx4[c] = sv[c];
-#pragma unroll
-        for (int k = 8; k < 128; ++k) mx4[k & 7] = fmaxf(mx4[k & 7], sv[k]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])),
-                               fmaxf(fmaxf(mx4[4], mx4[5]), fmaxf(mx4[6], mx4[7])));
-        const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
-        float mnew = m2;
-        bool resc = false;
-        if (mt > -INFINITY) {
-          if (!have) mnew = mt;
-          else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
-        }
-        // O and P are free once the previous tile's P.V is done (for j == 0 the previous
-        // item's epilogue waited for it)
-        if (j > 0) {
-          if (!warp_wait(&bar[F_OFULL], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-          tc_fence_after();
-        }
-        if (__any_sync(0xffffffffu, resc)) {
-          const float f = resc ? ex2(m2 - mnew) : 1.f;
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            float v[32];
-            tmem_ld32(tO + c * 32, v);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] *= f;
-            tmem_st32(tO + c * 32, v);
-          }
-          l *= f;
-        }
-        m2 = mnew;
-        if (mt > -INFINITY) have = true;
-        const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
-        float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2(fmaf(sv[c * 32 + k], P.scale_log2, -mu));
-            const float p1 = ex2(fmaf(sv[c * 32 + k + 1], P.scale_log2, -mu));
-            ls0 += p0;
-            ls1 += p1;
-            pk[k >> 1] = pack_bf16(p0, p1);
-          }
-          st_tmem_bf16x32(tP + c * 16, pk);
-        }
-        l += ls0 + ls1;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[F_PFULL]);
+      for (int i = 0; i < 32; ++i) {
+        sv[i] = __uint_as_float(s0[i]);
+        sv[32 + i] = __uint_as_float(s1[i]);
+        sv[64 + i] = __uint_as_float(s2[i]);
+        sv[96 + i] = __uint_as_float(s3[i]);
       }
-      if (!ok || !warp_wait(&bar[F_OFULL], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
+      if (!interior) {
+        // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= i <= hi
+        const int hi = qi - k0;
+        const int lo = w >= 0 ? qi - w - k0 : -1;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sv[i] = (i <= hi && i >= lo) ? sv[i] : -INFINITY;
+      }
+      float mx = sv[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+      const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
+      float mnew = m2;
+      bool resc = false;
+      if (mt > -INFINITY) {
+        if (!have) mnew = mt;
+        else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
+      }
+      if (j > 0) {
+        if (!warp_wait(&bar[F_OFULL], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? ex2(m2 - mnew) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          tmem_ld32(tO + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= f;
+          tmem_st32(tO + c * 32, v);
+        }
+        l *= f;
+      }
+      m2 = mnew;
+      if (mt > -INFINITY) have = true;
+      const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
+      float ls = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2(fmaf(sv[c * 32 + i], P.scale_log2, -mu));
+          const float p1 = ex2(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
+          ls += p0 + p1;
+          pk[i >> 1] = pack_bf16(p0, p1);
+        }
+        st_tmem_bf16x32(tP + c * 16, pk);
+      }
+      l += ls;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[F_PFULL]);
+    }
+    if (ok && warp_wait(&bar[F_OFULL], (n - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint32_t pk[32];
@@ -363,13 +325,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
         float v[32];
         tmem_ld32(tO + c * 32, v);
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) pk[c * 16 + (k >> 1)] = pack_bf16(v[k] * inv, v[k + 1] * inv);
+        for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * inv, v[i + 1] * inv);
       }
       if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.o + (size_t)(row0 + qi) * P.C + it.h * HD);
+        uint4 *dst = reinterpret_cast<uint4 *>(P.o + (size_t)(row0 + qi) * P.C + h * HD);
 #pragma unroll
         for (int t = 0; t < 8; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-        P.lse[((size_t)it.b * P.H + it.h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
+        P.lse[((size_t)b * P.H + h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
       }
     }
   }
@@ -907,9 +869,8 @@ cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B,
   AttnParams p = make_params(B, T, C, H, window, err);
   p.o = o;
   p.lse = lse;
-  const int items = B * H * ((T + TILE - 1) / TILE);
-  const int grid = items < 2 * attn_sms() ? items : 2 * attn_sms();  // two CTAs per SM
-  attn_fwd_tc<<<grid, 192, FWD_SMEM, st>>>(m, p);
+  const int nqt = (T + TILE - 1) / TILE;
+  attn_fwd_tc<<<B * H * nqt, 192, FWD_SMEM, st>>>(m, p);  // two CTAs per SM
   return cudaGetLastError();
 }
 

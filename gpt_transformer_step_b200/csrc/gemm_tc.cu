@@ -55,152 +55,90 @@ struct TcParams {
 // ---------------------------------------------------------------------------------------
 // epilogue helpers (one thread = one row, 32 consecutive columns per call)
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ void st_bf16x32(bf16 *dst, const float (&v)[32]) {
-  uint4 *d = reinterpret_cast<uint4 *>(dst);
+constexpr float LOG2E_F = 1.4426950408889634f;
+
+// Per-row epilogue operands that do not depend on the accumulators; they are fetched before
+// the epilogue waits for a tile, so their latency overlaps the MMAs.
+struct EpiRow {
+  float L2;   // cross-entropy dS: lse of the row, log2 units
+  float s;    // cross-entropy dS: 1 / (number of loss terms)
+  int t;      // cross-entropy: target column of the row (-1 for rows past M)
+};
+template <int EPI>
+__device__ __forceinline__ EpiRow epi_row(const TcParams &P, int row) {
+  EpiRow r{0.f, 0.f, -1};
+  const Epi &e = P.epi;
+  if (EPI == TE_CE_DS || EPI == TE_CE_STATS) {
+    if (row < P.M) r.t = e.targets[e.row_offset + row];
+  }
+  if (EPI == TE_CE_DS) {
+    if (row < P.M) r.L2 = e.lse[e.row_offset + row] * LOG2E_F;
+    r.s = e.sc->inv_M;
+  }
+  return r;
+}
+
+// 32 bf16 of the auxiliary input (residual stream or GELU pre-activation) of one row, packed;
+// zeros past M or N.
+__device__ __forceinline__ void load_aux_chunk(const TcParams &P, int row, int col0, uint4 (&a)[4]) {
+  const Epi &e = P.epi;
+  const bf16 *src = (const bf16 *)e.aux + (long)row * e.ld_aux + col0;
+  if (row < P.M && col0 + 32 <= P.N) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 u;
-    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * q + 0], v[8 * q + 1]);
-    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * q + 2], v[8 * q + 3]);
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 4], v[8 * q + 5]);
-    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * q + 6], v[8 * q + 7]);
-    u.x = *reinterpret_cast<uint32_t *>(&h0);
-    u.y = *reinterpret_cast<uint32_t *>(&h1);
-    u.z = *reinterpret_cast<uint32_t *>(&h2);
-    u.w = *reinterpret_cast<uint32_t *>(&h3);
-    d[q] = u;
+    for (int q = 0; q < 4; ++q) a[q] = reinterpret_cast<const uint4 *>(src)[q];
+  } else {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t lo = (row < P.M && col0 + 2 * i < P.N) ? __bfloat16_as_ushort(src[2 * i]) : 0u;
+      const uint32_t hi = (row < P.M && col0 + 2 * i + 1 < P.N) ? __bfloat16_as_ushort(src[2 * i + 1]) : 0u;
+      w[i] = lo | (hi << 16);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) a[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
 }
-__device__ __forceinline__ void ld_bf16x32(const bf16 *src, float (&v)[32]) {
-  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+__device__ __forceinline__ void unpack_bf16x32(const uint4 (&a)[4], float (&v)[32]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint4 u = s[q];
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float2 f = __bfloat1622float2(h[i]);
-      v[8 * q + 2 * i] = f.x;
-      v[8 * q + 2 * i + 1] = f.y;
+      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     }
   }
 }
 
-template <int EPI>
-__device__ __forceinline__ void epi_chunk(const TcParams &P, int row, int col0, int z,
-                                          float (&v)[32], float &ce_max, float &ce_sum) {
+// Cross-entropy statistics of one 32-column chunk of a row: the running (max, sum of
+// exp(logit - max)) over the valid vocabulary columns, and the target logit when the chunk
+// holds it.
+__device__ __forceinline__ void ce_stats_chunk(const TcParams &P, int row, int col0, const EpiRow &er,
+                                               const float (&v)[32], float &ce_max, float &ce_sum) {
   const Epi &e = P.epi;
-  const bool full = col0 + 32 <= P.N;
-  if (EPI == TE_CE_STATS) {
-    const int lim = min(P.N, e.V) - col0;  // valid columns in this chunk
-    float mx = -INFINITY;
+  const int lim = min(P.N, e.V) - col0;  // valid columns in this chunk
+  float mx = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (i < lim) mx = fmaxf(mx, v[i]);
-    const float mnew = fmaxf(ce_max, mx);
-    if (mnew > -INFINITY) {
-      float s = 0.f;
+  for (int i = 0; i < 32; ++i)
+    if (i < lim) mx = fmaxf(mx, v[i]);
+  const float mnew = fmaxf(ce_max, mx);
+  if (mnew > -INFINITY) {
+    const float m2 = mnew * LOG2E_F;
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i < lim) s += __expf(v[i] - mnew);
-      ce_sum = ce_sum * __expf(ce_max - mnew) + s;
-      ce_max = mnew;
+    for (int i = 0; i < 32; i += 2) {
+      if (i < lim) s0 += ex2(fmaf(v[i], LOG2E_F, -m2));
+      if (i + 1 < lim) s1 += ex2(fmaf(v[i + 1], LOG2E_F, -m2));
     }
-    const int grow = e.row_offset + row;
-    const int t = e.targets[grow] - col0;
-    if (t >= 0 && t < 32 && t < lim) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i == t) e.tgt_logit[grow] = v[i];
-    }
-    return;
+    ce_sum = ce_sum * ex2(fmaf(ce_max, LOG2E_F, -m2)) + (s0 + s1);
+    ce_max = mnew;
   }
-  if (EPI == TE_CE_DS) {
-    const int grow = e.row_offset + row;
-    const float L = e.lse[grow];
-    const int t = e.targets[grow];
-    const float s = e.sc->inv_M;
+  const int t = er.t - col0;
+  if (t >= 0 && t < 32 && t < lim) {
+    float tv = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int c = col0 + i;
-      float p = 0.f;
-      if (c < e.V) {
-        p = __expf(v[i] - L);
-        if (c == t) p -= 1.f;
-        p *= s;
-      }
-      v[i] = p;
-    }
-    bf16 *dst = (bf16 *)e.out + (long)row * e.ldo + col0;
-    if (full) {
-      st_bf16x32(dst, v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (col0 + i < P.N) dst[i] = __float2bfloat16_rn(v[i]);
-    }
-    return;
-  }
-  if (EPI == TE_PARTIAL || EPI == TE_F32_STORE || EPI == TE_F32_ACCUM) {
-    float *dst = EPI == TE_PARTIAL ? P.partial + ((long)z * P.M + row) * P.N + col0
-                                   : e.outf + (long)row * e.ldf + col0;
-    if (EPI == TE_F32_ACCUM) {
-      if (full) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float4 o = reinterpret_cast<float4 *>(dst)[q];
-          o.x += v[4 * q]; o.y += v[4 * q + 1]; o.z += v[4 * q + 2]; o.w += v[4 * q + 3];
-          reinterpret_cast<float4 *>(dst)[q] = o;
-        }
-      } else {
-        for (int i = 0; i < 32; ++i)
-          if (col0 + i < P.N) dst[i] += v[i];
-      }
-    } else {
-      if (full && (EPI != TE_PARTIAL || (P.N & 3) == 0)) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          reinterpret_cast<float4 *>(dst)[q] =
-              make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else {
-        for (int i = 0; i < 32; ++i)
-          if (col0 + i < P.N) dst[i] = v[i];
-      }
-    }
-    return;
-  }
-  // activation (bf16) outputs
-  bf16 *dst = (bf16 *)e.out + (long)row * e.ldo + col0;
-  if (EPI == TE_RESID || EPI == TE_DGELU) {
-    const bf16 *aux = (const bf16 *)e.aux + (long)row * e.ld_aux + col0;
-    float a[32];
-    if (full) {
-      ld_bf16x32(aux, a);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) a[i] = (col0 + i < P.N) ? __bfloat162float(aux[i]) : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_fast(a[i]);
-  }
-  if (full) {
-    st_bf16x32(dst, v);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (col0 + i < P.N) dst[i] = __float2bfloat16_rn(v[i]);
-  }
-  if (EPI == TE_STORE_GELU) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i]);
-    bf16 *d2 = (bf16 *)e.out2 + (long)row * e.ldo2 + col0;
-    if (full) {
-      st_bf16x32(d2, v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (col0 + i < P.N) d2[i] = __float2bfloat16_rn(v[i]);
-    }
+    for (int i = 0; i < 32; ++i) tv = (i == t) ? v[i] : tv;
+    e.tgt_logit[e.row_offset + row] = tv;
   }
 }
 
@@ -330,37 +268,24 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Epilogue math for one 32-column chunk of one row (everything but the store): v holds the
-// fp32 accumulators on entry and the values to store on exit; v2 the second output (GELU).
+// fp32 accumulators on entry and the values to store on exit; v2 the second output (GELU);
+// aux the chunk's auxiliary input (residual / dGELU).
 template <int EPI>
-__device__ __forceinline__ void epi_math(const TcParams &P, int row, int col0, float (&v)[32],
-                                         float (&v2)[32]) {
-  const Epi &e = P.epi;
+__device__ __forceinline__ void epi_math(const TcParams &P, int col0, const EpiRow &er,
+                                         const uint4 (&aux)[4], float (&v)[32], float (&v2)[32]) {
   if (EPI == TE_CE_DS) {
-    const int grow = e.row_offset + row;
-    const bool ok = row < P.M;
-    const float L = ok ? e.lse[grow] : 0.f;
-    const int t = ok ? e.targets[grow] : -1;
-    const float s = e.sc->inv_M;
+    // dS = (softmax - onehot(target)) / n over the valid vocabulary columns, 0 past V
+    const int V = P.epi.V;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int c = col0 + i;
-      float p = 0.f;
-      if (c < e.V) {
-        p = __expf(v[i] - L);
-        if (c == t) p -= 1.f;
-        p *= s;
-      }
-      v[i] = p;
+      float p = ex2(fmaf(v[i], LOG2E_F, -er.L2));
+      p = (c == er.t) ? p - 1.f : p;
+      v[i] = c < V ? p * er.s : 0.f;
     }
   } else if (EPI == TE_RESID || EPI == TE_DGELU) {
     float a[32];
-    if (row < P.M && col0 + 32 <= P.N) {
-      ld_bf16x32((const bf16 *)e.aux + (long)row * e.ld_aux + col0, a);
-    } else {
-      const bf16 *aux = (const bf16 *)e.aux + (long)row * e.ld_aux + col0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) a[i] = (row < P.M && col0 + i < P.N) ? __bfloat162float(aux[i]) : 0.f;
-    }
+    unpack_bf16x32(aux, a);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_fast(a[i]);
   } else if (EPI == TE_STORE_GELU) {
@@ -543,29 +468,46 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
       const int acc = i & 1;
       const uint32_t use = (uint32_t)(i >> 1);
+      const int row0 = mt * BM * CG + (int)rank * BM + q * 32;  // this warp's 32 rows
+      const int row = row0 + lane;
+      const int c0 = half * EPI_COLS;
+      // operands that do not depend on the accumulators: loaded before the wait
+      const EpiRow er = epi_row<EPI>(P, row);
+      uint4 aux[4];
+      if ((EPI == TE_RESID || EPI == TE_DGELU) && c0 < min(BN, P.N - nt * BN))
+        load_aux_chunk(P, row, nt * BN + c0, aux);
       int okw = 1;
       if (lane == 0) okw = mbar_wait(&tfull_bar[acc], use & 1u, abort_flag, P.err) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
       tc_fence_after();
-      const int row0 = mt * BM * CG + (int)rank * BM + q * 32;  // this warp's 32 rows
-      const int row = row0 + lane;
-      const int c0 = half * EPI_COLS;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0);
       float ce_max = -INFINITY, ce_sum = 0.f;
       const int ncols = min(BN, P.N - nt * BN) - c0;
 #pragma unroll 1
       for (int c = 0; c < EPI_COLS / 32; ++c) {
         if (c * 32 >= ncols) break;  // uniform across the warp
-        float v[32];
-        tmem_ld32(tbase + (uint32_t)(c * 32), v);
         const int col0 = nt * BN + c0 + c * 32;
+        float v[32];
+        uint32_t raw[32];
+        tmem_ld32_nw(tbase + (uint32_t)(c * 32), raw);
+        // the next chunk's auxiliary input is in flight during this chunk's math
+        uint4 aux_nx[4];
+        if ((EPI == TE_RESID || EPI == TE_DGELU) && (c + 1) * 32 < ncols && c + 1 < EPI_COLS / 32)
+          load_aux_chunk(P, row, col0 + 32, aux_nx);
+        tmem_wait_ld32(raw);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(raw[k]);
         if (EPI == TE_CE_STATS) {
-          if (row < P.M) epi_chunk<EPI>(P, row, col0, z, v, ce_max, ce_sum);
+          if (row < P.M) ce_stats_chunk(P, row, col0, er, v, ce_max, ce_sum);
           continue;
         }
         float v2[32];
-        epi_math<EPI>(P, row, col0, v, v2);
+        epi_math<EPI>(P, col0, er, aux, v, v2);
+        if (EPI == TE_RESID || EPI == TE_DGELU) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) aux[q] = aux_nx[q];
+        }
         // staging slot of this chunk (round robin); wait until its previous store has read it
         if (lane == 0) {
           if (CHUNK_SLOTS == 1) bulk_wait_read<0>();
