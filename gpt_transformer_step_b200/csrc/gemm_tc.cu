@@ -722,33 +722,39 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   TcParams P;
   memset(&P, 0, sizeof(P));
   const int sms = num_sms();
-  // CTA pairs (256-row tiles) whenever they fill the machine, directly or with a K split of
-  // at most 16 (weight gradients: small output, long K); single CTAs otherwise
   const int nt = (d.N + BN - 1) / BN;
   const long kblocks = (d.K + BK - 1) / BK;
   const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
   const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
-  const bool can_split = d.split_k <= 0 && (f32out || elementwise) && d.partial;
-  auto split_for = [&](long tiles, int cg) {
-    int s = 1;
-    while (tiles * s * cg < (long)sms && kblocks / (s * 2) >= 4 && s < 16 &&
-           (size_t)s * 2 * d.M * d.N <= t->splitk_capacity)
-      s *= 2;
-    return s;
-  };
-  const long tiles2 = (long)((d.M + 2 * BM - 1) / (2 * BM)) * nt;
-  int CG = 1;
-  if (tiles2 * 2 >= sms) CG = 2;
-  else if (can_split && tiles2 * 2 * split_for(tiles2, 2) >= sms) CG = 2;
+  int CG = ((long)((d.M + 2 * BM - 1) / (2 * BM)) * nt >= sms / 2) ? 2 : 1;
+  int S = d.split_k;
+  if (S <= 0) {
+    S = 1;
+    if ((f32out || elementwise) && d.partial) {
+      // automatic: the CTA group and K split with the smallest estimated time, in units of
+      // one k-block of one CTA tile (~0.4 us as measured): the wave-quantised main loop, CTA
+      // pairs credited with their smaller shared-memory traffic, plus for a split the ordered
+      // reduce, which reads the s fp32 partials and writes the result (~6 TB/s), and its
+      // launch (the partial stores themselves overlap the main loop)
+      double best = 1e30;
+      for (int cg = 1; cg <= 2; ++cg) {
+        const long tiles = (long)((d.M + cg * BM - 1) / (cg * BM)) * nt;
+        const long slots = sms / cg;
+        for (int s = 1; s <= 16; ++s) {
+          if (s > 1 && (kblocks / s < 4 || (size_t)s * d.M * d.N > t->splitk_capacity)) break;
+          const long units = tiles * s;
+          const long waves = (units + slots - 1) / slots;
+          double est = (double)waves * (double)((kblocks + s - 1) / s) * (cg == 2 ? 0.93 : 1.0);
+          if (s > 1) est += ((s + 1.0) * d.M * d.N * 4.0 / 6.0e12 + 3e-6) / 0.4e-6;
+          if (est < best) { best = est; CG = cg; S = s; }
+        }
+      }
+    }
+  }
   P.M = d.M; P.N = d.N; P.K = d.K;
   P.num_mt = (d.M + BM * CG - 1) / (BM * CG);
   P.num_nt = nt;
   P.total_kblocks = (int)kblocks;
-  int S = d.split_k;
-  if (S <= 0) {  // automatic: split K while the tile grid leaves SMs idle
-    const long tiles = (long)P.num_mt * P.num_nt;
-    S = (f32out || (elementwise && tiles * CG < sms)) && d.partial ? split_for(tiles, CG) : 1;
-  }
   if (S > P.total_kblocks) S = P.total_kblocks;
   P.kblocks_per_split = (P.total_kblocks + S - 1) / S;
   S = (P.total_kblocks + P.kblocks_per_split - 1) / P.kblocks_per_split;  // no empty split
