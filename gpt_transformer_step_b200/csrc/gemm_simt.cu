@@ -108,6 +108,31 @@ __global__ void splitk_reduce_kernel(GemmDesc d) {
   }
 }
 
+// N % 4 == 0: a block per row (grid-stride over rows), four columns per thread from 16-byte
+// partial loads; the splits are added in split order, as above.
+template <typename T>
+__global__ void __launch_bounds__(256) splitk_reduce4_kernel(GemmDesc d) {
+  const int n4 = d.N >> 2;
+  const long zstride4 = (long)d.M * n4;
+  const float4 *part = reinterpret_cast<const float4 *>(d.partial);
+  for (int m = blockIdx.x; m < d.M; m += gridDim.x) {
+    for (int c = threadIdx.x; c < n4; c += blockDim.x) {
+      const float4 *p = part + (long)m * n4 + c;
+      float4 s = p[0];
+#pragma unroll 4
+      for (int z = 1; z < d.split_k; ++z) {
+        const float4 v = p[z * zstride4];
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      const int n = 4 * c;
+      epi_elem<T>(d.epi, m, n, s.x);
+      epi_elem<T>(d.epi, m, n + 1, s.y);
+      epi_elem<T>(d.epi, m, n + 2, s.z);
+      epi_elem<T>(d.epi, m, n + 3, s.w);
+    }
+  }
+}
+
 }  // namespace
 
 template <typename T>
@@ -123,6 +148,11 @@ cudaError_t launch_gemm_simt(const GemmDesc &d, cudaStream_t st) {
 
 template <typename T>
 cudaError_t launch_splitk_reduce(const GemmDesc &d, cudaStream_t st) {
+  if ((d.N & 3) == 0 && ((uintptr_t)d.partial & 15) == 0) {
+    const int blocks = d.M < 148 * 8 ? d.M : 148 * 8;
+    splitk_reduce4_kernel<T><<<blocks, 256, 0, st>>>(d);
+    return cudaGetLastError();
+  }
   long total = (long)d.M * d.N;
   long blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;

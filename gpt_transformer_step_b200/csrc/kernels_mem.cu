@@ -144,14 +144,34 @@ __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restric
 // K12 LayerNorm backward (+ residual-gradient add, + per-block dgamma partials)
 // ------------------------------------------------------------------------------------------
 constexpr int LNB_WARPS = 8;
-constexpr int LNB_MAX_BLOCKS = 592;
+constexpr int LNB_MAX_BLOCKS = 296;
 
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const typename Vec<T>::type &v, float (&f)[Vec<T>::N]);
+template <>
+__device__ __forceinline__ void unpack_vec<float>(const float4 &v, float (&f)[4]) {
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void unpack_vec<bf16>(const uint4 &v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Each warp walks its rows with the next row's x, dy and residual gradient in flight while the
+// current row is reduced; x-hat and g*dy are recomputed from the raw vectors in the second
+// pass instead of being kept, which leaves room for two blocks of 8 warps per SM.
 template <typename T, int NV>
-__global__ void __launch_bounds__(LNB_WARPS * 32)
+__global__ void __launch_bounds__(LNB_WARPS * 32, 2)
 layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
                      const float *__restrict__ mean, const float *__restrict__ rstd,
                      const T *__restrict__ dy, T *__restrict__ dres,
                      float *__restrict__ dg_partial, int M, int C, int rows_per_block) {
+  using VT = typename Vec<T>::type;
   constexpr int VN = Vec<T>::N;
   extern __shared__ float sm_dg[];  // [LNB_WARPS][C]
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -163,26 +183,42 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
     for (int k = 0; k < VN; ++k) dgacc[j][k] = 0.f;
   const int r0 = blockIdx.x * rows_per_block;
   const int r1 = min(M, r0 + rows_per_block);
-  for (int row = r0 + w; row < r1; row += LNB_WARPS) {
-    const float mu = mean[row], rs = rstd[row];
-    float xh[NV][VN], dxh[NV][VN], rv[NV][VN];
+  VT xr[NV], dr[NV], rr[NV];
+  float mu = 0.f, rs = 0.f;
+  auto load_row = [&](int row, VT (&xa)[NV], VT (&da)[NV], VT (&ra)[NV], float &m, float &s) {
+    m = mean[row];
+    s = rstd[row];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      if (lane + 32 * j < nv) {
+        const long off = (long)row * C + (lane + 32 * j) * VN;
+        xa[j] = *reinterpret_cast<const VT *>(x + off);
+        da[j] = *reinterpret_cast<const VT *>(dy + off);
+        ra[j] = *reinterpret_cast<const VT *>(dres + off);
+      }
+    }
+  };
+  int row = r0 + w;
+  if (row < r1) load_row(row, xr, dr, rr, mu, rs);
+  for (; row < r1; row += LNB_WARPS) {
+    VT xn[NV], dn[NV], rn[NV];
+    float mun = 0.f, rsn = 0.f;
+    if (row + LNB_WARPS < r1) load_row(row + LNB_WARPS, xn, dn, rn, mun, rsn);
     float a = 0.f, b = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
-      int c = (lane + 32 * j) * VN;
       if (lane + 32 * j < nv) {
         float xv[VN], dv[VN], gv[VN];
-        load_vec<T>(x + (long)row * C + c, xv);
-        load_vec<T>(dy + (long)row * C + c, dv);
-        load_vec<T>(g + c, gv);
-        load_vec<T>(dres + (long)row * C + c, rv[j]);  // issued with the others
+        unpack_vec<T>(xr[j], xv);
+        unpack_vec<T>(dr[j], dv);
+        unpack_vec<T>(__ldg(reinterpret_cast<const VT *>(g + (lane + 32 * j) * VN)), gv);
 #pragma unroll
         for (int k = 0; k < VN; ++k) {
-          xh[j][k] = (xv[k] - mu) * rs;
-          dxh[j][k] = dv[k] * gv[k];
-          a += dxh[j][k];
-          b += dxh[j][k] * xh[j][k];
-          dgacc[j][k] += dv[k] * xh[j][k];
+          const float xh = (xv[k] - mu) * rs;
+          const float dxh = dv[k] * gv[k];
+          a += dxh;
+          b += dxh * xh;
+          dgacc[j][k] += dv[k] * xh;
         }
       }
     }
@@ -190,14 +226,29 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
     b = warp_sum(b) / (float)C;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
-      int c = (lane + 32 * j) * VN;
       if (lane + 32 * j < nv) {
-        float r[VN];
+        float xv[VN], dv[VN], gv[VN], rv[VN], o[VN];
+        unpack_vec<T>(xr[j], xv);
+        unpack_vec<T>(dr[j], dv);
+        unpack_vec<T>(__ldg(reinterpret_cast<const VT *>(g + (lane + 32 * j) * VN)), gv);
+        unpack_vec<T>(rr[j], rv);
 #pragma unroll
-        for (int k = 0; k < VN; ++k) r[k] = rv[j][k] + rs * (dxh[j][k] - a - xh[j][k] * b);
-        store_vec<T>(dres + (long)row * C + c, r);
+        for (int k = 0; k < VN; ++k) {
+          const float xh = (xv[k] - mu) * rs;
+          const float dxh = dv[k] * gv[k];
+          o[k] = rv[k] + rs * (dxh - a - xh * b);
+        }
+        store_vec<T>(dres + (long)row * C + (lane + 32 * j) * VN, o);
       }
     }
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      xr[j] = xn[j];
+      dr[j] = dn[j];
+      rr[j] = rn[j];
+    }
+    mu = mun;
+    rs = rsn;
   }
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
@@ -214,22 +265,25 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
   }
 }
 
-// out[c] = sum_r partial[r][c]: block = 32 columns x 8 row groups; each thread sums rows
-// g, g+8, ... in order, then the 8 group sums are added in group order (deterministic).
-__global__ void __launch_bounds__(256) colsum_kernel(const float *__restrict__ partial, int nrows,
-                                                     int C, float *__restrict__ out) {
-  __shared__ float sh[8][33];
+// out[c] = sum_r partial[r][c]: block = 32 columns x 32 row groups; each thread sums rows
+// g, g+32, ... in order (four loads in flight), then the 32 group sums are added in group
+// order (deterministic).
+__global__ void __launch_bounds__(1024) colsum_kernel(const float *__restrict__ partial, int nrows,
+                                                      int C, float *__restrict__ out) {
+  __shared__ float sh[32][33];
   const int cx = threadIdx.x & 31, g = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + cx;
   float s = 0.f;
-  if (c < C)
-    for (int r = g; r < nrows; r += 8) s += partial[(long)r * C + c];
+  if (c < C) {
+#pragma unroll 4
+    for (int r = g; r < nrows; r += 32) s += partial[(long)r * C + c];
+  }
   sh[g][cx] = s;
   __syncthreads();
   if (g == 0 && c < C) {
     float t = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) t += sh[i][cx];
+    for (int i = 0; i < 32; ++i) t += sh[i][cx];
     out[c] = t;
   }
 }
@@ -584,7 +638,7 @@ cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, cons
   LN_DISPATCH(ln_nv<T>(C), LNB)
 #undef LNB
   CUDA_TRY(cudaGetLastError());
-  colsum_kernel<<<(C + 31) / 32, 256, 0, st>>>(dg_partial, nb, C, dg);
+  colsum_kernel<<<(C + 31) / 32, 1024, 0, st>>>(dg_partial, nb, C, dg);
   return cudaGetLastError();
 }
 
