@@ -484,20 +484,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0);
       float ce_max = -INFINITY, ce_sum = 0.f;
       const int ncols = min(BN, P.N - nt * BN) - c0;
+      // the accumulator load of chunk c + 1 (and its auxiliary input) is in flight during
+      // chunk c's math and store
+      uint32_t raw[32];
+      if (ncols > 0) tmem_ld32_nw(tbase, raw);
 #pragma unroll 1
       for (int c = 0; c < EPI_COLS / 32; ++c) {
         if (c * 32 >= ncols) break;  // uniform across the warp
         const int col0 = nt * BN + c0 + c * 32;
-        float v[32];
-        uint32_t raw[32];
-        tmem_ld32_nw(tbase + (uint32_t)(c * 32), raw);
-        // the next chunk's auxiliary input is in flight during this chunk's math
-        uint4 aux_nx[4];
-        if ((EPI == TE_RESID || EPI == TE_DGELU) && (c + 1) * 32 < ncols && c + 1 < EPI_COLS / 32)
-          load_aux_chunk(P, row, col0 + 32, aux_nx);
+        const bool more = (c + 1) * 32 < ncols && c + 1 < EPI_COLS / 32;
         tmem_wait_ld32(raw);
+        float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(raw[k]);
+        if (more) tmem_ld32_nw(tbase + (uint32_t)((c + 1) * 32), raw);
+        uint4 aux_nx[4];
+        if ((EPI == TE_RESID || EPI == TE_DGELU) && more) load_aux_chunk(P, row, col0 + 32, aux_nx);
         if (EPI == TE_CE_STATS) {
           if (row < P.M) ce_stats_chunk(P, row, col0, er, v, ce_max, ce_sum);
           continue;
