@@ -161,7 +161,8 @@ enum { F_QFULL, F_K0, F_K1, F_V0, F_V1, F_KFREE0, F_KFREE1, F_VFREE0, F_VFREE1, 
 constexpr int FWD_SMEM = 5 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
-attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
+attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
+            const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sQ = smem, *sK0 = smem + TILE_BYTES, *sV0 = smem + 3 * TILE_BYTES;  // 2 stages each
@@ -327,12 +328,21 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const AttnParams P) {
 #pragma unroll
         for (int i = 0; i < 32; i += 2) pk[c * 16 + (i >> 1)] = pack_bf16(v[i] * inv, v[i + 1] * inv);
       }
-      if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.o + (size_t)(row0 + qi) * P.C + h * HD);
+      // O through shared memory (this warp's 32 rows of the Q tile, free now, 128-byte
+      // swizzle) and one TMA store; rows past T are clipped by the [B, T, C] tensor map
+      uint8_t *stg = sQ + q * 4096;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-        P.lse[((size_t)b * P.H + h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
+      for (int t = 0; t < 8; ++t)
+        *reinterpret_cast<uint4 *>(stg + lane * 128 + ((t ^ (lane & 7)) << 4)) =
+            make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0 && q0 + q * 32 < P.T) {  // (a box wholly past T is not issued)
+        tma_store_3d(&tmO, stg, h * HD, q0 + q * 32, b);
+        bulk_commit();
       }
+      if (qi < P.T) P.lse[((size_t)b * P.H + h) * P.T + qi] = (m2 + __log2f(l)) * LN2;
+      if (lane == 0) bulk_wait_read<0>();  // the staging smem must outlive the store's reads
     }
   }
   tc_fence_before();
@@ -384,7 +394,8 @@ static_assert(DQ_SMEM <= 232448, "dQ kernel shared memory");
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmO, const AttnParams P) {
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ,
+               const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sK0 = smem + 2 * DQ_QBUF;  // stage s: K at 2s, V at 2s+1 (in tiles)
@@ -397,7 +408,9 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     for (int i = 0; i < Q_NBAR; ++i) {
       uint32_t cnt = 1;
       if (i == Q_DS || i == Q_SDPFREE) cnt = ROW_WARPS;
-      if (i == Q_QFREE0 || i == Q_QFREE0 + 1) cnt = 1 + ROW_WARPS;  // last S/dP MMA + D reads
+      // the item's last S/dP MMA, then every row warp once its dQ staging (in the item's O
+      // tile) has been read by the TMA store
+      if (i == Q_QFREE0 || i == Q_QFREE0 + 1) cnt = 1 + ROW_WARPS;
       mbar_init(&bar[i], cnt);
     }
     *abort_flag = 0;
@@ -482,6 +495,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     QTile it, nx;
     bool have_it = query_item(P, 0, it);
     float lse_cur = have_it ? lse_of(it) : 0.f;
+    int pend_qb = -1;  // buffer whose dQ staging a TMA store may still be reading
     for (int i = 0; ok && have_it; ++i) {
       const bool have_nx = query_item(P, i + 1, nx);
       const float lse_nx = have_nx ? lse_of(nx) : 0.f;  // in flight during this item
@@ -505,8 +519,13 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[Q_QFREE0 + qb]);
+      // the previous item's dQ store has read its staging: that item's buffer is free
+      if (pend_qb >= 0) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[Q_QFREE0 + pend_qb]);
+        pend_qb = -1;
+      }
       if (ch == 0 && qi < P.T) P.Dbuf[((size_t)it.b * P.H + it.h) * P.T + qi] = D;
       const float lse2 = lse_cur * LOG2E;
       for (int j = 0; j < it.n; ++j, ++g) {
@@ -555,20 +574,28 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
       tc_fence_after();
       float v[32];
       tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 32, v);  // dQ columns ch*32..
-      if (qi < P.T) {
-        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(it.b * P.T + qi) * 3 * P.C +
-                                               it.h * HD + ch * 32);
+      // dQ through shared memory (this warp's 32 rows x 32 columns in the item's O tile,
+      // 64-byte swizzle) and one TMA store; rows past T are clipped by the [B, T, 3C] map
+      uint8_t *stg = smem + qb * DQ_QBUF + 2 * TILE_BYTES + (warp - 2) * 2048;
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          dst[t] = make_uint4(pack_bf16(v[8 * t] * P.scale, v[8 * t + 1] * P.scale),
-                              pack_bf16(v[8 * t + 2] * P.scale, v[8 * t + 3] * P.scale),
-                              pack_bf16(v[8 * t + 4] * P.scale, v[8 * t + 5] * P.scale),
-                              pack_bf16(v[8 * t + 6] * P.scale, v[8 * t + 7] * P.scale));
+      for (int t = 0; t < 4; ++t)
+        *reinterpret_cast<uint4 *>(stg + lane * 64 + ((t ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(pack_bf16(v[8 * t] * P.scale, v[8 * t + 1] * P.scale),
+                       pack_bf16(v[8 * t + 2] * P.scale, v[8 * t + 3] * P.scale),
+                       pack_bf16(v[8 * t + 4] * P.scale, v[8 * t + 5] * P.scale),
+                       pack_bf16(v[8 * t + 6] * P.scale, v[8 * t + 7] * P.scale));
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0 && q0 + q * 32 < P.T) {
+        tma_store_3d(&tmDQ, stg, it.h * HD + ch * 32, q0 + q * 32, it.b);
+        bulk_commit();
       }
+      pend_qb = qb;
       it = nx;
       have_it = have_nx;
       lse_cur = lse_nx;
     }
+    if (lane == 0) bulk_wait_read<0>();  // staging smem must outlive the last store's reads
   }
   tc_fence_before();
   __syncthreads();
@@ -592,7 +619,7 @@ static_assert(DKV_SMEM <= 232448, "dK/dV kernel shared memory");
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-                const AttnParams P) {
+                const __grid_constant__ CUtensorMap tmDKV, const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sKV0 = smem;                  // buffer b: K at 2b, V at 2b+1 (in tiles)
@@ -604,8 +631,14 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < K_NBAR; ++i)
-      mbar_init(&bar[i], (i == K_PS || i == K_SDPFREE) ? ROW_WARPS : 1);
+    for (int i = 0; i < K_NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == K_PS || i == K_SDPFREE) cnt = ROW_WARPS;
+      // the item's last S/dP MMA, then every row warp once its dV/dK staging (in the item's
+      // K/V buffer) has been read by the TMA store
+      if (i == K_KVFREE0 || i == K_KVFREE0 + 1) cnt = 1 + ROW_WARPS;
+      mbar_init(&bar[i], cnt);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -692,14 +725,22 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     KCursor cur;
     cur.start(P);
     float pre = cur.valid ? fetch(cur.it, 0) : 0.f;
+    int pend_kb = -1;  // buffer whose dV/dK staging a TMA store may still be reading
     for (int g = 0; cur.valid; ++g) {
       const KTile it = cur.it;
-      const int j = cur.j, k0 = it.k0, ki = k0 + r, qq0 = (it.qt0 + j) * TILE;
+      const int j = cur.j, kb = cur.i & 1, k0 = it.k0, ki = k0 + r, qq0 = (it.qt0 + j) * TILE;
       // this query tile's lse and D, into buffer g & 1; one barrier per tile (the other
       // buffer may still be read by a warp finishing the previous tile)
       float *lsd = s_lsd + (g & 1) * 2 * TILE;
       lsd[t] = pre;
       asm volatile("bar.sync 1, 256;" ::: "memory");
+      // the previous item's dV/dK store has read its staging: that K/V buffer is free
+      if (pend_kb >= 0) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[K_KVFREE0 + pend_kb]);
+        pend_kb = -1;
+      }
       KCursor nx = cur;
       nx.next(P);
       pre = nx.valid ? fetch(nx.it, nx.j) : 0.f;  // in flight during this tile
@@ -769,21 +810,30 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       if (!ok) continue;
       tc_fence_after();
       const float f = ch ? P.scale : 1.f;
-      uint32_t pk[32];
+      // through shared memory (this warp's 32 rows in the item's K/V buffer, free now,
+      // 128-byte swizzle) and one TMA store; rows past T are clipped by the [B, T, 3C] map
+      uint8_t *stg = sKV0 + kb * 2 * TILE_BYTES + (warp - 2) * 4096;
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 256 + ch * 64 + c * 32, v);
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) pk[c * 16 + (k >> 1)] = pack_bf16(v[k] * f, v[k + 1] * f);
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4 *>(stg + lane * 128 + (((4 * c + u) ^ (lane & 7)) << 4)) =
+              make_uint4(pack_bf16(v[8 * u] * f, v[8 * u + 1] * f),
+                         pack_bf16(v[8 * u + 2] * f, v[8 * u + 3] * f),
+                         pack_bf16(v[8 * u + 4] * f, v[8 * u + 5] * f),
+                         pack_bf16(v[8 * u + 6] * f, v[8 * u + 7] * f));
       }
-      if (ki < P.T) {
-        const int col = (ch ? P.C : 2 * P.C) + it.h * HD;
-        uint4 *dst = reinterpret_cast<uint4 *>(P.dqkv + (size_t)(it.b * P.T + ki) * 3 * P.C + col);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0 && k0 + q * 32 < P.T) {
+        tma_store_3d(&tmDKV, stg, (ch ? P.C : 2 * P.C) + it.h * HD, k0 + q * 32, it.b);
+        bulk_commit();
       }
+      pend_kb = kb;
     }
+    if (lane == 0) bulk_wait_read<0>();  // staging smem must outlive the last store's reads
   }
   tc_fence_before();
   __syncthreads();
@@ -826,6 +876,22 @@ bool map_rows(CUtensorMap *m, const void *base, long cols, long rows, long ld) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map over a [B, T, cols] bf16 tensor (row stride ld elements) for the epilogue TMA
+// stores: box {box_cols, 32 rows, 1}; rows t >= T of a batch are outside the map, so a store
+// of a ragged last tile is clipped at the batch boundary.
+bool map_btc(CUtensorMap *m, const void *base, long cols, long T, long B, long ld, int box_cols,
+             CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(ld * 2 * T)};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, 32u, 1u};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 AttnParams make_params(int B, int T, int C, int H, int window, unsigned *err) {
   AttnParams p;
   memset(&p, 0, sizeof(p));
@@ -864,13 +930,15 @@ bool attention_tc_supported(int C, int H) { return C / H == HD && C % H == 0 && 
 cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B, int T, int C,
                                     int H, int window, unsigned *err, cudaStream_t st) {
   CUDA_TRY(set_attrs());
-  CUtensorMap m;
-  if (!map_rows(&m, qkv, 3L * C, (long)B * T, 3L * C)) return cudaErrorInvalidValue;
+  CUtensorMap m, mo;
+  if (!map_rows(&m, qkv, 3L * C, (long)B * T, 3L * C) ||
+      !map_btc(&mo, o, C, T, B, C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   AttnParams p = make_params(B, T, C, H, window, err);
   p.o = o;
   p.lse = lse;
   const int nqt = (T + TILE - 1) / TILE;
-  attn_fwd_tc<<<B * H * nqt, 192, FWD_SMEM, st>>>(m, p);  // two CTAs per SM
+  attn_fwd_tc<<<B * H * nqt, 192, FWD_SMEM, st>>>(m, mo, p);  // two CTAs per SM
   return cudaGetLastError();
 }
 
@@ -878,10 +946,12 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
                                     const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
                                     int C, int H, int window, unsigned *err, cudaStream_t st) {
   CUDA_TRY(set_attrs());
-  CUtensorMap mq, md, mo;
+  CUtensorMap mq, md, mo, mdq, mdkv;
   if (!map_rows(&mq, qkv, 3L * C, (long)B * T, 3L * C) ||
       !map_rows(&md, dout, (long)C, (long)B * T, (long)C) ||
-      !map_rows(&mo, o, (long)C, (long)B * T, (long)C))
+      !map_rows(&mo, o, (long)C, (long)B * T, (long)C) ||
+      !map_btc(&mdq, dqkv, 3L * C, T, B, 3L * C, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map_btc(&mdkv, dqkv, 3L * C, T, B, 3L * C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   AttnParams p = make_params(B, T, C, H, window, err);
   p.O = o;
@@ -891,9 +961,9 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
   p.dqkv = dqkv;
   const int items = B * H * ((T + TILE - 1) / TILE);
   const int grid = items < attn_sms() ? items : attn_sms();  // one CTA per SM
-  attn_bwd_dq_tc<<<grid, BWD_THREADS, DQ_SMEM, st>>>(mq, md, mo, p);
+  attn_bwd_dq_tc<<<grid, BWD_THREADS, DQ_SMEM, st>>>(mq, md, mo, mdq, p);
   CUDA_TRY(cudaGetLastError());
-  attn_bwd_dkv_tc<<<grid, BWD_THREADS, DKV_SMEM, st>>>(mq, md, p);
+  attn_bwd_dkv_tc<<<grid, BWD_THREADS, DKV_SMEM, st>>>(mq, md, mdkv, p);
   return cudaGetLastError();
 }
 

@@ -133,13 +133,20 @@ def test_gpt2_124m_forward_prefixes_match_oracle(gpt2):
     assert abs(loss - math.log(wl.shape.vocab)) < 0.25
     o = oracle.Oracle.from_shape(wl.shape, dtype=np.float32)
     P = 24  # causal prefix the oracle recomputes: positions < P depend only on tokens < P
-    diffs = []
-    for b in (0, wl.B - 1):
-        _, ref = o.forward(p, tok[b:b + 1, :P], tgt[b:b + 1, :P], per_token=True)
-        diffs.append(ptl[b, :P] - ref[0])
-    d = np.concatenate(diffs)
-    # the loss tolerance bounds a mean over tokens; single tokens carry bf16 noise
-    assert abs(d.mean()) <= U.BF16_LOSS_ABS, d.mean()
+    rows = (0, wl.B - 1)
+    refs = [o.forward(p, tok[b:b + 1, :P], tgt[b:b + 1, :P], per_token=True)[1][0] for b in rows]
+    # the loss bound is about the mean over all B*T tokens: the fp32 validation path matches
+    # the oracle token by token on the prefixes, and the bf16 loss matches the fp32 loss over
+    # the full batch; single bf16 prefix tokens carry bf16 noise and are bounded directly
+    st32 = U.make_step(wl.shape, wl.B, wl.T, 0)
+    try:
+        loss32, ptl32 = U.gpu_forward(st32, p, tok, tgt)
+    finally:
+        st32.close()
+    for b, ref in zip(rows, refs):
+        assert np.abs(ptl32[b, :P] - ref).max() <= U.FP32_LOSS_ABS
+    assert abs(loss - loss32) <= U.BF16_LOSS_ABS, (loss, loss32)
+    d = np.concatenate([ptl[b, :P] - ref for b, ref in zip(rows, refs)])
     assert np.abs(d).max() <= 10 * U.BF16_LOSS_ABS, np.abs(d).max()
 
 

@@ -14,21 +14,32 @@ from tests import gpu_util as U
 pytestmark = pytest.mark.gpu
 
 
+# The bf16 loss bound is about the loss, the mean over all B*T tokens, which the oracle cannot
+# compute at these sizes. It is checked as a chain: the fp32 validation path matches the
+# oracle token by token on causal prefixes (positions < P depend only on tokens < P), and the
+# bf16 loss over the full batch matches the fp32 path. Single prefix tokens of the bf16 path
+# are also bounded against the oracle directly (they spread by ~0.01, more at early positions,
+# so a few dozen of them do not estimate the loss).
 def _full_size_checks(name, prefix=16, rows=(0,), perturb_at=200):
     wl = fx.WORKLOADS[name]
     sh = wl.shape
     p, tok, tgt = fx.make_inputs(wl)
+    o = oracle.Oracle.from_shape(sh, dtype=np.float32)
+    refs = [o.forward(p, tok[b:b + 1, :prefix], tgt[b:b + 1, :prefix], per_token=True)[1][0]
+            for b in rows]
+    st32 = U.make_step(sh, wl.B, wl.T, 0)
+    try:
+        loss32, ptl32 = U.gpu_forward(st32, p, tok, tgt)
+    finally:
+        st32.close()
+    for b, ref in zip(rows, refs):
+        assert np.abs(ptl32[b, :prefix] - ref).max() <= U.FP32_LOSS_ABS
     st = U.make_step(sh, wl.B, wl.T, 1)
     try:
         loss, ptl = U.gpu_forward(st, p, tok, tgt)
         assert abs(loss - math.log(sh.vocab)) < 0.3
-        o = oracle.Oracle.from_shape(sh, dtype=np.float32)
-        diffs = []
-        for b in rows:
-            _, ref = o.forward(p, tok[b:b + 1, :prefix], tgt[b:b + 1, :prefix], per_token=True)
-            diffs.append(ptl[b, :prefix] - ref[0])
-        d = np.concatenate(diffs)
-        assert abs(d.mean()) <= U.BF16_LOSS_ABS, d.mean()
+        assert abs(loss - loss32) <= U.BF16_LOSS_ABS, (loss, loss32)
+        d = np.concatenate([ptl[b, :prefix] - ref for b, ref in zip(rows, refs)])
         assert np.abs(d).max() <= 10 * U.BF16_LOSS_ABS, np.abs(d).max()
         # causality, bitwise
         tok2 = tok.copy()
@@ -56,8 +67,8 @@ def test_shakespeare_char_full_batch():
 
 
 def test_gpt2_350m_full_size():
-    _full_size_checks("gpt2_350m_bf16", prefix=12, rows=(5,), perturb_at=300)
+    _full_size_checks("gpt2_350m_bf16", prefix=24, rows=(5, 6), perturb_at=300)
 
 
 def test_gpt2_124m_sliding_window_full_size():
-    _full_size_checks("gpt2_124m_swa_bf16", prefix=12, rows=(7,), perturb_at=1500)
+    _full_size_checks("gpt2_124m_swa_bf16", prefix=24, rows=(6, 7), perturb_at=1500)
