@@ -167,7 +167,7 @@ def run_ours(args, wl, rank, world, local_rank):
     B, T = wl.B, wl.T
     p, tok, tgt = fx.make_inputs(wl, seed=0)
     tok, tgt = fx.zipf_tokens(sh.vocab, wl.zipf_s, B, T, seed=rank)  # own batch per replica
-    st = gb.GPTStep.from_workload(wl)
+    st = gb.GPTStep.from_workload(wl, lmhead_chunk_rows=args.lmhead_chunk_rows)
     stream = torch.cuda.Stream(device=dev)
     P = torch.from_numpy(p).to(dev)
     G = torch.zeros_like(P)
@@ -272,6 +272,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gpt2_124m_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lmhead-chunk-rows", type=int, default=0,
+                    help="rows per lm_head backward chunk (0 = the library default)")
     args = ap.parse_args()
     from gpt_transformer_step_b200 import fixtures as fx
     wl = fx.WORKLOADS[args.workload]

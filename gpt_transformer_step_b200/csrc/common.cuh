@@ -74,6 +74,15 @@ __device__ __forceinline__ float gelu_grad_fast(float x) {
   const float w = fmaf(6.f * kc, x2, 2.f * k) * x;
   return fmaf(h, fmaf(-w, h, w), h);
 }
+// gelu(x) and gelu'(x) together (one tanh): the forward stores gelu'(pre) for the backward.
+__device__ __forceinline__ float gelu_and_grad_fast(float x, float &g) {
+  const float k = 0.7978845608028654f, kc = 0.7978845608028654f * 0.044715f;
+  const float x2 = x * x;
+  const float h = fmaf(0.5f, tanh_fast(fmaf(kc, x2, k) * x), 0.5f);
+  const float w = fmaf(6.f * kc, x2, 2.f * k) * x;
+  g = fmaf(h, fmaf(-w, h, w), h);
+  return x * h;
+}
 template <typename T> __device__ __forceinline__ float gelu_t(float x) { return gelu_fast(x); }
 template <> __device__ __forceinline__ float gelu_t<float>(float x) { return gelu_f(x); }
 template <typename T> __device__ __forceinline__ float gelu_grad_t(float x) { return gelu_grad_fast(x); }
@@ -88,9 +97,9 @@ template <> __device__ __forceinline__ float exp_t<float>(float x) { return expf
 // accumulator to one of these epilogues.
 enum EpiKind {
   EPI_STORE = 0,      // out[m][n] = acc                                  (activation type)
-  EPI_STORE_GELU,     // out[m][n] = acc ; out2[m][n] = gelu(acc)         (activation type)
+  EPI_STORE_GELU,     // out[m][n] = gelu'(acc) ; out2[m][n] = gelu(acc)  (activation type)
   EPI_RESID,          // out[m][n] = aux[m][n] + acc  (aux may equal out)  (activation type)
-  EPI_DGELU,          // out[m][n] = acc * gelu'(aux[m][n])                 (activation type)
+  EPI_DGELU,          // out[m][n] = acc * aux[m][n], aux = gelu'(pre)    (activation type)
   EPI_F32_STORE,      // outf[m][n] = acc                                  (fp32)
   EPI_F32_ACCUM,      // outf[m][n] += acc                                 (fp32)
   EPI_CE_STATS,       // per (row, column tile): max and sum(exp(acc - max)) over cols < V;
@@ -132,7 +141,7 @@ __device__ __forceinline__ void epi_elem(const Epi &e, int m, int n, float acc) 
       ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(acc);
       break;
     case EPI_STORE_GELU:
-      ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(acc);
+      ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(gelu_grad_t<T>(acc));
       ((T *)e.out2)[(long)m * e.ldo2 + n] = from_f<T>(gelu_t<T>(acc));
       break;
     case EPI_RESID: {
@@ -141,8 +150,8 @@ __device__ __forceinline__ void epi_elem(const Epi &e, int m, int n, float acc) 
       break;
     }
     case EPI_DGELU: {
-      float x = to_f(((const T *)e.aux)[(long)m * e.ld_aux + n]);
-      ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(acc * gelu_grad_t<T>(x));
+      float gd = to_f(((const T *)e.aux)[(long)m * e.ld_aux + n]);
+      ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(acc * gd);
       break;
     }
     case EPI_F32_STORE:

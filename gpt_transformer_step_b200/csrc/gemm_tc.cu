@@ -256,13 +256,19 @@ __device__ __forceinline__ void epi_math(const TcParams &P, int col0, const EpiR
       v[i] = c < V ? p * er.s : 0.f;
     }
   } else if (EPI == TE_RESID || EPI == TE_DGELU) {
+    // residual: aux + acc; dGELU: acc * gelu'(pre), the derivative stored by the forward
     float a[32];
     unpack_bf16x32(aux, a);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * gelu_grad_fast(a[i]);
+    for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * a[i];
   } else if (EPI == TE_STORE_GELU) {
+    // out = gelu'(acc) (kept for the backward instead of the pre-activation), out2 = gelu(acc)
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v2[i] = gelu_fast(v[i]);
+    for (int i = 0; i < 32; ++i) {
+      float g;
+      v2[i] = gelu_and_grad_fast(v[i], g);
+      v[i] = g;
+    }
   }
 }
 
@@ -460,7 +466,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // chunk c's math and store
       uint32_t raw[32];
       if (ncols > 0) tmem_ld32_nw(tbase, raw);
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < EPI_COLS / 32; ++c) {
         if (c * 32 >= ncols) break;  // uniform across the warp
         const int col0 = nt * BN + c0 + c * 32;

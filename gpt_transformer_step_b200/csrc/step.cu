@@ -34,7 +34,7 @@ struct Layer {
 };
 
 struct Acts {  // per-layer saved activations
-  void *x_in, *a, *qkv, *o, *x_mid, *c, *pre, *h;
+  void *x_in, *a, *qkv, *o, *x_mid, *c, *dgelu, *h;  // dgelu = gelu'(pre-activation)
   float *lse, *mu1, *rs1, *mu2, *rs2;
 };
 
@@ -263,7 +263,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(launch_layernorm_fwd<T>((T *)A.x_mid, W + P.ln2, (T *)A.c, A.mu2, A.rs2, M, C,
                                      h->cfg.ln_eps, st)); nl++;
     d = gdesc(M, mC, C, A.c, C, 1, W + P.wfc, C, 1);
-    d.epi.kind = EPI_STORE_GELU; d.epi.out = A.pre; d.epi.ldo = mC; d.epi.out2 = A.h; d.epi.ldo2 = mC;
+    d.epi.kind = EPI_STORE_GELU; d.epi.out = A.dgelu; d.epi.ldo = mC; d.epi.out2 = A.h; d.epi.ldo2 = mC;
     CUDA_TRY(gemm(h, d));
     d = gdesc(M, C, mC, A.h, mC, 1, W + P.wmp, mC, 1);
     d.epi.kind = EPI_RESID; d.epi.out = xnext; d.epi.ldo = C; d.epi.aux = A.x_mid; d.epi.ld_aux = C;
@@ -319,7 +319,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     const Layer &P = h->layer[l];
     // MLP: x_out = x_mid + gelu(c Wfc^T) Wmp^T
     GemmDesc d = gdesc(M, mC, C, dx, C, 1, W + P.wmp, mC, 0);
-    d.epi.kind = EPI_DGELU; d.epi.out = h->dh; d.epi.ldo = mC; d.epi.aux = A.pre; d.epi.ld_aux = mC;
+    d.epi.kind = EPI_DGELU; d.epi.out = h->dh; d.epi.ldo = mC; d.epi.aux = A.dgelu; d.epi.ld_aux = mC;
     CUDA_TRY(gemm(h, d));
     d = gdesc(C, mC, M, dx, C, 0, A.h, mC, 0);
     d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wmp; d.epi.ldf = mC;
@@ -560,7 +560,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
     Acts &A = h->acts[l];
     need(&A.x_in, M * C * es); need(&A.a, M * C * es); need(&A.qkv, M * 3 * C * es);
     need(&A.o, M * C * es); need(&A.x_mid, M * C * es); need(&A.c, M * C * es);
-    need(&A.pre, M * h->mC * es); need(&A.h, M * h->mC * es);
+    need(&A.dgelu, M * h->mC * es); need(&A.h, M * h->mC * es);
     need((void **)&A.lse, M * H * 4); need((void **)&A.mu1, M * 4); need((void **)&A.rs1, M * 4);
     need((void **)&A.mu2, M * 4); need((void **)&A.rs2, M * 4);
   }

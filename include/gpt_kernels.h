@@ -10,9 +10,10 @@
  *   B[n][k] = B[n*ldb + k] if b_kmajor else B[k*ldb + n]     (bf16, device)
  * then epilogue `epi`:
  *   GPTK_EPI_STORE      out[m*ldo+n]  = bf16(acc)
- *   GPTK_EPI_STORE_GELU out[m*ldo+n]  = bf16(acc); out2[m*ldo2+n] = bf16(gelu_tanh(acc))
+ *   GPTK_EPI_STORE_GELU out[m*ldo+n]  = bf16(gelu_tanh'(acc)); out2[m*ldo2+n] = bf16(gelu_tanh(acc))
  *   GPTK_EPI_RESID      out[m*ldo+n]  = bf16(aux[m*ld_aux+n] + acc)
- *   GPTK_EPI_DGELU      out[m*ldo+n]  = bf16(acc * gelu_tanh'(aux[m*ld_aux+n]))
+ *   GPTK_EPI_DGELU      out[m*ldo+n]  = bf16(acc * aux[m*ld_aux+n])  (aux: the derivative the
+ *                       forward stored with GPTK_EPI_STORE_GELU)
  *   GPTK_EPI_F32_STORE  outf[m*ldf+n] = acc
  *   GPTK_EPI_F32_ACCUM  outf[m*ldf+n] += acc
  * split_k > 1 splits K into split_k ranges whose fp32 partials are summed in a fixed order

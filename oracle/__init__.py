@@ -66,6 +66,10 @@ def _load():
             f.restype = R
             f.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int] + [R] * 6 + \
                 [ctypes.c_long, P]
+            f = getattr(L, f"oracle_train_step_accum_{suf}")
+            f.restype = R
+            f.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
+                [R] * 6 + [ctypes.c_long, P]
         L.oracle_layernorm_fwd_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                                P, P, P]
         L.oracle_layernorm_bwd_f64.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int, P, P]
@@ -161,6 +165,22 @@ class Oracle:
         f = getattr(self.lib, f"oracle_train_step_{self.suf}")
         loss = f(ctypes.byref(self.cfg), _ptr(p), _ptr(g), _ptr(m), _ptr(v), _ptr(tok), _ptr(tgt),
                  B, T, lr, wd, clip, beta1, beta2, eps, step, ctypes.byref(gn))
+        return loss, g, gn.value
+
+    def train_step_accum(self, p, m, v, tokens, targets, lr, wd, clip, step, beta1=0.9,
+                         beta2=0.95, eps=1e-8):
+        """Gradient accumulation: tokens/targets [n_micro, B, T]; one optimizer step over all
+        micro-batches, in place on p, m, v. Returns (mean loss, raw mean grads, norm)."""
+        for a in (p, m, v):
+            assert a.dtype == self.dtype and a.flags.c_contiguous
+        tok = np.ascontiguousarray(tokens, np.int32)
+        tgt = np.ascontiguousarray(targets, np.int32)
+        n_micro, B, T = tok.shape
+        g = np.zeros(self.n, self.dtype)
+        gn = ctypes.c_double(0.0)
+        f = getattr(self.lib, f"oracle_train_step_accum_{self.suf}")
+        loss = f(ctypes.byref(self.cfg), _ptr(p), _ptr(g), _ptr(m), _ptr(v), _ptr(tok), _ptr(tgt),
+                 n_micro, B, T, lr, wd, clip, beta1, beta2, eps, step, ctypes.byref(gn))
         return loss, g, gn.value
 
     # -- single pieces (double) --

@@ -428,6 +428,37 @@ R train_step(const oracle_cfg *cf, R *p, R *g, R *m, R *v, const int *tok, const
   return loss;
 }
 
+// Gradient accumulation (llm.c summary, "Ejecución": the total batch of -d tokens is reached
+// with several micro-batches per optimizer step): the loss is the mean over all
+// n_micro*B*T positions, so with equal micro-batches it is the mean of the micro-batch losses
+// and its gradient the mean of the micro-batch gradients; then one clip and one AdamW update.
+// Micro-batch i holds tokens [i*B*T, (i+1)*B*T).
+template <typename R>
+R train_step_accum(const oracle_cfg *cf, R *p, R *g, R *m, R *v, const int *tok, const int *tgt,
+                   int n_micro, int B, int T, R lr, R wd, R clip, R b1, R b2, R eps, long step,
+                   double *gnorm) {
+  const Layout L = make_layout(cf);
+  std::vector<R> gi(L.total);
+  std::vector<R> dl((size_t)B * T * cf->vocab_padded);
+  for (size_t k = 0; k < L.total; ++k) g[k] = (R)0;
+  R loss = (R)0;
+  for (int i = 0; i < n_micro; ++i) {
+    Acts<R> A;
+    const int *ti = tok + (size_t)i * B * T, *gi_t = tgt + (size_t)i * B * T;
+    loss += forward(cf, p, ti, gi_t, B, T, (R *)nullptr, A, dl.data());
+    backward(cf, p, ti, B, T, A, dl.data(), gi.data());
+    for (size_t k = 0; k < L.total; ++k) g[k] += gi[k];
+  }
+  loss /= (R)n_micro;
+  for (size_t k = 0; k < L.total; ++k) g[k] /= (R)n_micro;
+  double n = grad_norm(L.total, g);
+  if (gnorm) *gnorm = n;
+  double coef = (double)clip / (n + 1e-6);
+  if (coef > 1.0) coef = 1.0;
+  adamw(L.total, p, g, m, v, lr, wd, b1, b2, eps, step, (R)coef);
+  return loss;
+}
+
 }  // namespace
 
 extern "C" {
@@ -506,6 +537,21 @@ float oracle_train_step_f32(const oracle_cfg *c, float *p, float *g, float *m, f
                             const int *tok, const int *tgt, int B, int T, float lr, float wd,
                             float clip, float b1, float b2, float eps, long step, double *gnorm) {
   return train_step<float>(c, p, g, m, v, tok, tgt, B, T, lr, wd, clip, b1, b2, eps, step, gnorm);
+}
+
+double oracle_train_step_accum_f64(const oracle_cfg *c, double *p, double *g, double *m,
+                                   double *v, const int *tok, const int *tgt, int n_micro, int B,
+                                   int T, double lr, double wd, double clip, double b1, double b2,
+                                   double eps, long step, double *gnorm) {
+  return train_step_accum<double>(c, p, g, m, v, tok, tgt, n_micro, B, T, lr, wd, clip, b1, b2,
+                                  eps, step, gnorm);
+}
+float oracle_train_step_accum_f32(const oracle_cfg *c, float *p, float *g, float *m, float *v,
+                                  const int *tok, const int *tgt, int n_micro, int B, int T,
+                                  float lr, float wd, float clip, float b1, float b2, float eps,
+                                  long step, double *gnorm) {
+  return train_step_accum<float>(c, p, g, m, v, tok, tgt, n_micro, B, T, lr, wd, clip, b1, b2,
+                                 eps, step, gnorm);
 }
 
 void oracle_layernorm_fwd_f64(const double *x, const double *g, int rows, int C, double eps,

@@ -70,6 +70,19 @@ float oracle_train_step_f32(const oracle_cfg *c, float *params, float *grads, fl
                             float wd, float clip, float beta1, float beta2, float eps, long step,
                             double *grad_norm);
 
+/* One optimizer step over n_micro micro-batches of B x T tokens (gradient accumulation; llm.c
+ * summary, "Ejecución"): loss = mean over all n_micro*B*T positions = mean of the micro-batch
+ * losses; grads = mean of the micro-batch gradients (raw); then the clip and AdamW of
+ * oracle_train_step. Micro-batch i holds tokens [i*B*T, (i+1)*B*T). */
+double oracle_train_step_accum_f64(const oracle_cfg *c, double *params, double *grads, double *m,
+                                   double *v, const int *tokens, const int *targets, int n_micro,
+                                   int B, int T, double lr, double wd, double clip, double beta1,
+                                   double beta2, double eps, long step, double *grad_norm);
+float oracle_train_step_accum_f32(const oracle_cfg *c, float *params, float *grads, float *m,
+                                  float *v, const int *tokens, const int *targets, int n_micro,
+                                  int B, int T, float lr, float wd, float clip, float beta1,
+                                  float beta2, float eps, long step, double *grad_norm);
+
 /* Single pieces, exposed for the oracle's own pins (double only). */
 void oracle_layernorm_fwd_f64(const double *x, const double *g, int rows, int C, double eps,
                               double *y, double *mean, double *rstd);

@@ -337,3 +337,51 @@ def test_window_special_cases():
         tg = np.concatenate([a.grad.transpose(1, 2).reshape(B, T, C).numpy()
                              for a in (qt, kt, vt)], -1)
         assert np.abs(o.attention_bwd(qkv, dout, H, w) - tg).max() < 1e-12, w
+
+
+# ---------------------------------------------------------------------------------------
+# gradient accumulation
+# ---------------------------------------------------------------------------------------
+
+def test_accumulated_step_equals_one_step_over_the_whole_batch():
+    """The loss of an accumulated step is the mean over all n_micro*B*T positions, so two
+    micro-batches of B=2 must give the loss, gradients and update of one B=4 step over the
+    same rows (that step is pinned to the torch float64 model above)."""
+    p, tok, tgt = tiny_inputs(seed=3, B=4)
+    sh = TINY.shape
+    o = oracle.Oracle.from_shape(sh)
+    pa, pb = p.astype(np.float64), p.astype(np.float64)
+    ma, va = np.zeros_like(pa), np.zeros_like(pa)
+    mb, vb = np.zeros_like(pb), np.zeros_like(pb)
+    la, ga, na = o.train_step_accum(pa, ma, va, tok.reshape(2, 2, -1), tgt.reshape(2, 2, -1),
+                                    TINY.lr, TINY.wd, TINY.clip, 1)
+    lb, gb, nb = o.train_step(pb, mb, vb, tok, tgt, TINY.lr, TINY.wd, TINY.clip, 1)
+    assert abs(la - lb) <= 1e-13 * abs(lb)
+    assert rel_max(ga, gb) <= 1e-12
+    assert abs(na - nb) <= 1e-12 * nb
+    for a, b in ((pa, pb), (ma, mb), (va, vb)):
+        assert np.abs(a - b).max() <= 1e-13
+
+
+def test_accumulated_step_with_one_micro_batch_is_the_plain_step():
+    p, tok, tgt = tiny_inputs(seed=4)
+    o = oracle.Oracle.from_shape(TINY.shape)
+    pa, pb = p.astype(np.float64), p.astype(np.float64)
+    za, zb = [np.zeros_like(pa) for _ in range(2)], [np.zeros_like(pb) for _ in range(2)]
+    la, ga, _ = o.train_step_accum(pa, *za, tok[None], tgt[None], TINY.lr, TINY.wd, TINY.clip, 1)
+    lb, gb, _ = o.train_step(pb, *zb, tok, tgt, TINY.lr, TINY.wd, TINY.clip, 1)
+    assert la == lb and np.array_equal(ga, gb) and np.array_equal(pa, pb)
+
+
+def test_accumulated_gradient_is_the_mean_of_micro_batch_gradients():
+    """Linearity: with unequal micro-batch contents the accumulated gradient is the plain
+    average of the per-micro-batch gradients (not their sum, not a token-weighted sum)."""
+    p, tok, tgt = tiny_inputs(seed=5, B=6)
+    o = oracle.Oracle.from_shape(TINY.shape)
+    parts = [o.forward_backward(p, tok[2 * i:2 * i + 2], tgt[2 * i:2 * i + 2]) for i in range(3)]
+    pa = p.astype(np.float64)
+    la, ga, _ = o.train_step_accum(pa, np.zeros_like(pa), np.zeros_like(pa),
+                                   tok.reshape(3, 2, -1), tgt.reshape(3, 2, -1), TINY.lr,
+                                   TINY.wd, TINY.clip, 1)
+    assert abs(la - sum(l for l, _ in parts) / 3) <= 1e-13 * abs(la)
+    assert rel_max(ga, sum(g for _, g in parts) / 3) <= 1e-13
