@@ -166,7 +166,10 @@ def run_ours(args, wl, rank, world, local_rank):
     sh = wl.shape
     B, T = wl.B, wl.T
     p, tok, tgt = fx.make_inputs(wl, seed=0)
-    tok, tgt = fx.zipf_tokens(sh.vocab, wl.zipf_s, B, T, seed=rank)  # own batch per replica
+    nm = max(1, args.micro_batches)  # micro-batches per optimizer step (gradient accumulation)
+    tok, tgt = fx.zipf_tokens(sh.vocab, wl.zipf_s, nm * B, T, seed=rank)  # own batch per replica
+    if nm > 1:
+        tok, tgt = tok.reshape(nm, B, T), tgt.reshape(nm, B, T)
     st = gb.GPTStep.from_workload(wl, lmhead_chunk_rows=args.lmhead_chunk_rows)
     stream = torch.cuda.Stream(device=dev)
     P = torch.from_numpy(p).to(dev)
@@ -183,6 +186,11 @@ def run_ours(args, wl, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    def step(a, b):
+        if nm > 1:
+            return st.train_step_accum(P, G, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
+        return st.train_step(P, G, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
+
     def timed(n, host_inputs=False):
         a, b = (tk_h, tg_h) if host_inputs else (tk, tg)
         e0 = torch.cuda.Event(enable_timing=True)
@@ -193,7 +201,7 @@ def run_ours(args, wl, rank, world, local_rank):
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(n):
-                losses.append(st.train_step(P, G, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip))
+                losses.append(step(a, b))
             e1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -203,7 +211,7 @@ def run_ours(args, wl, rank, world, local_rank):
     st.set_stream(stream.cuda_stream)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            st.train_step(P, G, Mm, Vv, tk, tg, wl.lr, wl.wd, wl.clip)
+            step(tk, tg)
     torch.cuda.synchronize()
     launches = st.last_launch_count()
 
@@ -225,7 +233,7 @@ def run_ours(args, wl, rank, world, local_rank):
     if rank != 0:
         return
     pk, pk_kind = peaks()
-    tokens = world * B * T
+    tokens = world * nm * B * T
     value = tokens / (ms / 1000)
     fpt = fx.flops_per_token(sh, T)
     fpt_lit = fx.flops_per_token(sh, T, exclude="wte+wpe")
@@ -237,7 +245,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (Zipf tokens, N(0,0.02) init)",
-        "config": {"workload": wl.name, "global_batch": world * B, "seq_len": T,
+        "config": {"workload": wl.name, "global_batch": world * nm * B, "seq_len": T,
+                   "micro_batches": nm,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "working set ~6 GB >> 126 MB L2 (no flush needed)"},
         "mfu": {"nominal_2250": value / world * fpt / 2.25e15,
@@ -246,7 +255,7 @@ def run_ours(args, wl, rank, world, local_rank):
                 "flops_per_token": fpt, "flops_per_token_literal_excl_wte": fpt_lit},
         "loss_first_timed": losses[0] if losses else None,
         "e2e": {"value": tokens / (ms_e2e / 1000), "unit": "tokens/s",
-                "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 128},
+                "h2d_bytes_per_step": 2 * nm * B * T * 4, "d2h_bytes_per_step": 128},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMMs (all launches, flop-weighted)",
                      "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": (achieved / peak_t) if achieved else None,
@@ -272,6 +281,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gpt2_124m_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--micro-batches", type=int, default=1,
+                    help="micro-batches of B x T per optimizer step (gradient accumulation)")
     ap.add_argument("--lmhead-chunk-rows", type=int, default=0,
                     help="rows per lm_head backward chunk (0 = the library default)")
     args = ap.parse_args()

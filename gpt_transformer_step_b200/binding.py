@@ -33,7 +33,8 @@ GPT_OPT_TIME_KERNELS = 2
 
 EXPORTED = [
     "gpt_create", "gpt_destroy", "gpt_num_params", "gpt_param_layout", "gpt_set_stream",
-    "gpt_forward_loss", "gpt_train_step", "gpt_get_step", "gpt_set_step", "gpt_last_grad_norm",
+    "gpt_forward_loss", "gpt_train_step", "gpt_train_step_accum", "gpt_get_step", "gpt_set_step",
+    "gpt_last_grad_norm",
     "gpt_params_changed", "gpt_set_option", "gpt_kernel_stats", "gpt_last_launch_count",
     "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
     "gptk_attention_bwd_bf16", "gptk_attention_bwd_bf16_noalloc", "gptk_selftest_bounded_wait",
@@ -80,6 +81,8 @@ gpt_set_stream = _sig("gpt_set_stream", _I, [_P, _P])
 gpt_forward_loss = _sig("gpt_forward_loss", _I, [_P, _P, _P, _P, _I, _I, ctypes.POINTER(_F), _P])
 gpt_train_step = _sig("gpt_train_step", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _F, _F, _F,
                                              ctypes.POINTER(_F)])
+gpt_train_step_accum = _sig("gpt_train_step_accum", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
+                                                         _F, _F, _F, ctypes.POINTER(_F)])
 gpt_get_step = _sig("gpt_get_step", _I, [_P, ctypes.POINTER(ctypes.c_long)])
 gpt_set_step = _sig("gpt_set_step", _I, [_P, ctypes.c_long])
 gpt_last_grad_norm = _sig("gpt_last_grad_norm", _F, [_P])
@@ -196,6 +199,16 @@ class GPTStep:
         s = gpt_train_step(self.h, _ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v),
                            _ptr(tokens), _ptr(targets), B, T, lr, wd, clip, ctypes.byref(loss))
         self._check(s, "gpt_train_step")
+        return loss.value
+
+    def train_step_accum(self, params, grads, adam_m, adam_v, tokens, targets, lr, wd, clip):
+        """One optimizer step over micro-batches: tokens/targets [n_micro, B, T] int32."""
+        n_micro, B, T = tokens.shape
+        loss = ctypes.c_float(0)
+        s = gpt_train_step_accum(self.h, _ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v),
+                                 _ptr(tokens), _ptr(targets), n_micro, B, T, lr, wd, clip,
+                                 ctypes.byref(loss))
+        self._check(s, "gpt_train_step_accum")
         return loss.value
 
     def train_step_status(self, params, grads, adam_m, adam_v, tokens, targets, lr, wd, clip):

@@ -17,17 +17,18 @@ struct DevScalars {
   // written by the host before each step
   float lr, wd, clip, beta1, beta2, eps;
   float bias1, bias2;  // 1 - beta^t, computed on the host in double
-  float inv_M;         // 1 / (B*T)
+  float inv_M;         // 1 / (positions in the optimizer step: n_micro * B * T)
   int step;
   int pad0[6];
   // written by the device
   double sumsq;        // sum of squared raw grads
   float norm, coef;    // global grad norm, clip coefficient
-  float loss;          // mean loss
-  int nonfinite;       // loss or norm not finite: the update is skipped
+  float loss;          // mean loss of the last micro-batch
+  float loss_sum;      // sum of the micro-batch mean losses of this optimizer step
+  int nonfinite;       // a loss or the norm not finite: the update is skipped
   unsigned err;        // GPT_DEVERR_* bits
   unsigned counter;    // arrival counter of the grad-norm last-block reduction
-  int pad1[8];
+  int pad1[7];
 };
 
 // ---- type helpers -----------------------------------------------------------------------

@@ -8,26 +8,29 @@ template <typename T>
 cudaError_t launch_embed_fwd(const int *tok, const int *tgt, const T *wte, const T *wpe, T *x,
                              int M, int Tlen, int C, int V, DevScalars *sc, cudaStream_t st);
 
-// K13: dwpe[t] = sum_b dx[b,t] (rows t >= T zeroed); dwte[id] += sum over positions with
-// that id, in position order (deterministic). dwte already holds the lm_head part.
+// K13: dwpe[t] = sum_b dx[b,t] (rows t >= T zeroed; added to dwpe when accumulate); dwte[id]
+// += sum over positions with that id, in position order (deterministic). dwte already holds
+// the lm_head part.
 struct EmbedBwdWs {
   unsigned *keys;      // [M] sorted (id << 14 | m)
   float *partial;      // [nwin][2][C]
 };
 template <typename T>
 cudaError_t launch_embed_bwd(const int *tok, const T *dx, float *dwte, float *dwpe, int M,
-                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st);
+                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st,
+                             bool accumulate = false);
 
 // K2: y = (x - mean) * rstd * g, one warp per row.
 template <typename T>
 cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
                                  int C, float eps, cudaStream_t st);
 
-// K12: dres += LN_backward(dy); dgamma partial sums per block -> dg (fp32) after reduce.
+// K12: dres += LN_backward(dy); dgamma partial sums per block -> dg (fp32) after reduce
+// (added to dg when accumulate).
 template <typename T>
 cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
                                  const T *dy, T *dres, float *dg_partial, float *dg, int M,
-                                 int C, cudaStream_t st);
+                                 int C, cudaStream_t st, bool accumulate = false);
 int layernorm_bwd_blocks(int M);
 
 // Cross-entropy: per-row lse and loss from the per-tile stats; mean loss into sc->loss.

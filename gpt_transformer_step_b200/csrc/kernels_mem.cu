@@ -269,7 +269,8 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
 // g, g+32, ... in order (four loads in flight), then the 32 group sums are added in group
 // order (deterministic).
 __global__ void __launch_bounds__(1024) colsum_kernel(const float *__restrict__ partial, int nrows,
-                                                      int C, float *__restrict__ out) {
+                                                      int C, float *__restrict__ out,
+                                                      int accumulate) {
   __shared__ float sh[32][33];
   const int cx = threadIdx.x & 31, g = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + cx;
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(1024) colsum_kernel(const float *__restrict__ 
     float t = 0.f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) t += sh[i][cx];
-    out[c] = t;
+    out[c] = accumulate ? out[c] + t : t;
   }
 }
 
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(1024) colsum_kernel(const float *__restrict__ 
 // ------------------------------------------------------------------------------------------
 template <typename T>
 __global__ void dwpe_kernel(const T *__restrict__ dx, float *__restrict__ dwpe, int Bn,
-                            int Tlen, int maxT, int C) {
+                            int Tlen, int maxT, int C, int accumulate) {
   long total = (long)maxT * C;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
        i += (long)gridDim.x * blockDim.x) {
@@ -301,7 +302,7 @@ __global__ void dwpe_kernel(const T *__restrict__ dx, float *__restrict__ dwpe, 
     float s = 0.f;
     if (t < Tlen)
       for (int b = 0; b < Bn; ++b) s += to_f(dx[((long)b * Tlen + t) * C + c]);
-    dwpe[i] = s;
+    dwpe[i] = accumulate ? dwpe[i] + s : s;
   }
 }
 
@@ -439,7 +440,8 @@ __global__ void mean_loss_kernel(const float *__restrict__ per_token, int M, Dev
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh[w];
     float loss = (float)(t / (double)M);
     sc->loss = loss;
-    sc->nonfinite = isfinite(loss) ? 0 : 1;
+    sc->loss_sum += loss;  // cleared with the other device results at the first micro-batch
+    if (!isfinite(loss)) sc->nonfinite = 1;
   }
 }
 
@@ -573,9 +575,11 @@ cudaError_t launch_embed_fwd(const int *tok, const int *tgt, const T *wte, const
 
 template <typename T>
 cudaError_t launch_embed_bwd(const int *tok, const T *dx, float *dwte, float *dwpe, int M,
-                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st) {
+                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st,
+                             bool accumulate) {
   const int Bn = M / Tlen;
-  dwpe_kernel<T><<<grid_for((long)maxT * C, 256), 256, 0, st>>>(dx, dwpe, Bn, Tlen, maxT, C);
+  dwpe_kernel<T><<<grid_for((long)maxT * C, 256), 256, 0, st>>>(dx, dwpe, Bn, Tlen, maxT, C,
+                                                                accumulate ? 1 : 0);
   CUDA_TRY(cudaGetLastError());
   int n = 1;
   while (n < M) n <<= 1;
@@ -628,7 +632,7 @@ int layernorm_bwd_blocks(int M) {
 template <typename T>
 cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
                                  const T *dy, T *dres, float *dg_partial, float *dg, int M,
-                                 int C, cudaStream_t st) {
+                                 int C, cudaStream_t st, bool accumulate) {
   const int nb = layernorm_bwd_blocks(M);
   const int rpb = (M + nb - 1) / nb;
   const size_t smem = (size_t)LNB_WARPS * C * sizeof(float);
@@ -638,7 +642,7 @@ cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, cons
   LN_DISPATCH(ln_nv<T>(C), LNB)
 #undef LNB
   CUDA_TRY(cudaGetLastError());
-  colsum_kernel<<<(C + 31) / 32, 1024, 0, st>>>(dg_partial, nb, C, dg);
+  colsum_kernel<<<(C + 31) / 32, 1024, 0, st>>>(dg_partial, nb, C, dg, accumulate ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -674,11 +678,11 @@ cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st)
   template cudaError_t launch_embed_fwd<T>(const int *, const int *, const T *, const T *, T *, \
                                            int, int, int, int, DevScalars *, cudaStream_t);    \
   template cudaError_t launch_embed_bwd<T>(const int *, const T *, float *, float *, int, int,  \
-                                           int, int, EmbedBwdWs, cudaStream_t);                \
+                                           int, int, EmbedBwdWs, cudaStream_t, bool);          \
   template cudaError_t launch_layernorm_fwd<T>(const T *, const T *, T *, float *, float *, int, \
                                                int, float, cudaStream_t);                      \
   template cudaError_t launch_layernorm_bwd<T>(const T *, const T *, const float *,             \
                                                const float *, const T *, T *, float *, float *, \
-                                               int, int, cudaStream_t);
+                                               int, int, cudaStream_t, bool);
 INST(float)
 INST(bf16)

@@ -38,12 +38,16 @@ struct Acts {  // per-layer saved activations
   float *lse, *mu1, *rs1, *mu2, *rs2;
 };
 
+// Phases of a training call: a whole step, or the first / a middle / the last micro-batch of
+// a gradient-accumulated step (gradients stored, accumulated, accumulated + update).
+enum StepPhase { PH_STEP = 0, PH_FIRST = 1, PH_MIDDLE = 2, PH_LAST = 3 };
+
 struct GraphKey {
-  int B, T, train;
+  int B, T, train, phase;
   const void *p, *g, *m, *v, *ptl;
   bool operator<(const GraphKey &o) const {
-    return std::tie(B, T, train, p, g, m, v, ptl) <
-           std::tie(o.B, o.T, o.train, o.p, o.g, o.m, o.v, o.ptl);
+    return std::tie(B, T, train, phase, p, g, m, v, ptl) <
+           std::tie(o.B, o.T, o.train, o.phase, o.p, o.g, o.m, o.v, o.ptl);
   }
 };
 
@@ -235,7 +239,8 @@ cudaError_t attention_bwd<bf16>(gpt_handle *h, const bf16 *qkv, const bf16 *o, c
 // --------------------------------------------------------------------------------------
 template <typename T>
 cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *adam_m,
-                    float *adam_v, int B, int Tlen, bool train, float *per_token_out) {
+                    float *adam_v, int B, int Tlen, bool train, float *per_token_out,
+                    int phase) {
   cudaStream_t st = h->stream;
   const int C = h->C, H = h->H, mC = h->mC, V = h->V, M = B * Tlen;
   const T *W = h->use_bf16 ? (const T *)h->shadow : (const T *)params;
@@ -289,8 +294,11 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   if (!train) return cudaSuccess;
 
   // ---------------- backward ----------------
+  // after the first micro-batch of an accumulated step every gradient write adds
+  const bool acc = phase == PH_MIDDLE || phase == PH_LAST;
+  const int wgrad = acc ? EPI_F32_ACCUM : EPI_F32_STORE;
   float *G = grads;
-  CUDA_TRY(cudaMemsetAsync(G + h->off_wte, 0, sizeof(float) * (size_t)h->Vp * C, st));
+  if (!acc) CUDA_TRY(cudaMemsetAsync(G + h->off_wte, 0, sizeof(float) * (size_t)h->Vp * C, st));
   for (int r0 = 0; r0 < M; r0 += h->chunk_rows) {
     const int R = M - r0 < h->chunk_rows ? M - r0 : h->chunk_rows;
     const T *yf_c = (const T *)h->yf + (size_t)r0 * C;
@@ -313,7 +321,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   T *dx = (T *)h->dx;
   CUDA_TRY(cudaMemsetAsync(dx, 0, sizeof(T) * (size_t)M * C, st));
   CUDA_TRY(launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf,
-                                   dx, h->dg_partial, G + h->off_lnf, M, C, st)); nl += 2;
+                                   dx, h->dg_partial, G + h->off_lnf, M, C, st, acc)); nl += 2;
   for (int l = h->L - 1; l >= 0; --l) {
     Acts &A = h->acts[l];
     const Layer &P = h->layer[l];
@@ -322,22 +330,22 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d.epi.kind = EPI_DGELU; d.epi.out = h->dh; d.epi.ldo = mC; d.epi.aux = A.dgelu; d.epi.ld_aux = mC;
     CUDA_TRY(gemm(h, d));
     d = gdesc(C, mC, M, dx, C, 0, A.h, mC, 0);
-    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wmp; d.epi.ldf = mC;
+    d.epi.kind = wgrad; d.epi.outf = G + P.wmp; d.epi.ldf = mC;
     CUDA_TRY(gemm(h, d));
     d = gdesc(M, C, mC, h->dh, mC, 1, W + P.wfc, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
     d = gdesc(mC, C, M, h->dh, mC, 0, A.c, C, 0);
-    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wfc; d.epi.ldf = C;
+    d.epi.kind = wgrad; d.epi.outf = G + P.wfc; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
     CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx,
-                                     h->dg_partial, G + P.ln2, M, C, st)); nl += 2;
+                                     h->dg_partial, G + P.ln2, M, C, st, acc)); nl += 2;
     // attention: x_mid = x_in + attn(a) Wap^T
     d = gdesc(M, C, C, dx, C, 1, W + P.wap, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dout; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
     d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
-    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wap; d.epi.ldf = C;
+    d.epi.kind = wgrad; d.epi.outf = G + P.wap; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
     CUDA_TRY(attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B,
                               Tlen, h->windows[l])); nl += 2;
@@ -345,14 +353,15 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
     d = gdesc(3 * C, C, M, h->dqkv, 3 * C, 0, A.a, C, 0);
-    d.epi.kind = EPI_F32_STORE; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
+    d.epi.kind = wgrad; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
     CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
-                                     h->dg_partial, G + P.ln1, M, C, st)); nl += 2;
+                                     h->dg_partial, G + P.ln1, M, C, st, acc)); nl += 2;
   }
   EmbedBwdWs ew{h->sort_keys, h->emb_partial};
   CUDA_TRY(launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C,
-                               ew, st)); nl += 4;
+                               ew, st, acc)); nl += 4;
+  if (phase == PH_FIRST || phase == PH_MIDDLE) return cudaSuccess;  // update after the last
   // ---------------- clip + AdamW ----------------
   CUDA_TRY(launch_grad_norm(G, h->nparams, h->gn_partials, sc, st)); nl++;
   CUDA_TRY(launch_adamw((float *)params, G, adam_m, adam_v, h->use_bf16 ? h->shadow : nullptr,
@@ -361,9 +370,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
 }
 
 cudaError_t run(gpt_handle *h, const float *params, float *grads, float *m, float *v, int B,
-                int Tlen, bool train, float *ptl) {
-  if (h->use_bf16) return enqueue<bf16>(h, params, grads, m, v, B, Tlen, train, ptl);
-  return enqueue<float>(h, params, grads, m, v, B, Tlen, train, ptl);
+                int Tlen, bool train, float *ptl, int phase = PH_STEP) {
+  if (h->use_bf16) return enqueue<bf16>(h, params, grads, m, v, B, Tlen, train, ptl, phase);
+  return enqueue<float>(h, params, grads, m, v, B, Tlen, train, ptl, phase);
 }
 
 int check_common(gpt_handle *h, const void *params, const int *tokens, const int *targets, int B,
@@ -375,8 +384,9 @@ int check_common(gpt_handle *h, const void *params, const int *tokens, const int
 }
 
 // Copies tokens/targets (host or device) into the workspace and the hyper-parameters into
-// device scalars.
-int stage_inputs(gpt_handle *h, const int *tokens, const int *targets, int M) {
+// device scalars; clear: also zero the device-written results (loss sum, flags, error word),
+// done once per optimizer step (at its first micro-batch).
+int stage_inputs(gpt_handle *h, const int *tokens, const int *targets, int M, bool clear = true) {
   const cudaMemcpyKind kt = is_device_ptr(tokens) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
   const cudaMemcpyKind kg = is_device_ptr(targets) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
   TRY(cudaMemcpyAsync(h->tok, tokens, sizeof(int) * M, kt, h->stream));
@@ -384,25 +394,26 @@ int stage_inputs(gpt_handle *h, const int *tokens, const int *targets, int M) {
   TRY(cudaMemcpyAsync(h->sc, h->sc_host, offsetof(DevScalars, sumsq), cudaMemcpyHostToDevice,
                       h->stream));
   // the device-written results of the previous call are cleared
-  TRY(cudaMemsetAsync((char *)h->sc + offsetof(DevScalars, loss), 0,
-                      offsetof(DevScalars, counter) - offsetof(DevScalars, loss), h->stream));
+  if (clear)
+    TRY(cudaMemsetAsync((char *)h->sc + offsetof(DevScalars, loss), 0,
+                        offsetof(DevScalars, counter) - offsetof(DevScalars, loss), h->stream));
   return GPT_OK;
 }
 
 int launch_step(gpt_handle *h, const float *params, float *grads, float *m, float *v, int B,
-                int Tlen, bool train, float *ptl) {
+                int Tlen, bool train, float *ptl, int phase = PH_STEP) {
   h->launches = 0;
   const bool capture_ok = h->use_graphs && h->stream != nullptr && !h->time_kernels;
   if (!capture_ok) {
-    TRY(run(h, params, grads, m, v, B, Tlen, train, ptl));
+    TRY(run(h, params, grads, m, v, B, Tlen, train, ptl, phase));
     return GPT_OK;
   }
-  GraphKey key{B, Tlen, train ? 1 : 0, params, grads, m, v, ptl};
+  GraphKey key{B, Tlen, train ? 1 : 0, phase, params, grads, m, v, ptl};
   auto it = h->graphs.find(key);
   if (it == h->graphs.end()) {
     cudaGraph_t g;
     TRY(cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
-    cudaError_t e = run(h, params, grads, m, v, B, Tlen, train, ptl);
+    cudaError_t e = run(h, params, grads, m, v, B, Tlen, train, ptl, phase);
     cudaError_t e2 = cudaStreamEndCapture(h->stream, &g);
     if (e != cudaSuccess) return fail(h, e);
     if (e2 != cudaSuccess) return fail(h, e2);
@@ -417,10 +428,10 @@ int launch_step(gpt_handle *h, const float *params, float *grads, float *m, floa
   return GPT_OK;
 }
 
-int finish(gpt_handle *h, float *loss) {
+int finish(gpt_handle *h, float *loss, int n_micro = 1) {
   TRY(cudaMemcpyAsync(h->sc_host, h->sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, h->stream));
   TRY(cudaStreamSynchronize(h->stream));
-  if (loss) *loss = h->sc_host->loss;
+  if (loss) *loss = n_micro == 1 ? h->sc_host->loss : h->sc_host->loss_sum / (float)n_micro;
   if (h->time_kernels) {
     for (int k = 0; k + 1 < h->ev_used; k += 2) {
       float ms = 0.f;
@@ -437,7 +448,8 @@ int finish(gpt_handle *h, float *loss) {
   return GPT_OK;
 }
 
-void set_hyper(gpt_handle *h, int M, float lr, float wd, float clip, long t) {
+// M: positions whose mean loss the step optimises (n_micro * B * T).
+void set_hyper(gpt_handle *h, long M, float lr, float wd, float clip, long t) {
   DevScalars *s = h->sc_host;
   s->lr = lr; s->wd = wd; s->clip = clip;
   s->beta1 = h->cfg.beta1; s->beta2 = h->cfg.beta2; s->eps = h->cfg.adam_eps;
@@ -672,23 +684,36 @@ int gpt_forward_loss(gpt_handle *h, const float *params, const int *tokens, cons
 int gpt_train_step(gpt_handle *h, float *params, float *grads, float *adam_m, float *adam_v,
                    const int *tokens, const int *targets, int B, int T, float lr, float wd,
                    float clip, float *loss) {
+  return gpt_train_step_accum(h, params, grads, adam_m, adam_v, tokens, targets, 1, B, T, lr, wd,
+                              clip, loss);
+}
+
+int gpt_train_step_accum(gpt_handle *h, float *params, float *grads, float *adam_m,
+                         float *adam_v, const int *tokens, const int *targets, int n_micro,
+                         int B, int T, float lr, float wd, float clip, float *loss) {
   int s = check_common(h, params, tokens, targets, B, T);
   if (s) return s;
-  if (!grads || !adam_m || !adam_v || !loss) return GPT_ERR_INVALID_ARG;
+  if (!grads || !adam_m || !adam_v || !loss || n_micro < 1) return GPT_ERR_INVALID_ARG;
   if (misaligned(grads) || misaligned(adam_m) || misaligned(adam_v)) return GPT_ERR_ALIGN;
   if (!isfinite(lr) || !isfinite(wd) || !(clip > 0.f)) return GPT_ERR_INVALID_ARG;
   cudaSetDevice(h->device);
   const int M = B * T;
   const long t = h->step + 1;
-  set_hyper(h, M, lr, wd, clip, t);
-  if ((s = stage_inputs(h, tokens, targets, M))) return s;
+  set_hyper(h, (long)n_micro * M, lr, wd, clip, t);
   if (h->use_bf16 && (!h->shadow_valid || h->shadow_src != params)) {
     TRY(launch_to_bf16(params, h->shadow, h->nparams, h->stream));
     h->shadow_src = params;
     h->shadow_valid = true;
   }
-  if ((s = launch_step(h, params, grads, adam_m, adam_v, B, T, true, nullptr))) return s;
-  s = finish(h, loss);
+  int launches = 0;
+  for (int i = 0; i < n_micro; ++i) {
+    const int phase = n_micro == 1 ? PH_STEP : i == 0 ? PH_FIRST : i + 1 < n_micro ? PH_MIDDLE : PH_LAST;
+    if ((s = stage_inputs(h, tokens + (size_t)i * M, targets + (size_t)i * M, M, i == 0))) return s;
+    if ((s = launch_step(h, params, grads, adam_m, adam_v, B, T, true, nullptr, phase))) return s;
+    launches += h->launches;
+  }
+  h->launches = launches;
+  s = finish(h, loss, n_micro);
   h->last_norm = h->sc_host->norm;
   if (s) return s;
   if (h->sc_host->nonfinite) return GPT_ERR_NONFINITE;

@@ -111,6 +111,19 @@ int gpt_train_step(gpt_handle *h, float *params, float *grads, float *adam_m, fl
                    const int *tokens, const int *targets, int B, int T, float lr, float wd,
                    float clip, float *loss);
 
+/* Gradient accumulation (llm.c summary, "Ejecución": a total batch of -d tokens reached with
+ * several micro-batches per optimizer step): one optimizer step over n_micro >= 1 micro-batches
+ * of B x T tokens. tokens/targets hold n_micro*B*T ids (device or host), micro-batch i at
+ * offset i*B*T. The loss is the mean over all n_micro*B*T positions (with equal micro-batches,
+ * the mean of the micro-batch losses); grads (RAW, written) are its gradient, the mean of the
+ * micro-batch gradients, accumulated in fp32 in the grads buffer; then one clip and one AdamW
+ * update exactly as in gpt_train_step, which is this call with n_micro = 1. Peak memory is that
+ * of one micro-batch. Errors and GPT_ERR_NONFINITE (any micro-batch's loss or the norm) as in
+ * gpt_train_step. */
+int gpt_train_step_accum(gpt_handle *h, float *params, float *grads, float *adam_m,
+                         float *adam_v, const int *tokens, const int *targets, int n_micro,
+                         int B, int T, float lr, float wd, float clip, float *loss);
+
 /* Step counter (number of completed AdamW updates); gpt_set_step is for resuming. */
 int gpt_get_step(const gpt_handle *h, long *step);
 int gpt_set_step(gpt_handle *h, long step);
