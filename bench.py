@@ -31,7 +31,7 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 # DRAM bytes (read + write) per tcgen05 GEMM launch, mean over all GEMM launches of the step,
 # from the ncu launch list in profiles/step_gpt2_124m_launch_list.md (same kernel version).
-GEMM_DRAM_BYTES_PER_LAUNCH = {"gpt2_124m_bf16": 204.75e6}
+GEMM_DRAM_BYTES_PER_LAUNCH = {"gpt2_124m_bf16": 204.31e6}
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
