@@ -25,12 +25,14 @@ template <typename T>
 cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
                                  int C, float eps, cudaStream_t st);
 
-// K12: dres += LN_backward(dy); dgamma partial sums per block -> dg (fp32) after reduce
-// (added to dg when accumulate).
+// K12: dres += LN_backward(dy) (dres = LN_backward(dy) when !dres_in: the incoming residual
+// gradient is zero and dres is not read); dgamma partial sums per block -> dg (fp32) after
+// reduce (added to dg when accumulate).
 template <typename T>
 cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
                                  const T *dy, T *dres, float *dg_partial, float *dg, int M,
-                                 int C, cudaStream_t st, bool accumulate = false);
+                                 int C, cudaStream_t st, bool accumulate = false,
+                                 bool dres_in = true);
 int layernorm_bwd_blocks(int M);
 
 // Cross-entropy: per-row lse and loss from the per-tile stats; mean loss into sc->loss.

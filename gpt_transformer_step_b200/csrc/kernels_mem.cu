@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(LNB_WARPS * 32, 2)
 layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
                      const float *__restrict__ mean, const float *__restrict__ rstd,
                      const T *__restrict__ dy, T *__restrict__ dres,
-                     float *__restrict__ dg_partial, int M, int C, int rows_per_block) {
+                     float *__restrict__ dg_partial, int M, int C, int rows_per_block,
+                     int res_in) {
   using VT = typename Vec<T>::type;
   constexpr int VN = Vec<T>::N;
   extern __shared__ float sm_dg[];  // [LNB_WARPS][C]
@@ -194,7 +195,8 @@ layernorm_bwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
         const long off = (long)row * C + (lane + 32 * j) * VN;
         xa[j] = *reinterpret_cast<const VT *>(x + off);
         da[j] = *reinterpret_cast<const VT *>(dy + off);
-        ra[j] = *reinterpret_cast<const VT *>(dres + off);
+        if (res_in) ra[j] = *reinterpret_cast<const VT *>(dres + off);
+        else ra[j] = VT{};  // dres starts at zero: written, not accumulated
       }
     }
   };
@@ -632,13 +634,14 @@ int layernorm_bwd_blocks(int M) {
 template <typename T>
 cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
                                  const T *dy, T *dres, float *dg_partial, float *dg, int M,
-                                 int C, cudaStream_t st, bool accumulate) {
+                                 int C, cudaStream_t st, bool accumulate, bool dres_in) {
   const int nb = layernorm_bwd_blocks(M);
   const int rpb = (M + nb - 1) / nb;
   const size_t smem = (size_t)LNB_WARPS * C * sizeof(float);
 #define LNB(NVC)                                                                              \
   layernorm_bwd_kernel<T, NVC><<<nb, LNB_WARPS * 32, smem, st>>>(x, g, mean, rstd, dy, dres, \
-                                                                 dg_partial, M, C, rpb)
+                                                                 dg_partial, M, C, rpb,     \
+                                                                 dres_in ? 1 : 0)
   LN_DISPATCH(ln_nv<T>(C), LNB)
 #undef LNB
   CUDA_TRY(cudaGetLastError());
@@ -683,6 +686,6 @@ cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st)
                                                int, float, cudaStream_t);                      \
   template cudaError_t launch_layernorm_bwd<T>(const T *, const T *, const float *,             \
                                                const float *, const T *, T *, float *, float *, \
-                                               int, int, cudaStream_t, bool);
+                                               int, int, cudaStream_t, bool, bool);
 INST(float)
 INST(bf16)

@@ -298,7 +298,10 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   const bool acc = phase == PH_MIDDLE || phase == PH_LAST;
   const int wgrad = acc ? EPI_F32_ACCUM : EPI_F32_STORE;
   float *G = grads;
-  if (!acc) CUDA_TRY(cudaMemsetAsync(G + h->off_wte, 0, sizeof(float) * (size_t)h->Vp * C, st));
+  // dwte: the first lm_head chunk stores (unless accumulating), later chunks and the embedding
+  // backward add; the padding rows V..Vp-1 are never written by the GEMMs and are zeroed
+  if (!acc && h->Vp > V)
+    CUDA_TRY(cudaMemsetAsync(G + h->off_wte + (size_t)V * C, 0, sizeof(float) * (size_t)(h->Vp - V) * C, st));
   for (int r0 = 0; r0 < M; r0 += h->chunk_rows) {
     const int R = M - r0 < h->chunk_rows ? M - r0 : h->chunk_rows;
     const T *yf_c = (const T *)h->yf + (size_t)r0 * C;
@@ -312,16 +315,15 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d = gdesc(R, C, V, h->dS, h->ldS, 1, W + h->off_wte, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = (T *)h->dyf + (size_t)r0 * C; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
-    // dwte += dS^T . yf
+    // dwte (+)= dS^T . yf
     d = gdesc(V, C, R, h->dS, h->ldS, 0, yf_c, C, 0);
-    d.epi.kind = EPI_F32_ACCUM; d.epi.outf = G + h->off_wte; d.epi.ldf = C;
+    d.epi.kind = (acc || r0 > 0) ? EPI_F32_ACCUM : EPI_F32_STORE; d.epi.outf = G + h->off_wte; d.epi.ldf = C;
     d.split_k = 1;
     CUDA_TRY(gemm(h, d));
   }
-  T *dx = (T *)h->dx;
-  CUDA_TRY(cudaMemsetAsync(dx, 0, sizeof(T) * (size_t)M * C, st));
+  T *dx = (T *)h->dx;  // the residual-stream gradient starts here (nothing to add to)
   CUDA_TRY(launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf,
-                                   dx, h->dg_partial, G + h->off_lnf, M, C, st, acc)); nl += 2;
+                                   dx, h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
   for (int l = h->L - 1; l >= 0; --l) {
     Acts &A = h->acts[l];
     const Layer &P = h->layer[l];
