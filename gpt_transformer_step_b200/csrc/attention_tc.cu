@@ -18,6 +18,8 @@
 // No atomics: every output element is written by exactly one work item, so results are bitwise
 // reproducible. Tiles entirely outside the causal/window band are skipped; edge tiles are
 // masked element by element. Every wait is bounded (device error word on timeout).
+#include <type_traits>
+
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
 
@@ -541,20 +543,26 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         const int hi = qi < P.T ? qi - k0 - ch * 64 : -1;  // admitted local columns: lo..hi
         const int lo = w >= 0 ? qi - w - k0 - ch * 64 : -1;
         uint32_t pk[32];
+        // two copies of the loop: interior tiles carry no per-element mask
+        auto ds_math = [&](auto masked) {
+          constexpr bool MASK = decltype(masked)::value;
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float sa = __uint_as_float(k < 32 ? s0[k] : s1[k - 32]);
-          const float sb = __uint_as_float(k < 32 ? s0[k + 1] : s1[k - 31]);
-          const float da = __uint_as_float(k < 32 ? d0[k] : d1[k - 32]);
-          const float db = __uint_as_float(k < 32 ? d0[k + 1] : d1[k - 31]);
-          float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
-          float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
-          if (!interior) {
-            x0 = (k <= hi && k >= lo) ? x0 : 0.f;
-            x1 = (k + 1 <= hi && k + 1 >= lo) ? x1 : 0.f;
+          for (int k = 0; k < 64; k += 2) {
+            const float sa = __uint_as_float(k < 32 ? s0[k] : s1[k - 32]);
+            const float sb = __uint_as_float(k < 32 ? s0[k + 1] : s1[k - 31]);
+            const float da = __uint_as_float(k < 32 ? d0[k] : d1[k - 32]);
+            const float db = __uint_as_float(k < 32 ? d0[k + 1] : d1[k - 31]);
+            float x0 = ex2(fmaf(sa, P.scale_log2, -lse2)) * (da - D);
+            float x1 = ex2(fmaf(sb, P.scale_log2, -lse2)) * (db - D);
+            if (MASK) {
+              x0 = (k <= hi && k >= lo) ? x0 : 0.f;
+              x1 = (k + 1 <= hi && k + 1 >= lo) ? x1 : 0.f;
+            }
+            pk[k >> 1] = pack_bf16(x0, x1);
           }
-          pk[k >> 1] = pack_bf16(x0, x1);
-        }
+        };
+        if (interior) ds_math(std::false_type{});
+        else ds_math(std::true_type{});
         // dS is free once the previous dQ MMA is done (for j == 0 the epilogue waited)
         if (j > 0 && !warp_wait(&bar[Q_MM2], (g - 1) & 1, abort_flag, P.err)) { ok = false; break; }
         {
@@ -768,6 +776,9 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         if (!ok) continue;
       }
       const uint32_t tPT = tmem + ((uint32_t)(q * 32) << 16) + 384 + ch * 32, tdST = tPT + 64;
+      // two copies of the loop: interior tiles carry no per-element mask
+      auto pds_math = [&](auto masked) {
+      constexpr bool MASK = decltype(masked)::value;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // 32 columns -> 16 packed TMEM columns each
         uint32_t pp[16], pd[16];
@@ -785,7 +796,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
               const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
               const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
               float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
-              if (!interior) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
+              if (MASK) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
               pr[e] = pv;
               dr[e] = pv * (dpv - dv[e]);
             }
@@ -799,6 +810,9 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         tmem_st16_nw(tPT + 16 * half, pp);
         tmem_st16_nw(tdST + 16 * half, pd);
       }
+      };
+      if (interior) pds_math(std::false_type{});
+      else pds_math(std::true_type{});
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
