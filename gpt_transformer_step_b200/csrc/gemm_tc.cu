@@ -14,9 +14,11 @@
 //               (128x256 per CTA, or 256x256 per CTA pair with cta_group::2);
 //               tcgen05.commit frees the stage; a second commit marks the accumulator full
 //   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (one row per thread, two warps
-//               per TMEM lane quarter, 128 columns each), the fused epilogue, global stores
-// Tiles of 256 rows run on CTA pairs whenever they fill the machine (the pair halves each
-// SM's shared-memory traffic per MMA); small-M GEMMs keep single-CTA 128-row tiles.
+//               per TMEM lane quarter, 128 columns each), the fused epilogue, staging in
+//               swizzled shared memory and TMA tensor stores (fp32 accumulate: TMA reduce-add)
+// The launcher picks CTA pairs (256-row tiles; the pair halves each SM's shared-memory
+// traffic per MMA) or single CTAs, and a K split whose fp32 partials an ordered reduce sums,
+// from an estimate of the wave-quantised main loop plus the reduce traffic.
 // The accumulator is double-buffered in TMEM (2 x 256 columns), so the epilogue of one tile
 // overlaps the MMAs of the next. Every mbarrier wait is bounded: after ~2 s it sets the
 // device error word and the CTA leaves through its normal teardown (TMEM is always freed).
@@ -78,7 +80,7 @@ __device__ __forceinline__ EpiRow epi_row(const TcParams &P, int row) {
   return r;
 }
 
-// 32 bf16 of the auxiliary input (residual stream or GELU pre-activation) of one row, packed;
+// 32 bf16 of the auxiliary input (residual stream, or gelu' stored by the forward) of one row, packed;
 // zeros past M or N.
 __device__ __forceinline__ void load_aux_chunk(const TcParams &P, int row, int col0, uint4 (&a)[4]) {
   const Epi &e = P.epi;

@@ -8,6 +8,8 @@
 // architecture page, "AdamW Fused Step": hyper-parameters held as tensors so that a
 // compiled step is reused when lr changes). The only host synchronisation is the read-back
 // of the loss, the grad norm and the device error word at the end of the call.
+// gpt_train_step_accum runs the same schedule once per micro-batch (one graph per phase:
+// gradients stored, accumulated, accumulated + clip and AdamW).
 #include <cuda.h>
 #include <math.h>
 #include <stdio.h>
