@@ -38,6 +38,7 @@ EXPORTED = [
     "gpt_params_changed", "gpt_set_option", "gpt_kernel_stats", "gpt_last_launch_count",
     "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
     "gptk_attention_bwd_bf16", "gptk_attention_bwd_bf16_noalloc", "gptk_selftest_bounded_wait",
+    "gptk_gemm_plan",
 ]
 
 
@@ -104,6 +105,16 @@ gptk_attention_bwd_bf16 = _sig("gptk_attention_bwd_bf16", _I, [_P, _P, _P, _P, _
 gptk_attention_bwd_bf16_noalloc = _sig("gptk_attention_bwd_bf16_noalloc", _I,
                                        [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P])
 gptk_selftest_bounded_wait = _sig("gptk_selftest_bounded_wait", _I, [ctypes.c_uint, _P, _P])
+gptk_gemm_plan = _sig("gptk_gemm_plan", _I, [_I, _I, _I, _I, ctypes.c_size_t, _I, ctypes.POINTER(_I),
+                                             ctypes.POINTER(_I)])
+
+
+def gemm_plan(M: int, N: int, K: int, epi: str, scratch_floats: int, sms: int = 148):
+    """(status, cta_group, split_k) of the tensor-core launch plan for this GEMM (host only)."""
+    cg, sk = _I(0), _I(0)
+    s = gptk_gemm_plan(M, N, K, GPTK_EPI[epi] if isinstance(epi, str) else epi, scratch_floats,
+                       sms, ctypes.byref(cg), ctypes.byref(sk))
+    return s, cg.value, sk.value
 GPTK_EPI = {"store": 0, "store_gelu": 1, "resid": 2, "dgelu": 3, "f32_store": 4, "f32_accum": 5}
 GPTK_PATH_TCGEN05 = 0
 GPTK_PATH_SIMT = 1

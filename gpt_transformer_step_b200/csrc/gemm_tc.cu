@@ -699,11 +699,9 @@ bool tc_gemm_supported(const GemmDesc &d) {
   }
 }
 
-cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches) {
-  (void)launches;
-  TcParams P;
-  memset(&P, 0, sizeof(P));
-  const int sms = num_sms();
+// The CTA group (1 or 2) and K split the launcher uses for `d` with `capacity` floats of
+// partial-sum scratch on `sms` SMs (host only; split_k > 0 in d is taken as given).
+void tc_gemm_plan(const GemmDesc &d, size_t capacity, int sms, int *cta_group, int *split) {
   const int nt = (d.N + BN - 1) / BN;
   const long kblocks = (d.K + BK - 1) / BK;
   const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
@@ -712,7 +710,7 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   int S = d.split_k;
   if (S <= 0) {
     S = 1;
-    if ((f32out || elementwise) && d.partial) {
+    if ((f32out || elementwise) && capacity > 0) {
       // automatic: the CTA group and K split with the smallest estimated time, in units of
       // one k-block of one CTA tile (~0.4 us as measured): the wave-quantised main loop, CTA
       // pairs credited with their smaller shared-memory traffic, plus for a split the ordered
@@ -723,7 +721,7 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
         const long tiles = (long)((d.M + cg * BM - 1) / (cg * BM)) * nt;
         const long slots = sms / cg;
         for (int s = 1; s <= 16; ++s) {
-          if (s > 1 && (kblocks / s < 4 || (size_t)s * d.M * d.N > t->splitk_capacity)) break;
+          if (s > 1 && (kblocks / s < 4 || (size_t)s * d.M * d.N > capacity)) break;
           const long units = tiles * s;
           const long waves = (units + slots - 1) / slots;
           double est = (double)waves * (double)((kblocks + s - 1) / s) * (cg == 2 ? 0.93 : 1.0);
@@ -733,13 +731,30 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
       }
     }
   }
+  if (S > kblocks) S = (int)kblocks;
+  if (S < 1) S = 1;
+  if (kblocks > 0) {
+    const long per = (kblocks + S - 1) / S;
+    S = (int)((kblocks + per - 1) / per);  // no empty split
+  }
+  *cta_group = CG;
+  *split = S;
+}
+
+cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches) {
+  (void)launches;
+  TcParams P;
+  memset(&P, 0, sizeof(P));
+  const int sms = num_sms();
+  const int nt = (d.N + BN - 1) / BN;
+  const long kblocks = (d.K + BK - 1) / BK;
+  int CG, S;
+  tc_gemm_plan(d, d.partial ? t->splitk_capacity : 0, sms, &CG, &S);
   P.M = d.M; P.N = d.N; P.K = d.K;
   P.num_mt = (d.M + BM * CG - 1) / (BM * CG);
   P.num_nt = nt;
   P.total_kblocks = (int)kblocks;
-  if (S > P.total_kblocks) S = P.total_kblocks;
   P.kblocks_per_split = (P.total_kblocks + S - 1) / S;
-  S = (P.total_kblocks + P.kblocks_per_split - 1) / P.kblocks_per_split;  // no empty split
   if (S > 1 && (!d.partial || (size_t)S * d.M * d.N > t->splitk_capacity)) return cudaErrorInvalidValue;
   d.split_k = S;
   P.splits = S;

@@ -14,6 +14,9 @@ void tc_gemm_destroy(TcGemm *t);
 void tc_gemm_set_splitk_capacity(TcGemm *t, size_t floats);
 // True when the shape, strides and epilogue can run on the tensor-core path.
 bool tc_gemm_supported(const GemmDesc &d);
+// CTA group (1 or 2) and K split the launcher chooses (host only); capacity = floats of split-K
+// scratch (0: no split).
+void tc_gemm_plan(const GemmDesc &d, size_t capacity, int sms, int *cta_group, int *split);
 // Enqueues the GEMM (and its split-K reduction, if any). d.split_k <= 0 lets the launcher
 // choose the split (only for elementwise epilogues); the chosen value is written back.
 cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launches);

@@ -19,7 +19,7 @@ extern "C" int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int 
                               void *out2, long ldo2, const void *aux, long ld_aux, float *outf,
                               long ldf, int split_k, float *scratch, size_t scratch_floats,
                               unsigned *dev_err, int path, void *stream) {
-  if (M < 0 || N < 0 || K < 0 || !A || !B || !dev_err) return GPT_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 1 || !A || !B || !dev_err) return GPT_ERR_INVALID_ARG;
   if (epi < GPTK_EPI_STORE || epi > GPTK_EPI_F32_ACCUM) return GPT_ERR_INVALID_ARG;
   const bool f32 = epi == GPTK_EPI_F32_STORE || epi == GPTK_EPI_F32_ACCUM;
   if (f32 ? !outf : !out) return GPT_ERR_INVALID_ARG;
@@ -54,6 +54,19 @@ extern "C" int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int 
     return GPT_ERR_INVALID_ARG;
   }
   return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
+extern "C" int gptk_gemm_plan(int M, int N, int K, int epi, size_t scratch_floats, int sms,
+                              int *cta_group, int *split_k) {
+  if (M < 1 || N < 1 || K < 1 || sms < 2 || !cta_group || !split_k) return GPT_ERR_INVALID_ARG;
+  if (epi < GPTK_EPI_STORE || epi > GPTK_EPI_F32_ACCUM) return GPT_ERR_INVALID_ARG;
+  GemmDesc d;
+  memset(&d, 0, sizeof(d));
+  d.M = M; d.N = N; d.K = K;
+  d.epi.kind = epi;
+  d.split_k = 0;
+  tc_gemm_plan(d, scratch_floats, sms, cta_group, split_k);
+  return GPT_OK;
 }
 
 extern "C" int gptk_attention_fwd_bf16(const void *qkv, void *o, float *lse, int B, int T, int C,

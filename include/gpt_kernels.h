@@ -16,7 +16,7 @@
  *                       forward stored with GPTK_EPI_STORE_GELU)
  *   GPTK_EPI_F32_STORE  outf[m*ldf+n] = acc
  *   GPTK_EPI_F32_ACCUM  outf[m*ldf+n] += acc
- * split_k > 1 splits K into split_k ranges whose fp32 partials are summed in a fixed order
+ * K >= 1. split_k > 1 splits K into split_k ranges whose fp32 partials are summed in a fixed order
  * (only for the two F32 epilogues; needs scratch of split_k*M*N floats, caller-owned).
  * split_k = 0 on the tensor-core path lets the launcher choose the CTA group and a split of at
  * most 16 that fits in scratch_floats (no split without scratch); on the SIMT path 0 means 1.
@@ -46,6 +46,14 @@ int gptk_gemm_bf16(int M, int N, int K, const void *A, long lda, int a_kmajor, c
                    const void *aux, long ld_aux, float *outf, long ldf, int split_k,
                    float *scratch, size_t scratch_floats, unsigned *dev_err, int path,
                    void *stream);
+
+/* The tensor-core launch plan gptk_gemm_bf16 (split_k = 0) and gpt_train_step use for an M x
+ * N x K GEMM with epilogue `epi`, given scratch_floats of split-K scratch, on a GPU with `sms`
+ * SMs: *cta_group = 1 (128-row tiles) or 2 (256-row tiles on CTA pairs), *split_k = number of
+ * K ranges (1 = no split). Host-only arithmetic (an estimate of the wave-quantised main loop
+ * plus the split-K reduce traffic); no GPU is touched. GPT_ERR_INVALID_ARG on bad sizes. */
+int gptk_gemm_plan(int M, int N, int K, int epi, size_t scratch_floats, int sms, int *cta_group,
+                   int *split_k);
 
 /* Causal attention with an optional left window (window < 0: full causal; w >= 0: query i
  * attends keys i-w..i), per head h of qkv [B*T, 3C] (q | k | v, head h at columns h*hd of

@@ -15,7 +15,7 @@ def declared_functions():
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names += re.findall(r"\b(gpt_\w+)\s*\(", src)
+            names += re.findall(r"\b(gptk?_\w+)\s*\(", src)
     return sorted(set(names))
 
 
