@@ -31,6 +31,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 # DRAM bytes (read + write) per tcgen05 GEMM launch, mean over all GEMM launches of the step,
 # from the ncu launch list in profiles/step_gpt2_124m_launch_list.md (same kernel version).
+METRIC = "train tokens/s (GPT-2 step, MFU from 6N+attn FLOPs)"
+
 GEMM_DRAM_BYTES_PER_LAUNCH = {"gpt2_124m_bf16": 204.31e6}
 
 def peaks():
@@ -138,12 +140,13 @@ def run_reference(args, wl, rank, world):
     from gpt_transformer_step_b200 import fixtures as fx
     fpt = fx.flops_per_token(wl.shape, wl.T)
     line = {
-        "impl": "reference", "metric": "train tokens/s (GPT-2 step)", "value": val,
+        "impl": "reference", "metric": METRIC, "value": val,
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "global_batch": 1, "seq_len": T_sample,
-                   "sample_of": f"B={wl.B} x T={wl.T}"},
+        "config": {"workload": wl.name, "global_batch": world * wl.B, "seq_len": wl.T,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "sample": f"each step: the oracle on B=1 x T={T_sample} tokens"},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"oracle train step on B=1 x T={T_sample} tokens per step"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -240,7 +243,7 @@ def run_ours(args, wl, rank, world, local_rank):
     achieved = (gemm_flops / (gemm_ms / 1000)) / 1e12 if gemm_ms > 0 else None
     peak_t = pk["bf16_tflops_sustained"]
     line = {
-        "metric": "train tokens/s (GPT-2 step, MFU from 6N+attn FLOPs)",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
