@@ -4,6 +4,8 @@
  * position embedding, n_layer pre-LayerNorm blocks (causal attention with an optional left
  * window per layer, GELU(tanh) MLP), final LayerNorm, tied lm_head with mean softmax
  * cross-entropy, the full backward pass, a global grad-norm clip and a fused AdamW update.
+ * gpt_train_step_accum runs one such update over several micro-batches (gradient
+ * accumulation).
  *
  * What the operations follow (pages cited by title and section):
  *   - model and config fields: nanoGPT README (intro: reproduces GPT-2 124M, loads OpenAI's
@@ -18,7 +20,9 @@
  *     with a new lr: nanochat architecture page, "Optimierungsstrategien Muon und AdamW",
  *     "AdamW Fused Step";
  *   - the flat parameter vector: Panthalia page, "Components of the Example Plugin" (the
- *     model adapter maps the model to and from a flattened tensor).
+ *     model adapter maps the model to and from a flattened tensor);
+ *   - gradient accumulation: llm.c summary, "Ejecución" (a total batch of -d tokens reached
+ *     with several micro-batches per optimizer step).
  *
  * Threading: a handle is not thread-safe; use one handle per host thread.
  * Errors: every int-returning call returns GPT_OK (0) or a negative GPT_ERR_* code; no C++
