@@ -119,7 +119,7 @@ def oracle_sample_step(wl, T_sample: int, seed: int = 0):
     return time.perf_counter() - t0, T_sample
 
 
-def cpu_baseline(wl, T_sample=16):
+def cpu_baseline(wl, T_sample=20):  # ~10 s of one host core for the 124M model
     sec, ntok = oracle_sample_step(wl, T_sample)
     return {"value": ntok / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"one oracle train step (fp32, 1 thread) on B=1 x T={T_sample} tokens of "
