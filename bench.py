@@ -27,13 +27,11 @@ sys.path.insert(0, ROOT)
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-
-
-# DRAM bytes (read + write) per tcgen05 GEMM launch, mean over all GEMM launches of the step,
-# from the ncu launch list in profiles/step_gpt2_124m_launch_list.md (same kernel version).
 METRIC = "train tokens/s (GPT-2 step, MFU from 6N+attn FLOPs)"
 
-GEMM_DRAM_BYTES_PER_LAUNCH = {"gpt2_124m_bf16": 204.31e6}
+# DRAM bytes (read + write) per tcgen05 GEMM launch from an ncu capture of the current GEMM
+# kernel (none yet: the roofline's traffic is reported as null until one is taken)
+GEMM_DRAM_BYTES_PER_LAUNCH: dict = {}
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -50,14 +48,21 @@ class Clocks:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, path: str | None = None):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        self.keep = path is not None
+        if path is None:
+            import tempfile
+            fd, path = tempfile.mkstemp(prefix=f"clocks_gpu{index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            d = os.path.dirname(self.path)
+            if d:
+                os.makedirs(d, exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
@@ -88,6 +93,11 @@ class Clocks:
             for nm, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
+        if not self.keep:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
@@ -103,27 +113,57 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def oracle_sample_step(wl, T_sample: int, seed: int = 0):
-    """One oracle training step (float instantiation, one thread) on B=1 x T_sample tokens of
-    the workload's model. Returns (seconds, tokens)."""
+def oracle_sample_step(wl, T_sample: int, seed: int = 0, B_sample: int = 1):
+    """One oracle training step (float instantiation, one thread) on B_sample x T_sample tokens
+    of the workload's model. Returns (seconds, tokens)."""
     import numpy as np
     import oracle
     from gpt_transformer_step_b200 import fixtures as fx
     o = oracle.Oracle.from_shape(wl.shape, dtype=np.float32)
     p = fx.init_params(wl.shape, seed)
-    tok, tgt = fx.zipf_tokens(wl.shape.vocab, wl.zipf_s, 1, T_sample, seed)
+    tok, tgt = fx.zipf_tokens(wl.shape.vocab, wl.zipf_s, B_sample, T_sample, seed)
     m = np.zeros_like(p)
     v = np.zeros_like(p)
     t0 = time.perf_counter()
     o.train_step(p, m, v, tok, tgt, wl.lr, wl.wd, wl.clip, 1)
-    return time.perf_counter() - t0, T_sample
+    return time.perf_counter() - t0, B_sample * T_sample
+
+
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return os.cpu_count(), model
 
 
 def cpu_baseline(wl, T_sample=20):  # ~10 s of one host core for the 124M model
+    """The oracle timed on one host thread: the headline sample (B=1 x T_sample of the bench
+    workload's full model) plus full oracle steps of the two small workload shapes."""
+    from gpt_transformer_step_b200 import fixtures as fx
     sec, ntok = oracle_sample_step(wl, T_sample)
-    return {"value": ntok / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"one oracle train step (fp32, 1 thread) on B=1 x T={T_sample} tokens of "
-                      f"the {wl.name} model (full width/depth/vocab); {sec:.1f} s"}
+    nproc, model = host_cpu()
+    out = {"value": ntok / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "sample": f"one oracle train step (fp32, 1 thread) on B=1 x T={T_sample} tokens of "
+                     f"the {wl.name} model (full width/depth/vocab); {sec:.1f} s",
+           "host_nproc": nproc, "host_cpu": model, "other_workloads": []}
+    tiny = fx.WORKLOADS["tiny_char_fp32"]
+    sec_t, n_t = oracle_sample_step(tiny, tiny.T, B_sample=tiny.B)
+    out["other_workloads"].append({"workload": tiny.name, "tokens_per_s": n_t / sec_t,
+                                   "sample": f"full step B={tiny.B} x T={tiny.T}",
+                                   "seconds": sec_t})
+    sh = fx.WORKLOADS["shakespeare_char_bf16"]
+    sec_s, n_s = oracle_sample_step(sh, sh.T, B_sample=1)
+    out["other_workloads"].append({"workload": sh.name, "tokens_per_s": n_s / sec_s,
+                                   "sample": f"one step at B=1 x T={sh.T} (full T; the workload's "
+                                             f"B={sh.B} is {sh.B}x this)",
+                                   "seconds": sec_s})
+    return out
 
 
 def run_reference(args, wl, rank, world):
@@ -195,21 +235,23 @@ def run_ours(args, wl, rank, world, local_rank):
         return st.train_step(P, G, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
 
     def timed(n, host_inputs=False):
+        """Device time of n steps (CUDA events on the launching stream), max over ranks, and
+        the median of the per-step event intervals."""
         a, b = (tk_h, tg_h) if host_inputs else (tk, tg)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
         barrier()
         torch.cuda.synchronize()
         losses = []
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(n):
+            ev[0].record(stream)
+            for i in range(n):
                 losses.append(step(a, b))
-            e1.record(stream)
+                ev[i + 1].record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
-        return ms, losses
+        ms = max_over_ranks(ev[0].elapsed_time(ev[n]) / n, world, dev)
+        med = statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(n))
+        return ms, losses, med
 
     st.set_stream(stream.cuda_stream)
     with torch.cuda.stream(stream):
@@ -218,19 +260,21 @@ def run_ours(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     launches = st.last_launch_count()
 
-    clk = Clocks(local_rank)
+    clk = Clocks(local_rank, args.clock_log)
     clk.start()
-    ms, losses = timed(args.steps)
+    ms, losses, ms_med = timed(args.steps)
     clocks = clk.stop()
 
     # end to end through the same C ABI call with host (pinned) token buffers
-    ms_e2e, _ = timed(args.steps, host_inputs=True)
+    ms_e2e, _, ms_e2e_med = timed(args.steps, host_inputs=True)
 
     # dominant kernel class (tensor-core GEMMs): CUDA events around every GEMM launch
+    n_inst = max(2, args.steps // 4)
     st.set_option(gb.GPT_OPT_TIME_KERNELS, 1)
     st.kernel_stats(reset=True)
-    timed(max(2, args.steps // 4))
-    n_l, gemm_ms, gemm_flops = st.kernel_stats(reset=True)
+    timed(n_inst)
+    n_rc, rc_ms, rc_flops = st.kernel_stats(kind=1)
+    n_l, gemm_ms, gemm_flops = st.kernel_stats(kind=0, reset=True)
     st.set_option(gb.GPT_OPT_TIME_KERNELS, 0)
 
     if rank != 0:
@@ -240,12 +284,16 @@ def run_ours(args, wl, rank, world, local_rank):
     value = tokens / (ms / 1000)
     fpt = fx.flops_per_token(sh, T)
     fpt_lit = fx.flops_per_token(sh, T, exclude="wte+wpe")
+    # algorithmic FLOPs (the method's own contractions) over the time of every GEMM launch,
+    # the logits recompute of the cross-entropy backward included in the time
     achieved = (gemm_flops / (gemm_ms / 1000)) / 1e12 if gemm_ms > 0 else None
-    peak_t = pk["bf16_tflops_sustained"]
+    peak_b = pk["bf16_tflops"]
+    peak_s = pk["bf16_tflops_sustained"]
     line = {
         "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_median": ms_med,
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (Zipf tokens, N(0,0.02) init)",
         "config": {"workload": wl.name, "global_batch": world * nm * B, "seq_len": T,
@@ -253,20 +301,29 @@ def run_ours(args, wl, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "working set ~6 GB >> 126 MB L2 (no flush needed)"},
         "mfu": {"nominal_2250": value / world * fpt / 2.25e15,
-                "measured_burst": value / world * fpt / (pk["bf16_tflops"] * 1e12),
-                "measured_sustained": value / world * fpt / (peak_t * 1e12),
+                "measured_burst": value / world * fpt / (peak_b * 1e12),
+                "measured_sustained": value / world * fpt / (peak_s * 1e12),
                 "flops_per_token": fpt, "flops_per_token_literal_excl_wte": fpt_lit},
         "loss_first_timed": losses[0] if losses else None,
         "e2e": {"value": tokens / (ms_e2e / 1000), "unit": "tokens/s",
-                "h2d_bytes_per_step": 2 * nm * B * T * 4, "d2h_bytes_per_step": 128},
+                "h2d_bytes_per_step": 2 * nm * B * T * 4, "d2h_bytes_per_step": 128,
+                "ms_per_step_median": ms_e2e_med},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMMs (all launches, flop-weighted)",
-                     "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": (achieved / peak_t) if achieved else None,
+                     "achieved": achieved, "peak": peak_b, "unit": "TFLOP/s",
+                     "frac": (achieved / peak_b) if achieved else None,
+                     "frac_vs_sustained": (achieved / peak_s) if achieved else None,
                      "traffic": GEMM_DRAM_BYTES_PER_LAUNCH.get(wl.name),
                      "traffic_unit": "bytes per GEMM launch (ncu dram__bytes_read.sum + "
-                                     "dram__bytes_write.sum, mean over one step's launches)",
-                     "peak_kind": f"{pk_kind} sustained bf16", "launches_timed": n_l,
-                     "gemm_ms_per_step": gemm_ms / max(1, max(2, args.steps // 4))},
+                                     "dram__bytes_write.sum)",
+                     "flops": "algorithmic: 2MNK of the block GEMMs and the lm_head forward, "
+                              "dX and dwte; the logits recompute is timed but not counted",
+                     "peak_kind": f"{pk_kind} burst bf16 (the step is ~19 ms, not a seconds-long "
+                                  f"loop); sustained {peak_s} beside it",
+                     "launches_timed": n_l,
+                     "gemm_ms_per_step": gemm_ms / n_inst,
+                     "gemm_tflop_per_step": gemm_flops / n_inst / 1e12,
+                     "recompute": {"launches": n_rc, "ms_per_step": rc_ms / n_inst,
+                                   "tflop_per_step": rc_flops / n_inst / 1e12}},
         "clocks": clocks,
         "gpu_launches": launches * args.steps,
     }
@@ -279,11 +336,13 @@ def run_ours(args, wl, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gpt2_124m_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="keep the nvidia-smi clock samples of the timed region in this file")
     ap.add_argument("--micro-batches", type=int, default=1,
                     help="micro-batches of B x T per optimizer step (gradient accumulation)")
     ap.add_argument("--lmhead-chunk-rows", type=int, default=0,

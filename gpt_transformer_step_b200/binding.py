@@ -249,11 +249,11 @@ class GPTStep:
     def set_option(self, opt: int, value: int):
         self._check(gpt_set_option(self.h, opt, value), "gpt_set_option")
 
-    def kernel_stats(self, reset: bool = False):
+    def kernel_stats(self, reset: bool = False, kind: int = 0):
         n = ctypes.c_longlong(0)
         ms = ctypes.c_double(0)
         fl = ctypes.c_double(0)
-        self._check(gpt_kernel_stats(self.h, 0, ctypes.byref(n), ctypes.byref(ms),
+        self._check(gpt_kernel_stats(self.h, kind, ctypes.byref(n), ctypes.byref(ms),
                                      ctypes.byref(fl), int(reset)), "gpt_kernel_stats")
         return n.value, ms.value, fl.value
 

@@ -18,6 +18,7 @@
 // No atomics: every output element is written by exactly one work item, so results are bitwise
 // reproducible. Tiles entirely outside the causal/window band are skipped; edge tiles are
 // masked element by element. Every wait is bounded (device error word on timeout).
+#include <atomic>
 #include <type_traits>
 
 #include "kernels.cuh"
@@ -998,20 +999,27 @@ static __device__ __align__(256) float g_noalloc_D[NOALLOC_D_MAX];
 
 namespace {
 constexpr int NOALLOC_MAX_DEVICES = 64;
-float *g_noalloc_D_addr[NOALLOC_MAX_DEVICES];  // device address per device ordinal
+// device address of g_noalloc_D per device ordinal; filled at most once per slot (host
+// threads that race on a first call all look up the same address, one store wins)
+std::atomic<float *> g_noalloc_D_addr[NOALLOC_MAX_DEVICES];
 
-// Device address of g_noalloc_D on the current device; looked up once per device. In host
-// code the symbol itself is only a host-side stand-in, never a device address.
+// Device address of g_noalloc_D on the current device, looked up on the first call there. In
+// host code the symbol itself is only a host-side stand-in, never a device address. The
+// cached address belongs to the device's current context: cudaDeviceReset invalidates it.
 cudaError_t noalloc_D_address(float **out) {
   int dev = 0;
   CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
-  if (!g_noalloc_D_addr[dev]) {
+  float *a = g_noalloc_D_addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void *ptr = nullptr;
     CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_D));
-    g_noalloc_D_addr[dev] = (float *)ptr;
+    float *expected = nullptr;
+    g_noalloc_D_addr[dev].compare_exchange_strong(expected, (float *)ptr,
+                                                  std::memory_order_acq_rel);
+    a = g_noalloc_D_addr[dev].load(std::memory_order_acquire);
   }
-  *out = g_noalloc_D_addr[dev];
+  *out = a;
   return cudaSuccess;
 }
 }  // namespace

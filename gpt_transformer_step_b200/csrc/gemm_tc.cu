@@ -47,12 +47,28 @@ struct TcParams {
   int M, N, K;
   int num_mt, num_nt, splits, kblocks_per_split, total_kblocks;
   int units;
+  int n_fast;      // 1: units walk the N tiles of one M tile first (see unit_coords)
   int a_mn, b_mn;  // 1 = MN-major
   uint32_t idesc;
   Epi epi;
   float *partial;
   unsigned *err;
 };
+
+// Tile coordinates of work unit u. Units are numbered M tile fastest, so that CTAs running at
+// the same time share the B tile; when A is the larger operand and does not fit in L2 (the
+// lm_head backward's dS chunk, read by the dX and dwte GEMMs) they are numbered N tile
+// fastest instead, so that the CTAs reading one A tile run together and A crosses HBM once.
+__device__ __forceinline__ void unit_coords(const TcParams &P, int u, int &mt, int &nt, int &z) {
+  if (P.n_fast) {
+    nt = u % P.num_nt;
+    mt = (u / P.num_nt) % P.num_mt;
+  } else {
+    mt = u % P.num_mt;
+    nt = (u / P.num_mt) % P.num_nt;
+  }
+  z = u / (P.num_mt * P.num_nt);
+}
 
 // ---------------------------------------------------------------------------------------
 // epilogue helpers (one thread = one row, 32 consecutive columns per call)
@@ -349,7 +365,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       bool ok = true;
       uint32_t issued = 0, last_par = 0;
       for (int u = unit0; u < P.units && ok; u += ustride) {
-        const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
+        int mt, nt, z;
+        unit_coords(P, u, mt, nt, z);
         const int m0 = mt * BM * CG + (int)rank * BM;
         const int n0 = nt * BN + (int)rank * Cf::B_ROWS;
         const int kb0 = z * P.kblocks_per_split;
@@ -445,7 +462,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int chunk_seq = 0;
     int i = 0;
     for (int u = unit0; u < P.units; u += ustride, ++i) {
-      const int mt = u % P.num_mt, nt = (u / P.num_mt) % P.num_nt, z = u / (P.num_mt * P.num_nt);
+      int mt, nt, z;
+      unit_coords(P, u, mt, nt, z);
       const int acc = i & 1;
       const uint32_t use = (uint32_t)(i >> 1);
       const int row0 = mt * BM * CG + (int)rank * BM + q * 32;  // this warp's 32 rows
@@ -759,6 +777,10 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   d.split_k = S;
   P.splits = S;
   P.units = P.num_mt * P.num_nt * S;
+  {
+    const double a_bytes = 2.0 * d.M * d.K, b_bytes = 2.0 * d.N * d.K;
+    P.n_fast = (P.num_nt > 1 && a_bytes > b_bytes && a_bytes > 48e6) ? 1 : 0;
+  }
   P.a_mn = d.a_kmajor ? 0 : 1;
   P.b_mn = d.b_kmajor ? 0 : 1;
   P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)P.a_mn << 15) |

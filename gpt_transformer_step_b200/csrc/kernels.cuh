@@ -9,15 +9,16 @@ cudaError_t launch_embed_fwd(const int *tok, const int *tgt, const T *wte, const
                              int M, int Tlen, int C, int V, DevScalars *sc, cudaStream_t st);
 
 // K13: dwpe[t] = sum_b dx[b,t] (rows t >= T zeroed; added to dwpe when accumulate); dwte[id]
-// += sum over positions with that id, in position order (deterministic). dwte already holds
-// the lm_head part.
+// += sum over positions with that id, in position order (deterministic; a stable radix sort of
+// the ids over several CTAs, then windowed segment sums). dwte already holds the lm_head part.
 struct EmbedBwdWs {
-  unsigned *keys;      // [M] sorted (id << 14 | m)
-  float *partial;      // [nwin][2][C]
+  void *base;  // embed_bwd_ws_bytes(maxM, C) bytes, 256-byte aligned
 };
+size_t embed_bwd_ws_bytes(int maxM, int C);
+int embed_bwd_launches(int Vp);
 template <typename T>
 cudaError_t launch_embed_bwd(const int *tok, const T *dx, float *dwte, float *dwpe, int M,
-                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st,
+                             int Tlen, int maxT, int C, int Vp, EmbedBwdWs ws, cudaStream_t st,
                              bool accumulate = false);
 
 // K2: y = (x - mean) * rstd * g, one warp per row.
@@ -45,7 +46,7 @@ cudaError_t launch_grad_norm(const float *g, size_t n, double *partials, DevScal
                              cudaStream_t st);
 int grad_norm_blocks();
 
-// K15: AdamW with g <- coef*g; skipped when sc->nonfinite. shadow (bf16, may be NULL)
+// K15: AdamW with g <- coef*g; skipped when sc->nonfinite or any sc->err bit is set. shadow (bf16, may be NULL)
 // receives the rounded new params.
 cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, bf16 *shadow, size_t n,
                          const DevScalars *sc, cudaStream_t st);

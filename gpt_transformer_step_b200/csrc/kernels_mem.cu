@@ -293,113 +293,229 @@ __global__ void __launch_bounds__(1024) colsum_kernel(const float *__restrict__ 
 
 // ------------------------------------------------------------------------------------------
 // K13 embedding backward
+//   dwpe[t] = sum_b dx[b, t]                      (b in order)
+//   dwte[v] += sum_{m : tok[m] = v} dx[m]          (m in increasing order)
+// The token ids are sorted stably (LSD radix sort, 9-bit digits, several CTAs per pass), so
+// the positions of one id end up in increasing order; windows of EW sorted entries then sum
+// their runs, and runs that cross a window boundary are finished by a merge in window order.
+// Every sum has a fixed order: the result is bitwise reproducible.
 // ------------------------------------------------------------------------------------------
 template <typename T>
 __global__ void dwpe_kernel(const T *__restrict__ dx, float *__restrict__ dwpe, int Bn,
                             int Tlen, int maxT, int C, int accumulate) {
-  long total = (long)maxT * C;
+  constexpr int VN = Vec<T>::N;
+  const int nvec = C / VN;
+  const long total = (long)maxT * nvec;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
        i += (long)gridDim.x * blockDim.x) {
-    int t = (int)(i / C), c = (int)(i % C);
-    float s = 0.f;
+    const int t = (int)(i / nvec), c = (int)(i % nvec) * VN;
+    float s[VN];
+#pragma unroll
+    for (int k = 0; k < VN; ++k) s[k] = 0.f;
     if (t < Tlen)
-      for (int b = 0; b < Bn; ++b) s += to_f(dx[((long)b * Tlen + t) * C + c]);
-    dwpe[i] = accumulate ? dwpe[i] + s : s;
-  }
-}
-
-// One CTA sorts the M keys (id << 14 | m) in shared memory with a bitonic network.
-constexpr int SORT_MAX = 16384;
-__global__ void __launch_bounds__(1024) sort_keys_kernel(const int *__restrict__ tok, int M,
-                                                         unsigned *__restrict__ keys_out) {
-  extern __shared__ unsigned sk[];
-  int n = 1;
-  while (n < M) n <<= 1;
-  for (int i = threadIdx.x; i < n; i += blockDim.x)
-    sk[i] = i < M ? ((unsigned)tok[i] << 14) | (unsigned)i : 0xffffffffu;
-  __syncthreads();
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        int p = i ^ j;
-        if (p > i) {
-          unsigned a = sk[i], b = sk[p];
-          bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            sk[i] = b;
-            sk[p] = a;
-          }
-        }
+      for (int b = 0; b < Bn; ++b) {
+        float v[VN];
+        load_vec<T>(dx + ((long)b * Tlen + t) * C + c, v);
+#pragma unroll
+        for (int k = 0; k < VN; ++k) s[k] += v[k];
       }
-      __syncthreads();
+    float *o = dwpe + (long)t * C + c;
+#pragma unroll
+    for (int k = 0; k < VN; k += 4) {
+      float4 r = make_float4(s[k], s[k + 1], s[k + 2], s[k + 3]);
+      if (accumulate) {
+        const float4 a = *reinterpret_cast<const float4 *>(o + k);
+        r.x += a.x; r.y += a.y; r.z += a.z; r.w += a.w;
+      }
+      *reinterpret_cast<float4 *>(o + k) = r;
     }
   }
-  for (int i = threadIdx.x; i < M; i += blockDim.x) keys_out[i] = sk[i];
 }
 
-constexpr int EW = 32;  // sorted entries per window
+constexpr int RS_BITS = 9;
+constexpr int RS_BUCKETS = 1 << RS_BITS;
+constexpr int RS_TILE = 2048;   // entries per CTA and pass
+constexpr int RS_WARPS = 8;     // each warp ranks RS_TILE / RS_WARPS consecutive entries
+
+// Digit histogram of one tile: hist[digit * ntiles + tile] (digit-major, so an exclusive scan
+// gives every (digit, tile) its first output slot in stable order).
+__global__ void __launch_bounds__(256) rs_hist_kernel(const int *__restrict__ ids, int M, int shift,
+                                                      unsigned *__restrict__ hist, int ntiles) {
+  __shared__ unsigned cnt[RS_BUCKETS];
+  for (int i = threadIdx.x; i < RS_BUCKETS; i += blockDim.x) cnt[i] = 0u;
+  __syncthreads();
+  const int e0 = blockIdx.x * RS_TILE, e1 = min(M, e0 + RS_TILE);
+  for (int i = e0 + threadIdx.x; i < e1; i += blockDim.x)
+    atomicAdd(&cnt[((unsigned)ids[i] >> shift) & (RS_BUCKETS - 1)], 1u);
+  __syncthreads();
+  for (int d = threadIdx.x; d < RS_BUCKETS; d += blockDim.x) hist[(long)d * ntiles + blockIdx.x] = cnt[d];
+}
+
+// Exclusive prefix sum of n counts in place (one CTA of 1024 threads, contiguous chunks).
+__global__ void __launch_bounds__(1024) rs_scan_kernel(unsigned *__restrict__ a, int n) {
+  __shared__ unsigned part[1024];
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int b0 = threadIdx.x * per, b1 = min(n, b0 + per);
+  unsigned s = 0;
+  for (int i = b0; i < b1; ++i) s += a[i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {  // Hillis-Steele inclusive scan
+    const unsigned v = threadIdx.x >= (unsigned)off ? part[threadIdx.x - off] : 0u;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  unsigned run = part[threadIdx.x] - s;  // exclusive base of this chunk
+  for (int i = b0; i < b1; ++i) {
+    const unsigned c = a[i];
+    a[i] = run;
+    run += c;
+  }
+}
+
+// Stable scatter of one tile by digit: an entry's slot is its (digit, tile) base plus the
+// number of earlier entries of the tile with the same digit. pos_in == NULL: positions are
+// the entry indices (first pass).
+__global__ void __launch_bounds__(RS_WARPS * 32)
+rs_scatter_kernel(const int *__restrict__ ids_in, const int *__restrict__ pos_in,
+                  int *__restrict__ ids_out, int *__restrict__ pos_out, int M, int shift,
+                  const unsigned *__restrict__ offs, int ntiles) {
+  __shared__ unsigned wbase[RS_WARPS][RS_BUCKETS];  // per-warp counts, then per-warp bases
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int PER_WARP = RS_TILE / RS_WARPS;
+  for (int i = threadIdx.x; i < RS_WARPS * RS_BUCKETS; i += blockDim.x) (&wbase[0][0])[i] = 0u;
+  __syncthreads();
+  const int t0 = blockIdx.x * RS_TILE;
+  const int w0 = t0 + warp * PER_WARP, w1 = min(M, w0 + PER_WARP);
+  for (int i = w0 + lane; i < w1; i += 32)
+    atomicAdd(&wbase[warp][((unsigned)ids_in[i] >> shift) & (RS_BUCKETS - 1)], 1u);
+  __syncthreads();
+  for (int d = threadIdx.x; d < RS_BUCKETS; d += blockDim.x) {
+    unsigned run = offs[(long)d * ntiles + blockIdx.x];
+    for (int w = 0; w < RS_WARPS; ++w) {
+      const unsigned c = wbase[w][d];
+      wbase[w][d] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c0 = w0; c0 < w1; c0 += 32) {  // chunks of 32 in entry order
+    const int i = c0 + lane;
+    const bool valid = i < w1;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    if (valid) {
+      const int id = ids_in[i];
+      const int pos = pos_in ? pos_in[i] : i;
+      const unsigned d = ((unsigned)id >> shift) & (RS_BUCKETS - 1);
+      const unsigned peers = __match_any_sync(vmask, d);
+      const unsigned dst = wbase[warp][d] + __popc(peers & lt);
+      ids_out[dst] = id;
+      pos_out[dst] = pos;
+      __syncwarp(vmask);
+      if ((peers & lt) == 0u) wbase[warp][d] += __popc(peers);  // the run's first lane
+    }
+    __syncwarp();
+  }
+}
+
+constexpr int EW = 64;  // sorted entries per window
 
 // Window w covers sorted entries [w*EW, (w+1)*EW). Runs of one id that lie wholly inside the
 // window are added to dwte here; a run that starts before the window goes to slot 0, a run
-// that continues past it (and did not start before) to slot 1, for the merge kernel.
+// that continues past it (and did not start before) to slot 1, for the merge kernel. Threads
+// own 16-byte column vectors; the entries of a run are summed in sorted (position) order.
 template <typename T>
-__global__ void embed_seg_kernel(const unsigned *__restrict__ keys, const T *__restrict__ dx,
-                                 float *__restrict__ dwte, float *__restrict__ partial, int M,
-                                 int C) {
+__global__ void __launch_bounds__(128) embed_seg_kernel(const int *__restrict__ sid,
+                                                        const int *__restrict__ spos,
+                                                        const T *__restrict__ dx,
+                                                        float *__restrict__ dwte,
+                                                        float *__restrict__ partial, int M, int C) {
+  constexpr int VN = Vec<T>::N;
   const int w = blockIdx.x;
   const int e0 = w * EW, e1 = min(M, e0 + EW);
-  __shared__ unsigned skey[EW];
-  if (threadIdx.x < EW) skey[threadIdx.x] = (e0 + (int)threadIdx.x < M) ? keys[e0 + threadIdx.x] : 0u;
+  __shared__ int s_id[EW], s_pos[EW];
+  if (threadIdx.x < EW && e0 + (int)threadIdx.x < M) {
+    s_id[threadIdx.x] = sid[e0 + threadIdx.x];
+    s_pos[threadIdx.x] = spos[e0 + threadIdx.x];
+  }
   __syncthreads();
-  const unsigned id_before = e0 > 0 ? (keys[e0 - 1] >> 14) : 0xffffffffu;
-  const unsigned id_after = e1 < M ? (keys[e1] >> 14) : 0xffffffffu;
+  const int id_before = e0 > 0 ? sid[e0 - 1] : -1;
+  const int id_after = e1 < M ? sid[e1] : -1;
+  const int nvec = C / VN;
   int s = e0;
   while (s < e1) {
-    const unsigned id = skey[s - e0] >> 14;
-    int e = s;
-    while (e < e1 && (skey[e - e0] >> 14) == id) ++e;
+    const int id = s_id[s - e0];
+    int e = s + 1;
+    while (e < e1 && s_id[e - e0] == id) ++e;
     const bool before = (s == e0) && (id == id_before);
     const bool after = (e == e1) && (id == id_after);
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      float acc = 0.f;
-      for (int k = s; k < e; ++k) {
-        int m = (int)(skey[k - e0] & 0x3fffu);
-        acc += to_f(dx[(long)m * C + c]);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      const int c = v * VN;
+      float acc[VN];
+#pragma unroll
+      for (int k = 0; k < VN; ++k) acc[k] = 0.f;
+      int k0 = s;
+      for (; k0 + 4 <= e; k0 += 4) {  // four rows in flight, added in order
+        float a[4][VN];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) load_vec<T>(dx + (long)s_pos[k0 + u - e0] * C + c, a[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int k = 0; k < VN; ++k) acc[k] += a[u][k];
       }
-      if (!before && !after)
-        dwte[(long)id * C + c] += acc;
-      else
-        partial[((long)w * 2 + (before ? 0 : 1)) * C + c] = acc;
+      for (; k0 < e; ++k0) {
+        float a[VN];
+        load_vec<T>(dx + (long)s_pos[k0 - e0] * C + c, a);
+#pragma unroll
+        for (int k = 0; k < VN; ++k) acc[k] += a[k];
+      }
+      float *dst = (!before && !after) ? dwte + (long)id * C + c
+                                       : partial + ((long)w * 2 + (before ? 0 : 1)) * C + c;
+#pragma unroll
+      for (int k = 0; k < VN; k += 4) {
+        float4 r = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+        if (!before && !after) {
+          const float4 o = *reinterpret_cast<const float4 *>(dst + k);
+          r.x += o.x; r.y += o.y; r.z += o.z; r.w += o.w;
+        }
+        *reinterpret_cast<float4 *>(dst + k) = r;
+      }
     }
     s = e;
   }
 }
 
 // For each run that continues past window w (and started inside it): sum slot 1 of w and
-// slot 0 of the following windows while the run goes on, in window order.
-__global__ void embed_merge_kernel(const unsigned *__restrict__ keys,
-                                   const float *__restrict__ partial, float *__restrict__ dwte,
-                                   int M, int C, int nwin) {
+// slot 0 of the following windows while the run goes on, in window order; add to dwte.
+__global__ void __launch_bounds__(128) embed_merge_kernel(const int *__restrict__ sid,
+                                                          const float *__restrict__ partial,
+                                                          float *__restrict__ dwte, int M, int C,
+                                                          int nwin) {
   const int w = blockIdx.x;
   const int e0 = w * EW, e1 = min(M, e0 + EW);
   if (e1 >= M) return;
-  const unsigned id = keys[e1 - 1] >> 14;
-  if ((keys[e1] >> 14) != id) return;  // does not continue
+  const int id = sid[e1 - 1];
+  if (sid[e1] != id) return;  // does not continue
   // the run must not have started before the window
   int s = e1 - 1;
-  while (s > e0 && (keys[s - 1] >> 14) == id) --s;
-  if (s == e0 && e0 > 0 && (keys[e0 - 1] >> 14) == id) return;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    float acc = partial[((long)w * 2 + 1) * C + c];
-    for (int ww = w + 1; ww < nwin; ++ww) {
-      int f0 = ww * EW;
-      if ((keys[f0] >> 14) != id) break;
-      acc += partial[((long)ww * 2 + 0) * C + c];
-      int f1 = min(M, f0 + EW);
-      if (f1 >= M || (keys[f1] >> 14) != id) break;  // run ends in this window
-      if ((keys[f1 - 1] >> 14) != id) break;
+  while (s > e0 && sid[s - 1] == id) --s;
+  if (s == e0 && e0 > 0 && sid[e0 - 1] == id) return;
+  // windows the run covers after w: up to the one where it ends
+  int wl = w + 1;
+  while (wl + 1 < nwin && sid[min(M, (wl + 1) * EW) - 1] == id && sid[(wl + 1) * EW] == id) ++wl;
+  for (int c = threadIdx.x * 4; c < C; c += blockDim.x * 4) {
+    float4 acc = *reinterpret_cast<const float4 *>(partial + ((long)w * 2 + 1) * C + c);
+    for (int ww = w + 1; ww <= wl; ++ww) {
+      const float4 p = *reinterpret_cast<const float4 *>(partial + ((long)ww * 2 + 0) * C + c);
+      acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
     }
-    dwte[(long)id * C + c] += acc;
+    float4 *o = reinterpret_cast<float4 *>(dwte + (long)id * C + c);
+    float4 r = *o;
+    r.x += acc.x; r.y += acc.y; r.z += acc.z; r.w += acc.w;
+    *o = r;
   }
 }
 
@@ -515,7 +631,9 @@ __device__ __forceinline__ void adamw_one(float &p, float g, float &m, float &v,
 __global__ void adamw_kernel(float *__restrict__ p, const float *__restrict__ g,
                              float *__restrict__ m, float *__restrict__ v,
                              bf16 *__restrict__ shadow, size_t n, const DevScalars *sc) {
-  if (sc->nonfinite) return;
+  // a failed step leaves the caller's state untouched: a non-finite loss or norm, an id out
+  // of range or a device wait that gave up (partial gradients) all skip the update
+  if (sc->nonfinite || sc->err) return;
   const float lr = sc->lr, wd = sc->wd, b1 = sc->beta1, b2 = sc->beta2, eps = sc->eps;
   const float bias1 = sc->bias1, bias2 = sc->bias2, coef = sc->coef;
   const size_t n4 = n / 4;
@@ -575,28 +693,57 @@ cudaError_t launch_embed_fwd(const int *tok, const int *tgt, const T *wte, const
   return cudaGetLastError();
 }
 
+size_t embed_bwd_ws_bytes(int maxM, int C) {
+  const size_t ntiles = (maxM + RS_TILE - 1) / RS_TILE;
+  const size_t nwin = (maxM + EW - 1) / EW;
+  return 4 * (size_t)maxM * sizeof(int) + (size_t)RS_BUCKETS * ntiles * sizeof(unsigned) + 256 +
+         nwin * 2 * (size_t)C * sizeof(float) + 256;
+}
+
 template <typename T>
 cudaError_t launch_embed_bwd(const int *tok, const T *dx, float *dwte, float *dwpe, int M,
-                             int Tlen, int maxT, int C, EmbedBwdWs ws, cudaStream_t st,
+                             int Tlen, int maxT, int C, int Vp, EmbedBwdWs ws, cudaStream_t st,
                              bool accumulate) {
   const int Bn = M / Tlen;
-  dwpe_kernel<T><<<grid_for((long)maxT * C, 256), 256, 0, st>>>(dx, dwpe, Bn, Tlen, maxT, C,
-                                                                accumulate ? 1 : 0);
+  dwpe_kernel<T><<<grid_for((long)maxT * (C / Vec<T>::N), 256), 256, 0, st>>>(
+      dx, dwpe, Bn, Tlen, maxT, C, accumulate ? 1 : 0);
   CUDA_TRY(cudaGetLastError());
-  int n = 1;
-  while (n < M) n <<= 1;
-  sort_keys_kernel<<<1, 1024, n * sizeof(unsigned), st>>>(tok, M, ws.keys);
-  CUDA_TRY(cudaGetLastError());
+  // carve the workspace: ids and positions (two buffers each), digit histogram, partials
+  const int ntiles = (M + RS_TILE - 1) / RS_TILE;
+  char *w = (char *)ws.base;
+  int *ids[2] = {(int *)w, (int *)w + M};
+  int *pos[2] = {(int *)w + 2 * (size_t)M, (int *)w + 3 * (size_t)M};
+  unsigned *hist = (unsigned *)((int *)w + 4 * (size_t)M);
+  float *partial = (float *)(((uintptr_t)(hist + (size_t)RS_BUCKETS * ntiles) + 255) & ~(uintptr_t)255);
+  // LSD radix passes over the id bits (a pass per 9 bits of Vp - 1)
+  int bits = 1;
+  while ((1 << bits) < Vp) ++bits;
+  const int passes = (bits + RS_BITS - 1) / RS_BITS;
+  const int *cur_id = tok;
+  const int *cur_pos = nullptr;
+  for (int p = 0; p < passes; ++p) {
+    const int shift = p * RS_BITS;
+    rs_hist_kernel<<<ntiles, 256, 0, st>>>(cur_id, M, shift, hist, ntiles);
+    CUDA_TRY(cudaGetLastError());
+    rs_scan_kernel<<<1, 1024, 0, st>>>(hist, RS_BUCKETS * ntiles);
+    CUDA_TRY(cudaGetLastError());
+    rs_scatter_kernel<<<ntiles, RS_WARPS * 32, 0, st>>>(cur_id, cur_pos, ids[p & 1], pos[p & 1], M,
+                                                        shift, hist, ntiles);
+    CUDA_TRY(cudaGetLastError());
+    cur_id = ids[p & 1];
+    cur_pos = pos[p & 1];
+  }
   const int nwin = (M + EW - 1) / EW;
-  embed_seg_kernel<T><<<nwin, 256, 0, st>>>(ws.keys, dx, dwte, ws.partial, M, C);
+  embed_seg_kernel<T><<<nwin, 128, 0, st>>>(cur_id, cur_pos, dx, dwte, partial, M, C);
   CUDA_TRY(cudaGetLastError());
-  embed_merge_kernel<<<nwin, 256, 0, st>>>(ws.keys, ws.partial, dwte, M, C, nwin);
+  embed_merge_kernel<<<nwin, 128, 0, st>>>(cur_id, partial, dwte, M, C, nwin);
   return cudaGetLastError();
 }
 
-cudaError_t embed_sort_smem_attr() {
-  return cudaFuncSetAttribute(sort_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              SORT_MAX * sizeof(unsigned));
+int embed_bwd_launches(int Vp) {
+  int bits = 1;
+  while ((1 << bits) < Vp) ++bits;
+  return 3 + 3 * ((bits + RS_BITS - 1) / RS_BITS);
 }
 
 #define LN_DISPATCH(NVV, CALL)                    \
@@ -681,7 +828,7 @@ cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st)
   template cudaError_t launch_embed_fwd<T>(const int *, const int *, const T *, const T *, T *, \
                                            int, int, int, int, DevScalars *, cudaStream_t);    \
   template cudaError_t launch_embed_bwd<T>(const int *, const T *, float *, float *, int, int,  \
-                                           int, int, EmbedBwdWs, cudaStream_t, bool);          \
+                                           int, int, int, EmbedBwdWs, cudaStream_t, bool);     \
   template cudaError_t launch_layernorm_fwd<T>(const T *, const T *, T *, float *, float *, int, \
                                                int, float, cudaStream_t);                      \
   template cudaError_t launch_layernorm_bwd<T>(const T *, const T *, const float *,             \

@@ -24,8 +24,6 @@
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 
-cudaError_t embed_sort_smem_attr();
-
 namespace {
 
 constexpr int ALIGN = 256;
@@ -85,8 +83,7 @@ struct gpt_handle {
   double *gn_partials;
   float *splitk;
   size_t splitk_elems;
-  unsigned *sort_keys;
-  float *emb_partial;
+  void *emb_ws;  // embedding backward: sort buffers, digit histogram, window partials
   bf16 *shadow;
   // state
   long step;
@@ -105,9 +102,10 @@ struct gpt_handle {
   bool time_kernels;
   std::vector<cudaEvent_t> ev;
   std::vector<double> ev_flops;
+  std::vector<int> ev_kind;  // 0: the method's own GEMM work, 1: the lm_head logits recompute
   int ev_used;
-  long long stat_launches;
-  double stat_ms, stat_flops;
+  long long stat_launches[2];
+  double stat_ms[2], stat_flops[2];
   TcGemm *tc;
 };
 
@@ -157,6 +155,7 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
     k = h->ev_used;
     h->ev_used += 2;
     h->ev_flops[k / 2] = flops;
+    h->ev_kind[k / 2] = d.epi.kind == EPI_CE_DS ? 1 : 0;
     cudaError_t e = cudaEventRecord(h->ev[k], h->stream);
     if (e != cudaSuccess) return e;
   }
@@ -362,9 +361,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
                                      h->dg_partial, G + P.ln1, M, C, st, acc)); nl += 2;
   }
-  EmbedBwdWs ew{h->sort_keys, h->emb_partial};
+  EmbedBwdWs ew{h->emb_ws};
   CUDA_TRY(launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C,
-                               ew, st, acc)); nl += 4;
+                               h->Vp, ew, st, acc)); nl += embed_bwd_launches(h->Vp);
   if (phase == PH_FIRST || phase == PH_MIDDLE) return cudaSuccess;  // update after the last
   // ---------------- clip + AdamW ----------------
   CUDA_TRY(launch_grad_norm(G, h->nparams, h->gn_partials, sc, st)); nl++;
@@ -440,9 +439,10 @@ int finish(gpt_handle *h, float *loss, int n_micro = 1) {
     for (int k = 0; k + 1 < h->ev_used; k += 2) {
       float ms = 0.f;
       if (cudaEventElapsedTime(&ms, h->ev[k], h->ev[k + 1]) == cudaSuccess) {
-        h->stat_ms += ms;
-        h->stat_flops += h->ev_flops[k / 2];
-        h->stat_launches++;
+        const int kind = h->ev_kind[k / 2];
+        h->stat_ms[kind] += ms;
+        h->stat_flops[kind] += h->ev_flops[k / 2];
+        h->stat_launches[kind]++;
       }
     }
   }
@@ -506,7 +506,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   const bool bf = c.precision == GPT_BF16;
   if (bf ? (C % 64 != 0) : (C % 4 != 0)) return nullptr;
   if (C > (bf ? 2048 : 1024)) return nullptr;
-  if ((long)c.max_B * c.max_T > 16384) return nullptr;
+  if ((long)c.max_B * c.max_T > GPT_MAX_TOKENS) return nullptr;
   if (c.vocab_padded > 131072) return nullptr;
 
   gpt_handle *h = new gpt_handle();
@@ -526,7 +526,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   h->use_graphs = true;
   h->time_kernels = false;
   h->ev_used = 0;
-  h->stat_launches = 0; h->stat_ms = 0; h->stat_flops = 0;
+  for (int k = 0; k < 2; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_flops[k] = 0; }
   h->tc = nullptr;
   cudaGetDevice(&h->device);
 
@@ -591,8 +591,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   need((void **)&h->dg_partial, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
   need((void **)&h->gn_partials, (size_t)grad_norm_blocks() * 8);
   need((void **)&h->splitk, h->splitk_elems * 4);
-  need((void **)&h->sort_keys, M * 4);
-  need((void **)&h->emb_partial, ((M + 31) / 32) * 2 * (size_t)C * 4);
+  need(&h->emb_ws, embed_bwd_ws_bytes((int)M, C));
   need((void **)&h->tok, M * 4); need((void **)&h->tgt, M * 4);
   need((void **)&h->sc, sizeof(DevScalars));
   if (bf) need((void **)&h->shadow, h->nparams * 2);
@@ -613,8 +612,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
     o2 += align_up(r.second);
   }
   *status = GPT_ERR_CUDA;
-  if (cudaMemset(h->ws, 0, total) != cudaSuccess || cudaMallocHost(&h->sc_host, sizeof(DevScalars)) != cudaSuccess ||
-      embed_sort_smem_attr() != cudaSuccess) {
+  if (cudaMemset(h->ws, 0, total) != cudaSuccess || cudaMallocHost(&h->sc_host, sizeof(DevScalars)) != cudaSuccess) {
     cudaGetLastError();
     cudaFree(h->ws);
     delete h;
@@ -752,6 +750,7 @@ int gpt_set_option(gpt_handle *h, int option, long value) {
       const int n = 2 * (16 * h->L + 64);
       h->ev.resize(n);
       h->ev_flops.assign(n / 2, 0.0);
+      h->ev_kind.assign(n / 2, 0);
       for (int i = 0; i < n; ++i)
         if (cudaEventCreate(&h->ev[i]) != cudaSuccess) return fail(h, cudaGetLastError());
     }
@@ -762,14 +761,16 @@ int gpt_set_option(gpt_handle *h, int option, long value) {
 
 int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
                      double *flops, int reset) {
-  if (!h || kind != 0) return GPT_ERR_INVALID_ARG;
-  if (launches) *launches = h->stat_launches;
-  if (total_ms) *total_ms = h->stat_ms;
-  if (flops) *flops = h->stat_flops;
+  if (!h || kind < 0 || kind > 1) return GPT_ERR_INVALID_ARG;
+  // kind 0: every GEMM launch (time), the method's own FLOPs (the recompute excluded);
+  // kind 1: the lm_head logits recompute of the cross-entropy backward alone
+  const long long n = kind == 0 ? h->stat_launches[0] + h->stat_launches[1] : h->stat_launches[1];
+  const double ms = kind == 0 ? h->stat_ms[0] + h->stat_ms[1] : h->stat_ms[1];
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  if (flops) *flops = h->stat_flops[kind];
   if (reset) {
-    h->stat_launches = 0;
-    h->stat_ms = 0;
-    h->stat_flops = 0;
+    for (int k = 0; k < 2; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_flops[k] = 0; }
   }
   return GPT_OK;
 }

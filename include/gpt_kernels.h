@@ -82,7 +82,9 @@ int gptk_selftest_bounded_wait(unsigned timeout_us, unsigned *dev_err, void *str
  * every GPU loading this library holds until the process exits.
  * Limits: head_dim 64; B * H * T <= 1048576, else GPT_ERR_SHAPE (nothing is launched).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
- * make that first call before any stream capture. All calls on one device share the array:
+ * make that first call before any stream capture. The address is kept for later calls; a
+ * cudaDeviceReset invalidates it (do not use this entry point after one). Host threads may
+ * make their first calls at the same time. All calls on one device share the array:
  * calls that overlap on the GPU (unordered streams) race on it. Nothing in it needs clearing
  * between calls: every row of D is written before it is read. Calls no allocating routine. */
 int gptk_attention_bwd_bf16_noalloc(const void *qkv, const void *o, const void *dout,

@@ -47,6 +47,8 @@ extern "C" {
 #define GPT_ERR_DEVICE_TIMEOUT -7  /* a bounded device-side wait expired                      */
 #define GPT_ERR_BAD_TOKEN      -8  /* a token id outside [0, vocab) or target outside [0, vocab) */
 
+#define GPT_MAX_TOKENS (1 << 20) /* largest max_B * max_T (tokens of one micro-batch)         */
+
 #define GPT_FP32 0  /* validation mode: fp32 activations and fp32 GEMMs (CUDA cores)          */
 #define GPT_BF16 1  /* bf16 operands on tcgen05 tensor cores, fp32 accumulation/master state  */
 
@@ -80,7 +82,7 @@ typedef struct gpt_handle gpt_handle;
  * max_B*max_T tokens, the bf16 weight shadow, device scalars) on the current CUDA device.
  * Returns NULL and sets *status (if non-NULL) on failure. Supported shapes: n_embd % n_head
  * == 0, head_dim in {32, 64, 128} (bf16: n_embd % 64 == 0, head_dim == 64),
- * max_B * max_T <= 16384, vocab_padded <= 131072. */
+ * max_B * max_T <= GPT_MAX_TOKENS, vocab_padded <= 131072. */
 gpt_handle *gpt_create(const gpt_config *cfg, int *status);
 void gpt_destroy(gpt_handle *h);
 
@@ -110,7 +112,9 @@ int gpt_forward_loss(gpt_handle *h, const float *params, const int *tokens, cons
  * params, adam_m, adam_v: device fp32 [num_params], updated in place (caller-owned; adam_m
  * and adam_v start zeroed). grads: device fp32 [num_params], written. tokens/targets as in
  * gpt_forward_loss. loss: host float. Weight decay applies to every element.
- * On GPT_ERR_NONFINITE, params/m/v are unchanged and the step counter does not advance. */
+ * On GPT_ERR_NONFINITE, GPT_ERR_BAD_TOKEN and GPT_ERR_DEVICE_TIMEOUT the update is skipped:
+ * params, adam_m, adam_v (and the handle's bf16 weight copy) are unchanged and the step
+ * counter does not advance; grads then hold whatever the failed backward wrote. */
 int gpt_train_step(gpt_handle *h, float *params, float *grads, float *adam_m, float *adam_v,
                    const int *tokens, const int *targets, int B, int T, float lr, float wd,
                    float clip, float *loss);
@@ -146,9 +150,12 @@ int gpt_params_changed(gpt_handle *h);
 #define GPT_OPT_TIME_KERNELS 2
 int gpt_set_option(gpt_handle *h, int option, long value);
 
-/* Per kernel class accumulated by GPT_OPT_TIME_KERNELS since the last reset: launches,
- * total milliseconds and algorithmic FLOPs. kind: 0 = tensor-core GEMMs (all of them).
- * reset != 0 clears the counters after reading. */
+/* Tensor-core GEMM timings accumulated by GPT_OPT_TIME_KERNELS since the last reset.
+ * kind 0: every GEMM launch of the step: launches, total milliseconds, and the ALGORITHMIC
+ *         FLOPs (2*M*N*K of the method's own contractions: the block GEMMs, the lm_head
+ *         forward, dX and dwte; the logits recompute of the cross-entropy backward excluded);
+ * kind 1: the cross-entropy backward's logits recompute alone (launches, ms, executed FLOPs).
+ * Reading either kind with reset != 0 clears both. */
 int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
                      double *flops, int reset);
 

@@ -103,3 +103,26 @@ def oracle_adamw_on(grads, params0, m0, v0, lr, wd, clip, step, beta1=0.9, beta2
     v = np.asarray(v0, np.float64).copy()
     o.adamw(p, g, m, v, lr, wd, step, coef=coef, beta1=beta1, beta2=beta2, eps=eps)
     return p, m, v, n
+
+
+def grad_report(sh, g_test, g_ref):
+    """Per tensor (name, cosine, max|dg| / max|g_ref|) of two flat gradient vectors."""
+    out = []
+    for (name, a), (_, b) in zip(per_tensor(sh, g_test), per_tensor(sh, g_ref)):
+        out.append((name, cosine(a, b), grad_rel_err(a, b) if np.abs(b).max() > 0 else 0.0))
+    return out
+
+
+def assert_bf16_grads(sh, g_test, g_ref, what=""):
+    """North-star bf16 gradient bound: cosine >= 0.999 per tensor (tensors whose reference is
+    exactly zero must be exactly zero). Prints the per-tensor figures."""
+    rep = grad_report(sh, g_test, g_ref)
+    worst = min(rep, key=lambda r: r[1])
+    print(f"\n[{what}] worst cosine {worst[1]:.6f} ({worst[0]}); max rel err "
+          f"{max(r[2] for r in rep):.3e}")
+    for (name, a), (_, b) in zip(per_tensor(sh, g_test), per_tensor(sh, g_ref)):
+        if np.abs(b).max() == 0:
+            assert np.abs(a).max() == 0, name
+    bad = [(n, c, r) for n, c, r in rep if c < BF16_GRAD_COS]
+    assert not bad, bad
+    return rep

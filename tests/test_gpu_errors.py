@@ -26,20 +26,56 @@ def _setup(precision=1, B=2, T=64, seed=0):
     return torch, gb, st, P, bufs, torch.from_numpy(tok).to(dev), torch.from_numpy(tgt).to(dev)
 
 
-def test_bad_token_and_target_ids():
+@pytest.mark.parametrize("n_micro", [1, 2])
+def test_bad_token_and_target_ids(n_micro):
+    """An id out of range is reported and skips the update: params, m, v and the step counter
+    stay bitwise unchanged (as for a non-finite loss), for one step and an accumulated one."""
     torch, gb, st, P, (G, M, V), tk, tg = _setup()
-    bad = tk.clone()
-    bad[0, 3] = SH.vocab  # == V: outside the softmax vocabulary
-    s, _ = st.train_step_status(P, G, M, V, bad, tg, 1e-3, 0.0, 1.0)
-    assert s == gb.GPT_ERR_BAD_TOKEN
-    badt = tg.clone()
-    badt[1, 0] = -1
-    s, _ = st.train_step_status(P, G, M, V, tk, badt, 1e-3, 0.0, 1.0)
-    assert s == gb.GPT_ERR_BAD_TOKEN
-    assert st.step == 0
-    # a good step still works afterwards
-    s, loss = st.train_step_status(P, G, M, V, tk, tg, 1e-3, 0.0, 1.0)
-    assert s == 0 and np.isfinite(loss) and st.step == 1
+    # non-zero optimizer state, so an update that slipped through would show
+    st.train_step(P, G, M, V, tk, tg, 1e-3, 0.1, 1.0)
+    torch.cuda.synchronize()
+    step0 = st.step
+    tkn = tk.unsqueeze(0).repeat(n_micro, 1, 1).contiguous()
+    tgn = tg.unsqueeze(0).repeat(n_micro, 1, 1).contiguous()
+
+    def call(a, b):
+        if n_micro == 1:
+            return st.train_step_status(P, G, M, V, a[0], b[0], 1e-3, 0.1, 1.0)[0]
+        try:
+            st.train_step_accum(P, G, M, V, a, b, 1e-3, 0.1, 1.0)
+            return 0
+        except gb.GPTError as e:
+            return e.status
+
+    for which in ("token", "target"):
+        P0, M0, V0 = P.clone(), M.clone(), V.clone()
+        a, b = tkn.clone(), tgn.clone()
+        if which == "token":
+            a[n_micro - 1, 0, 3] = SH.vocab  # == V: outside the softmax vocabulary
+        else:
+            b[n_micro - 1, 1, 0] = -1
+        assert call(a, b) == gb.GPT_ERR_BAD_TOKEN
+        torch.cuda.synchronize()
+        assert torch.equal(P, P0) and torch.equal(M, M0) and torch.equal(V, V0), which
+        assert st.step == step0
+    # a good step still works afterwards and uses the unchanged state
+    Pr, Mr, Vr = P.clone(), M.clone(), V.clone()
+    assert call(tkn, tgn) == 0 and st.step == step0 + 1
+    torch.cuda.synchronize()
+    assert not torch.equal(P, Pr)
+    # the bf16 weight copy was not touched by the failed calls: a fresh handle from the same
+    # state gives the same update
+    st2 = U.make_step(SH, 2, 64, 1)
+    st2.use_current_torch_stream()
+    st2.step = step0
+    P2, M2, V2 = Pr.clone(), Mr.clone(), Vr.clone()
+    if n_micro == 1:
+        st2.train_step(P2, G, M2, V2, tk, tg, 1e-3, 0.1, 1.0)
+    else:
+        st2.train_step_accum(P2, G, M2, V2, tkn, tgn, 1e-3, 0.1, 1.0)
+    torch.cuda.synchronize()
+    assert torch.equal(P2, P) and torch.equal(M2, M) and torch.equal(V2, V)
+    st2.close()
 
 
 def test_shape_alignment_and_argument_checks():
