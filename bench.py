@@ -3,10 +3,14 @@
 iteration through the library's C ABI, on synthetic Zipf tokens and random-init weights.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--parallel dp|replicas] [--micro-batches n]
 
-Prints one JSON line (rank 0). With N > 1 (launched by torch.distributed.run), each rank
-runs an independent replica of the whole step on its own batch (the step has no data-path
-collective); the timed region is bracketed by barriers and the slowest rank's time is used.
+Prints one JSON line (rank 0). With N > 1 (launched by torch.distributed.run) each rank takes
+its own batch of the workload's size (weak scaling). --parallel dp (the default) runs one
+data-parallel optimizer step over all ranks' batches: gradients reduce-scattered over NCCL,
+the optimizer state split across the ranks (ZeRO-1), parameters all-gathered;
+--parallel replicas runs N independent copies of the single-GPU step. The timed region is
+bracketed by barriers and the slowest rank's time is used.
 
 --impl reference times the oracle (plain single-threaded C++ CPU definition of the step) on
 the host cores, each step a bounded sample (B=1, a short causal prefix) of the workload.
@@ -196,6 +200,33 @@ def run_reference(args, wl, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def kernel_table(kst, n_steps, pk, pk_kind):
+    """Per kernel class: launches and ms per step, achieved rate on algorithmic work, and the
+    fraction of the measured copy bandwidth (bytes) or bf16 burst peak (FLOPs)."""
+    out = {}
+    for name, (n, ms, work, unit) in kst.items():
+        if n == 0 or ms <= 0:
+            continue
+        rec = {"launches_per_step": n / n_steps, "ms_per_step": ms / n_steps}
+        if unit == "byte":
+            gbs = work / (ms / 1000) / 1e9
+            rec.update({"achieved": gbs, "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                        "bound": "hbm", "work_per_launch": work / n})
+        else:
+            tf = work / (ms / 1000) / 1e12
+            rec.update({"achieved": tf, "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"],
+                        "bound": "tensor", "work_per_launch": work / n})
+        out[name] = rec
+    out["_peaks"] = f"{pk_kind}: {pk['hbm_gbs']} GB/s copy, {pk['bf16_tflops']} TFLOP/s bf16 burst"
+    return out
+
+
+def use_dp(args, world: int) -> bool:
+    """The data-parallel step runs for --parallel dp under torch.distributed.run (any world
+    size, so one GPU can run it too); a plain single-process run takes the one-GPU step."""
+    return args.parallel == "dp" and (world > 1 or "WORLD_SIZE" in os.environ)
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import numpy as np
     import torch
@@ -215,10 +246,17 @@ def run_ours(args, wl, rank, world, local_rank):
         tok, tgt = tok.reshape(nm, B, T), tgt.reshape(nm, B, T)
     st = gb.GPTStep.from_workload(wl, lmhead_chunk_rows=args.lmhead_chunk_rows)
     stream = torch.cuda.Stream(device=dev)
-    P = torch.from_numpy(p).to(dev)
-    G = torch.zeros_like(P)
-    Mm = torch.zeros_like(P)
-    Vv = torch.zeros_like(P)
+    dp = None
+    if use_dp(args, world):
+        # data parallelism with the optimizer state split across the ranks (ZeRO-1)
+        from gpt_transformer_step_b200.dp import DataParallelStep
+        dp = DataParallelStep(st, st.n_params, world, rank, dev, dist)
+        P, G, GS, Mm, Vv = dp.alloc(p)
+    else:
+        P = torch.from_numpy(p).to(dev)
+        G = torch.zeros_like(P)
+        Mm = torch.zeros_like(P)
+        Vv = torch.zeros_like(P)
     tk = torch.from_numpy(tok).to(dev)
     tg = torch.from_numpy(tgt).to(dev)
     tk_h = torch.from_numpy(tok).pin_memory()
@@ -230,6 +268,8 @@ def run_ours(args, wl, rank, world, local_rank):
             dist.barrier()
 
     def step(a, b):
+        if dp is not None:
+            return dp.train_step(P, G, GS, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
         if nm > 1:
             return st.train_step_accum(P, G, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
         return st.train_step(P, G, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
@@ -258,7 +298,7 @@ def run_ours(args, wl, rank, world, local_rank):
         for _ in range(args.warmup):
             step(tk, tg)
     torch.cuda.synchronize()
-    launches = st.last_launch_count()
+    launches = st.last_launch_count() + (2 if dp is not None else 0)  # + sumsq, ranged AdamW
 
     clk = Clocks(local_rank, args.clock_log)
     clk.start()
@@ -268,14 +308,16 @@ def run_ours(args, wl, rank, world, local_rank):
     # end to end through the same C ABI call with host (pinned) token buffers
     ms_e2e, _, ms_e2e_med = timed(args.steps, host_inputs=True)
 
-    # dominant kernel class (tensor-core GEMMs): CUDA events around every GEMM launch
+    # every kernel class, CUDA events around each launch on the step's stream (separate
+    # instrumented steps: graphs are off while timing)
     n_inst = max(2, args.steps // 4)
     st.set_option(gb.GPT_OPT_TIME_KERNELS, 1)
     st.kernel_stats(reset=True)
     timed(n_inst)
-    n_rc, rc_ms, rc_flops = st.kernel_stats(kind=1)
-    n_l, gemm_ms, gemm_flops = st.kernel_stats(kind=0, reset=True)
+    kst = st.all_kernel_stats(reset=True)
     st.set_option(gb.GPT_OPT_TIME_KERNELS, 0)
+    n_rc, rc_ms, rc_flops, _ = kst["gemm_recompute"]
+    n_l, gemm_ms, gemm_flops, _ = kst["gemm"]
 
     if rank != 0:
         return
@@ -298,7 +340,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "data": "synthetic (Zipf tokens, N(0,0.02) init)",
         "config": {"workload": wl.name, "global_batch": world * nm * B, "seq_len": T,
                    "micro_batches": nm,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "parallelism": f"dp{world}-zero1" if dp is not None
+                   else (f"replicas{world}" if world > 1 else "single"),
                    "l2": "working set ~6 GB >> 126 MB L2 (no flush needed)"},
         "mfu": {"nominal_2250": value / world * fpt / 2.25e15,
                 "measured_burst": value / world * fpt / (peak_b * 1e12),
@@ -324,6 +367,7 @@ def run_ours(args, wl, rank, world, local_rank):
                      "gemm_tflop_per_step": gemm_flops / n_inst / 1e12,
                      "recompute": {"launches": n_rc, "ms_per_step": rc_ms / n_inst,
                                    "tflop_per_step": rc_flops / n_inst / 1e12}},
+        "kernels": kernel_table(kst, n_inst, pk, pk_kind),
         "clocks": clocks,
         "gpu_launches": launches * args.steps,
     }
@@ -343,6 +387,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-log", default=None,
                     help="keep the nvidia-smi clock samples of the timed region in this file")
+    ap.add_argument("--parallel", default="dp", choices=["dp", "replicas"],
+                    help="with --gpus N > 1: data parallelism with ZeRO-1 optimizer sharding "
+                         "(gradients exchanged over NCCL) or N independent replicas")
     ap.add_argument("--micro-batches", type=int, default=1,
                     help="micro-batches of B x T per optimizer step (gradient accumulation)")
     ap.add_argument("--lmhead-chunk-rows", type=int, default=0,
@@ -356,7 +403,8 @@ def main():
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
         return
-    if world > 1:
+    pg = world > 1 or use_dp(args, world)
+    if pg:
         import datetime
 
         import torch
@@ -366,7 +414,7 @@ def main():
     try:
         run_ours(args, wl, rank, world, local_rank)
     finally:
-        if world > 1:
+        if pg:
             import torch.distributed as dist
             dist.destroy_process_group()
 

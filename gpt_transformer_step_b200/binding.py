@@ -30,6 +30,11 @@ GPT_FP32 = 0
 GPT_BF16 = 1
 GPT_OPT_USE_GRAPHS = 1
 GPT_OPT_TIME_KERNELS = 2
+# kernel classes of gpt_kernel_stats: (id, name, unit of the algorithmic work)
+KSTATS = [(0, "gemm", "flop"), (1, "gemm_recompute", "flop"), (2, "attn_fwd", "flop"),
+          (3, "attn_bwd", "flop"), (4, "ln_fwd", "byte"), (5, "ln_bwd", "byte"),
+          (6, "embed_fwd", "byte"), (7, "embed_bwd", "byte"), (8, "ce_combine", "byte"),
+          (9, "grad_norm", "byte"), (10, "adamw", "byte")]
 
 EXPORTED = [
     "gpt_create", "gpt_destroy", "gpt_num_params", "gpt_param_layout", "gpt_set_stream",
@@ -38,7 +43,7 @@ EXPORTED = [
     "gpt_params_changed", "gpt_set_option", "gpt_kernel_stats", "gpt_last_launch_count",
     "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
     "gptk_attention_bwd_bf16", "gptk_attention_bwd_bf16_noalloc", "gptk_selftest_bounded_wait",
-    "gptk_gemm_plan",
+    "gptk_gemm_plan", "gpt_forward_backward", "gpt_sumsq", "gpt_adamw_ranges",
 ]
 
 
@@ -84,6 +89,11 @@ gpt_train_step = _sig("gpt_train_step", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I,
                                              ctypes.POINTER(_F)])
 gpt_train_step_accum = _sig("gpt_train_step_accum", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
                                                          _F, _F, _F, ctypes.POINTER(_F)])
+gpt_forward_backward = _sig("gpt_forward_backward", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _F,
+                                                         ctypes.POINTER(_F)])
+gpt_sumsq = _sig("gpt_sumsq", _I, [_P, _P, ctypes.c_size_t, _P])
+gpt_adamw_ranges = _sig("gpt_adamw_ranges", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _F, _F, _F, _P,
+                                                 ctypes.c_long])
 gpt_get_step = _sig("gpt_get_step", _I, [_P, ctypes.POINTER(ctypes.c_long)])
 gpt_set_step = _sig("gpt_set_step", _I, [_P, ctypes.c_long])
 gpt_last_grad_norm = _sig("gpt_last_grad_norm", _F, [_P])
@@ -222,6 +232,33 @@ class GPTStep:
         self._check(s, "gpt_train_step_accum")
         return loss.value
 
+    def forward_backward(self, params, grads, tokens, targets, grad_scale=1.0) -> float:
+        """Forward + backward only (no clip, no update): tokens/targets [B, T] or
+        [n_micro, B, T]; grads = grad_scale * gradient of the mean loss. Returns the loss."""
+        if len(tokens.shape) == 2:
+            n_micro, (B, T) = 1, tokens.shape
+        else:
+            n_micro, B, T = tokens.shape
+        loss = ctypes.c_float(0)
+        s = gpt_forward_backward(self.h, _ptr(params), _ptr(grads), _ptr(tokens), _ptr(targets),
+                                 n_micro, B, T, grad_scale, ctypes.byref(loss))
+        self._check(s, "gpt_forward_backward")
+        return loss.value
+
+    def sumsq(self, x, out):
+        """out (device float64 tensor, 1 element) = sum of x^2 (device fp32), enqueued."""
+        self._check(gpt_sumsq(self.h, _ptr(x), x.numel(), _ptr(out)), "gpt_sumsq")
+
+    def adamw_ranges(self, params, grads, adam_m, adam_v, ranges, lr, wd, clip, sumsq, step):
+        """AdamW on params[off:off+cnt] for (off, cnt) in ranges; grads, adam_m, adam_v hold
+        the ranges compactly; sumsq: device float64 global sum of squares."""
+        n = len(ranges)
+        offs = (ctypes.c_longlong * max(n, 1))(*[r[0] for r in ranges])
+        cnts = (ctypes.c_longlong * max(n, 1))(*[r[1] for r in ranges])
+        s = gpt_adamw_ranges(self.h, _ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v), offs,
+                             cnts, n, lr, wd, clip, _ptr(sumsq), step)
+        self._check(s, "gpt_adamw_ranges")
+
     def train_step_status(self, params, grads, adam_m, adam_v, tokens, targets, lr, wd, clip):
         """Like train_step, but returns (status, loss) without raising."""
         B, T = tokens.shape
@@ -256,6 +293,16 @@ class GPTStep:
         self._check(gpt_kernel_stats(self.h, kind, ctypes.byref(n), ctypes.byref(ms),
                                      ctypes.byref(fl), int(reset)), "gpt_kernel_stats")
         return n.value, ms.value, fl.value
+
+    def all_kernel_stats(self, reset: bool = True):
+        """{name: (launches, ms, work, unit)} for every kernel class; clears them if reset."""
+        out = {}
+        for k, name, unit in KSTATS:
+            n, ms, w = self.kernel_stats(kind=k)
+            out[name] = (n, ms, w, unit)
+        if reset:
+            self.kernel_stats(reset=True)
+        return out
 
     def last_launch_count(self) -> int:
         return int(gpt_last_launch_count(self.h))

@@ -28,7 +28,8 @@ struct DevScalars {
   int nonfinite;       // a loss or the norm not finite: the update is skipped
   unsigned err;        // GPT_DEVERR_* bits
   unsigned counter;    // arrival counter of the grad-norm last-block reduction
-  int pad1[7];
+  unsigned counter2;   // arrival counter of gpt_sumsq's last-block reduction
+  int pad1[6];
 };
 
 // ---- type helpers -----------------------------------------------------------------------

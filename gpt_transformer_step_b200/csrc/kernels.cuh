@@ -51,6 +51,21 @@ int grad_norm_blocks();
 cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, bf16 *shadow, size_t n,
                          const DevScalars *sc, cudaStream_t st);
 
+// Sharded optimizer pieces (data parallelism): sum of squares into a device double, and
+// AdamW over parameter ranges with compactly stored gradients and moments.
+constexpr int ADAM_MAX_RANGES = 64;
+struct AdamRanges {
+  int n;
+  long long offset[ADAM_MAX_RANGES];  // first parameter of range k (multiple of 4)
+  long long count[ADAM_MAX_RANGES];   // elements of range k (multiple of 4)
+  long long base[ADAM_MAX_RANGES];    // compact offset of range k in g, m, v
+  float lr, wd, clip, beta1, beta2, eps, bias1, bias2;
+};
+cudaError_t launch_sumsq(const float *x, size_t n, double *partials, unsigned *counter,
+                         double *out, cudaStream_t st);
+cudaError_t launch_adamw_ranges(float *p, const float *g, float *m, float *v,
+                                const AdamRanges &rg, const double *sumsq, cudaStream_t st);
+
 // fp32 -> bf16 copy of the weights.
 cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st);
 

@@ -667,6 +667,78 @@ __global__ void adamw_kernel(float *__restrict__ p, const float *__restrict__ g,
     }
 }
 
+// ------------------------------------------------------------------------------------------
+// Sharded optimizer pieces (data parallelism with the optimizer state split across ranks)
+// ------------------------------------------------------------------------------------------
+// out = sum of x[i]^2 over [0, n): the same fixed partition and in-order combine of the
+// partials as grad_norm_kernel, into a caller-owned device double.
+__global__ void __launch_bounds__(GN_THREADS)
+sumsq_kernel(const float *__restrict__ x, size_t n, double *__restrict__ partials,
+             unsigned *__restrict__ counter, double *__restrict__ out) {
+  __shared__ double sh[GN_THREADS / 32];
+  __shared__ bool last;
+  const size_t n4 = n / 4;
+  const size_t per = (n4 + gridDim.x - 1) / gridDim.x;
+  const size_t b0 = blockIdx.x * per, b1 = min(n4, b0 + per);
+  float s = 0.f;
+  const float4 *x4 = reinterpret_cast<const float4 *>(x);
+  for (size_t i = b0 + threadIdx.x; i < b1; i += blockDim.x) {
+    float4 v = x4[i];
+    s += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (blockIdx.x == gridDim.x - 1)
+    for (size_t i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) s += x[i] * x[i];
+  double d = (double)s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = d;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < GN_THREADS / 32; ++w) t += sh[w];
+    partials[blockIdx.x] = t;
+    __threadfence();
+    last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    double t = 0.0;
+    for (int b = 0; b < (int)gridDim.x; ++b) t += ((volatile double *)partials)[b];
+    *out = t;
+    *counter = 0u;
+  }
+}
+
+// AdamW over a list of parameter ranges whose gradients and moments are stored compactly
+// (range k at compact offset base[k]); the clip coefficient comes from the global sum of
+// squares in device memory. Same arithmetic as adamw_kernel.
+__global__ void adamw_ranges_kernel(float *__restrict__ p, const float *__restrict__ g,
+                                    float *__restrict__ m, float *__restrict__ v,
+                                    AdamRanges rg, const double *__restrict__ sumsq) {
+  const int k = blockIdx.y;
+  const double t = *sumsq;
+  float coef = (float)((double)rg.clip / (sqrt(t) + 1e-6));
+  coef = coef > 1.f ? 1.f : coef;
+  if (!isfinite(t)) return;
+  const size_t n4 = (size_t)rg.count[k] / 4;
+  float4 *p4 = reinterpret_cast<float4 *>(p + rg.offset[k]);
+  const float4 *g4 = reinterpret_cast<const float4 *>(g + rg.base[k]);
+  float4 *m4 = reinterpret_cast<float4 *>(m + rg.base[k]);
+  float4 *v4 = reinterpret_cast<float4 *>(v + rg.base[k]);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 P = p4[i], G = g4[i], Mm = m4[i], Vv = v4[i];
+    adamw_one(P.x, G.x, Mm.x, Vv.x, rg.lr, rg.wd, rg.beta1, rg.beta2, rg.eps, rg.bias1, rg.bias2, coef);
+    adamw_one(P.y, G.y, Mm.y, Vv.y, rg.lr, rg.wd, rg.beta1, rg.beta2, rg.eps, rg.bias1, rg.bias2, coef);
+    adamw_one(P.z, G.z, Mm.z, Vv.z, rg.lr, rg.wd, rg.beta1, rg.beta2, rg.eps, rg.bias1, rg.bias2, coef);
+    adamw_one(P.w, G.w, Mm.w, Vv.w, rg.lr, rg.wd, rg.beta1, rg.beta2, rg.eps, rg.bias1, rg.bias2, coef);
+    p4[i] = P;
+    m4[i] = Mm;
+    v4[i] = Vv;
+  }
+}
+
 __global__ void to_bf16_kernel(const float *__restrict__ p, bf16 *__restrict__ out, size_t n) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
@@ -816,6 +888,23 @@ cudaError_t launch_grad_norm(const float *g, size_t n, double *partials, DevScal
 cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, bf16 *shadow, size_t n,
                          const DevScalars *sc, cudaStream_t st) {
   adamw_kernel<<<grid_for((long)(n / 4), 256, 148 * 8), 256, 0, st>>>(p, g, m, v, shadow, n, sc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sumsq(const float *x, size_t n, double *partials, unsigned *counter,
+                         double *out, cudaStream_t st) {
+  sumsq_kernel<<<GN_BLOCKS, GN_THREADS, 0, st>>>(x, n, partials, counter, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_adamw_ranges(float *p, const float *g, float *m, float *v,
+                                const AdamRanges &rg, const double *sumsq, cudaStream_t st) {
+  long most = 1;
+  for (int k = 0; k < rg.n; ++k) most = rg.count[k] > most ? rg.count[k] : most;
+  int bx = grid_for(most / 4, 256, 148 * 8);
+  const int per_range = (148 * 8 + rg.n - 1) / rg.n;
+  if (bx > per_range) bx = per_range < 1 ? 1 : per_range;
+  adamw_ranges_kernel<<<dim3(bx, rg.n), 256, 0, st>>>(p, g, m, v, rg, sumsq);
   return cudaGetLastError();
 }
 

@@ -101,11 +101,11 @@ struct gpt_handle {
   // kernel timing
   bool time_kernels;
   std::vector<cudaEvent_t> ev;
-  std::vector<double> ev_flops;
-  std::vector<int> ev_kind;  // 0: the method's own GEMM work, 1: the lm_head logits recompute
+  std::vector<double> ev_work;  // algorithmic FLOPs or bytes of the launch
+  std::vector<int> ev_kind;     // GPT_KSTAT_* class of the launch
   int ev_used;
-  long long stat_launches[2];
-  double stat_ms[2], stat_flops[2];
+  long long stat_launches[GPT_KSTAT_COUNT];
+  double stat_ms[GPT_KSTAT_COUNT], stat_work[GPT_KSTAT_COUNT];
   TcGemm *tc;
 };
 
@@ -136,6 +136,28 @@ bool is_device_ptr(const void *p) {
 }
 
 // --------------------------------------------------------------------------------------
+// per-launch timing (GPT_OPT_TIME_KERNELS): CUDA events on the step's stream around a launch,
+// with the launch's algorithmic work, accumulated per kernel class by finish()
+// --------------------------------------------------------------------------------------
+int tbegin(gpt_handle *h, int kind, double work) {
+  if (!h->time_kernels || h->ev_used + 2 > (int)h->ev.size()) return -1;
+  const int k = h->ev_used;
+  h->ev_used += 2;
+  h->ev_work[k / 2] = work;
+  h->ev_kind[k / 2] = kind;
+  return cudaEventRecord(h->ev[k], h->stream) == cudaSuccess ? k : -1;
+}
+cudaError_t tend(gpt_handle *h, int k) {
+  return k >= 0 ? cudaEventRecord(h->ev[k + 1], h->stream) : cudaSuccess;
+}
+#define TIMED(h, kind, work, call)                 \
+  do {                                             \
+    const int tk__ = tbegin((h), (kind), (work));  \
+    CUDA_TRY(call);                                \
+    CUDA_TRY(tend((h), tk__));                     \
+  } while (0)
+
+// --------------------------------------------------------------------------------------
 // GEMM dispatch
 // --------------------------------------------------------------------------------------
 int choose_split(const gpt_handle *h, int M, int N, int K, int tm, int tn) {
@@ -150,15 +172,8 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
   if (d.M <= 0 || d.N <= 0) return cudaSuccess;
   d.epi.sc = h->sc;  // device error word and 1/M for every epilogue
   const double flops = 2.0 * d.M * d.N * d.K;
-  int k = -1;
-  if (h->time_kernels && h->ev_used + 2 <= (int)h->ev.size()) {
-    k = h->ev_used;
-    h->ev_used += 2;
-    h->ev_flops[k / 2] = flops;
-    h->ev_kind[k / 2] = d.epi.kind == EPI_CE_DS ? 1 : 0;
-    cudaError_t e = cudaEventRecord(h->ev[k], h->stream);
-    if (e != cudaSuccess) return e;
-  }
+  const int k = tbegin(h, d.epi.kind == EPI_CE_DS ? GPT_KSTAT_GEMM_RECOMPUTE : GPT_KSTAT_GEMM,
+                       flops);
   cudaError_t e;
   const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
   const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
@@ -192,8 +207,7 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
   }
   h->launches += 1 + (d.split_k > 1 ? 1 : 0);
   if (e != cudaSuccess) return e;
-  if (k >= 0) return cudaEventRecord(h->ev[k + 1], h->stream);
-  return cudaSuccess;
+  return tend(h, k);
 }
 
 GemmDesc gdesc(int M, int N, int K, const void *A, long lda, int ak, const void *B, long ldb,
@@ -235,6 +249,13 @@ cudaError_t attention_bwd<bf16>(gpt_handle *h, const bf16 *qkv, const bf16 *o, c
                                     h->stream);
 }
 
+// Admitted (query, key) pairs of one head's causal attention over T positions with left
+// window w (w < 0: full causal): sum over queries of min(i, w) + 1.
+double admitted_scores(long T, long w) {
+  if (w < 0 || w >= T - 1) return (double)T * (T + 1) / 2.0;
+  return (double)(w + 1) * T - (double)w * (w + 1) / 2.0;
+}
+
 // --------------------------------------------------------------------------------------
 // the step schedule
 // --------------------------------------------------------------------------------------
@@ -247,27 +268,40 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   const T *W = h->use_bf16 ? (const T *)h->shadow : (const T *)params;
   DevScalars *sc = h->sc;
   int &nl = h->launches;
-  h->ev_used = 0;
+
+  // algorithmic work per launch (kernel timing): bytes of the memory-bound kernels, FLOPs
+  // of the contractions (4 hd per admitted score forward, 8 hd backward; the backward's
+  // recompute of the scores is not counted)
+  const double es = h->use_bf16 ? 2.0 : 4.0;
+  const double ln_fwd_bytes = (double)M * (2.0 * C * es + 8.0) + C * es;
+  const double ln_bwd_bytes = (double)M * (4.0 * C * es + 8.0) + C * es + 4.0 * C;
+  auto attn_flops = [&](int w, double per_score) {
+    return per_score * h->hd * admitted_scores(Tlen, w) * B * H;
+  };
 
   // ---------------- forward ----------------
   T *x0 = (T *)h->acts[0].x_in;
-  CUDA_TRY(launch_embed_fwd<T>(h->tok, h->tgt, W + h->off_wte, W + h->off_wpe, x0, M, Tlen, C,
-                               V, sc, st)); nl++;
+  TIMED(h, GPT_KSTAT_EMBED_FWD, (double)M * 3.0 * C * es + 8.0 * M,
+        (launch_embed_fwd<T>(h->tok, h->tgt, W + h->off_wte, W + h->off_wpe, x0, M, Tlen, C, V,
+                             sc, st))); nl++;
   for (int l = 0; l < h->L; ++l) {
     Acts &A = h->acts[l];
     const Layer &P = h->layer[l];
     T *xnext = (T *)(l + 1 < h->L ? h->acts[l + 1].x_in : h->x_final);
-    CUDA_TRY(launch_layernorm_fwd<T>((T *)A.x_in, W + P.ln1, (T *)A.a, A.mu1, A.rs1, M, C,
-                                     h->cfg.ln_eps, st)); nl++;
+    TIMED(h, GPT_KSTAT_LN_FWD, ln_fwd_bytes,
+          launch_layernorm_fwd<T>((T *)A.x_in, W + P.ln1, (T *)A.a, A.mu1, A.rs1, M, C,
+                                  h->cfg.ln_eps, st)); nl++;
     GemmDesc d = gdesc(M, 3 * C, C, A.a, C, 1, W + P.wqkv, C, 1);
     d.epi.kind = EPI_STORE; d.epi.out = A.qkv; d.epi.ldo = 3 * C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(attention_fwd<T>(h, (T *)A.qkv, (T *)A.o, A.lse, B, Tlen, h->windows[l])); nl++;
+    TIMED(h, GPT_KSTAT_ATTN_FWD, attn_flops(h->windows[l], 4.0),
+          attention_fwd<T>(h, (T *)A.qkv, (T *)A.o, A.lse, B, Tlen, h->windows[l])); nl++;
     d = gdesc(M, C, C, A.o, C, 1, W + P.wap, C, 1);
     d.epi.kind = EPI_RESID; d.epi.out = A.x_mid; d.epi.ldo = C; d.epi.aux = A.x_in; d.epi.ld_aux = C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(launch_layernorm_fwd<T>((T *)A.x_mid, W + P.ln2, (T *)A.c, A.mu2, A.rs2, M, C,
-                                     h->cfg.ln_eps, st)); nl++;
+    TIMED(h, GPT_KSTAT_LN_FWD, ln_fwd_bytes,
+          launch_layernorm_fwd<T>((T *)A.x_mid, W + P.ln2, (T *)A.c, A.mu2, A.rs2, M, C,
+                                  h->cfg.ln_eps, st)); nl++;
     d = gdesc(M, mC, C, A.c, C, 1, W + P.wfc, C, 1);
     d.epi.kind = EPI_STORE_GELU; d.epi.out = A.dgelu; d.epi.ldo = mC; d.epi.out2 = A.h; d.epi.ldo2 = mC;
     CUDA_TRY(gemm(h, d));
@@ -275,8 +309,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d.epi.kind = EPI_RESID; d.epi.out = xnext; d.epi.ldo = C; d.epi.aux = A.x_mid; d.epi.ld_aux = C;
     CUDA_TRY(gemm(h, d));
   }
-  CUDA_TRY(launch_layernorm_fwd<T>((T *)h->x_final, W + h->off_lnf, (T *)h->yf, h->muf, h->rsf,
-                                   M, C, h->cfg.ln_eps, st)); nl++;
+  TIMED(h, GPT_KSTAT_LN_FWD, ln_fwd_bytes,
+        launch_layernorm_fwd<T>((T *)h->x_final, W + h->off_lnf, (T *)h->yf, h->muf, h->rsf, M, C,
+                                h->cfg.ln_eps, st)); nl++;
   // lm_head statistics (the logits stay on chip)
   {
     GemmDesc d = gdesc(M, V, C, h->yf, C, 1, W + h->off_wte, C, 1);
@@ -285,8 +320,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     e.kind = EPI_CE_STATS; e.targets = h->tgt; e.stats = h->stats; e.tgt_logit = h->tgt_logit;
     e.V = V; e.row_offset = 0; e.sc = sc;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(launch_ce_combine(h->stats, h->tgt_logit, h->lse_ce, h->per_token, M, h->ce_ntiles,
-                               sc, st)); nl += 2;
+    TIMED(h, GPT_KSTAT_CE, (double)M * (h->ce_ntiles * 8.0 + 16.0),
+          launch_ce_combine(h->stats, h->tgt_logit, h->lse_ce, h->per_token, M, h->ce_ntiles, sc,
+                            st)); nl += 2;
   }
   if (per_token_out) {
     CUDA_TRY(cudaMemcpyAsync(per_token_out, h->per_token, sizeof(float) * M,
@@ -323,8 +359,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(gemm(h, d));
   }
   T *dx = (T *)h->dx;  // the residual-stream gradient starts here (nothing to add to)
-  CUDA_TRY(launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf,
-                                   dx, h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
+  TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes - (double)M * C * es,
+        launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf, dx,
+                                h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
   for (int l = h->L - 1; l >= 0; --l) {
     Acts &A = h->acts[l];
     const Layer &P = h->layer[l];
@@ -341,8 +378,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d = gdesc(mC, C, M, h->dh, mC, 0, A.c, C, 0);
     d.epi.kind = wgrad; d.epi.outf = G + P.wfc; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx,
-                                     h->dg_partial, G + P.ln2, M, C, st, acc)); nl += 2;
+    TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
+          launch_layernorm_bwd<T>((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx,
+                                  h->dg_partial, G + P.ln2, M, C, st, acc)); nl += 2;
     // attention: x_mid = x_in + attn(a) Wap^T
     d = gdesc(M, C, C, dx, C, 1, W + P.wap, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dout; d.epi.ldo = C;
@@ -350,25 +388,30 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
     d.epi.kind = wgrad; d.epi.outf = G + P.wap; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B,
-                              Tlen, h->windows[l])); nl += 2;
+    TIMED(h, GPT_KSTAT_ATTN_BWD, attn_flops(h->windows[l], 8.0),
+          attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B, Tlen,
+                           h->windows[l])); nl += 2;
     d = gdesc(M, C, 3 * C, h->dqkv, 3 * C, 1, W + P.wqkv, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
     d = gdesc(3 * C, C, M, h->dqkv, 3 * C, 0, A.a, C, 0);
     d.epi.kind = wgrad; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
     CUDA_TRY(gemm(h, d));
-    CUDA_TRY(launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
-                                     h->dg_partial, G + P.ln1, M, C, st, acc)); nl += 2;
+    TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
+          launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
+                                  h->dg_partial, G + P.ln1, M, C, st, acc)); nl += 2;
   }
   EmbedBwdWs ew{h->emb_ws};
-  CUDA_TRY(launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C,
-                               h->Vp, ew, st, acc)); nl += embed_bwd_launches(h->Vp);
+  TIMED(h, GPT_KSTAT_EMBED_BWD, (double)M * C * es + 4.0 * C * h->maxT * (acc ? 2 : 1) + 8.0 * M,
+        launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C, h->Vp,
+                            ew, st, acc)); nl += embed_bwd_launches(h->Vp);
   if (phase == PH_FIRST || phase == PH_MIDDLE) return cudaSuccess;  // update after the last
   // ---------------- clip + AdamW ----------------
-  CUDA_TRY(launch_grad_norm(G, h->nparams, h->gn_partials, sc, st)); nl++;
-  CUDA_TRY(launch_adamw((float *)params, G, adam_m, adam_v, h->use_bf16 ? h->shadow : nullptr,
-                        h->nparams, sc, st)); nl++;
+  TIMED(h, GPT_KSTAT_GRAD_NORM, 4.0 * h->nparams,
+        launch_grad_norm(G, h->nparams, h->gn_partials, sc, st)); nl++;
+  TIMED(h, GPT_KSTAT_ADAMW, (h->use_bf16 ? 30.0 : 28.0) * h->nparams,
+        launch_adamw((float *)params, G, adam_m, adam_v, h->use_bf16 ? h->shadow : nullptr,
+                     h->nparams, sc, st)); nl++;
   return cudaSuccess;
 }
 
@@ -441,10 +484,11 @@ int finish(gpt_handle *h, float *loss, int n_micro = 1) {
       if (cudaEventElapsedTime(&ms, h->ev[k], h->ev[k + 1]) == cudaSuccess) {
         const int kind = h->ev_kind[k / 2];
         h->stat_ms[kind] += ms;
-        h->stat_flops[kind] += h->ev_flops[k / 2];
+        h->stat_work[kind] += h->ev_work[k / 2];
         h->stat_launches[kind]++;
       }
     }
+    h->ev_used = 0;
   }
   const unsigned err = h->sc_host->err;
   if (err & GPT_DEVERR_TIMEOUT) return GPT_ERR_DEVICE_TIMEOUT;
@@ -526,7 +570,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   h->use_graphs = true;
   h->time_kernels = false;
   h->ev_used = 0;
-  for (int k = 0; k < 2; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_flops[k] = 0; }
+  for (int k = 0; k < GPT_KSTAT_COUNT; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_work[k] = 0; }
   h->tc = nullptr;
   cudaGetDevice(&h->device);
 
@@ -669,6 +713,7 @@ int gpt_forward_loss(gpt_handle *h, const float *params, const int *tokens, cons
   if (!loss) return GPT_ERR_INVALID_ARG;
   cudaSetDevice(h->device);
   const int M = B * T;
+  h->ev_used = 0;
   set_hyper(h, M, 0.f, 0.f, 1.f, h->step + 1);
   if ((s = stage_inputs(h, tokens, targets, M))) return s;
   if (h->use_bf16) {  // forward-only calls refresh the bf16 weights every time
@@ -701,6 +746,7 @@ int gpt_train_step_accum(gpt_handle *h, float *params, float *grads, float *adam
   cudaSetDevice(h->device);
   const int M = B * T;
   const long t = h->step + 1;
+  h->ev_used = 0;
   set_hyper(h, (long)n_micro * M, lr, wd, clip, t);
   if (h->use_bf16 && (!h->shadow_valid || h->shadow_src != params)) {
     TRY(launch_to_bf16(params, h->shadow, h->nparams, h->stream));
@@ -720,6 +766,83 @@ int gpt_train_step_accum(gpt_handle *h, float *params, float *grads, float *adam
   if (s) return s;
   if (h->sc_host->nonfinite) return GPT_ERR_NONFINITE;
   h->step = t;
+  return GPT_OK;
+}
+
+int gpt_forward_backward(gpt_handle *h, const float *params, float *grads, const int *tokens,
+                         const int *targets, int n_micro, int B, int T, float grad_scale,
+                         float *loss) {
+  int s = check_common(h, params, tokens, targets, B, T);
+  if (s) return s;
+  if (!grads || !loss || n_micro < 1 || !isfinite(grad_scale)) return GPT_ERR_INVALID_ARG;
+  if (misaligned(grads)) return GPT_ERR_ALIGN;
+  cudaSetDevice(h->device);
+  const int M = B * T;
+  h->ev_used = 0;
+  // the gradient of the mean loss over all n_micro * B * T positions, times grad_scale
+  set_hyper(h, (long)n_micro * M, 0.f, 0.f, 1.f, h->step + 1);
+  h->sc_host->inv_M = (float)((double)grad_scale / ((double)n_micro * M));
+  if (h->use_bf16 && (!h->shadow_valid || h->shadow_src != params)) {
+    TRY(launch_to_bf16(params, h->shadow, h->nparams, h->stream));
+    h->shadow_src = params;
+    h->shadow_valid = true;
+  }
+  int launches = 0;
+  for (int i = 0; i < n_micro; ++i) {
+    // gradients stored by the first micro-batch, added by the others; no update
+    const int phase = i == 0 ? PH_FIRST : PH_MIDDLE;
+    if ((s = stage_inputs(h, tokens + (size_t)i * M, targets + (size_t)i * M, M, i == 0))) return s;
+    if ((s = launch_step(h, params, grads, nullptr, nullptr, B, T, true, nullptr, phase))) return s;
+    launches += h->launches;
+  }
+  h->launches = launches;
+  s = finish(h, loss, n_micro);
+  if (s) return s;
+  return h->sc_host->nonfinite ? GPT_ERR_NONFINITE : GPT_OK;
+}
+
+int gpt_sumsq(gpt_handle *h, const float *x, size_t n, double *sumsq_dev) {
+  if (!h || !x || !sumsq_dev) return GPT_ERR_INVALID_ARG;
+  if (misaligned(x) || ((uintptr_t)sumsq_dev & 7u)) return GPT_ERR_ALIGN;
+  cudaSetDevice(h->device);
+  unsigned *counter = (unsigned *)((char *)h->sc + offsetof(DevScalars, counter2));
+  TRY(launch_sumsq(x, n, h->gn_partials, counter, sumsq_dev, h->stream));
+  return GPT_OK;
+}
+
+int gpt_adamw_ranges(gpt_handle *h, float *params, const float *grads, float *adam_m,
+                     float *adam_v, const long long *offsets, const long long *counts,
+                     int nranges, float lr, float wd, float clip, const double *sumsq_dev,
+                     long step) {
+  if (!h || !params || !grads || !adam_m || !adam_v || !offsets || !counts || !sumsq_dev)
+    return GPT_ERR_INVALID_ARG;
+  if (nranges < 0 || nranges > ADAM_MAX_RANGES || step < 1 || !isfinite(lr) || !isfinite(wd) ||
+      !(clip > 0.f))
+    return GPT_ERR_INVALID_ARG;
+  if (misaligned(params) || misaligned(grads) || misaligned(adam_m) || misaligned(adam_v) ||
+      ((uintptr_t)sumsq_dev & 7u))
+    return GPT_ERR_ALIGN;
+  if (nranges == 0) return GPT_OK;
+  AdamRanges rg;
+  memset(&rg, 0, sizeof(rg));
+  rg.n = nranges;
+  long long base = 0;
+  for (int k = 0; k < nranges; ++k) {
+    if (offsets[k] < 0 || counts[k] < 0 || offsets[k] + counts[k] > (long long)h->nparams)
+      return GPT_ERR_SHAPE;
+    if ((offsets[k] & 3) || (counts[k] & 3)) return GPT_ERR_ALIGN;
+    rg.offset[k] = offsets[k];
+    rg.count[k] = counts[k];
+    rg.base[k] = base;
+    base += counts[k];
+  }
+  rg.lr = lr; rg.wd = wd; rg.clip = clip;
+  rg.beta1 = h->cfg.beta1; rg.beta2 = h->cfg.beta2; rg.eps = h->cfg.adam_eps;
+  rg.bias1 = (float)(1.0 - pow((double)h->cfg.beta1, (double)step));
+  rg.bias2 = (float)(1.0 - pow((double)h->cfg.beta2, (double)step));
+  cudaSetDevice(h->device);
+  TRY(launch_adamw_ranges(params, grads, adam_m, adam_v, rg, sumsq_dev, h->stream));
+  h->shadow_valid = false;  // params changed outside the step
   return GPT_OK;
 }
 
@@ -747,9 +870,9 @@ int gpt_set_option(gpt_handle *h, int option, long value) {
   if (option == GPT_OPT_TIME_KERNELS) {
     h->time_kernels = value != 0;
     if (h->time_kernels && h->ev.empty()) {
-      const int n = 2 * (16 * h->L + 64);
+      const int n = 2 * (48 * h->L + 256);
       h->ev.resize(n);
-      h->ev_flops.assign(n / 2, 0.0);
+      h->ev_work.assign(n / 2, 0.0);
       h->ev_kind.assign(n / 2, 0);
       for (int i = 0; i < n; ++i)
         if (cudaEventCreate(&h->ev[i]) != cudaSuccess) return fail(h, cudaGetLastError());
@@ -760,17 +883,17 @@ int gpt_set_option(gpt_handle *h, int option, long value) {
 }
 
 int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
-                     double *flops, int reset) {
-  if (!h || kind < 0 || kind > 1) return GPT_ERR_INVALID_ARG;
-  // kind 0: every GEMM launch (time), the method's own FLOPs (the recompute excluded);
-  // kind 1: the lm_head logits recompute of the cross-entropy backward alone
-  const long long n = kind == 0 ? h->stat_launches[0] + h->stat_launches[1] : h->stat_launches[1];
-  const double ms = kind == 0 ? h->stat_ms[0] + h->stat_ms[1] : h->stat_ms[1];
+                     double *work, int reset) {
+  if (!h || kind < 0 || kind >= GPT_KSTAT_COUNT) return GPT_ERR_INVALID_ARG;
+  // GEMM: every GEMM launch's time with the method's own FLOPs (the recompute excluded)
+  const bool all_gemm = kind == GPT_KSTAT_GEMM;
+  const long long n = h->stat_launches[kind] + (all_gemm ? h->stat_launches[GPT_KSTAT_GEMM_RECOMPUTE] : 0);
+  const double ms = h->stat_ms[kind] + (all_gemm ? h->stat_ms[GPT_KSTAT_GEMM_RECOMPUTE] : 0.0);
   if (launches) *launches = n;
   if (total_ms) *total_ms = ms;
-  if (flops) *flops = h->stat_flops[kind];
+  if (work) *work = h->stat_work[kind];
   if (reset) {
-    for (int k = 0; k < 2; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_flops[k] = 0; }
+    for (int k = 0; k < GPT_KSTAT_COUNT; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_work[k] = 0; }
   }
   return GPT_OK;
 }

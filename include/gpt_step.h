@@ -132,6 +132,40 @@ int gpt_train_step_accum(gpt_handle *h, float *params, float *grads, float *adam
                          float *adam_v, const int *tokens, const int *targets, int n_micro,
                          int B, int T, float lr, float wd, float clip, float *loss);
 
+/* ---- data parallelism with sharded optimizer state --------------------------------------
+ * The pieces of one data-parallel step (the nanoGPT README's DDP reproduction, "reproducing
+ * GPT-2", and the llm.c summary, "Ejecución": ZeRO-1, the optimizer state split across
+ * ranks). Each rank runs gpt_forward_backward on its own batch; the caller reduce-scatters
+ * the gradients (the rank keeps the sum over ranks of its own ranges), all-reduces one
+ * gpt_sumsq per rank into the global sum of squares, runs gpt_adamw_ranges on its ranges and
+ * all-gathers the parameters. The collectives belong to the caller (NCCL, for instance). */
+
+/* Forward and backward over n_micro micro-batches (layout as gpt_train_step_accum), no
+ * clip, no update, step counter unchanged: grads (written) = grad_scale * d(mean loss over
+ * the n_micro*B*T positions)/d(params). With grad_scale = 1/world_size the SUM of the ranks'
+ * grads is the gradient of the global mean loss. loss: host, this call's mean loss.
+ * GPT_ERR_NONFINITE when a loss is not finite (grads are written all the same). */
+int gpt_forward_backward(gpt_handle *h, const float *params, float *grads, const int *tokens,
+                         const int *targets, int n_micro, int B, int T, float grad_scale,
+                         float *loss);
+
+/* *sumsq_dev (a device double, 8-byte aligned) = sum over x[0..n) of x^2: device fp32 x,
+ * 16-byte aligned; float sums per thread, double across them, in a fixed order. Enqueued on
+ * the handle's stream; does not synchronise. */
+int gpt_sumsq(gpt_handle *h, const float *x, size_t n, double *sumsq_dev);
+
+/* AdamW (the arithmetic of gpt_train_step) on nranges <= 64 parameter ranges: range k is
+ * params[offsets[k] .. offsets[k]+counts[k]) (offsets, counts: host arrays, multiples of 4);
+ * its gradients and moments are stored compactly: grads, adam_m, adam_v hold the ranges one
+ * after the other (range k at sum_{j<k} counts[j]). The clip coefficient is
+ * min(1, clip / (sqrt(*sumsq_dev) + 1e-6)) with *sumsq_dev the global sum of squares in device
+ * memory; nothing is updated when it is not finite. step: t >= 1 of the bias corrections
+ * (the handle's counter is not used or changed). The bf16 weight copy is marked stale. */
+int gpt_adamw_ranges(gpt_handle *h, float *params, const float *grads, float *adam_m,
+                     float *adam_v, const long long *offsets, const long long *counts,
+                     int nranges, float lr, float wd, float clip, const double *sumsq_dev,
+                     long step);
+
 /* Step counter (number of completed AdamW updates); gpt_set_step is for resuming. */
 int gpt_get_step(const gpt_handle *h, long *step);
 int gpt_set_step(gpt_handle *h, long step);
@@ -150,14 +184,39 @@ int gpt_params_changed(gpt_handle *h);
 #define GPT_OPT_TIME_KERNELS 2
 int gpt_set_option(gpt_handle *h, int option, long value);
 
-/* Tensor-core GEMM timings accumulated by GPT_OPT_TIME_KERNELS since the last reset.
- * kind 0: every GEMM launch of the step: launches, total milliseconds, and the ALGORITHMIC
- *         FLOPs (2*M*N*K of the method's own contractions: the block GEMMs, the lm_head
- *         forward, dX and dwte; the logits recompute of the cross-entropy backward excluded);
- * kind 1: the cross-entropy backward's logits recompute alone (launches, ms, executed FLOPs).
- * Reading either kind with reset != 0 clears both. */
+/* Kernel timings accumulated by GPT_OPT_TIME_KERNELS since the last reset: CUDA events on the
+ * step's stream around each launch of the class `kind` (CUDA graphs are off while timing).
+ * *launches, *total_ms, and *work = the launches' ALGORITHMIC work:
+ *   GPT_KSTAT_GEMM            every tensor-core GEMM launch's time; work = FLOPs (2*M*N*K) of the
+ *                             method's own contractions (block GEMMs, lm_head forward, dX, dwte),
+ *                             the cross-entropy backward's logits recompute excluded
+ *   GPT_KSTAT_GEMM_RECOMPUTE  that logits recompute alone (executed FLOPs)
+ *   GPT_KSTAT_ATTN_FWD / _BWD FLOPs: 4*hd (forward) and 8*hd (backward) per admitted score
+ *                             (the backward's recompute of the scores not counted)
+ *   GPT_KSTAT_LN_FWD          bytes: bf16 x read, y written, mean/rstd written (4C+8 per row)
+ *   GPT_KSTAT_LN_BWD          bytes: x, dy, residual gradient read, residual gradient written
+ *                             (8C+8 per row in bf16; the first has no residual input)
+ *   GPT_KSTAT_EMBED_FWD/_BWD  bytes: wte and wpe rows read, x written (6C per token);
+ *                             dx read once and dwpe written (the per-id fp32 rows not counted)
+ *   GPT_KSTAT_CE              bytes of the cross-entropy combine (statistics read)
+ *   GPT_KSTAT_GRAD_NORM       bytes: 4 per parameter
+ *   GPT_KSTAT_ADAMW           bytes: 30 per parameter in bf16 mode (p, g, m, v read; p, m, v
+ *                             and the bf16 copy written), 28 in fp32 mode
+ * Reading any kind with reset != 0 clears all of them. */
+#define GPT_KSTAT_GEMM 0
+#define GPT_KSTAT_GEMM_RECOMPUTE 1
+#define GPT_KSTAT_ATTN_FWD 2
+#define GPT_KSTAT_ATTN_BWD 3
+#define GPT_KSTAT_LN_FWD 4
+#define GPT_KSTAT_LN_BWD 5
+#define GPT_KSTAT_EMBED_FWD 6
+#define GPT_KSTAT_EMBED_BWD 7
+#define GPT_KSTAT_CE 8
+#define GPT_KSTAT_GRAD_NORM 9
+#define GPT_KSTAT_ADAMW 10
+#define GPT_KSTAT_COUNT 11
 int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
-                     double *flops, int reset);
+                     double *work, int reset);
 
 /* Number of kernels the last gpt_train_step / gpt_forward_loss enqueued. */
 int gpt_last_launch_count(const gpt_handle *h);

@@ -56,7 +56,7 @@ def _cfg(gb, **kw):
 @pytest.mark.parametrize("bad,code", [
     (dict(vocab=0), -1), (dict(vocab_padded=10), -1), (dict(precision=7), -1),
     (dict(beta1=1.0), -1), (dict(adam_eps=0.0), -1), (dict(n_head=3), -2),
-    (dict(n_embd=96, n_head=1), -2), (dict(max_B=64, max_T=1024), -2),
+    (dict(n_embd=96, n_head=1), -2), (dict(max_B=2048, max_T=1024), -2),
     (dict(precision=1, n_embd=96, n_head=3), -2), (dict(vocab_padded=200000), -2),
 ])
 def test_create_rejects_bad_config_without_touching_the_gpu(gb, bad, code):
