@@ -244,7 +244,8 @@ def run_ours(args, wl, rank, world, local_rank):
     tok, tgt = fx.zipf_tokens(sh.vocab, wl.zipf_s, nm * B, T, seed=rank)  # own batch per replica
     if nm > 1:
         tok, tgt = tok.reshape(nm, B, T), tgt.reshape(nm, B, T)
-    st = gb.GPTStep.from_workload(wl, lmhead_chunk_rows=args.lmhead_chunk_rows)
+    st = gb.GPTStep.from_workload(wl, lmhead_chunk_rows=args.lmhead_chunk_rows,
+                                  recompute_gelu=args.recompute)
     stream = torch.cuda.Stream(device=dev)
     dp = None
     if use_dp(args, world):
@@ -267,7 +268,16 @@ def run_ours(args, wl, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    muon_cfg = None
+    if args.optimizer == "muon":
+        from gpt_transformer_step_b200.muon import MuonConfig
+        muon_cfg = MuonConfig()
+
     def step(a, b):
+        if muon_cfg is not None:  # hybrid Muon + AdamW: forward/backward, then the update
+            loss = st.forward_backward(P, G, a, b)
+            st.muon_update(P, G, Mm, Vv, wl.lr, wl.wd, wl.clip, muon_cfg)
+            return loss
         if dp is not None:
             return dp.train_step(P, G, GS, Mm, Vv, a, b, wl.lr, wl.wd, wl.clip)
         if nm > 1:
@@ -299,6 +309,11 @@ def run_ours(args, wl, rank, world, local_rank):
             step(tk, tg)
     torch.cuda.synchronize()
     launches = st.last_launch_count() + (2 if dp is not None else 0)  # + sumsq, ranged AdamW
+    if muon_cfg is not None:  # the update's launches (the last call was the update)
+        st.forward_backward(P, G, tk, tg)
+        launches = st.last_launch_count()
+        st.muon_update(P, G, Mm, Vv, wl.lr, wl.wd, wl.clip, muon_cfg)
+        launches += st.last_launch_count()
 
     clk = Clocks(local_rank, args.clock_log)
     clk.start()
@@ -339,7 +354,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (Zipf tokens, N(0,0.02) init)",
         "config": {"workload": wl.name, "global_batch": world * nm * B, "seq_len": T,
-                   "micro_batches": nm,
+                   "micro_batches": nm, "recompute_gelu": bool(args.recompute),
+                   "optimizer": args.optimizer,
                    "parallelism": f"dp{world}-zero1" if dp is not None
                    else (f"replicas{world}" if world > 1 else "single"),
                    "l2": "working set ~6 GB >> 126 MB L2 (no flush needed)"},
@@ -392,6 +408,10 @@ def main():
                          "(gradients exchanged over NCCL) or N independent replicas")
     ap.add_argument("--micro-batches", type=int, default=1,
                     help="micro-batches of B x T per optimizer step (gradient accumulation)")
+    ap.add_argument("--optimizer", default="adamw", choices=["adamw", "muon"],
+                    help="muon: the hybrid Muon (block matrices) + AdamW update")
+    ap.add_argument("--recompute", action="store_true",
+                    help="activation recompute: GELU recomputed in the backward (llm.c -r)")
     ap.add_argument("--lmhead-chunk-rows", type=int, default=0,
                     help="rows per lm_head backward chunk (0 = the library default)")
     args = ap.parse_args()

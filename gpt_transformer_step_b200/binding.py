@@ -34,7 +34,7 @@ GPT_OPT_TIME_KERNELS = 2
 KSTATS = [(0, "gemm", "flop"), (1, "gemm_recompute", "flop"), (2, "attn_fwd", "flop"),
           (3, "attn_bwd", "flop"), (4, "ln_fwd", "byte"), (5, "ln_bwd", "byte"),
           (6, "embed_fwd", "byte"), (7, "embed_bwd", "byte"), (8, "ce_combine", "byte"),
-          (9, "grad_norm", "byte"), (10, "adamw", "byte")]
+          (9, "grad_norm", "byte"), (10, "adamw", "byte"), (11, "muon", "flop")]
 
 EXPORTED = [
     "gpt_create", "gpt_destroy", "gpt_num_params", "gpt_param_layout", "gpt_set_stream",
@@ -43,7 +43,7 @@ EXPORTED = [
     "gpt_params_changed", "gpt_set_option", "gpt_kernel_stats", "gpt_last_launch_count",
     "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
     "gptk_attention_bwd_bf16", "gptk_attention_bwd_bf16_noalloc", "gptk_selftest_bounded_wait",
-    "gptk_gemm_plan", "gpt_forward_backward", "gpt_sumsq", "gpt_adamw_ranges",
+    "gptk_gemm_plan", "gpt_forward_backward", "gpt_sumsq", "gpt_adamw_ranges", "gpt_muon_update",
 ]
 
 
@@ -54,7 +54,13 @@ class gpt_config(ctypes.Structure):
                 ("window_left", ctypes.POINTER(ctypes.c_int)), ("ln_eps", ctypes.c_float),
                 ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("adam_eps", ctypes.c_float), ("precision", ctypes.c_int),
-                ("lmhead_chunk_rows", ctypes.c_int)]
+                ("lmhead_chunk_rows", ctypes.c_int), ("recompute_gelu", ctypes.c_int)]
+
+
+class gpt_muon_config(ctypes.Structure):
+    _fields_ = [("matrix_lr", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("momentum", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("ns_steps", ctypes.c_int), ("coeffs", ctypes.POINTER(ctypes.c_float))]
 
 
 class gpt_tensor_desc(ctypes.Structure):
@@ -94,6 +100,8 @@ gpt_forward_backward = _sig("gpt_forward_backward", _I, [_P, _P, _P, _P, _P, _I,
 gpt_sumsq = _sig("gpt_sumsq", _I, [_P, _P, ctypes.c_size_t, _P])
 gpt_adamw_ranges = _sig("gpt_adamw_ranges", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _F, _F, _F, _P,
                                                  ctypes.c_long])
+gpt_muon_update = _sig("gpt_muon_update", _I, [_P, _P, _P, _P, _P, ctypes.POINTER(gpt_muon_config),
+                                               _F, _F, _F])
 gpt_get_step = _sig("gpt_get_step", _I, [_P, ctypes.POINTER(ctypes.c_long)])
 gpt_set_step = _sig("gpt_set_step", _I, [_P, ctypes.c_long])
 gpt_last_grad_norm = _sig("gpt_last_grad_norm", _F, [_P])
@@ -155,11 +163,11 @@ class GPTStep:
                  max_T: int, max_B: int, mlp_mult: int = 4,
                  window_left: Optional[Sequence[int]] = None, precision: int = GPT_BF16,
                  ln_eps: float = 1e-5, beta1: float = 0.9, beta2: float = 0.95,
-                 adam_eps: float = 1e-8, lmhead_chunk_rows: int = 0):
+                 adam_eps: float = 1e-8, lmhead_chunk_rows: int = 0, recompute_gelu: bool = False):
         self._win = (ctypes.c_int * n_layer)(*(window_left or [-1] * n_layer))
         cfg = gpt_config(vocab, vocab_padded, n_layer, n_head, n_embd, max_T, max_B, mlp_mult,
                          ctypes.cast(self._win, ctypes.POINTER(ctypes.c_int)), ln_eps, beta1,
-                         beta2, adam_eps, precision, lmhead_chunk_rows)
+                         beta2, adam_eps, precision, lmhead_chunk_rows, int(recompute_gelu))
         st = ctypes.c_int(0)
         self.h = gpt_create(ctypes.byref(cfg), ctypes.byref(st))
         if not self.h:
@@ -258,6 +266,19 @@ class GPTStep:
         s = gpt_adamw_ranges(self.h, _ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v), offs,
                              cnts, n, lr, wd, clip, _ptr(sumsq), step)
         self._check(s, "gpt_adamw_ranges")
+
+    def muon_update(self, params, grads, adam_m, adam_v, lr, wd, clip, muon=None):
+        """The hybrid Muon + AdamW update on the raw gradient `grads` (gpt_muon_update);
+        muon: a muon.MuonConfig (defaults: the page's matrix_lr 0.02, Polar Express x5)."""
+        from gpt_transformer_step_b200.muon import MuonConfig
+        mc_py = muon or MuonConfig()
+        cf = (ctypes.c_float * max(1, 3 * mc_py.ns_steps))(
+            *[float(x) for x in list(mc_py.coeffs.reshape(-1))[:3 * mc_py.ns_steps]])
+        mc = gpt_muon_config(mc_py.matrix_lr, mc_py.weight_decay, mc_py.momentum, mc_py.beta2,
+                             mc_py.eps, mc_py.ns_steps, ctypes.cast(cf, ctypes.POINTER(ctypes.c_float)))
+        s = gpt_muon_update(self.h, _ptr(params), _ptr(grads), _ptr(adam_m), _ptr(adam_v),
+                            ctypes.byref(mc), lr, wd, clip)
+        self._check(s, "gpt_muon_update")
 
     def train_step_status(self, params, grads, adam_m, adam_v, tokens, targets, lr, wd, clip):
         """Like train_step, but returns (status, loss) without raising."""

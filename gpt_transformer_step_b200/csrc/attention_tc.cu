@@ -272,9 +272,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
 #pragma unroll
         for (int i = 0; i < 128; ++i) sv[i] = (i <= hi && i >= lo) ? sv[i] : -INFINITY;
       }
-      float mx = sv[0];
+      // row max as a tree of independent partial maxima (a 128-long dependent chain of
+      // fmaxf would dominate the row's latency)
+      float mp[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+      for (int k = 0; k < 8; ++k) mp[k] = sv[k];
+#pragma unroll
+      for (int i = 8; i < 128; i += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = fmaxf(mp[k], sv[i + k]);
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
       float mnew = m2;
       bool resc = false;
@@ -301,7 +309,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       m2 = mnew;
       if (mt > -INFINITY) have = true;
       const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
-      float ls = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (no long FADD chain)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -309,12 +317,12 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         for (int i = 0; i < 32; i += 2) {
           const float p0 = ex2(fmaf(sv[c * 32 + i], P.scale_log2, -mu));
           const float p1 = ex2(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
-          ls += p0 + p1;
+          ls[(i >> 1) & 3] += p0 + p1;
           pk[i >> 1] = pack_bf16(p0, p1);
         }
         st_tmem_bf16x32(tP + c * 16, pk);
       }
-      l += ls;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

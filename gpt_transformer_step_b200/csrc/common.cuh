@@ -107,6 +107,11 @@ enum EpiKind {
   EPI_CE_STATS,       // per (row, column tile): max and sum(exp(acc - max)) over cols < V;
                       // the target's logit to tgt_logit[row]
   EPI_CE_DS,          // out[m][n] = (exp(acc - lse[row]) - [n == target]) * inv_M, 0 for n >= V
+  // GELU recompute (the backward recomputes the activation instead of the forward keeping it)
+  EPI_STORE_PRE_GELU, // out[m][n] = acc (pre-activation) ; out2[m][n] = gelu(acc)
+  EPI_DGELU_RECOMP,   // out[m][n] = acc * gelu'(aux[m][n]) ; out2[m][n] = gelu(aux[m][n]),
+                      // aux = the pre-activation the forward kept
+  EPI_AXPBY,          // out[m][n] = alpha * acc + beta * aux[m][n]        (activation type)
 };
 
 struct Epi {
@@ -124,6 +129,8 @@ struct Epi {
   int V;
   int row_offset;
   const DevScalars *sc;  // inv_M
+  float alpha, beta;     // EPI_AXPBY
+  long aux_bstride;      // batched GEMMs: elements between the aux matrices of two batches
 };
 
 struct GemmDesc {
@@ -134,6 +141,10 @@ struct GemmDesc {
   int split_k;       // > 1: fp32 partials [split][M][N] then an ordered reduction
   float *partial;
   unsigned *err;     // device error word (bounded-wait timeouts); NULL = &epi.sc->err
+  // batched GEMM (tensor-core path; no K split): `batch` independent products, operand and
+  // output matrices `*_bstride` elements apart (0 or 1: one product)
+  int batch;
+  long a_bstride, b_bstride, out_bstride;
 };
 
 template <typename T>
@@ -154,6 +165,23 @@ __device__ __forceinline__ void epi_elem(const Epi &e, int m, int n, float acc) 
     case EPI_DGELU: {
       float gd = to_f(((const T *)e.aux)[(long)m * e.ld_aux + n]);
       ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(acc * gd);
+      break;
+    }
+    case EPI_STORE_PRE_GELU: {  // gelu of the stored (rounded) value: recompute is exact
+      const T pre = from_f<T>(acc);
+      ((T *)e.out)[(long)m * e.ldo + n] = pre;
+      ((T *)e.out2)[(long)m * e.ldo2 + n] = from_f<T>(gelu_t<T>(to_f(pre)));
+      break;
+    }
+    case EPI_DGELU_RECOMP: {
+      const float pre = to_f(((const T *)e.aux)[(long)m * e.ld_aux + n]);
+      ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(acc * gelu_grad_t<T>(pre));
+      ((T *)e.out2)[(long)m * e.ldo2 + n] = from_f<T>(gelu_t<T>(pre));
+      break;
+    }
+    case EPI_AXPBY: {
+      const float a = to_f(((const T *)e.aux)[(long)m * e.ld_aux + n]);
+      ((T *)e.out)[(long)m * e.ldo + n] = from_f<T>(e.alpha * acc + e.beta * a);
       break;
     }
     case EPI_F32_STORE:

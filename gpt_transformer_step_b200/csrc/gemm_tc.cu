@@ -40,13 +40,18 @@ constexpr int TMEM_COLS = 512;
 
 enum TcEpi {
   TE_STORE = 0, TE_STORE_GELU, TE_RESID, TE_DGELU, TE_F32_STORE, TE_F32_ACCUM, TE_CE_STATS,
-  TE_CE_DS, TE_PARTIAL
+  TE_CE_DS, TE_PARTIAL, TE_STORE_PRE_GELU, TE_DGELU_RECOMP, TE_AXPBY
 };
+// epilogues that read an auxiliary bf16 input of the output's shape
+__host__ __device__ constexpr bool epi_has_aux(int e) {
+  return e == TE_RESID || e == TE_DGELU || e == TE_DGELU_RECOMP || e == TE_AXPBY;
+}
 
 struct TcParams {
   int M, N, K;
   int num_mt, num_nt, splits, kblocks_per_split, total_kblocks;
   int units;
+  int batch;       // independent products (batched GEMM); units = tiles * splits * batch
   int n_fast;      // 1: units walk the N tiles of one M tile first (see unit_coords)
   int a_mn, b_mn;  // 1 = MN-major
   uint32_t idesc;
@@ -59,7 +64,9 @@ struct TcParams {
 // the same time share the B tile; when A is the larger operand and does not fit in L2 (the
 // lm_head backward's dS chunk, read by the dX and dwte GEMMs) they are numbered N tile
 // fastest instead, so that the CTAs reading one A tile run together and A crosses HBM once.
-__device__ __forceinline__ void unit_coords(const TcParams &P, int u, int &mt, int &nt, int &z) {
+// z is the K split of the unit and bz its product of a batched GEMM.
+__device__ __forceinline__ void unit_coords(const TcParams &P, int u, int &mt, int &nt, int &z,
+                                            int &bz) {
   if (P.n_fast) {
     nt = u % P.num_nt;
     mt = (u / P.num_nt) % P.num_mt;
@@ -67,7 +74,9 @@ __device__ __forceinline__ void unit_coords(const TcParams &P, int u, int &mt, i
     mt = u % P.num_mt;
     nt = (u / P.num_mt) % P.num_nt;
   }
-  z = u / (P.num_mt * P.num_nt);
+  const int zz = u / (P.num_mt * P.num_nt);
+  z = zz % P.splits;
+  bz = zz / P.splits;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -98,9 +107,10 @@ __device__ __forceinline__ EpiRow epi_row(const TcParams &P, int row) {
 
 // 32 bf16 of the auxiliary input (residual stream, or gelu' stored by the forward) of one row, packed;
 // zeros past M or N.
-__device__ __forceinline__ void load_aux_chunk(const TcParams &P, int row, int col0, uint4 (&a)[4]) {
+__device__ __forceinline__ void load_aux_chunk(const TcParams &P, int row, int col0, int bz,
+                                               uint4 (&a)[4]) {
   const Epi &e = P.epi;
-  const bf16 *src = (const bf16 *)e.aux + (long)row * e.ld_aux + col0;
+  const bf16 *src = (const bf16 *)e.aux + (long)bz * e.aux_bstride + (long)row * e.ld_aux + col0;
   if (row < P.M && col0 + 32 <= P.N) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) a[q] = reinterpret_cast<const uint4 *>(src)[q];
@@ -217,18 +227,18 @@ __device__ __forceinline__ void mbar_expect_tx_addr(uint32_t addr, uint32_t byte
 // address, possibly in the peer CTA of the pair).
 template <int CG>
 __device__ __forceinline__ void tma_load_pair(void *dst, const CUtensorMap *map,
-                                              uint32_t mbar_cluster, int c0, int c1) {
+                                              uint32_t mbar_cluster, int c0, int c1, int c2) {
   if (CG == 2)
     asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1)
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
   else
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1)
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 template <int CG>
@@ -279,6 +289,12 @@ __device__ __forceinline__ void epi_math(const TcParams &P, int col0, const EpiR
     unpack_bf16x32(aux, a);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = EPI == TE_RESID ? a[i] + v[i] : v[i] * a[i];
+  } else if (EPI == TE_AXPBY) {
+    float a[32];
+    unpack_bf16x32(aux, a);
+    const float al = P.epi.alpha, be = P.epi.beta;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = fmaf(al, v[i], be * a[i]);
   } else if (EPI == TE_STORE_GELU) {
     // out = gelu'(acc) (kept for the backward instead of the pre-activation), out2 = gelu(acc)
 #pragma unroll
@@ -286,6 +302,24 @@ __device__ __forceinline__ void epi_math(const TcParams &P, int col0, const EpiR
       float g;
       v2[i] = gelu_and_grad_fast(v[i], g);
       v[i] = g;
+    }
+  } else if (EPI == TE_STORE_PRE_GELU) {
+    // out = bf16(acc) (the pre-activation, kept for the backward), out2 = gelu of that same
+    // bf16 value, so that the backward's recomputed activation is bitwise the forward's
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+      v2[i] = gelu_fast(v[i]);
+    }
+  } else if (EPI == TE_DGELU_RECOMP) {
+    // out = acc * gelu'(pre), out2 = gelu(pre): both from the kept pre-activation
+    float a[32];
+    unpack_bf16x32(aux, a);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float g;
+      v2[i] = gelu_and_grad_fast(a[i], g);
+      v[i] *= g;
     }
   }
 }
@@ -365,8 +399,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       bool ok = true;
       uint32_t issued = 0, last_par = 0;
       for (int u = unit0; u < P.units && ok; u += ustride) {
-        int mt, nt, z;
-        unit_coords(P, u, mt, nt, z);
+        int mt, nt, z, bz;
+        unit_coords(P, u, mt, nt, z, bz);
         const int m0 = mt * BM * CG + (int)rank * BM;
         const int n0 = nt * BN + (int)rank * Cf::B_ROWS;
         const int kb0 = z * P.kblocks_per_split;
@@ -380,17 +414,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (rank == 0) mbar_expect_tx_addr(fb, Cf::STAGE * CG);
           const int k0 = kb * BK;
           if (!P.a_mn) {
-            tma_load_pair<CG>(sA, &tmA, fbl, k0, m0);
+            tma_load_pair<CG>(sA, &tmA, fbl, k0, m0, bz);
           } else {
-            tma_load_pair<CG>(sA, &tmA, fbl, m0, k0);
-            tma_load_pair<CG>(sA + A_BYTES / 2, &tmA, fbl, m0 + 64, k0);
+            tma_load_pair<CG>(sA, &tmA, fbl, m0, k0, bz);
+            tma_load_pair<CG>(sA + A_BYTES / 2, &tmA, fbl, m0 + 64, k0, bz);
           }
           if (!P.b_mn) {
-            tma_load_pair<CG>(sB, &tmB, fbl, k0, n0);
+            tma_load_pair<CG>(sB, &tmB, fbl, k0, n0, bz);
           } else {
 #pragma unroll
             for (int j = 0; j < Cf::B_ROWS / 64; ++j)
-              tma_load_pair<CG>(sB + j * 8192, &tmB, fbl, n0 + 64 * j, k0);
+              tma_load_pair<CG>(sB + j * 8192, &tmB, fbl, n0 + 64 * j, k0, bz);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -421,7 +455,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t a_lbo = P.a_mn ? 8192u : 16u;
       const uint32_t b_lbo = P.b_mn ? 8192u : 16u;
       for (int u = unit0; u < P.units && ok; u += ustride, ++i) {
-        const int z = u / (P.num_mt * P.num_nt);
+        const int z = (u / (P.num_mt * P.num_nt)) % P.splits;
         const int kb0 = z * P.kblocks_per_split;
         const int kb1 = min(P.total_kblocks, kb0 + P.kblocks_per_split);
         const int acc = i & 1;
@@ -454,7 +488,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int half = (warp - 2) >> 2;
     constexpr int OUT_BYTES = (EPI == TE_F32_STORE || EPI == TE_F32_ACCUM || EPI == TE_PARTIAL) ? 4 : 2;
     constexpr int SLOT_BYTES = 32 * 32 * OUT_BYTES;
-    constexpr int NOUT = EPI == TE_STORE_GELU ? 2 : 1;
+    constexpr int NOUT = (EPI == TE_STORE_GELU || EPI == TE_STORE_PRE_GELU || EPI == TE_DGELU_RECOMP) ? 2 : 1;
     constexpr int CHUNK_SLOTS = Cf::WARP_STAGE / (SLOT_BYTES * NOUT) >= 4 ? 4
                               : Cf::WARP_STAGE / (SLOT_BYTES * NOUT);
     static_assert(CHUNK_SLOTS >= 1, "epilogue staging too small");
@@ -462,8 +496,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int chunk_seq = 0;
     int i = 0;
     for (int u = unit0; u < P.units; u += ustride, ++i) {
-      int mt, nt, z;
-      unit_coords(P, u, mt, nt, z);
+      int mt, nt, z, bz;
+      unit_coords(P, u, mt, nt, z, bz);
       const int acc = i & 1;
       const uint32_t use = (uint32_t)(i >> 1);
       const int row0 = mt * BM * CG + (int)rank * BM + q * 32;  // this warp's 32 rows
@@ -472,8 +506,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // operands that do not depend on the accumulators: loaded before the wait
       const EpiRow er = epi_row<EPI>(P, row);
       uint4 aux[4];
-      if ((EPI == TE_RESID || EPI == TE_DGELU) && c0 < min(BN, P.N - nt * BN))
-        load_aux_chunk(P, row, nt * BN + c0, aux);
+      if (epi_has_aux(EPI) && c0 < min(BN, P.N - nt * BN))
+        load_aux_chunk(P, row, nt * BN + c0, bz, aux);
       int okw = 1;
       if (lane == 0) okw = mbar_wait(&tfull_bar[acc], use & 1u, abort_flag, P.err) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -497,14 +531,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(raw[k]);
         if (more) tmem_ld32_nw(tbase + (uint32_t)((c + 1) * 32), raw);
         uint4 aux_nx[4];
-        if ((EPI == TE_RESID || EPI == TE_DGELU) && more) load_aux_chunk(P, row, col0 + 32, aux_nx);
+        if (epi_has_aux(EPI) && more) load_aux_chunk(P, row, col0 + 32, bz, aux_nx);
         if (EPI == TE_CE_STATS) {
           if (row < P.M) ce_stats_chunk(P, row, col0, er, v, ce_max, ce_sum);
           continue;
         }
         float v2[32];
         epi_math<EPI>(P, col0, er, aux, v, v2);
-        if (EPI == TE_RESID || EPI == TE_DGELU) {
+        if (epi_has_aux(EPI)) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) aux[q] = aux_nx[q];
         }
@@ -523,9 +557,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         __syncwarp();
         if (lane == 0) {
           if (EPI == TE_PARTIAL) tma_store_3d(&tmO, slot, col0, row0, z);
-          else if (EPI == TE_F32_ACCUM) tma_reduce_add_2d(&tmO, slot, col0, row0);
-          else tma_store_2d(&tmO, slot, col0, row0);
-          if (NOUT == 2) tma_store_2d(&tmO2, slot + SLOT_BYTES, col0, row0);
+          else if (EPI == TE_F32_ACCUM) tma_reduce_add_3d(&tmO, slot, col0, row0, bz);
+          else tma_store_3d(&tmO, slot, col0, row0, bz);
+          if (NOUT == 2) tma_store_3d(&tmO2, slot + SLOT_BYTES, col0, row0, bz);
           bulk_commit();
         }
         ++chunk_seq;
@@ -594,37 +628,39 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Output tensor map for the TMA-store epilogue: [rows, cols] (plus `depth` planes of
-// `plane` elements for split-K partials), box 32 x 32, bf16 with the 64-byte swizzle or fp32
-// with the 128-byte swizzle.
+// Output tensor map for the TMA-store epilogue: [depth][rows][cols] with row stride `ld` and
+// `plane` elements between planes (the products of a batched GEMM, or the split-K partials),
+// box 32 x 32 x 1, bf16 with the 64-byte swizzle or fp32 with the 128-byte one.
 bool make_out_map(CUtensorMap *m, const void *base, bool f32, long cols, long rows, long ld,
                   long depth = 1, long plane = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int es = f32 ? 4 : 2;
+  if (depth <= 1) { depth = 1; plane = ld * rows; }
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)depth};
   cuuint64_t strides[2] = {(cuuint64_t)ld * es, (cuuint64_t)plane * es};
   cuuint32_t box[3] = {32u, 32u, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
-  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-             depth > 1 ? 3 : 2, (void *)base, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE,
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             (void *)base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld, int box_outer) {
+// Operand map: bf16 [batch][outer][inner] (inner contiguous, row stride ld, `bstride`
+// elements between batches), box {64, box_outer, 1}, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld, int box_outer,
+              long batch = 1, long bstride = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)base, dims,
-                                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                      CU_TENSOR_MAP_SWIZZLE_128B,
-                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (batch <= 1) { batch = 1; bstride = ld * outer; }
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)bstride * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_outer, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -670,6 +706,9 @@ cudaError_t launch_epi(int kind, bool split, const CUtensorMap &ma, const CUtens
     case EPI_F32_ACCUM: return TC_L(TE_F32_ACCUM);
     case EPI_CE_STATS: return TC_L(TE_CE_STATS);
     case EPI_CE_DS: return TC_L(TE_CE_DS);
+    case EPI_STORE_PRE_GELU: return TC_L(TE_STORE_PRE_GELU);
+    case EPI_DGELU_RECOMP: return TC_L(TE_DGELU_RECOMP);
+    case EPI_AXPBY: return TC_L(TE_AXPBY);
     default: return cudaErrorInvalidValue;
   }
 #undef TC_L
@@ -698,15 +737,25 @@ bool tc_gemm_supported(const GemmDesc &d) {
   if ((d.lda & 7) || (d.ldb & 7)) return false;
   if (!aligned16(d.A) || !aligned16(d.B)) return false;
   const Epi &e = d.epi;
+  if (d.batch > 1) {  // batched products: bf16 outputs, 16-byte batch strides, no K split
+    if (e.kind != EPI_STORE && e.kind != EPI_AXPBY) return false;
+    if ((d.a_bstride & 7) || (d.b_bstride & 7) || (d.out_bstride & 7) || d.split_k > 1) return false;
+  }
   switch (e.kind) {
     case EPI_STORE:
     case EPI_CE_DS:
       return (e.ldo & 7) == 0 && aligned16(e.out);
     case EPI_STORE_GELU:
+    case EPI_STORE_PRE_GELU:
       return (e.ldo & 7) == 0 && (e.ldo2 & 7) == 0 && aligned16(e.out) && aligned16(e.out2);
+    case EPI_DGELU_RECOMP:
+      return (e.ldo & 7) == 0 && (e.ldo2 & 7) == 0 && (e.ld_aux & 7) == 0 && aligned16(e.out) &&
+             aligned16(e.out2) && aligned16(e.aux);
     case EPI_RESID:
     case EPI_DGELU:
-      return (e.ldo & 7) == 0 && (e.ld_aux & 7) == 0 && aligned16(e.out) && aligned16(e.aux);
+    case EPI_AXPBY:
+      return (e.ldo & 7) == 0 && (e.ld_aux & 7) == 0 && (e.aux_bstride & 7) == 0 &&
+             aligned16(e.out) && aligned16(e.aux);
     case EPI_F32_STORE:
     case EPI_F32_ACCUM:
       return (e.ldf & 3) == 0 && aligned16(e.outf);
@@ -724,8 +773,10 @@ void tc_gemm_plan(const GemmDesc &d, size_t capacity, int sms, int *cta_group, i
   const long kblocks = (d.K + BK - 1) / BK;
   const bool f32out = d.epi.kind == EPI_F32_STORE || d.epi.kind == EPI_F32_ACCUM;
   const bool elementwise = d.epi.kind != EPI_CE_STATS && d.epi.kind != EPI_CE_DS;
-  int CG = ((long)((d.M + 2 * BM - 1) / (2 * BM)) * nt >= sms / 2) ? 2 : 1;
+  const long nbatch = d.batch > 1 ? d.batch : 1;
+  int CG = ((long)((d.M + 2 * BM - 1) / (2 * BM)) * nt * nbatch >= sms / 2) ? 2 : 1;
   int S = d.split_k;
+  if (nbatch > 1) S = 1;  // batched products are not split
   if (S <= 0) {
     S = 1;
     if ((f32out || elementwise) && capacity > 0) {
@@ -736,7 +787,7 @@ void tc_gemm_plan(const GemmDesc &d, size_t capacity, int sms, int *cta_group, i
       // launch (the partial stores themselves overlap the main loop)
       double best = 1e30;
       for (int cg = 1; cg <= 2; ++cg) {
-        const long tiles = (long)((d.M + cg * BM - 1) / (cg * BM)) * nt;
+        const long tiles = (long)((d.M + cg * BM - 1) / (cg * BM)) * nt * nbatch;
         const long slots = sms / cg;
         for (int s = 1; s <= 16; ++s) {
           if (s > 1 && (kblocks / s < 4 || (size_t)s * d.M * d.N > capacity)) break;
@@ -776,7 +827,9 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   if (S > 1 && (!d.partial || (size_t)S * d.M * d.N > t->splitk_capacity)) return cudaErrorInvalidValue;
   d.split_k = S;
   P.splits = S;
-  P.units = P.num_mt * P.num_nt * S;
+  P.batch = d.batch > 1 ? d.batch : 1;
+  if (P.batch > 1 && S > 1) return cudaErrorInvalidValue;
+  P.units = P.num_mt * P.num_nt * S * P.batch;
   {
     const double a_bytes = 2.0 * d.M * d.K, b_bytes = 2.0 * d.N * d.K;
     P.n_fast = (P.num_nt > 1 && a_bytes > b_bytes && a_bytes > 48e6) ? 1 : 0;
@@ -792,10 +845,10 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   if (!P.err) return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
   const int b_rows = BN / CG;
-  bool ok = P.a_mn ? make_map(&ma, d.A, d.M, d.K, d.lda, 64)
-                   : make_map(&ma, d.A, d.K, d.M, d.lda, BM);
-  ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, 64)
-                     : make_map(&mb, d.B, d.K, d.N, d.ldb, b_rows));
+  bool ok = P.a_mn ? make_map(&ma, d.A, d.M, d.K, d.lda, 64, P.batch, d.a_bstride)
+                   : make_map(&ma, d.A, d.K, d.M, d.lda, BM, P.batch, d.a_bstride);
+  ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, 64, P.batch, d.b_bstride)
+                     : make_map(&mb, d.B, d.K, d.N, d.ldb, b_rows, P.batch, d.b_bstride));
   if (!ok) return cudaErrorInvalidValue;
   // output maps of the TMA-store epilogue (rows and columns past M, N are clipped by TMA)
   CUtensorMap mo, mo2;
@@ -806,10 +859,10 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
     ok = make_out_map(&mo, d.partial, true, d.N, d.M, d.N, S, (long)d.M * d.N);
   } else {
     switch (e0.kind) {
-      case EPI_STORE: case EPI_RESID: case EPI_DGELU: case EPI_CE_DS:
-        ok = make_out_map(&mo, e0.out, false, d.N, d.M, e0.ldo);
+      case EPI_STORE: case EPI_RESID: case EPI_DGELU: case EPI_CE_DS: case EPI_AXPBY:
+        ok = make_out_map(&mo, e0.out, false, d.N, d.M, e0.ldo, P.batch, d.out_bstride);
         break;
-      case EPI_STORE_GELU:
+      case EPI_STORE_GELU: case EPI_STORE_PRE_GELU: case EPI_DGELU_RECOMP:
         ok = make_out_map(&mo, e0.out, false, d.N, d.M, e0.ldo) &&
              make_out_map(&mo2, e0.out2, false, d.N, d.M, e0.ldo2);
         break;

@@ -42,6 +42,22 @@ __device__ __forceinline__ void store_vec<bf16>(bf16 *p, const float (&f)[8]) {
   *reinterpret_cast<uint4 *>(p) = v;
 }
 
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const typename Vec<T>::type &v, float (&f)[Vec<T>::N]);
+template <>
+__device__ __forceinline__ void unpack_vec<float>(const float4 &v, float (&f)[4]) {
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void unpack_vec<bf16>(const uint4 &v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -89,54 +105,71 @@ __global__ void embed_fwd_kernel(const int *__restrict__ tok, const int *__restr
 constexpr int LN_MAXV = 8;  // vectors per lane: C <= 32*8*VN
 
 // NV = 16-byte vectors per lane (ceil(C / (32*VN))), a compile-time bound on the row slice
-// each lane keeps in registers.
+// each lane keeps in registers. Persistent: a grid of a few blocks per SM; each warp walks its
+// rows with the next row's vectors in flight while the current row is reduced, and keeps the
+// gains in registers.
+constexpr int LNF_WARPS = 8;
 template <typename T, int NV>
-__global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
-                                     T *__restrict__ y, float *__restrict__ mean,
-                                     float *__restrict__ rstd, int M, int C, float eps) {
+__global__ void __launch_bounds__(LNF_WARPS * 32)
+layernorm_fwd_kernel(const T *__restrict__ x, const T *__restrict__ g, T *__restrict__ y,
+                     float *__restrict__ mean, float *__restrict__ rstd, int M, int C, float eps) {
+  using VT = typename Vec<T>::type;
   constexpr int VN = Vec<T>::N;
   const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= M) return;
+  const int nwarps = gridDim.x * LNF_WARPS;
   const int nv = C / VN;
-  float v[NV][VN];
-  float s = 0.f;
-#pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    int c = (lane + 32 * j) * VN;
-    if (lane + 32 * j < nv) {
-      load_vec<T>(x + (long)row * C + c, v[j]);
-#pragma unroll
-      for (int k = 0; k < VN; ++k) s += v[j][k];
-    }
-  }
-  const float mu = warp_sum(s) / (float)C;
-  float q = 0.f;
+  VT gr[NV], cur[NV], nxt[NV];
 #pragma unroll
   for (int j = 0; j < NV; ++j)
-    if (lane + 32 * j < nv) {
+    if (lane + 32 * j < nv) gr[j] = __ldg(reinterpret_cast<const VT *>(g + (lane + 32 * j) * VN));
+  auto load_row = [&](int row, VT (&v)[NV]) {
 #pragma unroll
-      for (int k = 0; k < VN; ++k) {
-        float d = v[j][k] - mu;
-        q += d * d;
+    for (int j = 0; j < NV; ++j)
+      if (lane + 32 * j < nv)
+        v[j] = *reinterpret_cast<const VT *>(x + (long)row * C + (lane + 32 * j) * VN);
+  };
+  int row = blockIdx.x * LNF_WARPS + (threadIdx.x >> 5);
+  if (row < M) load_row(row, cur);
+  for (; row < M; row += nwarps) {
+    if (row + nwarps < M) load_row(row + nwarps, nxt);
+    float v[NV][VN];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      if (lane + 32 * j < nv) {
+        unpack_vec<T>(cur[j], v[j]);
+#pragma unroll
+        for (int k = 0; k < VN; ++k) s += v[j][k];
+      }
+    const float mu = warp_sum(s) / (float)C;
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      if (lane + 32 * j < nv) {
+#pragma unroll
+        for (int k = 0; k < VN; ++k) {
+          const float d = v[j][k] - mu;
+          q += d * d;
+        }
+      }
+    const float var = warp_sum(q) / (float)C;
+    const float rs = 1.0f / sqrtf(var + eps);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      if (lane + 32 * j < nv) {
+        float gg[VN], o[VN];
+        unpack_vec<T>(gr[j], gg);
+#pragma unroll
+        for (int k = 0; k < VN; ++k) o[k] = (v[j][k] - mu) * rs * gg[k];
+        store_vec<T>(y + (long)row * C + (lane + 32 * j) * VN, o);
       }
     }
-  const float var = warp_sum(q) / (float)C;
-  const float rs = 1.0f / sqrtf(var + eps);
-#pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    int c = (lane + 32 * j) * VN;
-    if (lane + 32 * j < nv) {
-      float gg[VN], o[VN];
-      load_vec<T>(g + c, gg);
-#pragma unroll
-      for (int k = 0; k < VN; ++k) o[k] = (v[j][k] - mu) * rs * gg[k];
-      store_vec<T>(y + (long)row * C + c, o);
+    if (lane == 0) {
+      mean[row] = mu;
+      rstd[row] = rs;
     }
-  }
-  if (lane == 0) {
-    mean[row] = mu;
-    rstd[row] = rs;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) cur[j] = nxt[j];
   }
 }
 
@@ -145,22 +178,6 @@ __global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restric
 // ------------------------------------------------------------------------------------------
 constexpr int LNB_WARPS = 8;
 constexpr int LNB_MAX_BLOCKS = 296;
-
-template <typename T>
-__device__ __forceinline__ void unpack_vec(const typename Vec<T>::type &v, float (&f)[Vec<T>::N]);
-template <>
-__device__ __forceinline__ void unpack_vec<float>(const float4 &v, float (&f)[4]) {
-  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void unpack_vec<bf16>(const uint4 &v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
 
 // Each warp walks its rows with the next row's x, dy and residual gradient in flight while the
 // current row is reduced; x-hat and g*dy are recomputed from the raw vectors in the second
@@ -617,15 +634,18 @@ grad_norm_kernel(const float *__restrict__ g, size_t n, double *__restrict__ par
 // ------------------------------------------------------------------------------------------
 // K15 AdamW (order of the nanochat fused step: decay, first moment, bias correction, update)
 // ------------------------------------------------------------------------------------------
+// Every operation rounds on its own (no contraction into fused multiply-adds), so the result
+// does not depend on the kernel this is inlined into: the whole-step update and the ranged
+// update of the data-parallel step give the same bits.
 __device__ __forceinline__ void adamw_one(float &p, float g, float &m, float &v, float lr,
                                           float wd, float b1, float b2, float eps, float bias1,
                                           float bias2, float coef) {
-  g *= coef;
-  p = p * (1.f - lr * wd);
-  m = m + (1.f - b1) * (g - m);
-  v = b2 * v + (1.f - b2) * g * g;
-  float denom = sqrtf(v / bias2) + eps;
-  p = p - (lr / bias1) * m / denom;
+  g = __fmul_rn(g, coef);
+  p = __fmul_rn(p, __fsub_rn(1.f, __fmul_rn(lr, wd)));
+  m = __fadd_rn(m, __fmul_rn(__fsub_rn(1.f, b1), __fsub_rn(g, m)));
+  v = __fadd_rn(__fmul_rn(b2, v), __fmul_rn(__fmul_rn(__fsub_rn(1.f, b2), g), g));
+  const float denom = __fadd_rn(__fsqrt_rn(__fdiv_rn(v, bias2)), eps);
+  p = __fsub_rn(p, __fdiv_rn(__fmul_rn(__fdiv_rn(lr, bias1), m), denom));
 }
 
 __global__ void adamw_kernel(float *__restrict__ p, const float *__restrict__ g,
@@ -834,12 +854,32 @@ int ln_nv(int C) {
   return (C + per - 1) / per;
 }
 
+// Blocks of `kernel` (block size `threads`) resident on the whole GPU at once.
+template <typename K>
+int resident_blocks(K kernel, int threads, size_t smem) {
+  int dev = 0, sms = 148, per = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, smem) != cudaSuccess ||
+      per < 1) {
+    cudaGetLastError();
+    per = 1;
+  }
+  return per * sms;
+}
+
 template <typename T>
 cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
                                  int C, float eps, cudaStream_t st) {
-  const int warps = 8;
-  const int grid = (M + warps - 1) / warps;
-#define LNF(NVC) layernorm_fwd_kernel<T, NVC><<<grid, warps * 32, 0, st>>>(x, g, y, mean, rstd, M, C, eps)
+  const int rows_grid = (M + LNF_WARPS - 1) / LNF_WARPS;
+  // one wave of resident blocks; each warp walks several rows
+#define LNF(NVC)                                                                              \
+  {                                                                                           \
+    static int res = 0;                                                                       \
+    if (!res) res = resident_blocks(layernorm_fwd_kernel<T, NVC>, LNF_WARPS * 32, 0);         \
+    const int grid = rows_grid < res ? rows_grid : res;                                       \
+    layernorm_fwd_kernel<T, NVC><<<grid, LNF_WARPS * 32, 0, st>>>(x, g, y, mean, rstd, M, C, eps); \
+  }
   LN_DISPATCH(ln_nv<T>(C), LNF)
 #undef LNF
   return cudaGetLastError();

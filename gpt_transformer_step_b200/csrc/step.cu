@@ -23,6 +23,7 @@
 #include "../../include/gpt_step.h"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "muon.cuh"
 
 namespace {
 
@@ -34,7 +35,9 @@ struct Layer {
 };
 
 struct Acts {  // per-layer saved activations
-  void *x_in, *a, *qkv, *o, *x_mid, *c, *dgelu, *h;  // dgelu = gelu'(pre-activation)
+  // dgelu = gelu'(pre-activation), or with GELU recompute the pre-activation itself; h =
+  // gelu(pre-activation), one buffer shared by all layers with GELU recompute
+  void *x_in, *a, *qkv, *o, *x_mid, *c, *dgelu, *h;
   float *lse, *mu1, *rs1, *mu2, *rs2;
 };
 
@@ -107,6 +110,7 @@ struct gpt_handle {
   long long stat_launches[GPT_KSTAT_COUNT];
   double stat_ms[GPT_KSTAT_COUNT], stat_work[GPT_KSTAT_COUNT];
   TcGemm *tc;
+  void *muon_ws;  // Muon scratch, allocated by the first gpt_muon_update
 };
 
 namespace {
@@ -155,6 +159,13 @@ cudaError_t tend(gpt_handle *h, int k) {
     const int tk__ = tbegin((h), (kind), (work));  \
     CUDA_TRY(call);                                \
     CUDA_TRY(tend((h), tk__));                     \
+  } while (0)
+// the same in a C-ABI function (returns a GPT_ERR_* status)
+#define TIMED_S(h, kind, work, call)               \
+  do {                                             \
+    const int tk__ = tbegin((h), (kind), (work));  \
+    TRY(call);                                     \
+    TRY(tend((h), tk__));                          \
   } while (0)
 
 // --------------------------------------------------------------------------------------
@@ -303,7 +314,8 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
           launch_layernorm_fwd<T>((T *)A.x_mid, W + P.ln2, (T *)A.c, A.mu2, A.rs2, M, C,
                                   h->cfg.ln_eps, st)); nl++;
     d = gdesc(M, mC, C, A.c, C, 1, W + P.wfc, C, 1);
-    d.epi.kind = EPI_STORE_GELU; d.epi.out = A.dgelu; d.epi.ldo = mC; d.epi.out2 = A.h; d.epi.ldo2 = mC;
+    d.epi.kind = h->cfg.recompute_gelu ? EPI_STORE_PRE_GELU : EPI_STORE_GELU;
+    d.epi.out = A.dgelu; d.epi.ldo = mC; d.epi.out2 = A.h; d.epi.ldo2 = mC;
     CUDA_TRY(gemm(h, d));
     d = gdesc(M, C, mC, A.h, mC, 1, W + P.wmp, mC, 1);
     d.epi.kind = EPI_RESID; d.epi.out = xnext; d.epi.ldo = C; d.epi.aux = A.x_mid; d.epi.ld_aux = C;
@@ -368,6 +380,9 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     // MLP: x_out = x_mid + gelu(c Wfc^T) Wmp^T
     GemmDesc d = gdesc(M, mC, C, dx, C, 1, W + P.wmp, mC, 0);
     d.epi.kind = EPI_DGELU; d.epi.out = h->dh; d.epi.ldo = mC; d.epi.aux = A.dgelu; d.epi.ld_aux = mC;
+    if (h->cfg.recompute_gelu) {  // dh = dy * gelu'(pre), and gelu(pre) again for dWmp
+      d.epi.kind = EPI_DGELU_RECOMP; d.epi.out2 = A.h; d.epi.ldo2 = mC;
+    }
     CUDA_TRY(gemm(h, d));
     d = gdesc(C, mC, M, dx, C, 0, A.h, mC, 0);
     d.epi.kind = wgrad; d.epi.outf = G + P.wmp; d.epi.ldf = mC;
@@ -572,6 +587,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   h->ev_used = 0;
   for (int k = 0; k < GPT_KSTAT_COUNT; ++k) { h->stat_launches[k] = 0; h->stat_ms[k] = 0; h->stat_work[k] = 0; }
   h->tc = nullptr;
+  h->muon_ws = nullptr;
   cudaGetDevice(&h->device);
 
   // ---- parameter layout ----
@@ -620,7 +636,8 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
     Acts &A = h->acts[l];
     need(&A.x_in, M * C * es); need(&A.a, M * C * es); need(&A.qkv, M * 3 * C * es);
     need(&A.o, M * C * es); need(&A.x_mid, M * C * es); need(&A.c, M * C * es);
-    need(&A.dgelu, M * h->mC * es); need(&A.h, M * h->mC * es);
+    need(&A.dgelu, M * h->mC * es);
+    if (!c.recompute_gelu || l == 0) need(&A.h, M * h->mC * es);
     need((void **)&A.lse, M * H * 4); need((void **)&A.mu1, M * 4); need((void **)&A.rs1, M * 4);
     need((void **)&A.mu2, M * 4); need((void **)&A.rs2, M * 4);
   }
@@ -655,6 +672,8 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
     *r.first = h->ws + o2;
     o2 += align_up(r.second);
   }
+  if (c.recompute_gelu)  // one activation buffer for all layers
+    for (int l = 1; l < h->L; ++l) h->acts[l].h = h->acts[0].h;
   *status = GPT_ERR_CUDA;
   if (cudaMemset(h->ws, 0, total) != cudaSuccess || cudaMallocHost(&h->sc_host, sizeof(DevScalars)) != cudaSuccess) {
     cudaGetLastError();
@@ -681,6 +700,7 @@ void gpt_destroy(gpt_handle *h) {
   for (auto &kv : h->graphs) cudaGraphExecDestroy(kv.second.exec);
   for (auto ev : h->ev) cudaEventDestroy(ev);
   if (h->tc) tc_gemm_destroy(h->tc);
+  if (h->muon_ws) cudaFree(h->muon_ws);
   cudaFree(h->ws);
   cudaFreeHost(h->sc_host);
   delete h;
@@ -843,6 +863,86 @@ int gpt_adamw_ranges(gpt_handle *h, float *params, const float *grads, float *ad
   cudaSetDevice(h->device);
   TRY(launch_adamw_ranges(params, grads, adam_m, adam_v, rg, sumsq_dev, h->stream));
   h->shadow_valid = false;  // params changed outside the step
+  return GPT_OK;
+}
+
+int gpt_muon_update(gpt_handle *h, float *params, const float *grads, float *adam_m,
+                    float *adam_v, const gpt_muon_config *mc, float lr, float wd, float clip) {
+  if (!h || !params || !grads || !adam_m || !adam_v || !mc || !mc->coeffs) return GPT_ERR_INVALID_ARG;
+  if (misaligned(params) || misaligned(grads) || misaligned(adam_m) || misaligned(adam_v))
+    return GPT_ERR_ALIGN;
+  if (!isfinite(lr) || !isfinite(wd) || !(clip > 0.f) || mc->ns_steps < 0 || mc->ns_steps > 16 ||
+      !isfinite(mc->matrix_lr) || !isfinite(mc->weight_decay) || !(mc->momentum >= 0.f) ||
+      !(mc->momentum < 1.f) || !(mc->beta2 >= 0.f) || !(mc->beta2 < 1.f) || !(mc->eps > 0.f))
+    return GPT_ERR_INVALID_ARG;
+  if (!h->use_bf16 || !h->tc) return GPT_ERR_SHAPE;  // the iteration runs on the tensor cores
+  cudaSetDevice(h->device);
+  cudaStream_t st = h->stream;
+  const int C = h->C, mC = h->mC, L = h->L;
+  const size_t lstride = L > 1 ? h->layer[1].wqkv - h->layer[0].wqkv : 0;
+  MuonGroup groups[4] = {{3 * C, C, L, h->layer[0].wqkv, lstride},
+                         {C, C, L, h->layer[0].wap, lstride},
+                         {mC, C, L, h->layer[0].wfc, lstride},
+                         {C, mC, L, h->layer[0].wmp, lstride}};
+  if (!h->muon_ws) {
+    const size_t bytes = muon_scratch_bytes(groups, 4);
+    TRY(cudaMalloc(&h->muon_ws, bytes));
+    TRY(cudaMemset(h->muon_ws, 0, bytes));
+  }
+  const MuonScratch scr = muon_scratch_carve(h->muon_ws, groups, 4);
+  const long t = h->step + 1;
+  h->ev_used = 0;
+  set_hyper(h, 1, lr, wd, clip, t);
+  TRY(cudaMemcpyAsync(h->sc, h->sc_host, offsetof(DevScalars, sumsq), cudaMemcpyHostToDevice, st));
+  TRY(cudaMemsetAsync((char *)h->sc + offsetof(DevScalars, loss), 0,
+                      offsetof(DevScalars, counter) - offsetof(DevScalars, loss), st));
+  int nl = 0;
+  // global norm and clip coefficient of the raw gradient
+  TIMED_S(h, GPT_KSTAT_GRAD_NORM, 4.0 * h->nparams,
+        launch_grad_norm(grads, h->nparams, h->gn_partials, h->sc, st)); nl++;
+  // AdamW: embeddings (wte is also the tied lm_head), positions, LayerNorm gains
+  MuonAdamRanges rg;
+  memset(&rg, 0, sizeof(rg));
+  rg.lr = lr; rg.wd = wd;
+  rg.beta1 = h->cfg.beta1; rg.beta2 = h->cfg.beta2; rg.eps = h->cfg.adam_eps;
+  rg.bias1 = h->sc_host->bias1; rg.bias2 = h->sc_host->bias2;
+  std::vector<std::pair<long long, long long>> ranges;
+  ranges.push_back({(long long)h->off_wte, (long long)h->Vp * C});
+  ranges.push_back({(long long)h->off_wpe, (long long)h->maxT * C});
+  for (int l = 0; l < L; ++l) {
+    ranges.push_back({(long long)h->layer[l].ln1, C});
+    ranges.push_back({(long long)h->layer[l].ln2, C});
+  }
+  ranges.push_back({(long long)h->off_lnf, C});
+  for (size_t k0 = 0; k0 < ranges.size(); k0 += MUON_ADAM_MAX_RANGES) {
+    rg.n = 0;
+    for (size_t k = k0; k < ranges.size() && rg.n < MUON_ADAM_MAX_RANGES; ++k, ++rg.n) {
+      rg.offset[rg.n] = ranges[k].first;
+      rg.count[rg.n] = ranges[k].second;
+    }
+    TIMED_S(h, GPT_KSTAT_ADAMW, 28.0 * (double)(h->off_wpe + (size_t)h->maxT * C),
+          muon_adamw_ranges(params, grads, adam_m, adam_v, rg, h->sc, st)); nl++;
+  }
+  // Muon on the block matrices, one group of equal shapes at a time
+  MuonStepArgs a;
+  a.params = params; a.grads = grads; a.mom = adam_m; a.sv = adam_v;
+  a.coeffs = mc->coeffs; a.ns = mc->ns_steps;
+  a.lr = mc->matrix_lr; a.wd = mc->weight_decay; a.mu = mc->momentum; a.beta2 = mc->beta2;
+  a.eps = mc->eps; a.sc = h->sc; a.err = &h->sc->err;
+  for (int gi = 0; gi < 4; ++gi) {
+    const MuonGroup &g = groups[gi];
+    const double d = g.rows < g.cols ? g.rows : g.cols, big = g.rows < g.cols ? g.cols : g.rows;
+    const double flops = (double)g.count * a.ns * (4.0 * d * d * big + 2.0 * d * d * d);
+    TIMED_S(h, GPT_KSTAT_MUON, flops, muon_update_group(h->tc, g, a, scr, st, &nl));
+  }
+  h->launches = nl;
+  h->shadow_valid = false;  // the bf16 weights are refreshed by the next forward
+  float dummy = 0.f;
+  int s = finish(h, &dummy);
+  h->last_norm = h->sc_host->norm;
+  if (s) return s;
+  if (h->sc_host->nonfinite) return GPT_ERR_NONFINITE;
+  h->step = t;
   return GPT_OK;
 }
 

@@ -67,6 +67,9 @@ typedef struct {
   int precision;         /* GPT_FP32 or GPT_BF16                                                */
   int lmhead_chunk_rows; /* rows per lm_head backward chunk (0 = library default); the largest
                             B*T*V-shaped buffer the step keeps is chunk_rows * Vp bf16          */
+  int recompute_gelu;    /* 1: activation recompute (llm.c summary, "Ejecución", -r): each layer
+                            keeps only its MLP pre-activation; the backward recomputes GELU and
+                            its derivative from it (saves n_layer-1 activations of B*T*4C) */
 } gpt_config;
 
 typedef struct {
@@ -166,6 +169,36 @@ int gpt_adamw_ranges(gpt_handle *h, float *params, const float *grads, float *ad
                      int nranges, float lr, float wd, float clip, const double *sumsq_dev,
                      long step);
 
+/* ---- hybrid Muon + AdamW optimizer --------------------------------------------------------
+ * nanochat architecture page, "Optimierungsstrategien Muon und AdamW": Muon for the 2-D block
+ * matrices (w_qkv, w_attnproj, w_fc, w_mlpproj of every layer), AdamW for wte (embedding and
+ * tied lm_head), wpe and the LayerNorm gains. Per matrix W (rows x cols) on the clipped
+ * gradient g = coef * grad, coef = min(1, clip / (||grad|| + 1e-6)):
+ *   momentum (Nesterov, lerp form): buf = lerp(buf, g, 1 - momentum); u = lerp(g, buf, momentum)
+ *   Polar Express: X = bf16(u) / (||X||_F * 1.01 + 1e-6); per coefficient triple (a, b, c):
+ *     rows > cols: A = X^T X, B = b A + c A^2, X = a X + X B; else A = X X^T, X = a X + B X
+ *     (bf16 operands, fp32 accumulation, tensor cores; all layers' matrices of one shape batched)
+ *   factored second moment: v = mean of X^2 per row (rows > cols) or per column;
+ *     s = lerp(s, v, 1 - beta2); X' = X / sqrt(max(s, eps)), rescaled to ||X||_F
+ *   cautious update: W -= matrix_lr * X' + matrix_lr * weight_decay * W * [X' * W >= 0]
+ * Everything else: the AdamW of gpt_train_step with lr, wd and t = (step counter) + 1.
+ * State in the caller's flat adam_m / adam_v: for a matrix, adam_m holds its momentum buffer
+ * and adam_v, from the matrix's offset, its second moment (rows or cols floats); both start
+ * zeroed. grads: the raw gradient (e.g. from gpt_forward_backward). bf16 mode only
+ * (GPT_ERR_SHAPE otherwise). On success the step counter advances; on GPT_ERR_NONFINITE
+ * (non-finite norm) nothing is updated. The first call allocates the handle's Muon scratch. */
+typedef struct {
+  float matrix_lr;      /* Muon learning rate (the page's matrix_lr, 0.02)                   */
+  float weight_decay;   /* Muon cautious weight decay (the page: 0.0)                        */
+  float momentum;       /* 0.95                                                              */
+  float beta2;          /* EMA factor of the factored second moment, 0.95                    */
+  float eps;            /* floor of the second moment, 1e-10                                 */
+  int ns_steps;         /* Polar Express iterations (the page: 5), <= 16                     */
+  const float *coeffs;  /* host, ns_steps triples (a, b, c)                                  */
+} gpt_muon_config;
+int gpt_muon_update(gpt_handle *h, float *params, const float *grads, float *adam_m,
+                    float *adam_v, const gpt_muon_config *mc, float lr, float wd, float clip);
+
 /* Step counter (number of completed AdamW updates); gpt_set_step is for resuming. */
 int gpt_get_step(const gpt_handle *h, long *step);
 int gpt_set_step(gpt_handle *h, long step);
@@ -214,7 +247,9 @@ int gpt_set_option(gpt_handle *h, int option, long value);
 #define GPT_KSTAT_CE 8
 #define GPT_KSTAT_GRAD_NORM 9
 #define GPT_KSTAT_ADAMW 10
-#define GPT_KSTAT_COUNT 11
+#define GPT_KSTAT_MUON 11          /* gpt_muon_update's Muon part per matrix group: FLOPs of
+                                      the Polar Express GEMMs */
+#define GPT_KSTAT_COUNT 12
 int gpt_kernel_stats(gpt_handle *h, int kind, long long *launches, double *total_ms,
                      double *work, int reset);
 

@@ -14,17 +14,17 @@ from typing import List, Optional, Sequence
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "gpt_oracle.cpp")
+_SRCS = [os.path.join(_HERE, "gpt_oracle.cpp"), os.path.join(_HERE, "muon_oracle.cpp")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 
 def build(force: bool = False) -> str:
     """Compile the oracle with g++ (-O2, IEEE semantics: no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
-            os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "gpt_oracle.h"))):
+    deps = _SRCS + [os.path.join(_HERE, "gpt_oracle.h")]
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(map(os.path.getmtime, deps)):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-fno-fast-math",
-                               "-ffp-contract=off", _SRC, "-o", tmp])
+                               "-ffp-contract=off", *_SRCS, "-o", tmp])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -81,6 +81,11 @@ def _load():
         L.oracle_gelu_f64.argtypes = [ctypes.c_double]
         L.oracle_gelu_grad_f64.restype = ctypes.c_double
         L.oracle_gelu_grad_f64.argtypes = [ctypes.c_double]
+        L.oracle_polar_express_f64.restype = None
+        L.oracle_polar_express_f64.argtypes = [P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+        L.oracle_muon_adamw_f64.restype = ctypes.c_double
+        L.oracle_muon_adamw_f64.argtypes = [ctypes.c_size_t, P, P, P, P, ctypes.c_int, P, P, P] + \
+            [ctypes.c_double] * 10 + [P, ctypes.c_int, ctypes.c_double, ctypes.c_long]
         L.oracle_cross_entropy_f64.restype = ctypes.c_double
         L.oracle_cross_entropy_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     return _lib
@@ -220,6 +225,44 @@ class Oracle:
                                           B, T, C3 // 3, H, window, _ptr(d))
         return d
 
+    def polar_express(self, X, coeffs, ns=None):
+        """Polar Express (normalisation, then ns iterations) of a 2-D array; returns a copy."""
+        X = np.array(X, dtype=np.float64, order="C", copy=True)
+        cf = np.ascontiguousarray(coeffs, np.float64).reshape(-1)
+        ns = len(cf) // 3 if ns is None else ns
+        self.lib.oracle_polar_express_f64(_ptr(X), X.shape[0], X.shape[1], _ptr(cf), ns)
+        return X
+
+    def matrices(self):
+        """(offset, rows, cols) of the 2-D block matrices Muon updates: per layer w_qkv,
+        w_attnproj, w_fc, w_mlpproj (the flat layout of this oracle)."""
+        lay = self.layout()
+        C, mC, L = self.cfg.n_embd, self.cfg.mlp_mult * self.cfg.n_embd, self.cfg.n_layer
+        out = []
+        for l in range(L):
+            base = 2 + 6 * l  # wte, wpe, then per layer ln1, w_qkv, w_ap, ln2, w_fc, w_mp
+            out += [(lay[base + 1][0], 3 * C, C), (lay[base + 2][0], C, C),
+                    (lay[base + 4][0], mC, C), (lay[base + 5][0], C, mC)]
+        return out
+
+    def muon_adamw(self, p, g, m, v, lr, wd, step, clip, coeffs, matrix_lr=0.02, muon_wd=0.0,
+                   mu=0.95, beta2_muon=0.95, s_eps=1e-10, beta1=0.9, beta2=0.95, eps=1e-8,
+                   ns=None):
+        """One hybrid step in place on p, m, v (double arrays); returns the grad norm."""
+        for a in (p, m, v):
+            assert a.dtype == np.float64 and a.flags.c_contiguous
+        mats = self.matrices()
+        off = np.array([x[0] for x in mats], np.int64)
+        rows = np.array([x[1] for x in mats], np.int32)
+        cols = np.array([x[2] for x in mats], np.int32)
+        cf = np.ascontiguousarray(coeffs, np.float64).reshape(-1)
+        ns = len(cf) // 3 if ns is None else ns
+        g = np.ascontiguousarray(g, np.float64)
+        return self.lib.oracle_muon_adamw_f64(p.size, _ptr(p), _ptr(g), _ptr(m), _ptr(v), len(mats),
+                                              _ptr(off), _ptr(rows), _ptr(cols), lr, wd, beta1,
+                                              beta2, eps, matrix_lr, muon_wd, mu, beta2_muon,
+                                              s_eps, _ptr(cf), ns, clip, step)
+
     def gelu(self, x: float) -> float:
         return self.lib.oracle_gelu_f64(x)
 
@@ -233,3 +276,28 @@ class Oracle:
         loss = self.lib.oracle_cross_entropy_f64(_ptr(lg), _ptr(np.ascontiguousarray(targets, np.int32)),
                                                  rows, V, Vp, _ptr(d))
         return loss, d
+
+
+def polar_express_coeffs(steps: int = 5, lo: float = 1e-3, npts: int = 6000) -> np.ndarray:
+    """The Polar Express coefficient table (nanochat architecture page, "Polar Express
+    Details", refers to it without printing it), built the way the method defines it: step t
+    takes the odd quintic a x + b x^3 + c x^5 with the least max |1 - p(x)| over the interval
+    the singular values are in, and the next interval is [1 - E, 1 + E], E that least error.
+    Each minimax problem is solved here as a linear programme over a dense grid (HiGHS via
+    scipy): minimise E subject to |1 - p(x)| <= E at every grid point. [steps, 3] float64."""
+    from scipy.optimize import linprog
+    out = []
+    lo_t, hi_t = lo, 1.0
+    for _ in range(steps):
+        x = np.unique(np.concatenate([np.geomspace(lo_t, hi_t, npts // 2),
+                                      np.linspace(lo_t, hi_t, npts // 2)]))
+        P = np.stack([x, x ** 3, x ** 5], axis=1)
+        ones = np.ones((len(x), 1))
+        A_ub = np.vstack([np.hstack([-P, -ones]), np.hstack([P, -ones])])
+        b_ub = np.concatenate([-np.ones(len(x)), np.ones(len(x))])
+        r = linprog([0, 0, 0, 1], A_ub=A_ub, b_ub=b_ub,
+                    bounds=[(None, None)] * 3 + [(0, None)], method="highs")
+        a, b, c, E = r.x
+        out.append((a, b, c))
+        lo_t, hi_t = 1 - E, 1 + E
+    return np.array(out, dtype=np.float64)

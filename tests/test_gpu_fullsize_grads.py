@@ -81,14 +81,17 @@ def test_gpt2_124m_plan_uses_pairs_splits_and_chunks():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name", ["gpt2_124m_bf16", "gpt2_350m_bf16", "gpt2_124m_swa_bf16"])
-def test_full_size_bf16_grads_match_fp32_path(name):
+@pytest.mark.parametrize("name,recompute", [("gpt2_124m_bf16", False), ("gpt2_350m_bf16", False),
+                                            ("gpt2_124m_swa_bf16", False),
+                                            ("gpt2_124m_bf16", True)])
+def test_full_size_bf16_grads_match_fp32_path(name, recompute):
+    """recompute: the bf16 step with GELU recomputed in the backward (activation recompute)."""
     wl = fx.WORKLOADS[name]
     sh = wl.shape
     p, tok, tgt = fx.make_inputs(wl)
     grads = {}
     for prec in (0, 1):
-        st = U.make_step(sh, wl.B, wl.T, prec)
+        st = U.make_step(sh, wl.B, wl.T, prec, recompute_gelu=recompute and prec == 1)
         try:
             r = U.gpu_train_step(st, p, tok, tgt, wl.lr, wl.wd, wl.clip)
         finally:

@@ -178,3 +178,35 @@ def test_gpt2_124m_causality_bitwise(gpt2):
     _, pert = U.gpu_forward(st, p, tok2, tgt)
     assert np.array_equal(base[:, :t + 1], pert[:, :t + 1])
     assert not np.array_equal(base[:, t + 1:], pert[:, t + 1:])
+
+
+# ---------------------------------------------------------------------------------------
+# activation recompute (GELU recomputed in the backward from the kept pre-activation)
+# ---------------------------------------------------------------------------------------
+
+def test_gelu_recompute_fp32_is_bitwise_the_stored_path():
+    """In fp32 mode the recomputed GELU and derivative are the very values the stored path
+    keeps, so the whole step is bitwise identical."""
+    sh = fx.ModelShape(vocab=1000, vocab_padded=1024, n_layer=2, n_head=4, n_embd=128,
+                       max_T=80, window_left=[17, -1])
+    p = fx.init_params(sh, 21)
+    tok, tgt = fx.zipf_tokens(sh.vocab, 1.1, 3, 70, 21)
+    runs = []
+    for rc in (False, True):
+        st = U.make_step(sh, 3, 70, FP32, recompute_gelu=rc)
+        runs.append(U.gpu_train_step(st, p, tok, tgt, 1e-3, 0.01, 1.0))
+        st.close()
+    a, b = runs
+    assert a.loss == b.loss and np.array_equal(a.grads, b.grads)
+    assert np.array_equal(a.params, b.params)
+
+
+def test_gelu_recompute_bf16_matches_oracle():
+    sh = fx.ModelShape(vocab=1000, vocab_padded=1024, n_layer=3, n_head=4, n_embd=256,
+                       max_T=200, window_left=[50, -1, 7])
+    r1 = check_bf16(sh, B=3, T=200, seed=22, recompute_gelu=True)
+    st = U.make_step(sh, 3, 200, BF16, recompute_gelu=True)
+    tok, tgt = fx.zipf_tokens(sh.vocab, 1.05, 3, 200, 22)
+    r2 = U.gpu_train_step(st, fx.init_params(sh, 22), tok, tgt, 6e-4, 0.1, 1.0)
+    st.close()
+    assert r1.loss == r2.loss and np.array_equal(r1.grads, r2.grads)  # deterministic
