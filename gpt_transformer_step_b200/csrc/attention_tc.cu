@@ -628,20 +628,29 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // Per item: K and V of the key tile (double-buffered); then for every query tile that sees it
 // S^T = K Q^T, dP^T = V dO^T, P^T and dS^T -> TMEM, dV += P^T dO, dK += dS^T Q. The lse and
 // D of the next query tile are fetched from global memory one tile ahead.
-constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight
+// With WRITE_DS the kernel also writes every dS^T tile (bf16, [B*H][T keys][T queries]) for
+// the tensor-core dQ pass (attn_bwd_dq_mma), through a 32 KB staging area that takes one of
+// the Q/dO stages (NST = 3 then).
+constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight (at most)
 enum { K_KV0, K_KVFREE0 = K_KV0 + 2, K_QDO0 = K_KVFREE0 + 2, K_FREE0 = K_QDO0 + DKV_STAGES,
        K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE, K_PS, K_MM2, K_NBAR };
-constexpr int DKV_SMEM = (4 + 2 * DKV_STAGES) * TILE_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
-static_assert(DKV_SMEM <= 232448, "dK/dV kernel shared memory");
+__host__ __device__ constexpr int dkv_smem(int nst, bool write_ds) {
+  return (4 + 2 * nst + (write_ds ? 2 : 0)) * TILE_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
+}
+static_assert(dkv_smem(DKV_STAGES, false) <= 232448, "dK/dV kernel shared memory");
+static_assert(dkv_smem(DKV_STAGES - 1, true) <= 232448, "dK/dV kernel shared memory");
 
+template <int NST, bool WRITE_DS>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-                const __grid_constant__ CUtensorMap tmDKV, const AttnParams P) {
+                const __grid_constant__ CUtensorMap tmDKV, const __grid_constant__ CUtensorMap tmDST,
+                const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sKV0 = smem;                  // buffer b: K at 2b, V at 2b+1 (in tiles)
   uint8_t *sQ0 = smem + 4 * TILE_BYTES;  // stage s: Q at 2s, dO at 2s+1
-  float *s_lsd = (float *)(smem + (4 + 2 * DKV_STAGES) * TILE_BYTES);  // [2][lse 128 | D 128]
+  uint8_t *sDS = smem + (4 + 2 * NST) * TILE_BYTES;  // dS^T staging: 4 KB per row warp
+  float *s_lsd = (float *)(smem + (4 + 2 * NST + (WRITE_DS ? 2 : 0)) * TILE_BYTES);  // [2][lse | D]
   uint64_t *bar = (uint64_t *)(s_lsd + 2 * 2 * TILE);
   uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
@@ -679,7 +688,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         tma_load_2d(sK, &tmQKV, &bar[K_KV0 + kb], P.C + it.h * HD, row0 + it.k0);
         tma_load_2d(sK + TILE_BYTES, &tmQKV, &bar[K_KV0 + kb], 2 * P.C + it.h * HD, row0 + it.k0);
         for (int j = 0; j < it.n; ++j, ++g) {
-          const int s = g % DKV_STAGES, use = g / DKV_STAGES, qq0 = (it.qt0 + j) * TILE;
+          const int s = g % NST, use = g / NST, qq0 = (it.qt0 + j) * TILE;
           if (use > 0 && !mbar_wait(&bar[K_FREE0 + s], (use - 1) & 1, abort_flag, P.err)) { ok = false; break; }
           uint8_t *sQ = sQ0 + s * 2 * TILE_BYTES;
           mbar_expect_tx(&bar[K_QDO0 + s], 2 * TILE_BYTES);
@@ -697,9 +706,9 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       mc.start(P);
       int gs = 0;
       auto issue_sdp = [&]() -> bool {  // S^T and dP^T of the next tile in the walk
-        const int kb = sc.i & 1, s = gs % DKV_STAGES;
+        const int kb = sc.i & 1, s = gs % NST;
         if (sc.j == 0 && !mbar_wait(&bar[K_KV0 + kb], (sc.i >> 1) & 1, abort_flag, P.err)) return false;
-        if (!mbar_wait(&bar[K_QDO0 + s], (gs / DKV_STAGES) & 1, abort_flag, P.err)) return false;
+        if (!mbar_wait(&bar[K_QDO0 + s], (gs / NST) & 1, abort_flag, P.err)) return false;
         tc_fence_after();
         const uint32_t aK = aKV0 + kb * 2 * TILE_BYTES, aV = aK + TILE_BYTES;
         const uint32_t aQ = aQ0 + s * 2 * TILE_BYTES, adO = aQ + TILE_BYTES;
@@ -718,11 +727,11 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         if (sc.valid && !issue_sdp()) break;
         if (!mbar_wait(&bar[K_PS], g & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        const uint32_t aQ = aQ0 + (g % DKV_STAGES) * 2 * TILE_BYTES, adO = aQ + TILE_BYTES;
+        const uint32_t aQ = aQ0 + (g % NST) * 2 * TILE_BYTES, adO = aQ + TILE_BYTES;
         mma_pv_ts(tmem + 256, tmem + 384, adO, mc.j > 0);  // dV += P^T dO   (P^T in TMEM)
         mma_pv_ts(tmem + 320, tmem + 448, aQ, mc.j > 0);   // dK += dS^T Q  (dS^T in TMEM)
         umma_commit(&bar[K_MM2]);
-        umma_commit(&bar[K_FREE0 + (g % DKV_STAGES)]);
+        umma_commit(&bar[K_FREE0 + (g % NST)]);
       }
     }
     __syncwarp();
@@ -818,14 +827,36 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         }
         tmem_st16_nw(tPT + 16 * half, pp);
         tmem_st16_nw(tdST + 16 * half, pd);
+        if (WRITE_DS) {  // the same bf16 dS^T row into the staging slot (128-byte swizzle)
+          uint8_t *slot = sDS + (warp - 2) * 4096;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = 4 * half + c4;  // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4 *>(slot + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(pd[4 * c4], pd[4 * c4 + 1], pd[4 * c4 + 2], pd[4 * c4 + 3]);
+          }
+        }
       }
       };
+      if (WRITE_DS) {  // this warp's dS^T staging slot must have been read by its last store
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
       if (interior) pds_math(std::false_type{});
       else pds_math(std::true_type{});
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[K_PS]);
+      if (WRITE_DS) {  // dS^T rows k0+q*32.. (keys) x queries qq0+ch*64.. to [B*H][T][T]
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && qq0 + ch * 64 < P.T && k0 + q * 32 < P.T) {
+          tma_store_3d(&tmDST, sDS + (warp - 2) * 4096, qq0 + ch * 64, k0 + q * 32,
+                       it.b * P.H + it.h);
+          bulk_commit();
+        }
+      }
       if (j + 1 < it.n) continue;
       // the item's last query tile: dV / dK out (column half 0 writes dV, half 1 writes dK
       // times the softmax scale)
@@ -856,7 +887,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       }
       pend_kb = kb;
     }
-    if (lane == 0) bulk_wait_read<0>();  // staging smem must outlive the last store's reads
+    if (lane == 0) bulk_wait_all();  // every store of this warp (dK/dV, dS^T) has completed
   }
   tc_fence_before();
   __syncthreads();
@@ -865,6 +896,180 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     tmem_dealloc(tmem, 512);
   }
 }
+// ------------------------------------------------------------------------------------------
+// backward, dQ from the stored dS^T (used with attn_bwd_dkv_tc<.., true>)
+// ------------------------------------------------------------------------------------------
+// D_i = dO_i . O_i for every row (b, t) and head: one thread per (row, head), 16-byte loads.
+__global__ void __launch_bounds__(256)
+attn_bwd_prep_d(const bf16 *__restrict__ O, const bf16 *__restrict__ dO, float *__restrict__ D,
+                int B, int T, int C, int H) {
+  const long n = (long)B * T * H;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const int h = (int)(i % H);
+    const long m = i / H;  // row b*T + t
+    const uint4 *o4 = reinterpret_cast<const uint4 *>(O + m * C + h * HD);
+    const uint4 *d4 = reinterpret_cast<const uint4 *>(dO + m * C + h * HD);
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 av = o4[c], cv = d4[c];
+      const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&av);
+      const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
+        acc += fa.x * fc.x + fa.y * fc.y;
+      }
+    }
+    const int b = (int)(m / T), t = (int)(m % T);
+    D[((long)b * H + h) * T + t] = acc;
+  }
+}
+
+// dQ_i = scale * sum_j dS_ij K_j over the key tiles a query tile sees, on the tensor cores:
+// persistent CTAs over query tiles (the heavy-first snake schedule of the other passes); per
+// 64-key block a TMA load of the dS^T block (MN-major A: 64 keys x 128 queries) and of the K
+// block (MN-major B: 64 keys x 64 head dims), 4 MMAs of 128x64x16 into a TMEM accumulator
+// (double-buffered across items); 4 epilogue warps scale, round and TMA-store dQ.
+constexpr int DQM_STAGES = 6;
+constexpr int DQM_A = TILE * 64 * 2;  // 16 KB
+constexpr int DQM_B = 64 * 64 * 2;    // 8 KB
+constexpr int DQM_STAGE = DQM_A + DQM_B;
+constexpr int DQM_THREADS = 192;      // TMA, MMA, 4 epilogue warps
+enum { M_FULL0, M_EMPTY0 = M_FULL0 + DQM_STAGES, M_TFULL0 = M_EMPTY0 + DQM_STAGES,
+       M_TEMPTY0 = M_TFULL0 + 2, M_NBAR = M_TEMPTY0 + 2 };
+constexpr int DQM_SMEM = DQM_STAGES * DQM_STAGE + 4 * 4096 + 1024 + 256;
+static_assert(DQM_SMEM <= 232448, "dQ kernel shared memory");
+
+__global__ void __launch_bounds__(DQM_THREADS, 1)
+attn_bwd_dq_mma(const __grid_constant__ CUtensorMap tmDST, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmDQ, const AttnParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *stg = smem + DQM_STAGES * DQM_STAGE;  // 4 x 4 KB output staging
+  uint64_t *bar = (uint64_t *)(stg + 4 * 4096);
+  uint32_t *tmem_holder = (uint32_t *)(bar + M_NBAR);
+  volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < M_NBAR; ++i)
+      mbar_init(&bar[i], (i == M_TEMPTY0 || i == M_TEMPTY0 + 1) ? 4 : 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;  // dQ accumulators: columns [0,64) and [64,128)
+
+  if (warp == 0) {
+    if (lane == 0) {  // TMA producer
+      QTile it;
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; ok && query_item(P, i, it); ++i) {
+        const int bh = it.b * P.H + it.h;
+        for (int j = 0; ok && j < it.n; ++j) {
+          const int k0 = (it.kt0 + j) * TILE;
+          for (int kb = 0; kb < 2; ++kb, ++g) {
+            const int s = g % DQM_STAGES, use = g / DQM_STAGES;
+            if (use > 0 && !mbar_wait(&bar[M_EMPTY0 + s], (use - 1) & 1, abort_flag, P.err)) {
+              ok = false;
+              break;
+            }
+            uint8_t *sA = smem + s * DQM_STAGE;
+            mbar_expect_tx(&bar[M_FULL0 + s], DQM_STAGE);
+            // dS^T[bh][keys k0+64kb..][queries q0..q0+127]: two 64-query boxes
+            tma_load_3d(sA, &tmDST, &bar[M_FULL0 + s], it.q0, k0 + 64 * kb, bh);
+            tma_load_3d(sA + DQM_A / 2, &tmDST, &bar[M_FULL0 + s], it.q0 + 64, k0 + 64 * kb, bh);
+            // K[keys][head dims] of head h, batch b
+            tma_load_2d(sA + DQM_A, &tmK, &bar[M_FULL0 + s], P.C + it.h * HD,
+                        it.b * P.T + k0 + 64 * kb);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      const uint32_t id = idesc_bf16(HD, 1, 1);  // M = 128, N = 64, both operands MN-major
+      QTile it;
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; ok && query_item(P, i, it); ++i) {
+        const int acc = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        if (!mbar_wait(&bar[M_TEMPTY0 + acc], (use & 1u) ^ 1u, abort_flag, P.err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * 64);
+        for (int j = 0; ok && j < it.n; ++j)
+          for (int kb = 0; kb < 2; ++kb, ++g) {
+            const int s = g % DQM_STAGES;
+            if (!mbar_wait(&bar[M_FULL0 + s], (g / DQM_STAGES) & 1, abort_flag, P.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sA = smem_u32(smem + s * DQM_STAGE);
+            const uint64_t ad = sdesc(sA, 8192u, 1024u), bd = sdesc(sA + DQM_A, 8192u, 1024u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 16 keys per MMA: 16 rows of 128 bytes
+              umma_bf16(d, ad + (uint64_t)((k * 2048) >> 4), bd + (uint64_t)((k * 2048) >> 4), id,
+                        (j > 0 || kb > 0 || k > 0) ? 1u : 0u);
+            umma_commit(&bar[M_EMPTY0 + s]);
+          }
+        if (!ok) break;
+        umma_commit(&bar[M_TFULL0 + acc]);
+      }
+    }
+    __syncwarp();
+  } else {  // epilogue: warp w reads TMEM lane quarter w % 4
+    const int q = warp & 3;
+    uint8_t *ws = stg + (warp - 2) * 4096;
+    QTile it;
+    for (int i = 0; query_item(P, i, it); ++i) {
+      const int acc = i & 1;
+      const uint32_t use = (uint32_t)(i >> 1);
+      if (!warp_wait(&bar[M_TFULL0 + acc], use & 1u, abort_flag, P.err)) break;
+      tc_fence_after();
+      float v0[32], v1[32];
+      const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 64);
+      tmem_ld32(ta, v0);
+      tmem_ld32(ta + 32, v1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[M_TEMPTY0 + acc]);  // the MMA may reuse it
+      if (lane == 0) bulk_wait_read<0>();                  // the staging slot is free
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float *v = t < 4 ? v0 : v1;
+        const int b8 = (t & 3) * 8;
+        *reinterpret_cast<uint4 *>(ws + lane * 128 + ((t ^ (lane & 7)) << 4)) =
+            make_uint4(pack_bf16(v[b8] * P.scale, v[b8 + 1] * P.scale),
+                       pack_bf16(v[b8 + 2] * P.scale, v[b8 + 3] * P.scale),
+                       pack_bf16(v[b8 + 4] * P.scale, v[b8 + 5] * P.scale),
+                       pack_bf16(v[b8 + 6] * P.scale, v[b8 + 7] * P.scale));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0 && it.q0 + q * 32 < P.T) {
+        tma_store_3d(&tmDQ, ws, it.h * HD, it.q0 + q * 32, it.b);
+        bulk_commit();
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -886,13 +1091,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, cols] bf16 matrix with row stride ld elements; box 64 columns x 128 rows, SW128.
-bool map_rows(CUtensorMap *m, const void *base, long cols, long rows, long ld) {
+// [rows, cols] bf16 matrix with row stride ld elements; box 64 columns x box_rows rows, SW128.
+bool map_rows(CUtensorMap *m, const void *base, long cols, long rows, long ld, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {64u, 128u};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1u, 1u};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)base, dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -913,6 +1118,19 @@ bool map_btc(CUtensorMap *m, const void *base, long cols, long T, long B, long l
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)base, dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// dS^T [B*H][T keys][T queries] bf16: box {64 queries, box_keys keys, 1}, SW128.
+bool map_dst(CUtensorMap *m, const void *base, long T, long BH, int box_keys) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)T, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)T * 2, (cuuint64_t)(T * T * 2)};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_keys, 1u};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 AttnParams make_params(int B, int T, int C, int H, int window, unsigned *err) {
@@ -941,7 +1159,13 @@ cudaError_t set_attrs() {
   if (smem_attrs_set) return cudaSuccess;
   CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, FWD_SMEM));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM));
-  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM));
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                dkv_smem(DKV_STAGES, false)));
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES - 1, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                dkv_smem(DKV_STAGES - 1, true)));
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, DQM_SMEM));
   smem_attrs_set = true;
   return cudaSuccess;
 }
@@ -967,7 +1191,8 @@ cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B,
 
 cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
                                     const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
-                                    int C, int H, int window, unsigned *err, cudaStream_t st) {
+                                    int C, int H, int window, unsigned *err, cudaStream_t st,
+                                    bf16 *dst) {
   CUDA_TRY(set_attrs());
   CUtensorMap mq, md, mo, mdq, mdkv;
   if (!map_rows(&mq, qkv, 3L * C, (long)B * T, 3L * C) ||
@@ -984,9 +1209,27 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
   p.dqkv = dqkv;
   const int items = B * H * ((T + TILE - 1) / TILE);
   const int grid = items < attn_sms() ? items : attn_sms();  // one CTA per SM
+  if (dst) {
+    // D, then dK/dV writing dS^T, then dQ = dS K from the stored dS^T on the tensor cores
+    CUtensorMap mst, mld, mk, mdq64;
+    if (!map_dst(&mst, dst, T, (long)B * H, 32) || !map_dst(&mld, dst, T, (long)B * H, 64) ||
+        !map_rows(&mk, qkv, 3L * C, (long)B * T, 3L * C, 64) ||
+        !map_btc(&mdq64, dqkv, 3L * C, T, B, 3L * C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    const long rows = (long)B * T * H;
+    const int pb = (int)((rows + 255) / 256 < 148 * 8 ? (rows + 255) / 256 : 148 * 8);
+    attn_bwd_prep_d<<<pb, 256, 0, st>>>(o, dout, Dbuf, B, T, C, H);
+    CUDA_TRY(cudaGetLastError());
+    attn_bwd_dkv_tc<DKV_STAGES - 1, true><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES - 1, true), st>>>(
+        mq, md, mdkv, mst, p);
+    CUDA_TRY(cudaGetLastError());
+    attn_bwd_dq_mma<<<grid, DQM_THREADS, DQM_SMEM, st>>>(mld, mk, mdq64, p);
+    return cudaGetLastError();
+  }
   attn_bwd_dq_tc<<<grid, BWD_THREADS, DQ_SMEM, st>>>(mq, md, mo, mdq, p);
   CUDA_TRY(cudaGetLastError());
-  attn_bwd_dkv_tc<<<grid, BWD_THREADS, DKV_SMEM, st>>>(mq, md, mdkv, p);
+  attn_bwd_dkv_tc<DKV_STAGES, false><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES, false), st>>>(
+      mq, md, mdkv, mdkv, p);
   return cudaGetLastError();
 }
 
@@ -1040,5 +1283,6 @@ cudaError_t launch_attention_bwd_tc_noalloc(const bf16 *qkv, const bf16 *o, cons
   if ((size_t)B * H * T > NOALLOC_D_MAX) return cudaErrorInvalidValue;
   float *D = nullptr;
   CUDA_TRY(noalloc_D_address(&D));
-  return launch_attention_bwd_tc(qkv, o, dout, lse, D, dqkv, B, T, C, H, window, err, st);
+  return launch_attention_bwd_tc(qkv, o, dout, lse, D, dqkv, B, T, C, H, window, err, st,
+                                 nullptr);
 }

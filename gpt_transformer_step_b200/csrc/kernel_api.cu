@@ -108,6 +108,21 @@ extern "C" int gptk_attention_bwd_bf16(const void *qkv, const void *o, const voi
   return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }
 
+extern "C" int gptk_attention_bwd_bf16_ds(const void *qkv, const void *o, const void *dout,
+                                          const float *lse, float *Dbuf, void *ds_scratch,
+                                          void *dqkv, int B, int T, int C, int H, int window,
+                                          unsigned *dev_err, void *stream) {
+  if (!qkv || !o || !dout || !lse || !Dbuf || !ds_scratch || !dqkv || !dev_err || B <= 0 ||
+      T <= 0 || H <= 0 || C % H)
+    return GPT_ERR_INVALID_ARG;
+  if (!attention_tc_supported(C, H) || (T & 7)) return GPT_ERR_SHAPE;
+  if (((uintptr_t)ds_scratch & 15u) != 0) return GPT_ERR_ALIGN;
+  cudaError_t e = launch_attention_bwd_tc((const bf16 *)qkv, (const bf16 *)o, (const bf16 *)dout,
+                                          lse, Dbuf, (bf16 *)dqkv, B, T, C, H, window, dev_err,
+                                          (cudaStream_t)stream, (bf16 *)ds_scratch);
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
 // Attention backward without any allocation: see include/gpt_kernels.h.
 extern "C" int gptk_attention_bwd_bf16_noalloc(const void *qkv, const void *o, const void *dout,
                                                const float *lse, void *dqkv, int B, int T, int C,

@@ -83,6 +83,7 @@ struct gpt_handle {
   int chunk_rows;
   void *dx, *dh, *dc, *dqkv, *dout, *dyf;
   float *Dbuf, *dg_partial;
+  bf16 *dst;  // attention backward: dS^T of one layer [B*H][T][T] (NULL: the two-pass backward)
   double *gn_partials;
   float *splitk;
   size_t splitk_elems;
@@ -244,6 +245,9 @@ cudaError_t attention_fwd<bf16>(gpt_handle *h, const bf16 *qkv, bf16 *o, float *
     return launch_attention_fwd_tc(qkv, o, lse, B, Tlen, h->C, h->H, w, &h->sc->err, h->stream);
   return launch_attention_fwd<bf16>(qkv, o, lse, B, Tlen, h->C, h->H, w, h->stream);
 }
+// The dS^T scratch when the call's T gives it 16-byte rows (else the two-pass backward).
+bf16 *attn_dst(const gpt_handle *h, int Tlen) { return (Tlen % 8 == 0) ? h->dst : nullptr; }
+
 template <typename T>
 cudaError_t attention_bwd(gpt_handle *h, const T *qkv, const T *o, const T *dout,
                           const float *lse, T *dqkv, int B, int Tlen, int w) {
@@ -255,7 +259,7 @@ cudaError_t attention_bwd<bf16>(gpt_handle *h, const bf16 *qkv, const bf16 *o, c
                                 const float *lse, bf16 *dqkv, int B, int Tlen, int w) {
   if (attention_tc_supported(h->C, h->H))
     return launch_attention_bwd_tc(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
-                                   &h->sc->err, h->stream);
+                                   &h->sc->err, h->stream, attn_dst(h, Tlen));
   return launch_attention_bwd<bf16>(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
                                     h->stream);
 }
@@ -405,7 +409,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(gemm(h, d));
     TIMED(h, GPT_KSTAT_ATTN_BWD, attn_flops(h->windows[l], 8.0),
           attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B, Tlen,
-                           h->windows[l])); nl += 2;
+                           h->windows[l])); nl += (h->use_bf16 && attn_dst(h, Tlen)) ? 3 : 2;
     d = gdesc(M, C, 3 * C, h->dqkv, 3 * C, 1, W + P.wqkv, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
@@ -649,6 +653,12 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   need(&h->dx, M * C * es); need(&h->dh, M * h->mC * es); need(&h->dc, M * C * es);
   need(&h->dqkv, M * 3 * C * es); need(&h->dout, M * C * es); need(&h->dyf, M * C * es);
   need((void **)&h->Dbuf, M * H * 4);
+  // dS^T scratch of the attention backward: B*H*T^2 bf16 (403 MB at 124M), when it is modest
+  const size_t dst_bytes = (size_t)c.max_B * H * (size_t)c.max_T * c.max_T * 2;
+  const bool use_dst = bf && (c.max_T % 8 == 0) && dst_bytes <= ((size_t)4 << 30) &&
+                       (C / H == 64);
+  if (use_dst) need((void **)&h->dst, dst_bytes);
+  else h->dst = nullptr;
   need((void **)&h->dg_partial, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
   need((void **)&h->gn_partials, (size_t)grad_norm_blocks() * 8);
   need((void **)&h->splitk, h->splitk_elems * 4);

@@ -5,7 +5,9 @@
 
 Each case runs `warmup` untimed launches, then `reps` launches timed with CUDA events on the
 launching stream; prints one JSON line per case with ms per launch and TFLOP/s (algorithmic
-FLOPs: 2*M*N*K per GEMM; 4*hd per admitted score forward, 10*hd backward).
+FLOPs: 2*M*N*K per GEMM; 4*hd per admitted score forward, 8*hd backward). attn_bwd is the
+two-pass backward (dQ with D, then dK/dV); attn_bwd_ds the one the step runs (D, dK/dV writing
+dS^T, dQ from it).
 Also the workload for small ncu captures of a single kernel (few hundred MB on the device).
 """
 from __future__ import annotations
@@ -30,7 +32,7 @@ GEMMS = {
     "gemm_wgrad_mlpproj": (C, 4 * C, M, 0, 0, "f32_store", 0),
     "gemm_lmhead": (M, 50304, C, 1, 1, "store", 1),
 }
-ATTN = ("attn_fwd", "attn_bwd")
+ATTN = ("attn_fwd", "attn_bwd", "attn_bwd_ds")
 
 
 def causal_scores(Bn, Tn, Hn, w=-1):
@@ -97,13 +99,23 @@ def main():
                                                         B, T, C, H, -1, err.data_ptr(), path, s)
                         assert rc == 0, rc
                     flops = 4.0 * hd * sc
-                else:
+                elif name == "attn_bwd":
                     def run():
                         rc = gb.gptk_attention_bwd_bf16(qkv.data_ptr(), o.data_ptr(), dout.data_ptr(),
                                                         lse.data_ptr(), D.data_ptr(), dq.data_ptr(),
                                                         B, T, C, H, -1, err.data_ptr(), path, s)
                         assert rc == 0, rc
-                    flops = 10.0 * hd * sc
+                    flops = 8.0 * hd * sc
+                else:
+                    ds = torch.zeros(B * H * T * T, dtype=torch.bfloat16, device=dev)
+
+                    def run():
+                        rc = gb.gptk_attention_bwd_bf16_ds(qkv.data_ptr(), o.data_ptr(),
+                                                           dout.data_ptr(), lse.data_ptr(),
+                                                           D.data_ptr(), ds.data_ptr(), dq.data_ptr(),
+                                                           B, T, C, H, -1, err.data_ptr(), s)
+                        assert rc == 0, rc
+                    flops = 8.0 * hd * sc
             for _ in range(args.warmup):
                 run()
             e0 = torch.cuda.Event(enable_timing=True)

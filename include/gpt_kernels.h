@@ -68,6 +68,17 @@ int gptk_attention_bwd_bf16(const void *qkv, const void *o, const void *dout, co
                             float *Dbuf, void *dqkv, int B, int T, int C, int H, int window,
                             unsigned *dev_err, int path, void *stream);
 
+/* The tensor-core backward in the form gpt_train_step runs it: D, then the dK/dV pass, which
+ * also writes dS^T (the softmax Jacobian applied to dP, bf16) to ds_scratch, then dQ = dS K
+ * as tensor-core products over the stored dS^T (the scores are not recomputed for dQ).
+ * ds_scratch: device bf16 [B*H][T][T] (keys x queries per head; only the tiles inside the
+ * causal/window band are written and read), 16-byte aligned. T must be a multiple of 8 (the
+ * row stride of ds_scratch is a whole number of 16-byte units), head_dim 64, else
+ * GPT_ERR_SHAPE. Other arguments and results as gptk_attention_bwd_bf16. */
+int gptk_attention_bwd_bf16_ds(const void *qkv, const void *o, const void *dout, const float *lse,
+                               float *Dbuf, void *ds_scratch, void *dqkv, int B, int T, int C,
+                               int H, int window, unsigned *dev_err, void *stream);
+
 /* Failure-detection self test: launches one CTA that waits on an mbarrier nothing arrives
  * on, with the bounded wait every kernel of the step uses for its barriers; after timeout_us
  * (1 .. 2,000,000) it gives up, ORs GPT_DEVERR_TIMEOUT (2) into *dev_err and returns, leaving

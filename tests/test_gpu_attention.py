@@ -1,6 +1,8 @@
 """Attention kernels (tensor-core and CUDA-core paths) through the kernel-level C ABI vs
 PyTorch's scaled_dot_product_attention in fp32 on the same bf16 inputs: causal and windowed
-masks, ragged T (not a multiple of the 128-row tile), forward and backward."""
+masks, ragged T (not a multiple of the 128-row tile), forward and backward. Path 2 is the
+tensor-core backward as the step runs it (dK/dV writing dS^T, then dQ from the stored dS^T);
+it needs T % 8 == 0."""
 import math
 
 import numpy as np
@@ -48,10 +50,12 @@ CASES = [  # B, T, H, window
 ]
 
 
-@pytest.mark.parametrize("path", [0, 1])
+@pytest.mark.parametrize("path", [0, 1, 2])
 @pytest.mark.parametrize("B,T,H,w", CASES)
 def test_attention_vs_sdpa(env, path, B, T, H, w):
     torch, gb, dev, err = env
+    if path == 2 and T % 8:
+        pytest.skip("the stored-dS backward needs T % 8 == 0 (the step falls back otherwise)")
     C = 64 * H
     g = torch.Generator(device="cpu").manual_seed(B * 1000 + T + H + w)
     qkv = (torch.randn(B * T, 3 * C, generator=g) * 1.5).to(torch.bfloat16).to(dev)
@@ -62,11 +66,18 @@ def test_attention_vs_sdpa(env, path, B, T, H, w):
     Dbuf = torch.zeros(B, H, T, device=dev)
     err.zero_()
     s = torch.cuda.current_stream().cuda_stream
+    fpath = 0 if path == 2 else path
     assert gb.gptk_attention_fwd_bf16(qkv.data_ptr(), o.data_ptr(), lse.data_ptr(), B, T, C, H, w,
-                                      err.data_ptr(), path, s) == 0
-    assert gb.gptk_attention_bwd_bf16(qkv.data_ptr(), o.data_ptr(), dout.data_ptr(),
-                                      lse.data_ptr(), Dbuf.data_ptr(), dq.data_ptr(), B, T, C, H,
-                                      w, err.data_ptr(), path, s) == 0
+                                      err.data_ptr(), fpath, s) == 0
+    if path == 2:
+        ds = torch.full((B * H * T * T,), float("nan"), dtype=torch.bfloat16, device=dev)
+        assert gb.gptk_attention_bwd_bf16_ds(qkv.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                             lse.data_ptr(), Dbuf.data_ptr(), ds.data_ptr(),
+                                             dq.data_ptr(), B, T, C, H, w, err.data_ptr(), s) == 0
+    else:
+        assert gb.gptk_attention_bwd_bf16(qkv.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                          lse.data_ptr(), Dbuf.data_ptr(), dq.data_ptr(), B, T, C,
+                                          H, w, err.data_ptr(), path, s) == 0
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     ro, rlse, rdq = _ref(torch, qkv, B, T, C, H, w, dout)
