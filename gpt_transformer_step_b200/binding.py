@@ -44,7 +44,8 @@ EXPORTED = [
     "gpt_strerror", "gpt_last_cuda_error", "gptk_gemm_bf16", "gptk_attention_fwd_bf16",
     "gptk_attention_bwd_bf16", "gptk_attention_bwd_bf16_noalloc", "gptk_selftest_bounded_wait",
     "gptk_gemm_plan", "gpt_forward_backward", "gpt_sumsq", "gpt_adamw_ranges", "gpt_muon_update",
-    "gptk_attention_bwd_bf16_ds",
+    "gptk_attention_bwd_bf16_ds", "gptk_layernorm_fwd_bf16", "gptk_layernorm_bwd_bf16",
+    "gptk_layernorm_bwd_scratch_floats",
 ]
 
 
@@ -123,6 +124,11 @@ gptk_attention_bwd_bf16 = _sig("gptk_attention_bwd_bf16", _I, [_P, _P, _P, _P, _
                                                                _I, _I, _P, _I, _P])
 gptk_attention_bwd_bf16_ds = _sig("gptk_attention_bwd_bf16_ds", _I, [_P, _P, _P, _P, _P, _P, _P, _I,
                                                                      _I, _I, _I, _I, _P, _P])
+gptk_layernorm_fwd_bf16 = _sig("gptk_layernorm_fwd_bf16", _I, [_P, _P, _P, _P, _P, _I, _I, _F, _P])
+gptk_layernorm_bwd_scratch_floats = _sig("gptk_layernorm_bwd_scratch_floats", ctypes.c_size_t,
+                                         [_I, _I])
+gptk_layernorm_bwd_bf16 = _sig("gptk_layernorm_bwd_bf16", _I, [_P, _P, _P, _P, _P, _P, _I, _P, _I,
+                                                               _P, ctypes.c_size_t, _I, _I, _P])
 gptk_attention_bwd_bf16_noalloc = _sig("gptk_attention_bwd_bf16_noalloc", _I,
                                        [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P])
 gptk_selftest_bounded_wait = _sig("gptk_selftest_bounded_wait", _I, [ctypes.c_uint, _P, _P])

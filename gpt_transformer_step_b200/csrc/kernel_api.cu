@@ -123,6 +123,37 @@ extern "C" int gptk_attention_bwd_bf16_ds(const void *qkv, const void *o, const 
   return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }
 
+extern "C" int gptk_layernorm_fwd_bf16(const void *x, const void *g, void *y, float *mean,
+                                       float *rstd, int M, int C, float eps, void *stream) {
+  if (!x || !g || !y || !mean || !rstd || M < 0 || C <= 0 || !(eps > 0.f)) return GPT_ERR_INVALID_ARG;
+  if ((C % 8) || C > 2048) return GPT_ERR_SHAPE;
+  if ((((uintptr_t)x | (uintptr_t)g | (uintptr_t)y) & 15u) != 0) return GPT_ERR_ALIGN;
+  if (M == 0) return GPT_OK;
+  const cudaError_t e = launch_layernorm_fwd<bf16>((const bf16 *)x, (const bf16 *)g, (bf16 *)y,
+                                                   mean, rstd, M, C, eps, (cudaStream_t)stream);
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
+extern "C" size_t gptk_layernorm_bwd_scratch_floats(int M, int C) {
+  return M <= 0 || C <= 0 ? 0 : (size_t)layernorm_bwd_blocks(M) * C;
+}
+
+extern "C" int gptk_layernorm_bwd_bf16(const void *x, const void *g, const float *mean,
+                                       const float *rstd, const void *dy, void *dres, int dres_in,
+                                       float *dg, int accumulate, float *scratch,
+                                       size_t scratch_floats, int M, int C, void *stream) {
+  if (!x || !g || !mean || !rstd || !dy || !dres || !dg || !scratch || M <= 0 || C <= 0)
+    return GPT_ERR_INVALID_ARG;
+  if ((C % 8) || C > 2048) return GPT_ERR_SHAPE;
+  if (scratch_floats < gptk_layernorm_bwd_scratch_floats(M, C)) return GPT_ERR_INVALID_ARG;
+  if ((((uintptr_t)x | (uintptr_t)g | (uintptr_t)dy | (uintptr_t)dres) & 15u) != 0)
+    return GPT_ERR_ALIGN;
+  const cudaError_t e = launch_layernorm_bwd<bf16>(
+      (const bf16 *)x, (const bf16 *)g, mean, rstd, (const bf16 *)dy, (bf16 *)dres, scratch, dg, M,
+      C, (cudaStream_t)stream, accumulate != 0, dres_in != 0);
+  return e == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
 // Attention backward without any allocation: see include/gpt_kernels.h.
 extern "C" int gptk_attention_bwd_bf16_noalloc(const void *qkv, const void *o, const void *dout,
                                                const float *lse, void *dqkv, int B, int T, int C,

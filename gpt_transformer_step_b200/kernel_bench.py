@@ -33,6 +33,7 @@ GEMMS = {
     "gemm_lmhead": (M, 50304, C, 1, 1, "store", 1),
 }
 ATTN = ("attn_fwd", "attn_bwd", "attn_bwd_ds")
+LN = ("ln_fwd", "ln_bwd")
 
 
 def causal_scores(Bn, Tn, Hn, w=-1):
@@ -48,7 +49,7 @@ def main():
 
     from gpt_transformer_step_b200 import binding as gb
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", nargs="*", default=list(GEMMS) + list(ATTN))
+    ap.add_argument("--case", nargs="*", default=list(GEMMS) + list(ATTN) + list(LN))
     ap.add_argument("--reps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--path", default="tc", choices=["tc", "simt"])
@@ -60,7 +61,36 @@ def main():
     for name in args.case:
         with torch.cuda.stream(stream):
             s = stream.cuda_stream
-            if name in GEMMS:
+            if name in LN:
+                x = torch.randn(M, C, device=dev).to(torch.bfloat16)
+                gam = torch.ones(C, device=dev).to(torch.bfloat16)
+                y = torch.empty(M, C, dtype=torch.bfloat16, device=dev)
+                mean = torch.empty(M, device=dev)
+                rstd = torch.empty(M, device=dev)
+                gb.gptk_layernorm_fwd_bf16(x.data_ptr(), gam.data_ptr(), y.data_ptr(),
+                                           mean.data_ptr(), rstd.data_ptr(), M, C, 1e-5, s)
+                dres = torch.randn(M, C, device=dev).to(torch.bfloat16)
+                dg = torch.zeros(C, device=dev)
+                nsc = gb.gptk_layernorm_bwd_scratch_floats(M, C)
+                scr = torch.empty(nsc, device=dev)
+                if name == "ln_fwd":
+                    def run():
+                        rc = gb.gptk_layernorm_fwd_bf16(x.data_ptr(), gam.data_ptr(), y.data_ptr(),
+                                                        mean.data_ptr(), rstd.data_ptr(), M, C,
+                                                        1e-5, s)
+                        assert rc == 0, rc
+                    nbytes = M * (4.0 * C + 8)
+                else:
+                    def run():
+                        rc = gb.gptk_layernorm_bwd_bf16(x.data_ptr(), gam.data_ptr(),
+                                                        mean.data_ptr(), rstd.data_ptr(),
+                                                        y.data_ptr(), dres.data_ptr(), 1,
+                                                        dg.data_ptr(), 0, scr.data_ptr(), nsc, M,
+                                                        C, s)
+                        assert rc == 0, rc
+                    nbytes = M * (8.0 * C + 8)
+                flops = None
+            elif name in GEMMS:
                 m, n, k, ak, bk, epi, split = GEMMS[name]
                 A = torch.randn(m * k, device=dev).to(torch.bfloat16)
                 Bm = torch.randn(n * k, device=dev).to(torch.bfloat16)
@@ -126,8 +156,12 @@ def main():
             e1.record(stream)
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / args.reps
-        print(json.dumps({"case": name, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
-                          "err": int(err.item())}), flush=True)
+        rec = {"case": name, "ms": ms, "err": int(err.item())}
+        if flops is None:
+            rec["gbs"] = nbytes / (ms * 1e-3) / 1e9
+        else:
+            rec["tflops"] = flops / (ms * 1e-3) / 1e12
+        print(json.dumps(rec), flush=True)
 
 
 if __name__ == "__main__":

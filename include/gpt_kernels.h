@@ -79,6 +79,21 @@ int gptk_attention_bwd_bf16_ds(const void *qkv, const void *o, const void *dout,
                                float *Dbuf, void *ds_scratch, void *dqkv, int B, int T, int C,
                                int H, int window, unsigned *dev_err, void *stream);
 
+/* LayerNorm as the step runs it (bf16 activations, fp32 statistics; gain only, no bias).
+ * forward: y = (x - mean) * rstd * g per row of x [M, C]; mean, rstd fp32 [M] written;
+ *   rstd = 1 / sqrt(biased variance + eps). C % 8 == 0, C <= 2048; 16-byte aligned pointers.
+ * backward: with xh = (x - mean) * rstd and dyh = dy * g,
+ *   dres[m] (+)= rstd * (dyh - mean_c(dyh) - xh * mean_c(dyh * xh))   (+= when dres_in)
+ *   dg (+)= sum_m dy * xh                                             (+= when accumulate)
+ *   summed in a fixed order (per-block partials in scratch, then a column sum);
+ *   scratch: gptk_layernorm_bwd_scratch_floats(M, C) floats. */
+int gptk_layernorm_fwd_bf16(const void *x, const void *g, void *y, float *mean, float *rstd, int M,
+                            int C, float eps, void *stream);
+size_t gptk_layernorm_bwd_scratch_floats(int M, int C);
+int gptk_layernorm_bwd_bf16(const void *x, const void *g, const float *mean, const float *rstd,
+                            const void *dy, void *dres, int dres_in, float *dg, int accumulate,
+                            float *scratch, size_t scratch_floats, int M, int C, void *stream);
+
 /* Failure-detection self test: launches one CTA that waits on an mbarrier nothing arrives
  * on, with the bounded wait every kernel of the step uses for its barriers; after timeout_us
  * (1 .. 2,000,000) it gives up, ORs GPT_DEVERR_TIMEOUT (2) into *dev_err and returns, leaving
