@@ -105,71 +105,54 @@ __global__ void embed_fwd_kernel(const int *__restrict__ tok, const int *__restr
 constexpr int LN_MAXV = 8;  // vectors per lane: C <= 32*8*VN
 
 // NV = 16-byte vectors per lane (ceil(C / (32*VN))), a compile-time bound on the row slice
-// each lane keeps in registers. Persistent: a grid of a few blocks per SM; each warp walks its
-// rows with the next row's vectors in flight while the current row is reduced, and keeps the
-// gains in registers.
-constexpr int LNF_WARPS = 8;
+// each lane keeps in registers.
 template <typename T, int NV>
-__global__ void __launch_bounds__(LNF_WARPS * 32)
-layernorm_fwd_kernel(const T *__restrict__ x, const T *__restrict__ g, T *__restrict__ y,
-                     float *__restrict__ mean, float *__restrict__ rstd, int M, int C, float eps) {
-  using VT = typename Vec<T>::type;
+__global__ void layernorm_fwd_kernel(const T *__restrict__ x, const T *__restrict__ g,
+                                     T *__restrict__ y, float *__restrict__ mean,
+                                     float *__restrict__ rstd, int M, int C, float eps) {
   constexpr int VN = Vec<T>::N;
   const int lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * LNF_WARPS;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= M) return;
   const int nv = C / VN;
-  VT gr[NV], cur[NV], nxt[NV];
+  float v[NV][VN];
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    int c = (lane + 32 * j) * VN;
+    if (lane + 32 * j < nv) {
+      load_vec<T>(x + (long)row * C + c, v[j]);
+#pragma unroll
+      for (int k = 0; k < VN; ++k) s += v[j][k];
+    }
+  }
+  const float mu = warp_sum(s) / (float)C;
+  float q = 0.f;
 #pragma unroll
   for (int j = 0; j < NV; ++j)
-    if (lane + 32 * j < nv) gr[j] = __ldg(reinterpret_cast<const VT *>(g + (lane + 32 * j) * VN));
-  auto load_row = [&](int row, VT (&v)[NV]) {
+    if (lane + 32 * j < nv) {
 #pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (lane + 32 * j < nv)
-        v[j] = *reinterpret_cast<const VT *>(x + (long)row * C + (lane + 32 * j) * VN);
-  };
-  int row = blockIdx.x * LNF_WARPS + (threadIdx.x >> 5);
-  if (row < M) load_row(row, cur);
-  for (; row < M; row += nwarps) {
-    if (row + nwarps < M) load_row(row + nwarps, nxt);
-    float v[NV][VN];
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (lane + 32 * j < nv) {
-        unpack_vec<T>(cur[j], v[j]);
-#pragma unroll
-        for (int k = 0; k < VN; ++k) s += v[j][k];
-      }
-    const float mu = warp_sum(s) / (float)C;
-    float q = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (lane + 32 * j < nv) {
-#pragma unroll
-        for (int k = 0; k < VN; ++k) {
-          const float d = v[j][k] - mu;
-          q += d * d;
-        }
-      }
-    const float var = warp_sum(q) / (float)C;
-    const float rs = 1.0f / sqrtf(var + eps);
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      if (lane + 32 * j < nv) {
-        float gg[VN], o[VN];
-        unpack_vec<T>(gr[j], gg);
-#pragma unroll
-        for (int k = 0; k < VN; ++k) o[k] = (v[j][k] - mu) * rs * gg[k];
-        store_vec<T>(y + (long)row * C + (lane + 32 * j) * VN, o);
+      for (int k = 0; k < VN; ++k) {
+        float d = v[j][k] - mu;
+        q += d * d;
       }
     }
-    if (lane == 0) {
-      mean[row] = mu;
-      rstd[row] = rs;
-    }
+  const float var = warp_sum(q) / (float)C;
+  const float rs = 1.0f / sqrtf(var + eps);
 #pragma unroll
-    for (int j = 0; j < NV; ++j) cur[j] = nxt[j];
+  for (int j = 0; j < NV; ++j) {
+    int c = (lane + 32 * j) * VN;
+    if (lane + 32 * j < nv) {
+      float gg[VN], o[VN];
+      load_vec<T>(g + c, gg);
+#pragma unroll
+      for (int k = 0; k < VN; ++k) o[k] = (v[j][k] - mu) * rs * gg[k];
+      store_vec<T>(y + (long)row * C + c, o);
+    }
+  }
+  if (lane == 0) {
+    mean[row] = mu;
+    rstd[row] = rs;
   }
 }
 
@@ -854,32 +837,12 @@ int ln_nv(int C) {
   return (C + per - 1) / per;
 }
 
-// Blocks of `kernel` (block size `threads`) resident on the whole GPU at once.
-template <typename K>
-int resident_blocks(K kernel, int threads, size_t smem) {
-  int dev = 0, sms = 148, per = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, smem) != cudaSuccess ||
-      per < 1) {
-    cudaGetLastError();
-    per = 1;
-  }
-  return per * sms;
-}
-
 template <typename T>
 cudaError_t launch_layernorm_fwd(const T *x, const T *g, T *y, float *mean, float *rstd, int M,
                                  int C, float eps, cudaStream_t st) {
-  const int rows_grid = (M + LNF_WARPS - 1) / LNF_WARPS;
-  // one wave of resident blocks; each warp walks several rows
-#define LNF(NVC)                                                                              \
-  {                                                                                           \
-    static int res = 0;                                                                       \
-    if (!res) res = resident_blocks(layernorm_fwd_kernel<T, NVC>, LNF_WARPS * 32, 0);         \
-    const int grid = rows_grid < res ? rows_grid : res;                                       \
-    layernorm_fwd_kernel<T, NVC><<<grid, LNF_WARPS * 32, 0, st>>>(x, g, y, mean, rstd, M, C, eps); \
-  }
+  const int warps = 8;
+  const int grid = (M + warps - 1) / warps;
+#define LNF(NVC) layernorm_fwd_kernel<T, NVC><<<grid, warps * 32, 0, st>>>(x, g, y, mean, rstd, M, C, eps)
   LN_DISPATCH(ln_nv<T>(C), LNF)
 #undef LNF
   return cudaGetLastError();

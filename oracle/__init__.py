@@ -82,10 +82,11 @@ def _load():
         L.oracle_gelu_grad_f64.restype = ctypes.c_double
         L.oracle_gelu_grad_f64.argtypes = [ctypes.c_double]
         L.oracle_polar_express_f64.restype = None
-        L.oracle_polar_express_f64.argtypes = [P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+        L.oracle_polar_express_f64.argtypes = [P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int,
+                                               ctypes.c_int]
         L.oracle_muon_adamw_f64.restype = ctypes.c_double
         L.oracle_muon_adamw_f64.argtypes = [ctypes.c_size_t, P, P, P, P, ctypes.c_int, P, P, P] + \
-            [ctypes.c_double] * 10 + [P, ctypes.c_int, ctypes.c_double, ctypes.c_long]
+            [ctypes.c_double] * 10 + [P, ctypes.c_int, ctypes.c_double, ctypes.c_long, ctypes.c_int]
         L.oracle_cross_entropy_f64.restype = ctypes.c_double
         L.oracle_cross_entropy_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     return _lib
@@ -225,12 +226,13 @@ class Oracle:
                                           B, T, C3 // 3, H, window, _ptr(d))
         return d
 
-    def polar_express(self, X, coeffs, ns=None):
-        """Polar Express (normalisation, then ns iterations) of a 2-D array; returns a copy."""
+    def polar_express(self, X, coeffs, ns=None, bf16=False):
+        """Polar Express (normalisation, then ns iterations) of a 2-D array; returns a copy.
+        bf16: every matrix the iteration stores rounded to bf16 (the page's precision)."""
         X = np.array(X, dtype=np.float64, order="C", copy=True)
         cf = np.ascontiguousarray(coeffs, np.float64).reshape(-1)
         ns = len(cf) // 3 if ns is None else ns
-        self.lib.oracle_polar_express_f64(_ptr(X), X.shape[0], X.shape[1], _ptr(cf), ns)
+        self.lib.oracle_polar_express_f64(_ptr(X), X.shape[0], X.shape[1], _ptr(cf), ns, int(bf16))
         return X
 
     def matrices(self):
@@ -247,8 +249,9 @@ class Oracle:
 
     def muon_adamw(self, p, g, m, v, lr, wd, step, clip, coeffs, matrix_lr=0.02, muon_wd=0.0,
                    mu=0.95, beta2_muon=0.95, s_eps=1e-10, beta1=0.9, beta2=0.95, eps=1e-8,
-                   ns=None):
-        """One hybrid step in place on p, m, v (double arrays); returns the grad norm."""
+                   ns=None, bf16=False):
+        """One hybrid step in place on p, m, v (double arrays); returns the grad norm. bf16:
+        the Polar Express at the page's precision (oracle_polar_express_f64)."""
         for a in (p, m, v):
             assert a.dtype == np.float64 and a.flags.c_contiguous
         mats = self.matrices()
@@ -261,7 +264,7 @@ class Oracle:
         return self.lib.oracle_muon_adamw_f64(p.size, _ptr(p), _ptr(g), _ptr(m), _ptr(v), len(mats),
                                               _ptr(off), _ptr(rows), _ptr(cols), lr, wd, beta1,
                                               beta2, eps, matrix_lr, muon_wd, mu, beta2_muon,
-                                              s_eps, _ptr(cf), ns, clip, step)
+                                              s_eps, _ptr(cf), ns, clip, step, int(bf16))
 
     def gelu(self, x: float) -> float:
         return self.lib.oracle_gelu_f64(x)

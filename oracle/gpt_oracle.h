@@ -104,17 +104,20 @@ double oracle_cross_entropy_f64(const double *logits, const int *targets, int ro
 /* ---- hybrid Muon + AdamW update (muon_oracle.cpp; nanochat architecture page,
  * "Optimierungsstrategien Muon und AdamW") ---- */
 /* Polar Express in place on X (rows x cols, row-major): Frobenius normalisation (x 1.01 + 1e-6)
- * then ns iterations with the coefficient triples coeffs[3*i .. 3*i+2] = (a, b, c). */
-void oracle_polar_express_f64(double *X, int rows, int cols, const double *coeffs, int ns);
+ * then ns iterations with the coefficient triples coeffs[3*i .. 3*i+2] = (a, b, c); exact, or
+ * with bf16 != 0 every matrix the iteration stores rounded to bf16 once formed. */
+void oracle_polar_express_f64(double *X, int rows, int cols, const double *coeffs, int ns,
+                              int bf16);
 /* One optimizer step on n parameters: Muon on the n_mat matrices (offset, rows, cols) with
  * the momentum in m and the factored second moment at v[offset ..], AdamW (step t = step) on
- * every other element; both on coef * g, coef = min(1, clip / (||g|| + 1e-6)). Returns ||g||. */
+ * every other element; both on coef * g, coef = min(1, clip / (||g|| + 1e-6)). bf16 != 0: the
+ * update cast to bf16 and the iteration at bf16 (oracle_polar_express_f64). Returns ||g||. */
 double oracle_muon_adamw_f64(size_t n, double *p, const double *g, double *m, double *v,
                              int n_mat, const int64_t *mat_off, const int *mat_rows,
                              const int *mat_cols, double lr, double wd, double beta1,
                              double beta2, double eps, double matrix_lr, double muon_wd,
                              double mu, double beta2_muon, double s_eps, const double *coeffs,
-                             int ns, double clip, long step);
+                             int ns, double clip, long step, int bf16);
 
 #ifdef __cplusplus
 }

@@ -17,8 +17,10 @@
 //  * tall means rows > cols (a square matrix takes the wide branch);
 //  * stage 1, momentum, Nesterov form in the lerp notation of the AdamW listing:
 //    buf = lerp(buf, g, 1 - mu); u = lerp(g, buf, mu);
-//  * the iteration runs here in exact (double) arithmetic; the page's bf16 is the precision of
-//    the GPU path, whose distance from this is bounded in the tests;
+//  * the iteration runs in exact (double) arithmetic, or, with `bf16`, at the page's precision:
+//    the update is cast to bf16 (X = g.bfloat16()), and every matrix the iteration stores
+//    (X after the normalisation, A, B, each new X) is rounded to bf16 once it is formed, its
+//    products and sums taken exactly before that rounding;
 //  * stage 3, the factored second moment: v = mean of X^2 over the reduced dimension,
 //    s = lerp(s, v, 1 - beta2), X' = X / sqrt(max(s, eps)) broadcast along that dimension,
 //    then X' is rescaled to the Frobenius norm of X (the step size stays Muon's);
@@ -26,11 +28,27 @@
 //    gradient of both optimizers.
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <vector>
 
 #include "gpt_oracle.h"
 
 namespace {
+
+// Round to bf16 (nearest even), through float: the value a float accumulator would hold.
+double bf16r(double x) {
+  float f = (float)x;
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7f800000u) == 0x7f800000u) return x;  // inf / nan unchanged
+  u = (u + 0x7fffu + ((u >> 16) & 1u)) & 0xffff0000u;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+void round_all(std::vector<double> &v, bool on) {
+  if (on)
+    for (double &x : v) x = bf16r(x);
+}
 
 // C[m][n] = sum_k A[m][k] * B[k][n]   (A: m x k, B: k x n, row-major)
 void matmul(const double *A, const double *B, int m, int k, int n, double *C) {
@@ -48,12 +66,13 @@ void transpose(const double *X, int r, int c, double *Y) {
 }
 
 // The Polar Express iteration in place on X (r x c), after the Frobenius normalisation.
-void polar_express(double *X, int r, int c, const double *coeffs, int ns) {
+void polar_express(double *X, int r, int c, const double *coeffs, int ns, bool bf16) {
   const size_t n = (size_t)r * c;
   double ss = 0;
   for (size_t i = 0; i < n; ++i) ss += X[i] * X[i];
-  const double scale = 1.0 / (std::sqrt(ss) * 1.01 + 1e-6);
-  for (size_t i = 0; i < n; ++i) X[i] *= scale;
+  double scale = 1.0 / (std::sqrt(ss) * 1.01 + 1e-6);
+  if (bf16) scale = (double)(float)scale;
+  for (size_t i = 0; i < n; ++i) X[i] = bf16 ? bf16r(X[i] * scale) : X[i] * scale;
   const bool tall = r > c;
   const int d = tall ? c : r;  // A and B are d x d
   std::vector<double> Xt(n), A((size_t)d * d), A2((size_t)d * d), Bm((size_t)d * d), XB(n);
@@ -62,11 +81,13 @@ void polar_express(double *X, int r, int c, const double *coeffs, int ns) {
     transpose(X, r, c, Xt.data());
     if (tall) matmul(Xt.data(), X, c, r, c, A.data());   // A = X^T X
     else matmul(X, Xt.data(), r, c, r, A.data());        // A = X X^T
+    round_all(A, bf16);
     matmul(A.data(), A.data(), d, d, d, A2.data());
     for (size_t i = 0; i < (size_t)d * d; ++i) Bm[i] = b * A[i] + cc * A2[i];
+    round_all(Bm, bf16);
     if (tall) matmul(X, Bm.data(), r, c, c, XB.data());  // X B
     else matmul(Bm.data(), X, r, r, c, XB.data());       // B X
-    for (size_t i = 0; i < n; ++i) X[i] = a * X[i] + XB[i];
+    for (size_t i = 0; i < n; ++i) X[i] = bf16 ? bf16r(a * X[i] + XB[i]) : a * X[i] + XB[i];
   }
 }
 
@@ -74,8 +95,9 @@ void polar_express(double *X, int r, int c, const double *coeffs, int ns) {
 
 extern "C" {
 
-void oracle_polar_express_f64(double *X, int rows, int cols, const double *coeffs, int ns) {
-  polar_express(X, rows, cols, coeffs, ns);
+void oracle_polar_express_f64(double *X, int rows, int cols, const double *coeffs, int ns,
+                              int bf16) {
+  polar_express(X, rows, cols, coeffs, ns, bf16 != 0);
 }
 
 double oracle_muon_adamw_f64(size_t n, double *p, const double *g, double *m, double *v,
@@ -83,7 +105,7 @@ double oracle_muon_adamw_f64(size_t n, double *p, const double *g, double *m, do
                              const int *mat_cols, double lr, double wd, double beta1,
                              double beta2, double eps, double matrix_lr, double muon_wd,
                              double mu, double beta2_muon, double s_eps, const double *coeffs,
-                             int ns, double clip, long step) {
+                             int ns, double clip, long step, int bf16) {
   // global clip coefficient
   double ss = 0;
   for (size_t i = 0; i < n; ++i) ss += g[i] * g[i];
@@ -114,8 +136,9 @@ double oracle_muon_adamw_f64(size_t n, double *p, const double *g, double *m, do
       const double gi = coef * g[off + i];
       m[off + i] = m[off + i] + (1.0 - mu) * (gi - m[off + i]);
       X[i] = gi + mu * (m[off + i] - gi);
+      if (bf16) X[i] = bf16r(X[i]);  // X = g.bfloat16()
     }
-    polar_express(X.data(), r, c, coeffs, ns);  // stage 2
+    polar_express(X.data(), r, c, coeffs, ns, bf16 != 0);  // stage 2
     // stage 3: factored second moment, per row (tall) or per column (wide)
     const bool tall = r > c;
     const int nl = tall ? r : c;

@@ -1,13 +1,16 @@
 """The hybrid Muon + AdamW update on the GPU (gpt_muon_update, tensor-core Polar Express
-batched over layers) against the oracle (double, exact iteration), on the same gradients and
-state, for two consecutive steps.
+batched over layers) against the oracle on the same gradients and state, for two
+consecutive steps.
 
-Tolerances. The AdamW part runs in fp32 on the same inputs: the spec update bound,
-max |dp| <= 2e-2 * lr. The momentum buffer is fp32 arithmetic on the same inputs: 1e-6
-relative. The Polar Express iteration runs with bf16 operands (the page's precision): every
-iteration rounds X, A = X X^T and B to bf16 (relative 2^-9 each), so the orthogonalised update
-carries a few 1e-3 of relative error; the matrix update is checked at cosine >= 0.999 and a
-relative Frobenius error <= 3e-2 per matrix, the factored second moment at 3e-2 relative.
+The oracle runs the iteration at the page's precision (X = g.bfloat16(); every matrix the
+iteration stores rounded to bf16 once formed, products and sums exact before that): the GPU
+differs from it only by fp32 accumulation order inside the GEMMs, which flips the bf16
+rounding of a small fraction of the stored elements by one unit (2^-8 relative); the first
+Polar Express step (a = 8.5, b = -25, c = 19) amplifies such flips, so the matrix update is
+checked at cosine >= 0.999 and relative Frobenius error <= 3e-2 per matrix, the factored
+second moment at 3e-2 relative. The distance to the exact (double) iteration is printed. The
+AdamW part runs in fp32 on the same inputs: the spec update bound, max |dp| <= 2e-2 * lr;
+the momentum buffer is fp32 arithmetic on the same inputs: 1e-6 relative.
 """
 import numpy as np
 import pytest
@@ -49,8 +52,11 @@ def test_muon_update_matches_oracle_two_steps():
         st.muon_update(P, G, M, V, LR, WD, CLIP, mc)
         torch.cuda.synchronize()
         assert st.step == step
-        o.muon_adamw(po, g.astype(np.float64), mo, vo, lr=LR, wd=WD, step=step, clip=CLIP,
+        pe, me, ve = po.copy(), mo.copy(), vo.copy()  # the exact iteration, for the report
+        o.muon_adamw(pe, g.astype(np.float64), me, ve, lr=LR, wd=WD, step=step, clip=CLIP,
                      coeffs=cf_oracle, matrix_lr=MATRIX_LR, muon_wd=MUON_WD)
+        o.muon_adamw(po, g.astype(np.float64), mo, vo, lr=LR, wd=WD, step=step, clip=CLIP,
+                     coeffs=cf_oracle, matrix_lr=MATRIX_LR, muon_wd=MUON_WD, bf16=True)
         Pg, Mg, Vg = P.cpu().numpy().astype(np.float64), M.cpu().numpy(), V.cpu().numpy()
         # AdamW part
         assert np.abs(Pg[~in_mat] - po[~in_mat]).max() <= 2e-2 * LR
@@ -60,9 +66,12 @@ def test_muon_update_matches_oracle_two_steps():
             sl = slice(off, off + r * c)
             assert np.abs(Mg[sl] - mo[sl]).max() <= 1e-6 * np.abs(mo[sl]).max()
             d_gpu, d_ref = Pg[sl] - p_before[sl], po[sl] - p_before[sl]
+            d_ex = pe[sl] - p_before[sl]
             cos = U.cosine(d_gpu, d_ref)
             rel = np.linalg.norm(d_gpu - d_ref) / np.linalg.norm(d_ref)
-            print(f"step {step} matrix {r}x{c}: cosine {cos:.6f} rel {rel:.3e}")
+            rel_ex = np.linalg.norm(d_gpu - d_ex) / np.linalg.norm(d_ex)
+            print(f"step {step} matrix {r}x{c}: vs bf16 oracle cosine {cos:.6f} rel {rel:.3e}; "
+                  f"vs exact iteration rel {rel_ex:.3e}")
             assert cos >= 0.999 and rel <= 3e-2, (step, r, c, cos, rel)
             nl = r if r > c else c
             s_gpu, s_ref = Vg[off:off + nl], vo[off:off + nl]

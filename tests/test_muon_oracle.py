@@ -161,3 +161,21 @@ def test_adamw_part_equals_the_pinned_adamw(coeffs):
     # the last bits)
     assert np.abs(p[~mask] - pa[~mask]).max() <= 1e-13 * np.abs(pa).max()
     assert np.abs(m[~mask] - ma[~mask]).max() <= 1e-13 * np.abs(ma).max()
+
+
+def _bf16(a):
+    """Round float64 values to bf16 (nearest even) through float32, with numpy bit operations."""
+    u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return u.view(np.float32).astype(np.float64)
+
+
+def test_bf16_mode_rounds_the_stored_matrices():
+    """With (a, b, c) = (1, 0, 0) the iteration stores X' = 1 X + 0: at bf16 the result is the
+    normalised input (scale taken in float) rounded once to bf16."""
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((40, 72))
+    o = oracle.Oracle.from_shape(SH)
+    Y = o.polar_express(X, np.array([[1.0, 0.0, 0.0]]), bf16=True)
+    scale = np.float32(1.0 / (np.sqrt((X ** 2).sum()) * 1.01 + 1e-6))
+    assert np.array_equal(Y, _bf16(X * np.float64(scale)))
