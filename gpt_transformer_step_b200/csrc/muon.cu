@@ -110,7 +110,7 @@ muon_scale_kernel(bf16 *__restrict__ X, size_t n, const float *__restrict__ scal
 
 // Stage 3, per line (row of a tall matrix, column of a wide one): q = sum of X^2 over the line,
 // s = lerp(s, q / len, 1 - beta2) (s in adam_v at the matrix's offset), rs = 1/sqrt(max(s, eps)),
-// qh = q * rs^2. Tall: a warp per row; wide: a thread per column.
+// qh = q * rs^2. Tall: a warp per row; wide: a block per 256 columns.
 __global__ void __launch_bounds__(MU_THREADS)
 muon_lines_kernel(const bf16 *__restrict__ X, float *__restrict__ sv, MuonGroup grp, float beta2,
                   float eps, const DevScalars *__restrict__ sc, float *__restrict__ q,
@@ -151,13 +151,38 @@ muon_lines_kernel(const bf16 *__restrict__ X, float *__restrict__ sv, MuonGroup 
       if (lane == 0) finish(row, sum);
     }
   } else {
-    for (int col = blockIdx.x * blockDim.x + threadIdx.x; col < c; col += gridDim.x * blockDim.x) {
-      float sum = 0.f;
-      for (int i = 0; i < r; ++i) {
-        const float f = __bfloat162float(x[(size_t)i * c + col]);
-        sum += f * f;
+    // a block per 256 columns: 32 column groups of 8 (16-byte loads) x 8 row groups, each
+    // thread summing every 8th row of its 8 columns; the 8 row-group sums are added in order
+    __shared__ float part[8][256];
+    const int cg = threadIdx.x & 31, rg = threadIdx.x >> 5;
+    for (int c0 = blockIdx.x * 256; c0 < c; c0 += gridDim.x * 256) {
+      const int col = c0 + cg * 8;
+      float acc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+      if (col < c) {
+        for (int i = rg; i < r; i += 8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(x + (size_t)i * c + col);
+          const __nv_bfloat162 *hh = reinterpret_cast<const __nv_bfloat162 *>(&w);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(hh[k]);
+            acc[2 * k] += f.x * f.x;
+            acc[2 * k + 1] += f.y * f.y;
+          }
+        }
       }
-      finish(col, sum);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) part[rg][cg * 8 + k] = acc[k];
+      __syncthreads();
+      const int cc = c0 + threadIdx.x;
+      if (cc < c) {
+        float sum = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) sum += part[g][threadIdx.x];
+        finish(cc, sum);
+      }
+      __syncthreads();
     }
   }
 }
@@ -356,7 +381,7 @@ cudaError_t muon_update_group(TcGemm *tc, const MuonGroup &grp, const MuonStepAr
     cur ^= 1;
   }
   // 3. factored second moment and the norm-preserving rescale
-  const int lb = tall ? (r + (MU_THREADS / 32) - 1) / (MU_THREADS / 32) : (c + MU_THREADS - 1) / MU_THREADS;
+  const int lb = tall ? (r + (MU_THREADS / 32) - 1) / (MU_THREADS / 32) : (c + 255) / 256;
   muon_lines_kernel<<<dim3(lb < 1 ? 1 : lb, L), MU_THREADS, 0, st>>>(s.X[cur], a.sv, grp, a.beta2,
                                                                    a.eps, a.sc, s.q, s.qh, s.rs);
   CUDA_TRY(cudaGetLastError());

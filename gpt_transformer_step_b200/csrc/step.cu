@@ -653,9 +653,12 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   need(&h->dx, M * C * es); need(&h->dh, M * h->mC * es); need(&h->dc, M * C * es);
   need(&h->dqkv, M * 3 * C * es); need(&h->dout, M * C * es); need(&h->dyf, M * C * es);
   need((void **)&h->Dbuf, M * H * 4);
-  // the attention backward runs its two-pass form (the stored-dS form, which the kernel-level
-  // gptk_attention_bwd_bf16_ds runs, measured slower at the 124M shape)
-  h->dst = nullptr;
+  // dS^T scratch of the attention backward: B*H*T^2 bf16 (403 MB at 124M), when it is modest
+  const size_t dst_bytes = (size_t)c.max_B * H * (size_t)c.max_T * c.max_T * 2;
+  const bool use_dst = bf && (c.max_T % 8 == 0) && dst_bytes <= ((size_t)4 << 30) &&
+                       (C / H == 64);
+  if (use_dst) need((void **)&h->dst, dst_bytes);
+  else h->dst = nullptr;
   need((void **)&h->dg_partial, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
   need((void **)&h->gn_partials, (size_t)grad_norm_blocks() * 8);
   need((void **)&h->splitk, h->splitk_elems * 4);

@@ -30,8 +30,20 @@ GEMMS = {
     "gemm_wgrad_qkv": (3 * C, C, M, 0, 0, "f32_store", 0),
     "gemm_wgrad_attnproj": (C, C, M, 0, 0, "f32_store", 0),
     "gemm_wgrad_mlpproj": (C, 4 * C, M, 0, 0, "f32_store", 0),
+    "gemm_dgrad_attnproj": (M, C, C, 1, 0, "store", 1),
+    "gemm_dgrad_qkv": (M, C, 3 * C, 1, 0, "store", 1),
     "gemm_lmhead": (M, 50304, C, 1, 1, "store", 1),
+    # the lm_head backward's two products on one 8192-row chunk (dS is A in both)
+    "gemm_lmhead_dx": (8192, C, 50304, 1, 0, "store", 0),
+    "gemm_lmhead_dwte": (50304, C, 8192, 0, 0, "f32_store", 1),
 }
+# launches of each shape in one 124M step (the lm_head forward statistics and dS recompute
+# run the gemm_lmhead shape with cross-entropy epilogues: two of them per chunk pair)
+STEP_LAUNCHES = {"gemm_qkv": 12, "gemm_attnproj": 12, "gemm_fc": 12, "gemm_mlpproj": 12,
+                 "gemm_dgrad_mlpproj": 12, "gemm_dgrad_fc": 12, "gemm_dgrad_attnproj": 12,
+                 "gemm_dgrad_qkv": 12, "gemm_wgrad_fc": 12, "gemm_wgrad_qkv": 12,
+                 "gemm_wgrad_attnproj": 12, "gemm_wgrad_mlpproj": 12, "gemm_lmhead_dx": 2,
+                 "gemm_lmhead_dwte": 2}
 ATTN = ("attn_fwd", "attn_bwd", "attn_bwd_ds")
 LN = ("ln_fwd", "ln_bwd")
 
