@@ -629,16 +629,19 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // S^T = K Q^T, dP^T = V dO^T, P^T and dS^T -> TMEM, dV += P^T dO, dK += dS^T Q. The lse and
 // D of the next query tile are fetched from global memory one tile ahead.
 // With WRITE_DS the kernel also writes every dS^T tile (bf16, [B*H][T keys][T queries]) for
-// the tensor-core dQ pass (attn_bwd_dq_mma), through a 32 KB staging area that takes one of
-// the Q/dO stages (NST = 3 then).
-constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight (at most)
+// the tensor-core dQ pass (attn_bwd_dq_mma), through a 32 KB staging area. With four Q/dO
+// stages that fits only without the 1 KB of alignment slack: the dynamic shared memory of a
+// kernel without static shared memory starts 1 KB aligned, which the kernel checks (a
+// misaligned start sets the error word and the kernel returns without work).
+constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight
 enum { K_KV0, K_KVFREE0 = K_KV0 + 2, K_QDO0 = K_KVFREE0 + 2, K_FREE0 = K_QDO0 + DKV_STAGES,
        K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE, K_PS, K_MM2, K_NBAR };
 __host__ __device__ constexpr int dkv_smem(int nst, bool write_ds) {
-  return (4 + 2 * nst + (write_ds ? 2 : 0)) * TILE_BYTES + 1024 + 2 * 2 * TILE * 4 + 256;
+  return (4 + 2 * nst + (write_ds ? 2 : 0)) * TILE_BYTES + (write_ds ? 0 : 1024) +
+         2 * 2 * TILE * 4 + 256;
 }
 static_assert(dkv_smem(DKV_STAGES, false) <= 232448, "dK/dV kernel shared memory");
-static_assert(dkv_smem(DKV_STAGES - 1, true) <= 232448, "dK/dV kernel shared memory");
+static_assert(dkv_smem(DKV_STAGES, true) <= 232448, "dK/dV kernel shared memory");
 
 template <int NST, bool WRITE_DS>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
@@ -646,7 +649,11 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
                 const __grid_constant__ CUtensorMap tmDKV, const __grid_constant__ CUtensorMap tmDST,
                 const AttnParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = align1024(smem_raw);
+  if (WRITE_DS && (smem_u32(smem_raw) & 1023u) != 0) {  // no slack for aligning (see above)
+    if (threadIdx.x == 0) atomicOr(P.err, GPT_DEVERR_TIMEOUT);
+    return;
+  }
+  uint8_t *smem = WRITE_DS ? smem_raw : align1024(smem_raw);
   uint8_t *sKV0 = smem;                  // buffer b: K at 2b, V at 2b+1 (in tiles)
   uint8_t *sQ0 = smem + 4 * TILE_BYTES;  // stage s: Q at 2s, dO at 2s+1
   uint8_t *sDS = smem + (4 + 2 * NST) * TILE_BYTES;  // dS^T staging: 4 KB per row warp
@@ -899,30 +906,35 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
 // ------------------------------------------------------------------------------------------
 // backward, dQ from the stored dS^T (used with attn_bwd_dkv_tc<.., true>)
 // ------------------------------------------------------------------------------------------
-// D_i = dO_i . O_i for every row (b, t) and head: one thread per (row, head), 16-byte loads.
+// D_i = dO_i . O_i for every row (b, t) and head: a warp per row, 16-byte loads across the
+// row; the 8 lanes that hold one head's 64 columns combine their partial dots (fixed order).
 __global__ void __launch_bounds__(256)
 attn_bwd_prep_d(const bf16 *__restrict__ O, const bf16 *__restrict__ dO, float *__restrict__ D,
                 int B, int T, int C, int H) {
-  const long n = (long)B * T * H;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
-    const int h = (int)(i % H);
-    const long m = i / H;  // row b*T + t
-    const uint4 *o4 = reinterpret_cast<const uint4 *>(O + m * C + h * HD);
-    const uint4 *d4 = reinterpret_cast<const uint4 *>(dO + m * C + h * HD);
-    float acc = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 av = o4[c], cv = d4[c];
-      const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&av);
-      const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
-        acc += fa.x * fc.x + fa.y * fc.y;
-      }
-    }
+  const int lane = threadIdx.x & 31;
+  const long rows = (long)B * T;
+  for (long m = blockIdx.x * 8L + (threadIdx.x >> 5); m < rows; m += gridDim.x * 8L) {
     const int b = (int)(m / T), t = (int)(m % T);
-    D[((long)b * H + h) * T + t] = acc;
+    for (int c0 = 0; c0 < C; c0 += 256) {  // 256 columns = 4 heads per pass
+      const int col = c0 + lane * 8;
+      float acc = 0.f;
+      if (col < C) {
+        const uint4 av = *reinterpret_cast<const uint4 *>(O + m * C + col);
+        const uint4 cv = *reinterpret_cast<const uint4 *>(dO + m * C + col);
+        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&av);
+        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 fa = __bfloat1622float2(ha[u]), fc = __bfloat1622float2(hc[u]);
+          acc += fa.x * fc.x + fa.y * fc.y;
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      const int h = col / HD;
+      if ((lane & 7) == 0 && col < C) D[((long)b * H + h) * T + t] = acc;
+    }
   }
 }
 
@@ -1162,9 +1174,9 @@ cudaError_t set_attrs() {
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 dkv_smem(DKV_STAGES, false)));
-  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES - 1, true>,
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                dkv_smem(DKV_STAGES - 1, true)));
+                                dkv_smem(DKV_STAGES, true)));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, DQM_SMEM));
   smem_attrs_set = true;
   return cudaSuccess;
@@ -1216,11 +1228,11 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
         !map_rows(&mk, qkv, 3L * C, (long)B * T, 3L * C, 64) ||
         !map_btc(&mdq64, dqkv, 3L * C, T, B, 3L * C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-    const long rows = (long)B * T * H;
-    const int pb = (int)((rows + 255) / 256 < 148 * 8 ? (rows + 255) / 256 : 148 * 8);
+    const long rows = (long)B * T;
+    const int pb = (int)((rows + 7) / 8 < 148 * 16 ? (rows + 7) / 8 : 148 * 16);
     attn_bwd_prep_d<<<pb, 256, 0, st>>>(o, dout, Dbuf, B, T, C, H);
     CUDA_TRY(cudaGetLastError());
-    attn_bwd_dkv_tc<DKV_STAGES - 1, true><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES - 1, true), st>>>(
+    attn_bwd_dkv_tc<DKV_STAGES, true><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES, true), st>>>(
         mq, md, mdkv, mst, p);
     CUDA_TRY(cudaGetLastError());
     attn_bwd_dq_mma<<<grid, DQM_THREADS, DQM_SMEM, st>>>(mld, mk, mdq64, p);
