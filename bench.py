@@ -33,9 +33,13 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 METRIC = "train tokens/s (GPT-2 step, MFU from 6N+attn FLOPs)"
 
-# DRAM bytes (read + write) per tcgen05 GEMM launch from an ncu capture of the current GEMM
-# kernel (none yet: the roofline's traffic is reported as null until one is taken)
-GEMM_DRAM_BYTES_PER_LAUNCH: dict = {}
+# DRAM bytes (read + write) per tcgen05 GEMM launch: ncu dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch of each block GEMM shape and of the lm_head dX / dwte
+# chunks (kernel_bench cases, profiles/gemm_shapes_gpt2_124m_ncu.md), averaged with the launch
+# counts of one step (148 launches; 148.7 MB algorithmic per launch on the same basis). The
+# split-K reduce kernels and the lm_head statistics / recompute launches are not in the mean.
+GEMM_DRAM_BYTES_PER_LAUNCH: dict = {"gpt2_124m_bf16": 137.1e6}
+GEMM_ALG_BYTES_PER_LAUNCH: dict = {"gpt2_124m_bf16": 148.7e6}
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -372,6 +376,7 @@ def run_ours(args, wl, rank, world, local_rank):
                      "frac": (achieved / peak_b) if achieved else None,
                      "frac_vs_sustained": (achieved / peak_s) if achieved else None,
                      "traffic": GEMM_DRAM_BYTES_PER_LAUNCH.get(wl.name),
+                     "traffic_algorithmic": GEMM_ALG_BYTES_PER_LAUNCH.get(wl.name),
                      "traffic_unit": "bytes per GEMM launch (ncu dram__bytes_read.sum + "
                                      "dram__bytes_write.sum)",
                      "flops": "algorithmic: 2MNK of the block GEMMs and the lm_head forward, "
