@@ -52,6 +52,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, int a_mn, int b_mn) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TILE >> 4) << 24);
 }
 
+// A global load issued where it stands: the compiler may not sink it towards its first use
+// (the value is wanted a whole tile later, and its latency must pass in the meantime).
+__device__ __forceinline__ float ldg_early(const float *p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
 // One warp-collective bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           unsigned *err) {
@@ -290,6 +298,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         if (!have) mnew = mt;
         else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
       }
+      const bool have_new = have || mt > -INFINITY;
+      const float mu = have_new ? mnew : 0.f;  // rows with nothing admitted yet: every sv is -inf
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (no long FADD chain)
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float p0 = ex2(fmaf(sv[i], P.scale_log2, -mu));
+        const float p1 = ex2(fmaf(sv[i + 1], P.scale_log2, -mu));
+        ls[(i >> 1) & 3] += p0 + p1;
+        pk[i >> 1] = pack_bf16(p0, p1);
+      }
       if (j > 0) {
         if (!warp_wait(&bar[F_OFULL], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
         tc_fence_after();
@@ -307,21 +326,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         l *= f;
       }
       m2 = mnew;
-      if (mt > -INFINITY) have = true;
-      const float mu = have ? m2 : 0.f;  // rows with nothing admitted yet: every sv is -inf
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (no long FADD chain)
+      have = have_new;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2(fmaf(sv[c * 32 + i], P.scale_log2, -mu));
-          const float p1 = ex2(fmaf(sv[c * 32 + i + 1], P.scale_log2, -mu));
-          ls[(i >> 1) & 3] += p0 + p1;
-          pk[i >> 1] = pack_bf16(p0, p1);
-        }
-        st_tmem_bf16x32(tP + c * 16, pk);
-      }
+      for (int c = 0; c < 4; ++c)
+        st_tmem_bf16x32(tP + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * c]));
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
@@ -497,19 +505,22 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     const int q = warp & 3, ch = (warp - 2) >> 2, r = q * 32 + lane;
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     const int w = P.window;
+    // the lse of this thread's row of an item, loaded from a valid address (index 0 for a row
+    // past T, whose value is never used: such a row's P is masked to zero) with no use of the
+    // value until the item starts
     auto lse_of = [&](const QTile &t) -> float {
       const int qi = t.q0 + r;
-      return qi < P.T ? P.lse_in[((size_t)t.b * P.H + t.h) * P.T + qi] : 0.f;
+      return ldg_early(P.lse_in + (qi < P.T ? ((size_t)t.b * P.H + t.h) * P.T + qi : 0));
     };
     int g = 0;
     bool ok = true;
     QTile it, nx;
     bool have_it = query_item(P, 0, it);
-    float lse_cur = have_it ? lse_of(it) : 0.f;
+    float lse_cur = have_it ? lse_of(it) : 0.f;  // (no item: nothing waits on it)
     int pend_qb = -1;  // buffer whose dQ staging a TMA store may still be reading
     for (int i = 0; ok && have_it; ++i) {
       const bool have_nx = query_item(P, i + 1, nx);
-      const float lse_nx = have_nx ? lse_of(nx) : 0.f;  // in flight during this item
+      const float lse_nx = lse_of(have_nx ? nx : it);  // in flight during this item
       const int qb = i & 1, q0 = it.q0, qi = q0 + r;
       if (!warp_wait(&bar[Q_QDO0 + qb], (i >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
       // D_i = dO_i . O_i (also written for the dK/dV pass) from the swizzled smem tiles
@@ -747,25 +758,32 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     const int t = threadIdx.x - 64;  // 0..255 among the row warps
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     const int w = P.window;
-    // this thread's share of a query tile's (lse | D): t < 128 lse (log2 domain), else D
-    auto fetch = [&](const KTile &k, int j) -> float {
-      const int qi = (k.qt0 + j) * TILE + (t & 127);
-      if (qi >= P.T) return 0.f;
-      const size_t li = ((size_t)k.b * P.H + k.h) * P.T + qi;
-      return t < 128 ? P.lse_in[li] * LOG2E : P.Dbuf[li];
+    // This thread's share of a query tile's (lse | D): t < 128 lse, else D. It is copied one
+    // tile ahead straight into that tile's shared buffer (cp.async: no register holds it, so
+    // nothing waits on the load's latency), always from a valid address; whether it counts (a
+    // query past T, or no tile) and the scaling of lse to the log2 domain are applied in place
+    // when that tile starts.
+    auto fetch = [&](const KCursor &k, float *dst) -> bool {
+      const int qi = k.valid ? (k.it.qt0 + k.j) * TILE + (t & 127) : P.T;
+      const bool valid = qi < P.T;
+      const size_t li = valid ? ((size_t)k.it.b * P.H + k.it.h) * P.T + qi : 0;
+      cp_async4(dst, (t < 128 ? P.lse_in : P.Dbuf) + li);
+      return valid;
     };
+    const float lsd_scale = t < 128 ? LOG2E : 1.f;
     bool ok = true;
     KCursor cur;
     cur.start(P);
-    float pre = cur.valid ? fetch(cur.it, 0) : 0.f;
+    bool pre_ok = fetch(cur, s_lsd + t);
     int pend_kb = -1;  // buffer whose dV/dK staging a TMA store may still be reading
     for (int g = 0; cur.valid; ++g) {
       const KTile it = cur.it;
       const int j = cur.j, kb = cur.i & 1, k0 = it.k0, ki = k0 + r, qq0 = (it.qt0 + j) * TILE;
-      // this query tile's lse and D, into buffer g & 1; one barrier per tile (the other
+      // this query tile's lse and D are in buffer g & 1; one barrier per tile (the other
       // buffer may still be read by a warp finishing the previous tile)
       float *lsd = s_lsd + (g & 1) * 2 * TILE;
-      lsd[t] = pre;
+      cp_async_wait_all();  // this thread's copy for this tile (issued a tile ago) has landed
+      lsd[t] = pre_ok ? lsd[t] * lsd_scale : 0.f;
       asm volatile("bar.sync 1, 256;" ::: "memory");
       // the previous item's dV/dK store has read its staging: that K/V buffer is free
       if (pend_kb >= 0) {
@@ -776,7 +794,9 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       }
       KCursor nx = cur;
       nx.next(P);
-      pre = nx.valid ? fetch(nx.it, nx.j) : 0.f;  // in flight during this tile
+      // every row warp is past the barrier, so done with the previous tile and its buffer,
+      // which now takes the next tile's values (in flight during this tile)
+      pre_ok = fetch(nx, s_lsd + ((g + 1) & 1) * 2 * TILE + t);
       cur = nx;
       // after an abort every row warp still passes the named barrier of each tile
       if (ok) ok = warp_wait(&bar[K_SDP], g & 1, abort_flag, P.err);
@@ -794,63 +814,58 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       const int hi = min(P.T - 1, w >= 0 ? ki + w : P.T - 1) - qq0 - ch * 64;
       const float4 *L4 = reinterpret_cast<const float4 *>(lsd + ch * 64);
       const float4 *D4 = reinterpret_cast<const float4 *>(lsd + TILE + ch * 64);
-      // P^T / dS^T are free once the previous dV / dK MMAs are done (for j == 0 the
-      // previous item's epilogue waited for them)
-      if (j > 0) {
-        ok = warp_wait(&bar[K_MM2], (g - 1) & 1, abort_flag, P.err);
-        if (!ok) continue;
-      }
       const uint32_t tPT = tmem + ((uint32_t)(q * 32) << 16) + 384 + ch * 32, tdST = tPT + 64;
+      // P^T and dS^T of this thread's 64 columns, packed bf16 pairs, in registers first; the
+      // tensor-memory copies wait for the previous tile's dV / dK MMAs (which read P^T / dS^T)
+      // only after the math, so those MMAs run under it
+      uint32_t pp[32], pd[32];
       // two copies of the loop: interior tiles carry no per-element mask
       auto pds_math = [&](auto masked) {
       constexpr bool MASK = decltype(masked)::value;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {  // 32 columns -> 16 packed TMEM columns each
-        uint32_t pp[16], pd[16];
+      for (int i = 0; i < 64; i += 4) {
+        const float4 L = L4[i >> 2], Dv = D4[i >> 2];
+        const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+        float pr[4], dr[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int i = 32 * half + 8 * u + 4 * hh;
-            const float4 L = L4[i >> 2], Dv = D4[i >> 2];
-            const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
-            float pr[4], dr[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int ii = i + e;
-              const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
-              const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
-              float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
-              if (MASK) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
-              pr[e] = pv;
-              dr[e] = pv * (dpv - dv[e]);
-            }
-            const int o = 4 * u + 2 * hh;
-            pp[o] = pack_bf16(pr[0], pr[1]);
-            pp[o + 1] = pack_bf16(pr[2], pr[3]);
-            pd[o] = pack_bf16(dr[0], dr[1]);
-            pd[o + 1] = pack_bf16(dr[2], dr[3]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const int ii = i + e;
+          const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
+          const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
+          float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
+          if (MASK) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
+          pr[e] = pv;
+          dr[e] = pv * (dpv - dv[e]);
         }
-        tmem_st16_nw(tPT + 16 * half, pp);
-        tmem_st16_nw(tdST + 16 * half, pd);
-        if (WRITE_DS) {  // the same bf16 dS^T row into the staging slot (128-byte swizzle)
-          uint8_t *slot = sDS + (warp - 2) * 4096;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int c = 4 * half + c4;  // 16-byte chunk of the 128-byte row
-            *reinterpret_cast<uint4 *>(slot + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(pd[4 * c4], pd[4 * c4 + 1], pd[4 * c4 + 2], pd[4 * c4 + 3]);
-          }
-        }
+        pp[i >> 1] = pack_bf16(pr[0], pr[1]);
+        pp[(i >> 1) + 1] = pack_bf16(pr[2], pr[3]);
+        pd[i >> 1] = pack_bf16(dr[0], dr[1]);
+        pd[(i >> 1) + 1] = pack_bf16(dr[2], dr[3]);
       }
       };
-      if (WRITE_DS) {  // this warp's dS^T staging slot must have been read by its last store
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
       if (interior) pds_math(std::false_type{});
       else pds_math(std::true_type{});
+      // P^T / dS^T in tensor memory are free once the previous dV / dK MMAs are done (for
+      // j == 0 the previous item's epilogue waited for them)
+      if (j > 0) {
+        ok = warp_wait(&bar[K_MM2], (g - 1) & 1, abort_flag, P.err);
+        if (!ok) continue;
+      }
+      tmem_st16_nw(tPT, *reinterpret_cast<const uint32_t(*)[16]>(&pp[0]));
+      tmem_st16_nw(tPT + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pp[16]));
+      tmem_st16_nw(tdST, *reinterpret_cast<const uint32_t(*)[16]>(&pd[0]));
+      tmem_st16_nw(tdST + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pd[16]));
+      if (WRITE_DS) {
+        // this warp's dS^T staging slot must have been read by its last store; then the same
+        // bf16 dS^T row goes into it (128-byte swizzle)
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        uint8_t *slot = sDS + (warp - 2) * 4096;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)  // 16-byte chunk c of the 128-byte row
+          *reinterpret_cast<uint4 *>(slot + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -894,6 +909,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       }
       pend_kb = kb;
     }
+    cp_async_wait_all();  // the last (unused) lse / D copy has landed
     if (lane == 0) bulk_wait_all();  // every store of this warp (dK/dV, dS^T) has completed
   }
   tc_fence_before();

@@ -87,7 +87,8 @@ constexpr float LOG2E_F = 1.4426950408889634f;
 // Per-row epilogue operands that do not depend on the accumulators; they are fetched before
 // the epilogue waits for a tile, so their latency overlaps the MMAs.
 struct EpiRow {
-  float L2;   // cross-entropy dS: lse of the row, log2 units
+  float lse;  // cross-entropy dS: lse of the row (natural log; scaled where it is used, so
+              // that nothing waits on the load before the accumulators are ready)
   float s;    // cross-entropy dS: 1 / (number of loss terms)
   int t;      // cross-entropy: target column of the row (-1 for rows past M)
 };
@@ -95,11 +96,13 @@ template <int EPI>
 __device__ __forceinline__ EpiRow epi_row(const TcParams &P, int row) {
   EpiRow r{0.f, 0.f, -1};
   const Epi &e = P.epi;
-  if (EPI == TE_CE_DS || EPI == TE_CE_STATS) {
-    if (row < P.M) r.t = e.targets[e.row_offset + row];
-  }
+  // Loaded unconditionally from a valid row (a row past M reads row M-1: nothing of such a row
+  // is stored or written), so that no select on the loaded values makes the warp wait for
+  // them before the accumulators are ready.
+  const int rr = row < P.M ? row : P.M - 1;
+  if (EPI == TE_CE_DS || EPI == TE_CE_STATS) r.t = e.targets[e.row_offset + rr];
   if (EPI == TE_CE_DS) {
-    if (row < P.M) r.L2 = e.lse[e.row_offset + row] * LOG2E_F;
+    r.lse = e.lse[e.row_offset + rr];
     r.s = e.sc->inv_M;
   }
   return r;
@@ -185,9 +188,13 @@ struct TcCfg {
   static constexpr int B_ROWS = BN / CG;                 // rows of B each CTA loads
   static constexpr int B_CTA_BYTES = B_ROWS * BK * 2;    // 32 KB / 16 KB
   static constexpr int STAGE = A_BYTES + B_CTA_BYTES;    // 48 KB / 32 KB
-  static constexpr int NSTAGE = CG == 1 ? 4 : 5;
-  static constexpr int WARP_STAGE = CG == 1 ? 4096 : 8192;  // epilogue staging per warp
+  // Pairs: six 32 KB stages and 4 KB of epilogue staging per warp (two bf16 chunk slots, or
+  // one for two outputs / fp32) measured faster than five stages with 8 KB: the deeper ring
+  // covers more TMA latency, and the epilogue's smaller slot count costs less than that.
+  static constexpr int NSTAGE = CG == 1 ? 4 : 6;
+  static constexpr int WARP_STAGE = 4096;  // epilogue staging per warp
   static constexpr int SMEM = NSTAGE * STAGE + EPI_WARPS * WARP_STAGE + 1024 + 256;
+  static_assert(SMEM <= 232448, "GEMM shared memory");
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -276,10 +283,11 @@ __device__ __forceinline__ void epi_math(const TcParams &P, int col0, const EpiR
   if (EPI == TE_CE_DS) {
     // dS = (softmax - onehot(target)) / n over the valid vocabulary columns, 0 past V
     const int V = P.epi.V;
+    const float L2 = er.lse * LOG2E_F;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int c = col0 + i;
-      float p = ex2(fmaf(v[i], LOG2E_F, -er.L2));
+      float p = ex2(fmaf(v[i], LOG2E_F, -L2));
       p = (c == er.t) ? p - 1.f : p;
       v[i] = c < V ? p * er.s : 0.f;
     }

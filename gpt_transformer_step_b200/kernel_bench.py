@@ -2,6 +2,7 @@
 (B=16, T=1024, C=768, H=12), through the kernel-level C ABI (include/gpt_kernels.h).
 
     python -m gpt_transformer_step_b200.kernel_bench [--case NAME ...] [--reps N] [--path tc|simt]
+                                                     [--torch] [--gemm M,N,K[,EPI] ...]
 
 Each case runs `warmup` untimed launches, then `reps` launches timed with CUDA events on the
 launching stream; prints one JSON line per case with ms per launch and TFLOP/s (algorithmic
@@ -65,7 +66,17 @@ def main():
     ap.add_argument("--reps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--path", default="tc", choices=["tc", "simt"])
+    ap.add_argument("--torch", action="store_true",
+                    help="also time torch.matmul (cuBLAS, bf16 output, no epilogue) on each "
+                         "GEMM case's shapes and layouts, for comparison")
+    ap.add_argument("--gemm", nargs="*", default=[], metavar="M,N,K[,EPI]",
+                    help="extra K-major x K-major GEMM cases (epilogue store by default)")
     args = ap.parse_args()
+    for spec in args.gemm:
+        f = spec.split(",")
+        GEMMS[f"gemm_{spec}"] = (int(f[0]), int(f[1]), int(f[2]), 1, 1,
+                                 f[3] if len(f) > 3 else "store", 1)
+        args.case.append(f"gemm_{spec}")
     path = gb.GPTK_PATH_TCGEN05 if args.path == "tc" else gb.GPTK_PATH_SIMT
     dev = torch.device("cuda", 0)
     stream = torch.cuda.Stream(device=dev)
@@ -124,6 +135,19 @@ def main():
                                            path, s)
                     assert rc == 0, rc
                 flops = 2.0 * m * n * k
+                if args.torch:
+                    At = A.view(m, k) if ak else A.view(k, m).t()
+                    Bt = Bm.view(n, k).t() if bk else Bm.view(k, n)
+                    for _ in range(args.warmup):
+                        torch.matmul(At, Bt)
+                    t0 = torch.cuda.Event(enable_timing=True)
+                    t1 = torch.cuda.Event(enable_timing=True)
+                    t0.record(stream)
+                    for _ in range(args.reps):
+                        torch.matmul(At, Bt)
+                    t1.record(stream)
+                    torch.cuda.synchronize()
+                    torch_ms = t0.elapsed_time(t1) / args.reps
             else:
                 qkv = torch.randn(M, 3 * C, device=dev).to(torch.bfloat16)
                 o = torch.empty(M, C, dtype=torch.bfloat16, device=dev)
@@ -173,6 +197,9 @@ def main():
             rec["gbs"] = nbytes / (ms * 1e-3) / 1e9
         else:
             rec["tflops"] = flops / (ms * 1e-3) / 1e12
+            if args.torch and name in GEMMS:
+                rec["torch_ms"] = torch_ms
+                rec["torch_tflops"] = flops / (torch_ms * 1e-3) / 1e12
         print(json.dumps(rec), flush=True)
 
 
