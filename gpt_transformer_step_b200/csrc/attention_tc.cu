@@ -802,11 +802,6 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       if (ok) ok = warp_wait(&bar[K_SDP], g & 1, abort_flag, P.err);
       if (!ok) continue;
       tc_fence_after();
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      ld_s_dp64(tS, tdP, s0, s1, d0, d1);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[K_SDPFREE]);
       const bool interior = (k0 + TILE - 1 <= qq0) && (w < 0 || k0 >= qq0 + TILE - 1 - w) &&
                             (qq0 + TILE <= P.T);
       // queries admitted for key ki: ki <= q <= ki + w, q < T  ->  local columns lo..hi
@@ -817,34 +812,49 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
       const uint32_t tPT = tmem + ((uint32_t)(q * 32) << 16) + 384 + ch * 32, tdST = tPT + 64;
       // P^T and dS^T of this thread's 64 columns, packed bf16 pairs, in registers first; the
       // tensor-memory copies wait for the previous tile's dV / dK MMAs (which read P^T / dS^T)
-      // only after the math, so those MMAs run under it
+      // only after the math, so those MMAs run under it. The 64 columns are taken in two
+      // halves of 32 (S and dP of one half in registers at a time, which keeps the row warps
+      // within their registers); the accumulators are released after the second half's loads.
       uint32_t pp[32], pd[32];
+      uint32_t sv[32], dv[32];
       // two copies of the loop: interior tiles carry no per-element mask
-      auto pds_math = [&](auto masked) {
+      auto pds_math = [&](auto masked, auto half_c) {
       constexpr bool MASK = decltype(masked)::value;
+      constexpr int half = decltype(half_c)::value;
 #pragma unroll
-      for (int i = 0; i < 64; i += 4) {
-        const float4 L = L4[i >> 2], Dv = D4[i >> 2];
-        const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+      for (int i = 0; i < 32; i += 4) {
+        const int c = 32 * half + i;  // column within this thread's 64
+        const float4 L = L4[c >> 2], Dv = D4[c >> 2];
+        const float lv[4] = {L.x, L.y, L.z, L.w}, dl[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
         float pr[4], dr[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int ii = i + e;
-          const float sv = __uint_as_float(ii < 32 ? s0[ii] : s1[ii - 32]);
-          const float dpv = __uint_as_float(ii < 32 ? d0[ii] : d1[ii - 32]);
-          float pv = ex2(fmaf(sv, P.scale_log2, -lv[e]));
-          if (MASK) pv = (ii <= hi && ii >= lo) ? pv : 0.f;
+          float pv = ex2(fmaf(__uint_as_float(sv[i + e]), P.scale_log2, -lv[e]));
+          if (MASK) pv = (c + e <= hi && c + e >= lo) ? pv : 0.f;
           pr[e] = pv;
-          dr[e] = pv * (dpv - dv[e]);
+          dr[e] = pv * (__uint_as_float(dv[i + e]) - dl[e]);
         }
-        pp[i >> 1] = pack_bf16(pr[0], pr[1]);
-        pp[(i >> 1) + 1] = pack_bf16(pr[2], pr[3]);
-        pd[i >> 1] = pack_bf16(dr[0], dr[1]);
-        pd[(i >> 1) + 1] = pack_bf16(dr[2], dr[3]);
+        pp[c >> 1] = pack_bf16(pr[0], pr[1]);
+        pp[(c >> 1) + 1] = pack_bf16(pr[2], pr[3]);
+        pd[c >> 1] = pack_bf16(dr[0], dr[1]);
+        pd[(c >> 1) + 1] = pack_bf16(dr[2], dr[3]);
       }
       };
-      if (interior) pds_math(std::false_type{});
-      else pds_math(std::true_type{});
+      tmem_ld32_nw(tS, sv);
+      tmem_ld32_nw(tdP, dv);
+      tmem_wait_ld32(sv);
+      reg_fence32(dv);
+      if (interior) pds_math(std::false_type{}, std::integral_constant<int, 0>{});
+      else pds_math(std::true_type{}, std::integral_constant<int, 0>{});
+      tmem_ld32_nw(tS + 32, sv);
+      tmem_ld32_nw(tdP + 32, dv);
+      tmem_wait_ld32(sv);
+      reg_fence32(dv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[K_SDPFREE]);  // S^T / dP^T may be overwritten now
+      if (interior) pds_math(std::false_type{}, std::integral_constant<int, 1>{});
+      else pds_math(std::true_type{}, std::integral_constant<int, 1>{});
       // P^T / dS^T in tensor memory are free once the previous dV / dK MMAs are done (for
       // j == 0 the previous item's epilogue waited for them)
       if (j > 0) {
