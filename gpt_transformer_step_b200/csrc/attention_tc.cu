@@ -638,21 +638,23 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 // ------------------------------------------------------------------------------------------
 // Per item: K and V of the key tile (double-buffered); then for every query tile that sees it
 // S^T = K Q^T, dP^T = V dO^T, P^T and dS^T -> TMEM, dV += P^T dO, dK += dS^T Q. The lse and
-// D of the next query tile are fetched from global memory one tile ahead.
+// D of a query tile are copied from global memory two tiles ahead.
 // With WRITE_DS the kernel also writes every dS^T tile (bf16, [B*H][T keys][T queries]) for
-// the tensor-core dQ pass (attn_bwd_dq_mma), through a 32 KB staging area. With four Q/dO
-// stages that fits only without the 1 KB of alignment slack: the dynamic shared memory of a
-// kernel without static shared memory starts 1 KB aligned, which the kernel checks (a
-// misaligned start sets the error word and the kernel returns without work).
-constexpr int DKV_STAGES = 4;  // Q/dO tiles in flight
+// the tensor-core dQ pass (attn_bwd_dq_mma), through a 32 KB staging area, and keeps three
+// Q/dO stages. It takes no alignment slack: the dynamic shared memory of a kernel without
+// static shared memory starts 1 KB aligned, which the kernel checks (a misaligned start sets
+// the error word and the kernel returns without work).
+constexpr int DKV_STAGES = 4;     // Q/dO tiles in flight
+constexpr int DKV_STAGES_DS = 3;  // the same with dS^T staging (shared memory)
+constexpr int LSD_BUFS = 3;       // per-tile lse / D buffers: copied two tiles ahead
 enum { K_KV0, K_KVFREE0 = K_KV0 + 2, K_QDO0 = K_KVFREE0 + 2, K_FREE0 = K_QDO0 + DKV_STAGES,
        K_SDP = K_FREE0 + DKV_STAGES, K_SDPFREE, K_PS, K_MM2, K_NBAR };
 __host__ __device__ constexpr int dkv_smem(int nst, bool write_ds) {
   return (4 + 2 * nst + (write_ds ? 2 : 0)) * TILE_BYTES + (write_ds ? 0 : 1024) +
-         2 * 2 * TILE * 4 + 256;
+         LSD_BUFS * 2 * TILE * 4 + 256;
 }
 static_assert(dkv_smem(DKV_STAGES, false) <= 232448, "dK/dV kernel shared memory");
-static_assert(dkv_smem(DKV_STAGES, true) <= 232448, "dK/dV kernel shared memory");
+static_assert(dkv_smem(DKV_STAGES_DS, true) <= 232448, "dK/dV kernel shared memory");
 
 template <int NST, bool WRITE_DS>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
@@ -668,8 +670,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
   uint8_t *sKV0 = smem;                  // buffer b: K at 2b, V at 2b+1 (in tiles)
   uint8_t *sQ0 = smem + 4 * TILE_BYTES;  // stage s: Q at 2s, dO at 2s+1
   uint8_t *sDS = smem + (4 + 2 * NST) * TILE_BYTES;  // dS^T staging: 4 KB per row warp
-  float *s_lsd = (float *)(smem + (4 + 2 * NST + (WRITE_DS ? 2 : 0)) * TILE_BYTES);  // [2][lse | D]
-  uint64_t *bar = (uint64_t *)(s_lsd + 2 * 2 * TILE);
+  float *s_lsd = (float *)(smem + (4 + 2 * NST + (WRITE_DS ? 2 : 0)) * TILE_BYTES);  // [3][lse | D]
+  uint64_t *bar = (uint64_t *)(s_lsd + LSD_BUFS * 2 * TILE);
   uint32_t *tmem_holder = (uint32_t *)(bar + K_NBAR);
   volatile int *abort_flag = (volatile int *)(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -758,11 +760,11 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     const int t = threadIdx.x - 64;  // 0..255 among the row warps
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16) + ch * 64, tdP = tS + 128;
     const int w = P.window;
-    // This thread's share of a query tile's (lse | D): t < 128 lse, else D. It is copied one
-    // tile ahead straight into that tile's shared buffer (cp.async: no register holds it, so
-    // nothing waits on the load's latency), always from a valid address; whether it counts (a
-    // query past T, or no tile) and the scaling of lse to the log2 domain are applied in place
-    // when that tile starts.
+    // This thread's share of a query tile's (lse | D): t < 128 lse, else D. It is copied two
+    // tiles ahead straight into that tile's shared buffer (cp.async: no register holds it, so
+    // nothing waits on the load's latency, which under the dS^T write stream can exceed a
+    // tile), always from a valid address; whether it counts (a query past T, or no tile) and
+    // the scaling of lse to the log2 domain are applied in place when that tile starts.
     auto fetch = [&](const KCursor &k, float *dst) -> bool {
       const int qi = k.valid ? (k.it.qt0 + k.j) * TILE + (t & 127) : P.T;
       const bool valid = qi < P.T;
@@ -772,18 +774,24 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
     };
     const float lsd_scale = t < 128 ? LOG2E : 1.f;
     bool ok = true;
-    KCursor cur;
+    KCursor cur, c1;  // this tile and the next one
     cur.start(P);
-    bool pre_ok = fetch(cur, s_lsd + t);
+    c1 = cur;
+    c1.next(P);
+    bool ok0 = fetch(cur, s_lsd + t);  // validity of this tile's value and the next one's
+    cp_async_commit();
+    bool ok1 = fetch(c1, s_lsd + 2 * TILE + t);
+    cp_async_commit();
+    int lb = 0;  // this tile's buffer (g mod 3)
     int pend_kb = -1;  // buffer whose dV/dK staging a TMA store may still be reading
     for (int g = 0; cur.valid; ++g) {
       const KTile it = cur.it;
       const int j = cur.j, kb = cur.i & 1, k0 = it.k0, ki = k0 + r, qq0 = (it.qt0 + j) * TILE;
       // this query tile's lse and D are in buffer g & 1; one barrier per tile (the other
       // buffer may still be read by a warp finishing the previous tile)
-      float *lsd = s_lsd + (g & 1) * 2 * TILE;
-      cp_async_wait_all();  // this thread's copy for this tile (issued a tile ago) has landed
-      lsd[t] = pre_ok ? lsd[t] * lsd_scale : 0.f;
+      float *lsd = s_lsd + lb * 2 * TILE;
+      cp_async_wait_group<1>();  // this tile's copy has landed (the next tile's may not have)
+      lsd[t] = ok0 ? lsd[t] * lsd_scale : 0.f;
       asm volatile("bar.sync 1, 256;" ::: "memory");
       // the previous item's dV/dK store has read its staging: that K/V buffer is free
       if (pend_kb >= 0) {
@@ -792,11 +800,15 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant
         if (lane == 0) mbar_arrive(&bar[K_KVFREE0 + pend_kb]);
         pend_kb = -1;
       }
-      KCursor nx = cur;
-      nx.next(P);
+      const KCursor nx = c1;
+      c1.next(P);
       // every row warp is past the barrier, so done with the previous tile and its buffer,
-      // which now takes the next tile's values (in flight during this tile)
-      pre_ok = fetch(nx, s_lsd + ((g + 1) & 1) * 2 * TILE + t);
+      // which now takes the values of the tile after the next one
+      const int lb2 = lb == 0 ? 2 : lb - 1;  // (g + 2) mod 3
+      ok0 = ok1;
+      ok1 = fetch(c1, s_lsd + lb2 * 2 * TILE + t);
+      cp_async_commit();
+      lb = lb == 2 ? 0 : lb + 1;
       cur = nx;
       // after an abort every row warp still passes the named barrier of each tile
       if (ok) ok = warp_wait(&bar[K_SDP], g & 1, abort_flag, P.err);
@@ -1200,9 +1212,9 @@ cudaError_t set_attrs() {
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 dkv_smem(DKV_STAGES, false)));
-  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES, true>,
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkv_tc<DKV_STAGES_DS, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                dkv_smem(DKV_STAGES, true)));
+                                dkv_smem(DKV_STAGES_DS, true)));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, DQM_SMEM));
   smem_attrs_set = true;
   return cudaSuccess;
@@ -1258,7 +1270,7 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
     const int pb = (int)((rows + 7) / 8 < 148 * 16 ? (rows + 7) / 8 : 148 * 16);
     attn_bwd_prep_d<<<pb, 256, 0, st>>>(o, dout, Dbuf, B, T, C, H);
     CUDA_TRY(cudaGetLastError());
-    attn_bwd_dkv_tc<DKV_STAGES, true><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES, true), st>>>(
+    attn_bwd_dkv_tc<DKV_STAGES_DS, true><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES_DS, true), st>>>(
         mq, md, mdkv, mst, p);
     CUDA_TRY(cudaGetLastError());
     attn_bwd_dq_mma<<<grid, DQM_THREADS, DQM_SMEM, st>>>(mld, mk, mdq64, p);
