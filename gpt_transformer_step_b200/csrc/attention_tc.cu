@@ -301,13 +301,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       const bool have_new = have || mt > -INFINITY;
       const float mu = have_new ? mnew : 0.f;  // rows with nothing admitted yet: every sv is -inf
       float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (no long FADD chain)
-      uint32_t pk[64];
+      uint32_t pk[4][16];  // P of the row, packed bf16 pairs, by 32-column chunk
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
         const float p0 = ex2(fmaf(sv[i], P.scale_log2, -mu));
         const float p1 = ex2(fmaf(sv[i + 1], P.scale_log2, -mu));
         ls[(i >> 1) & 3] += p0 + p1;
-        pk[i >> 1] = pack_bf16(p0, p1);
+        pk[i >> 5][(i >> 1) & 15] = pack_bf16(p0, p1);
       }
       if (j > 0) {
         if (!warp_wait(&bar[F_OFULL], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
@@ -329,7 +329,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       have = have_new;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        st_tmem_bf16x32(tP + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * c]));
+        st_tmem_bf16x32(tP + c * 16, pk[c]);
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();

@@ -222,8 +222,11 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
 }
+// Relaxed: it only tells the MMA issuer that this warp's accumulator reads are done, and those
+// have completed (tcgen05.wait::ld) before the tcgen05 fence that precedes it; a release would
+// also wait for this thread's earlier writes, which nothing on the other side reads.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx_addr(uint32_t addr, uint32_t bytes) {
