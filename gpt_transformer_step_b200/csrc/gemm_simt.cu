@@ -108,27 +108,49 @@ __global__ void splitk_reduce_kernel(GemmDesc d) {
   }
 }
 
-// N % 4 == 0: a block per row (grid-stride over rows), four columns per thread from 16-byte
-// partial loads; the splits are added in split order, as above.
+// N % 4 == 0: grid-stride over groups of four columns, 16-byte partial loads; the splits are
+// added in split order, as above. vec_out: the fp32 store / accumulate and the plain
+// activation store write their four values with one vector access (the host checks the
+// alignment), the other epilogues go element by element.
 template <typename T>
-__global__ void __launch_bounds__(256) splitk_reduce4_kernel(GemmDesc d) {
+__global__ void __launch_bounds__(256) splitk_reduce4_kernel(GemmDesc d, int vec_out) {
   const int n4 = d.N >> 2;
-  const long zstride4 = (long)d.M * n4;
+  const long total4 = (long)d.M * n4;
   const float4 *part = reinterpret_cast<const float4 *>(d.partial);
-  for (int m = blockIdx.x; m < d.M; m += gridDim.x) {
-    for (int c = threadIdx.x; c < n4; c += blockDim.x) {
-      const float4 *p = part + (long)m * n4 + c;
-      float4 s = p[0];
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total4;
+       i += (long)gridDim.x * blockDim.x) {
+    const int m = (int)(i / n4), n = 4 * (int)(i - (long)m * n4);
+    const float4 *p = part + i;
+    float4 s = p[0];
 #pragma unroll 4
-      for (int z = 1; z < d.split_k; ++z) {
-        const float4 v = p[z * zstride4];
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    for (int z = 1; z < d.split_k; ++z) {
+      const float4 v = p[z * total4];
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    const Epi &e = d.epi;
+    if (vec_out && e.kind == EPI_F32_STORE) {
+      *reinterpret_cast<float4 *>(e.outf + (long)m * e.ldf + n) = s;
+    } else if (vec_out && e.kind == EPI_F32_ACCUM) {
+      float4 *o = reinterpret_cast<float4 *>(e.outf + (long)m * e.ldf + n);
+      float4 t = *o;
+      t.x += s.x; t.y += s.y; t.z += s.z; t.w += s.w;
+      *o = t;
+    } else if (vec_out && e.kind == EPI_STORE) {
+      T *o = (T *)e.out + (long)m * e.ldo + n;
+      if (sizeof(T) == 2) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(s.x, s.y), hi = __floats2bfloat162_rn(s.z, s.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t *>(&lo);
+        u.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(o) = u;
+      } else {
+        *reinterpret_cast<float4 *>(o) = s;
       }
-      const int n = 4 * c;
-      epi_elem<T>(d.epi, m, n, s.x);
-      epi_elem<T>(d.epi, m, n + 1, s.y);
-      epi_elem<T>(d.epi, m, n + 2, s.z);
-      epi_elem<T>(d.epi, m, n + 3, s.w);
+    } else {
+      epi_elem<T>(e, m, n, s.x);
+      epi_elem<T>(e, m, n + 1, s.y);
+      epi_elem<T>(e, m, n + 2, s.z);
+      epi_elem<T>(e, m, n + 3, s.w);
     }
   }
 }
@@ -149,8 +171,16 @@ cudaError_t launch_gemm_simt(const GemmDesc &d, cudaStream_t st) {
 template <typename T>
 cudaError_t launch_splitk_reduce(const GemmDesc &d, cudaStream_t st) {
   if ((d.N & 3) == 0 && ((uintptr_t)d.partial & 15) == 0) {
-    const int blocks = d.M < 148 * 8 ? d.M : 148 * 8;
-    splitk_reduce4_kernel<T><<<blocks, 256, 0, st>>>(d);
+    const Epi &e = d.epi;
+    int vec = 0;
+    if (e.kind == EPI_F32_STORE || e.kind == EPI_F32_ACCUM)
+      vec = (e.ldf & 3) == 0 && ((uintptr_t)e.outf & 15) == 0;
+    else if (e.kind == EPI_STORE)
+      vec = (e.ldo & 3) == 0 && ((uintptr_t)e.out & (4 * sizeof(T) - 1)) == 0;
+    const long total4 = (long)d.M * (d.N >> 2);
+    long blocks = (total4 + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    splitk_reduce4_kernel<T><<<(int)blocks, 256, 0, st>>>(d, vec);
     return cudaGetLastError();
   }
   long total = (long)d.M * d.N;

@@ -37,6 +37,8 @@ GEMMS = {
     # the lm_head backward's two products on one 8192-row chunk (dS is A in both)
     "gemm_lmhead_dx": (8192, C, 50304, 1, 0, "store", 0),
     "gemm_lmhead_dwte": (50304, C, 8192, 0, 0, "f32_store", 1),
+    # the second chunk's dwte, accumulated into the fp32 gradient
+    "gemm_lmhead_dwte_acc": (50304, C, 8192, 0, 0, "f32_accum", 1),
 }
 # launches of each shape in one 124M step (the lm_head forward statistics and dS recompute
 # run the gemm_lmhead shape with cross-entropy epilogues: two of them per chunk pair)
