@@ -92,6 +92,20 @@ __device__ __forceinline__ void mma_pv_ts(uint32_t d, uint32_t a_tmem, uint32_t 
                  (accumulate || k > 0) ? 1u : 0u);
 }
 
+// The same product over keys [64 half, 64 half + 64) only: P's TMEM columns and V's rows of
+// that half.
+__device__ __forceinline__ void mma_pv_ts_half(uint32_t d, uint32_t a_tmem, uint32_t sV, int half,
+                                               bool accumulate) {
+  const uint32_t id = idesc_bf16(HD, 0, 1);
+  const uint64_t b0 = sdesc(sV, 8192, 1024);
+#pragma unroll
+  for (int kk = 0; kk < TILE / 32; ++kk) {
+    const int k = half * (TILE / 32) + kk;
+    umma_bf16_ts(d, a_tmem + 8 * k, b0 + (uint64_t)((k * 2048) >> 4), id,
+                 (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
 // Packs 32 fp32 values into 16 bf16 pairs and stores them to 16 TMEM columns.
 __device__ __forceinline__ void st_tmem_bf16x32(uint32_t taddr, const uint32_t (&pk)[16]) {
   tmem_st16_nw(taddr, pk);
@@ -168,7 +182,7 @@ struct KCursor {  // (item, query tile) walk of this CTA
 // stage after its P.V MMA); the softmax warps release S as soon as it is in registers, so the
 // next tile's S = Q K^T runs on the tensor core while they compute P.
 enum { F_QFULL, F_K0, F_K1, F_V0, F_V1, F_KFREE0, F_KFREE1, F_VFREE0, F_VFREE1, F_SFULL, F_SFREE,
-       F_PFULL, F_OFULL, F_NBAR };
+       F_PFULL_A, F_PFULL_B, F_OFULL_A, F_OFULL_B, F_NBAR };
 constexpr int FWD_SMEM = 5 * TILE_BYTES + 1024 + 256;
 
 __global__ void __launch_bounds__(192, 2)
@@ -191,7 +205,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   const int n = kt1 - kt0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < F_NBAR; ++i) mbar_init(&bar[i], (i == F_PFULL || i == F_SFREE) ? 4 : 1);
+    for (int i = 0; i < F_NBAR; ++i)
+      mbar_init(&bar[i], (i == F_PFULL_A || i == F_PFULL_B || i == F_SFREE) ? 4 : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -233,11 +248,16 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         if (!mbar_wait(&bar[F_SFREE], j & 1, abort_flag, P.err)) break;  // S_j is in registers
         tc_fence_after();
         if (j + 1 < n && !issue_s(j + 1)) break;
-        if (!mbar_wait(&bar[F_PFULL], j & 1, abort_flag, P.err)) break;
+        // O += P V in two halves of 64 keys, each as soon as its half of P is in TMEM
+        if (!mbar_wait(&bar[F_PFULL_A], j & 1, abort_flag, P.err)) break;
         if (!mbar_wait(&bar[F_V0 + (j & 1)], (j >> 1) & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        mma_pv_ts(tmem + 128, tmem + 192, aV0 + (j & 1) * TILE_BYTES, j > 0);
-        umma_commit(&bar[F_OFULL]);
+        mma_pv_ts_half(tmem + 128, tmem + 192, aV0 + (j & 1) * TILE_BYTES, 0, j > 0);
+        umma_commit(&bar[F_OFULL_A]);
+        if (!mbar_wait(&bar[F_PFULL_B], j & 1, abort_flag, P.err)) break;
+        tc_fence_after();
+        mma_pv_ts_half(tmem + 128, tmem + 192, aV0 + (j & 1) * TILE_BYTES, 1, true);
+        umma_commit(&bar[F_OFULL_B]);
         umma_commit(&bar[F_VFREE0 + (j & 1)]);  // V_j is no longer read
       }
     }
@@ -247,96 +267,107 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     const uint32_t tS = tmem + ((uint32_t)(q * 32) << 16), tO = tS + 128, tP = tS + 192;
     float m2 = -INFINITY, l = 0.f;
     bool have = false, ok = true;
+    // Each 128-key tile in two halves of 64 keys, each an online-softmax step of its own (a
+    // thread holds 64 scores at a time): its P goes to TMEM and its half of O += P V is
+    // issued while the next half is computed. S is released once both halves are loaded.
     for (int j = 0; j < n; ++j) {
       const int k0 = (kt0 + j) * TILE;
       if (!warp_wait(&bar[F_SFULL], j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
-      // the whole 128-key score row of this thread, one wait for the four loads
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32_nw(tS, s0);
-      tmem_ld32_nw(tS + 32, s1);
-      tmem_ld32_nw(tS + 64, s2);
-      tmem_ld32_nw(tS + 96, s3);
-      tmem_wait_ld32(s0);
-      reg_fence32(s1);
-      reg_fence32(s2);
-      reg_fence32(s3);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
-      float sv[128];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        sv[i] = __uint_as_float(s0[i]);
-        sv[32 + i] = __uint_as_float(s1[i]);
-        sv[64 + i] = __uint_as_float(s2[i]);
-        sv[96 + i] = __uint_as_float(s3[i]);
-      }
       const bool interior = (k0 + TILE - 1 <= q0) && (w < 0 || k0 >= q0 + TILE - 1 - w);
-      if (!interior) {
-        // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= i <= hi
-        const int hi = qi - k0;
-        const int lo = w >= 0 ? qi - w - k0 : -1;
-#pragma unroll
-        for (int i = 0; i < 128; ++i) sv[i] = (i <= hi && i >= lo) ? sv[i] : -INFINITY;
-      }
-      // row max as a tree of independent partial maxima (a 128-long dependent chain of
-      // fmaxf would dominate the row's latency)
-      float mp[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = sv[k];
-#pragma unroll
-      for (int i = 8; i < 128; i += 8)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mp[k] = fmaxf(mp[k], sv[i + k]);
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
-      float mnew = m2;
-      bool resc = false;
-      if (mt > -INFINITY) {
-        if (!have) mnew = mt;
-        else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
-      }
-      const bool have_new = have || mt > -INFINITY;
-      const float mu = have_new ? mnew : 0.f;  // rows with nothing admitted yet: every sv is -inf
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (no long FADD chain)
-      uint32_t pk[4][16];  // P of the row, packed bf16 pairs, by 32-column chunk
-#pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        const float p0 = ex2(fmaf(sv[i], P.scale_log2, -mu));
-        const float p1 = ex2(fmaf(sv[i + 1], P.scale_log2, -mu));
-        ls[(i >> 1) & 3] += p0 + p1;
-        pk[i >> 5][(i >> 1) & 15] = pack_bf16(p0, p1);
-      }
-      if (j > 0) {
-        if (!warp_wait(&bar[F_OFULL], (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        const float f = resc ? ex2(m2 - mnew) : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          tmem_ld32(tO + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= f;
-          tmem_st32(tO + c * 32, v);
+      // keys admitted for query qi: max(0, qi-w) <= key <= qi  ->  lo <= i <= hi (tile-local)
+      const int hi = qi - k0;
+      const int lo = w >= 0 ? qi - w - k0 : -1;
+      auto half_step = [&](auto half_c) -> bool {
+        constexpr int HF = decltype(half_c)::value;
+        uint32_t s0[32], s1[32];
+        tmem_ld32_nw(tS + 64 * HF, s0);
+        tmem_ld32_nw(tS + 64 * HF + 32, s1);
+        tmem_wait_ld32(s0);
+        reg_fence32(s1);
+        if (HF == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[F_SFREE]);  // the MMA warp may overwrite S now
         }
-        l *= f;
-      }
-      m2 = mnew;
-      have = have_new;
+        float sv[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        st_tmem_bf16x32(tP + c * 16, pk[c]);
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[F_PFULL]);
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = __uint_as_float(s0[i]);
+          sv[32 + i] = __uint_as_float(s1[i]);
+        }
+        if (!interior) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            sv[i] = (64 * HF + i <= hi && 64 * HF + i >= lo) ? sv[i] : -INFINITY;
+        }
+        // row max as a tree of independent partial maxima
+        float mp[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = sv[k];
+#pragma unroll
+        for (int i = 8; i < 64; i += 8)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mp[k] = fmaxf(mp[k], sv[i + k]);
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
+        float mnew = m2;
+        bool resc = false;
+        if (mt > -INFINITY) {
+          if (!have) mnew = mt;
+          else if (mt > m2 + 8.f) { mnew = mt; resc = true; }
+        }
+        const bool have_new = have || mt > -INFINITY;
+        const float mu = have_new ? mnew : 0.f;  // nothing admitted yet: every sv is -inf
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};      // independent partial sums
+        uint32_t pk[2][16];                       // P of the half, packed bf16 pairs
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          const float p0 = ex2(fmaf(sv[i], P.scale_log2, -mu));
+          const float p1 = ex2(fmaf(sv[i + 1], P.scale_log2, -mu));
+          ls[(i >> 1) & 3] += p0 + p1;
+          pk[i >> 5][(i >> 1) & 15] = pack_bf16(p0, p1);
+        }
+        const bool any_resc = __any_sync(0xffffffffu, resc);
+        if (HF == 0) {
+          // this half's P columns and O are free once the previous tile's P V is done
+          if (j > 0) {
+            if (!warp_wait(&bar[F_OFULL_B], (j - 1) & 1, abort_flag, P.err)) return false;
+            tc_fence_after();
+          }
+        } else if (any_resc) {
+          // O is rescaled below: the first half's P V of this tile must be done
+          if (!warp_wait(&bar[F_OFULL_A], j & 1, abort_flag, P.err)) return false;
+          tc_fence_after();
+        }
+        if (any_resc) {
+          const float f = resc ? ex2(m2 - mnew) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            float v[32];
+            tmem_ld32(tO + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= f;
+            tmem_st32(tO + c * 32, v);
+          }
+          l *= f;
+        }
+        m2 = mnew;
+        have = have_new;
+        st_tmem_bf16x32(tP + 32 * HF, pk[0]);
+        st_tmem_bf16x32(tP + 32 * HF + 16, pk[1]);
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[HF == 0 ? F_PFULL_A : F_PFULL_B]);
+        return true;
+      };
+      if (!half_step(std::integral_constant<int, 0>{})) { ok = false; break; }
+      if (!half_step(std::integral_constant<int, 1>{})) { ok = false; break; }
     }
-    if (ok && warp_wait(&bar[F_OFULL], (n - 1) & 1, abort_flag, P.err)) {
+    if (ok && warp_wait(&bar[F_OFULL_B], (n - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint32_t pk[32];
