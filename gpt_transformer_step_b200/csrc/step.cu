@@ -87,6 +87,12 @@ struct gpt_handle {
   double *gn_partials;
   float *splitk;
   size_t splitk_elems;
+  // The weight-gradient GEMMs of the backward run on a second stream beside the chain of
+  // data-gradient kernels (they fill its GEMM wave tails and memory-bound stretches), with
+  // their own split-K scratch; events order them against the buffers they share.
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_wmp, ev_wfc, ev_wap, ev_wqkv, ev_side_done;
+  float *splitk2;
   void *emb_ws;  // embedding backward: sort buffers, digit histogram, window partials
   bf16 *shadow;
   // state
@@ -180,8 +186,15 @@ int choose_split(const gpt_handle *h, int M, int N, int K, int tm, int tn) {
   return s;
 }
 
-cudaError_t gemm(gpt_handle *h, GemmDesc d) {
+// on_side: launch on the weight-gradient stream (only when side_ok: not while timing kernels,
+// which needs every launch on the main stream)
+bool side_ok(const gpt_handle *h) { return h->side != nullptr && !h->time_kernels; }
+
+cudaError_t gemm(gpt_handle *h, GemmDesc d, bool on_side = false) {
   if (d.M <= 0 || d.N <= 0) return cudaSuccess;
+  on_side = on_side && side_ok(h);
+  cudaStream_t gst = on_side ? h->side : h->stream;
+  float *scratch = on_side ? h->splitk2 : h->splitk;
   d.epi.sc = h->sc;  // device error word and 1/M for every epilogue
   const double flops = 2.0 * d.M * d.N * d.K;
   const int k = tbegin(h, d.epi.kind == EPI_CE_DS ? GPT_KSTAT_GEMM_RECOMPUTE : GPT_KSTAT_GEMM,
@@ -196,8 +209,8 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
       h->ce_ntiles = d.epi.ntiles;
     }
     if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 64, 64) : 1;
-    d.partial = h->splitk;
-    e = launch_gemm_simt<float>(d, h->stream);
+    d.partial = scratch;
+    e = launch_gemm_simt<float>(d, gst);
   } else if (h->tc && tc_gemm_supported(d)) {
     if (d.epi.kind == EPI_CE_STATS) {
       d.epi.tile_n = TC_CE_TILE;
@@ -205,8 +218,8 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
       h->ce_ntiles = d.epi.ntiles;
     }
     // the launcher picks the CTA group and, for elementwise epilogues, the K split
-    d.partial = h->splitk;
-    e = tc_gemm_launch(h->tc, d, h->stream, &h->launches);
+    d.partial = scratch;
+    e = tc_gemm_launch(h->tc, d, gst, &h->launches);
   } else {
     if (d.epi.kind == EPI_CE_STATS) {
       d.epi.tile_n = SIMT_TILE_N;
@@ -214,8 +227,8 @@ cudaError_t gemm(gpt_handle *h, GemmDesc d) {
       h->ce_ntiles = d.epi.ntiles;
     }
     if (d.split_k == 0) d.split_k = f32out ? choose_split(h, d.M, d.N, d.K, 64, 64) : 1;
-    d.partial = h->splitk;
-    e = launch_gemm_simt<bf16>(d, h->stream);
+    d.partial = scratch;
+    e = launch_gemm_simt<bf16>(d, gst);
   }
   h->launches += 1 + (d.split_k > 1 ? 1 : 0);
   if (e != cudaSuccess) return e;
@@ -378,47 +391,78 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes - (double)M * C * es,
         launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf, dx,
                                 h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
+  // The weight gradients go to the side stream (see gpt_handle::side). fork: the side stream
+  // waits for all the main stream has issued; mark / join: an event after side work, and the
+  // main stream waiting for it before it rewrites a buffer that work reads.
+  const bool sd = side_ok(h);
+  auto fork = [&]() -> cudaError_t {
+    if (!sd) return cudaSuccess;
+    CUDA_TRY(cudaEventRecord(h->ev_fork, st));
+    return cudaStreamWaitEvent(h->side, h->ev_fork, 0);
+  };
+  auto mark = [&](cudaEvent_t ev) { return sd ? cudaEventRecord(ev, h->side) : cudaSuccess; };
+  auto join = [&](cudaEvent_t ev) { return sd ? cudaStreamWaitEvent(st, ev, 0) : cudaSuccess; };
+  bool have_wfc = false, have_wqkv = false;
   for (int l = h->L - 1; l >= 0; --l) {
     Acts &A = h->acts[l];
     const Layer &P = h->layer[l];
     // MLP: x_out = x_mid + gelu(c Wfc^T) Wmp^T
+    if (have_wfc) CUDA_TRY(join(h->ev_wfc));  // dh is rewritten: the last dWfc has read it
     GemmDesc d = gdesc(M, mC, C, dx, C, 1, W + P.wmp, mC, 0);
     d.epi.kind = EPI_DGELU; d.epi.out = h->dh; d.epi.ldo = mC; d.epi.aux = A.dgelu; d.epi.ld_aux = mC;
     if (h->cfg.recompute_gelu) {  // dh = dy * gelu'(pre), and gelu(pre) again for dWmp
       d.epi.kind = EPI_DGELU_RECOMP; d.epi.out2 = A.h; d.epi.ldo2 = mC;
     }
     CUDA_TRY(gemm(h, d));
+    CUDA_TRY(fork());
     d = gdesc(C, mC, M, dx, C, 0, A.h, mC, 0);
     d.epi.kind = wgrad; d.epi.outf = G + P.wmp; d.epi.ldf = mC;
-    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(gemm(h, d, true));
+    CUDA_TRY(mark(h->ev_wmp));
+    d = gdesc(mC, C, M, h->dh, mC, 0, A.c, C, 0);
+    d.epi.kind = wgrad; d.epi.outf = G + P.wfc; d.epi.ldf = C;
+    CUDA_TRY(gemm(h, d, true));
+    CUDA_TRY(mark(h->ev_wfc));
+    have_wfc = true;
     d = gdesc(M, C, mC, h->dh, mC, 1, W + P.wfc, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
-    d = gdesc(mC, C, M, h->dh, mC, 0, A.c, C, 0);
-    d.epi.kind = wgrad; d.epi.outf = G + P.wfc; d.epi.ldf = C;
-    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(join(h->ev_wmp));  // dx is rewritten: dWmp has read it
     TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
           launch_layernorm_bwd<T>((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx,
                                   h->dg_partial, G + P.ln2, M, C, st, acc)); nl += 2;
     // attention: x_mid = x_in + attn(a) Wap^T
+    CUDA_TRY(fork());
+    d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
+    d.epi.kind = wgrad; d.epi.outf = G + P.wap; d.epi.ldf = C;
+    CUDA_TRY(gemm(h, d, true));
+    CUDA_TRY(mark(h->ev_wap));
     d = gdesc(M, C, C, dx, C, 1, W + P.wap, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dout; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
-    d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
-    d.epi.kind = wgrad; d.epi.outf = G + P.wap; d.epi.ldf = C;
-    CUDA_TRY(gemm(h, d));
+    if (have_wqkv) CUDA_TRY(join(h->ev_wqkv));  // dqkv is rewritten: the last dWqkv has read it
     TIMED(h, GPT_KSTAT_ATTN_BWD, attn_flops(h->windows[l], 8.0),
           attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B, Tlen,
                            h->windows[l])); nl += (h->use_bf16 && attn_dst(h, Tlen)) ? 3 : 2;
+    CUDA_TRY(fork());
+    d = gdesc(3 * C, C, M, h->dqkv, 3 * C, 0, A.a, C, 0);
+    d.epi.kind = wgrad; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
+    CUDA_TRY(gemm(h, d, true));
+    CUDA_TRY(mark(h->ev_wqkv));
+    have_wqkv = true;
     d = gdesc(M, C, 3 * C, h->dqkv, 3 * C, 1, W + P.wqkv, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dc; d.epi.ldo = C;
     CUDA_TRY(gemm(h, d));
-    d = gdesc(3 * C, C, M, h->dqkv, 3 * C, 0, A.a, C, 0);
-    d.epi.kind = wgrad; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
-    CUDA_TRY(gemm(h, d));
+    CUDA_TRY(join(h->ev_wap));  // dx is rewritten: dWap has read it
     TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
           launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
                                   h->dg_partial, G + P.ln1, M, C, st, acc)); nl += 2;
+  }
+  // every weight gradient is complete before anything reads the gradients, or the next phase
+  // rewrites the activations the side stream reads (and a captured graph rejoins here)
+  if (sd) {
+    CUDA_TRY(mark(h->ev_side_done));
+    CUDA_TRY(join(h->ev_side_done));
   }
   EmbedBwdWs ew{h->emb_ws};
   TIMED(h, GPT_KSTAT_EMBED_BWD, (double)M * C * es + 4.0 * C * h->maxT * (acc ? 2 : 1) + 8.0 * M,
@@ -662,6 +706,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   need((void **)&h->dg_partial, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
   need((void **)&h->gn_partials, (size_t)grad_norm_blocks() * 8);
   need((void **)&h->splitk, h->splitk_elems * 4);
+  need((void **)&h->splitk2, h->splitk_elems * 4);
   need(&h->emb_ws, embed_bwd_ws_bytes((int)M, C));
   need((void **)&h->tok, M * 4); need((void **)&h->tgt, M * 4);
   need((void **)&h->sc, sizeof(DevScalars));
@@ -700,6 +745,22 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
       tc_gemm_set_splitk_capacity(h->tc, h->splitk_elems);
     }
   }
+  // the weight-gradient stream and its events; without them everything runs on one stream
+  h->side = nullptr;
+  if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess) {
+    cudaEvent_t *evs[6] = {&h->ev_fork, &h->ev_wmp, &h->ev_wfc, &h->ev_wap, &h->ev_wqkv,
+                           &h->ev_side_done};
+    bool ok = true;
+    for (auto *ev : evs) ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      cudaStreamDestroy(h->side);
+      h->side = nullptr;
+    }
+  } else {
+    cudaGetLastError();
+    h->side = nullptr;
+  }
   *status = GPT_OK;
   return h;
 }
@@ -709,6 +770,11 @@ void gpt_destroy(gpt_handle *h) {
   cudaSetDevice(h->device);
   for (auto &kv : h->graphs) cudaGraphExecDestroy(kv.second.exec);
   for (auto ev : h->ev) cudaEventDestroy(ev);
+  if (h->side) {
+    for (auto ev : {h->ev_fork, h->ev_wmp, h->ev_wfc, h->ev_wap, h->ev_wqkv, h->ev_side_done})
+      cudaEventDestroy(ev);
+    cudaStreamDestroy(h->side);
+  }
   if (h->tc) tc_gemm_destroy(h->tc);
   if (h->muon_ws) cudaFree(h->muon_ws);
   cudaFree(h->ws);
