@@ -91,7 +91,7 @@ struct gpt_handle {
   // data-gradient kernels (they fill its GEMM wave tails and memory-bound stretches), with
   // their own split-K scratch; events order them against the buffers they share.
   cudaStream_t side;
-  cudaEvent_t ev_fork, ev_wmp, ev_wfc, ev_wap, ev_wqkv, ev_side_done;
+  cudaEvent_t ev_fork, ev_wmp, ev_wfc, ev_wap, ev_wqkv, ev_wte, ev_side_done;
   float *splitk2;
   void *emb_ws;  // embedding backward: sort buffers, digit histogram, window partials
   bf16 *shadow;
@@ -368,32 +368,10 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   // backward add; the padding rows V..Vp-1 are never written by the GEMMs and are zeroed
   if (!acc && h->Vp > V)
     CUDA_TRY(cudaMemsetAsync(G + h->off_wte + (size_t)V * C, 0, sizeof(float) * (size_t)(h->Vp - V) * C, st));
-  for (int r0 = 0; r0 < M; r0 += h->chunk_rows) {
-    const int R = M - r0 < h->chunk_rows ? M - r0 : h->chunk_rows;
-    const T *yf_c = (const T *)h->yf + (size_t)r0 * C;
-    GemmDesc d = gdesc(R, V, C, yf_c, C, 1, W + h->off_wte, C, 1);
-    d.split_k = 1;
-    Epi &e = d.epi;
-    e.kind = EPI_CE_DS; e.out = h->dS; e.ldo = h->ldS; e.targets = h->tgt; e.lse = h->lse_ce;
-    e.V = V; e.row_offset = r0; e.sc = sc;
-    CUDA_TRY(gemm(h, d));
-    // dyf = dS . wte
-    d = gdesc(R, C, V, h->dS, h->ldS, 1, W + h->off_wte, C, 0);
-    d.epi.kind = EPI_STORE; d.epi.out = (T *)h->dyf + (size_t)r0 * C; d.epi.ldo = C;
-    CUDA_TRY(gemm(h, d));
-    // dwte (+)= dS^T . yf
-    d = gdesc(V, C, R, h->dS, h->ldS, 0, yf_c, C, 0);
-    d.epi.kind = (acc || r0 > 0) ? EPI_F32_ACCUM : EPI_F32_STORE; d.epi.outf = G + h->off_wte; d.epi.ldf = C;
-    d.split_k = 1;
-    CUDA_TRY(gemm(h, d));
-  }
-  T *dx = (T *)h->dx;  // the residual-stream gradient starts here (nothing to add to)
-  TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes - (double)M * C * es,
-        launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf, dx,
-                                h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
-  // The weight gradients go to the side stream (see gpt_handle::side). fork: the side stream
-  // waits for all the main stream has issued; mark / join: an event after side work, and the
-  // main stream waiting for it before it rewrites a buffer that work reads.
+  // The weight gradients (dwte here, the layers' weights below) go to the side stream (see
+  // gpt_handle::side). fork: the side stream waits for all the main stream has issued; mark /
+  // join: an event after side work, and the main stream waiting for it before it rewrites a
+  // buffer that work reads.
   const bool sd = side_ok(h);
   auto fork = [&]() -> cudaError_t {
     if (!sd) return cudaSuccess;
@@ -402,6 +380,35 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   };
   auto mark = [&](cudaEvent_t ev) { return sd ? cudaEventRecord(ev, h->side) : cudaSuccess; };
   auto join = [&](cudaEvent_t ev) { return sd ? cudaStreamWaitEvent(st, ev, 0) : cudaSuccess; };
+  bool have_wte = false;
+  for (int r0 = 0; r0 < M; r0 += h->chunk_rows) {
+    const int R = M - r0 < h->chunk_rows ? M - r0 : h->chunk_rows;
+    const T *yf_c = (const T *)h->yf + (size_t)r0 * C;
+    GemmDesc d = gdesc(R, V, C, yf_c, C, 1, W + h->off_wte, C, 1);
+    d.split_k = 1;
+    Epi &e = d.epi;
+    e.kind = EPI_CE_DS; e.out = h->dS; e.ldo = h->ldS; e.targets = h->tgt; e.lse = h->lse_ce;
+    e.V = V; e.row_offset = r0; e.sc = sc;
+    if (have_wte) CUDA_TRY(join(h->ev_wte));  // dS is rewritten: the last dwte has read it
+    CUDA_TRY(gemm(h, d));
+    // dwte (+)= dS^T . yf, on the side stream beside dyf
+    CUDA_TRY(fork());
+    GemmDesc dw = gdesc(V, C, R, h->dS, h->ldS, 0, yf_c, C, 0);
+    dw.epi.kind = (acc || r0 > 0) ? EPI_F32_ACCUM : EPI_F32_STORE; dw.epi.outf = G + h->off_wte;
+    dw.epi.ldf = C;
+    dw.split_k = 1;
+    CUDA_TRY(gemm(h, dw, true));
+    CUDA_TRY(mark(h->ev_wte));
+    have_wte = true;
+    // dyf = dS . wte
+    d = gdesc(R, C, V, h->dS, h->ldS, 1, W + h->off_wte, C, 0);
+    d.epi.kind = EPI_STORE; d.epi.out = (T *)h->dyf + (size_t)r0 * C; d.epi.ldo = C;
+    CUDA_TRY(gemm(h, d));
+  }
+  T *dx = (T *)h->dx;  // the residual-stream gradient starts here (nothing to add to)
+  TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes - (double)M * C * es,
+        launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf, dx,
+                                h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
   bool have_wfc = false, have_wqkv = false;
   for (int l = h->L - 1; l >= 0; --l) {
     Acts &A = h->acts[l];
@@ -748,8 +755,8 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   // the weight-gradient stream and its events; without them everything runs on one stream
   h->side = nullptr;
   if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess) {
-    cudaEvent_t *evs[6] = {&h->ev_fork, &h->ev_wmp, &h->ev_wfc, &h->ev_wap, &h->ev_wqkv,
-                           &h->ev_side_done};
+    cudaEvent_t *evs[7] = {&h->ev_fork, &h->ev_wmp, &h->ev_wfc, &h->ev_wap, &h->ev_wqkv,
+                           &h->ev_wte, &h->ev_side_done};
     bool ok = true;
     for (auto *ev : evs) ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
     if (!ok) {
@@ -771,7 +778,8 @@ void gpt_destroy(gpt_handle *h) {
   for (auto &kv : h->graphs) cudaGraphExecDestroy(kv.second.exec);
   for (auto ev : h->ev) cudaEventDestroy(ev);
   if (h->side) {
-    for (auto ev : {h->ev_fork, h->ev_wmp, h->ev_wfc, h->ev_wap, h->ev_wqkv, h->ev_side_done})
+    for (auto ev : {h->ev_fork, h->ev_wmp, h->ev_wfc, h->ev_wap, h->ev_wqkv, h->ev_wte,
+                    h->ev_side_done})
       cudaEventDestroy(ev);
     cudaStreamDestroy(h->side);
   }
