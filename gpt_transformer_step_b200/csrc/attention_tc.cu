@@ -60,6 +60,29 @@ __device__ __forceinline__ float ldg_early(const float *p) {
   return v;
 }
 
+// Packed two-lane fp32 arithmetic (sm_100): one instruction for two independent elements.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // One warp-collective bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           unsigned *err) {
@@ -306,9 +329,11 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
 #pragma unroll
         for (int k = 0; k < 8; ++k) mp[k] = sv[k];
 #pragma unroll
-        for (int i = 8; i < 64; i += 8)
+        for (int i = 8; i < 56; i += 16)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mp[k] = fmaxf(mp[k], sv[i + k]);
+          for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], sv[i + k], sv[i + 8 + k]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = fmaxf(mp[k], sv[56 + k]);
         const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                                fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         const float mt = mx * P.scale_log2;  // -inf stays -inf (scale > 0)
@@ -320,15 +345,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         }
         const bool have_new = have || mt > -INFINITY;
         const float mu = have_new ? mnew : 0.f;  // nothing admitted yet: every sv is -inf
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};      // independent partial sums
+        float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // partial sums
         uint32_t pk[2][16];                       // P of the half, packed bf16 pairs
+        const float2 sc2 = make_float2(P.scale_log2, P.scale_log2), nmu2 = make_float2(-mu, -mu);
 #pragma unroll
         for (int i = 0; i < 64; i += 2) {
-          const float p0 = ex2(fmaf(sv[i], P.scale_log2, -mu));
-          const float p1 = ex2(fmaf(sv[i + 1], P.scale_log2, -mu));
-          ls[(i >> 1) & 3] += p0 + p1;
+          const float2 a2 = fma2(make_float2(sv[i], sv[i + 1]), sc2, nmu2);
+          const float p0 = ex2(a2.x), p1 = ex2(a2.y);
+          ls2[(i >> 1) & 1] = add2(ls2[(i >> 1) & 1], make_float2(p0, p1));
           pk[i >> 5][(i >> 1) & 15] = pack_bf16(p0, p1);
         }
+        const float ls[4] = {ls2[0].x, ls2[1].x, ls2[0].y, ls2[1].y};
         const bool any_resc = __any_sync(0xffffffffu, resc);
         if (HF == 0) {
           // this half's P columns and O are free once the previous tile's P V is done
