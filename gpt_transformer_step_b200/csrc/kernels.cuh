@@ -33,7 +33,10 @@ template <typename T>
 cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
                                  const T *dy, T *dres, float *dg_partial, float *dg, int M,
                                  int C, cudaStream_t st, bool accumulate = false,
-                                 bool dres_in = true);
+                                 bool dres_in = true, bool colsum = true);
+// dgamma from the per-block partials of launch_layernorm_bwd(..., colsum = false), in block order
+cudaError_t launch_ln_colsum(const float *dg_partial, int M, int C, float *dg, bool accumulate,
+                             cudaStream_t st);
 int layernorm_bwd_blocks(int M);
 
 // Cross-entropy: per-row lse and loss from the per-tile stats; mean loss into sc->loss.

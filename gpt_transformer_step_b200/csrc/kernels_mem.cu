@@ -856,7 +856,8 @@ int layernorm_bwd_blocks(int M) {
 template <typename T>
 cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, const float *rstd,
                                  const T *dy, T *dres, float *dg_partial, float *dg, int M,
-                                 int C, cudaStream_t st, bool accumulate, bool dres_in) {
+                                 int C, cudaStream_t st, bool accumulate, bool dres_in,
+                                 bool colsum) {
   const int nb = layernorm_bwd_blocks(M);
   const int rpb = (M + nb - 1) / nb;
   const size_t smem = (size_t)LNB_WARPS * C * sizeof(float);
@@ -867,7 +868,15 @@ cudaError_t launch_layernorm_bwd(const T *x, const T *g, const float *mean, cons
   LN_DISPATCH(ln_nv<T>(C), LNB)
 #undef LNB
   CUDA_TRY(cudaGetLastError());
+  if (!colsum) return cudaSuccess;
   colsum_kernel<<<(C + 31) / 32, 1024, 0, st>>>(dg_partial, nb, C, dg, accumulate ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_colsum(const float *dg_partial, int M, int C, float *dg, bool accumulate,
+                             cudaStream_t st) {
+  colsum_kernel<<<(C + 31) / 32, 1024, 0, st>>>(dg_partial, layernorm_bwd_blocks(M), C, dg,
+                                                accumulate ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -925,6 +934,6 @@ cudaError_t launch_to_bf16(const float *p, bf16 *out, size_t n, cudaStream_t st)
                                                int, float, cudaStream_t);                      \
   template cudaError_t launch_layernorm_bwd<T>(const T *, const T *, const float *,             \
                                                const float *, const T *, T *, float *, float *, \
-                                               int, int, cudaStream_t, bool, bool);
+                                               int, int, cudaStream_t, bool, bool, bool);
 INST(float)
 INST(bf16)

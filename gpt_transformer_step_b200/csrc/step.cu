@@ -91,8 +91,9 @@ struct gpt_handle {
   // data-gradient kernels (they fill its GEMM wave tails and memory-bound stretches), with
   // their own split-K scratch; events order them against the buffers they share.
   cudaStream_t side;
-  cudaEvent_t ev_fork, ev_wmp, ev_wfc, ev_wap, ev_wqkv, ev_wte, ev_side_done;
+  cudaEvent_t ev_fork, ev_wmp, ev_wfc, ev_wap, ev_wqkv, ev_wte, ev_side_done, ev_cs[2];
   float *splitk2;
+  float *dg_partial2;  // LayerNorm backward: the dgamma partials alternate between two buffers
   void *emb_ws;  // embedding backward: sort buffers, digit histogram, window partials
   bf16 *shadow;
   // state
@@ -380,6 +381,25 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   };
   auto mark = [&](cudaEvent_t ev) { return sd ? cudaEventRecord(ev, h->side) : cudaSuccess; };
   auto join = [&](cudaEvent_t ev) { return sd ? cudaStreamWaitEvent(st, ev, 0) : cudaSuccess; };
+  // LayerNorm backward; with the side stream its dgamma column sum runs there, reading one of
+  // two partial buffers, which the next-but-one LayerNorm backward reuses after that sum
+  int lnbuf = 0;
+  bool have_cs[2] = {false, false};
+  auto ln_bwd = [&](const T *x, const T *g, const float *mu, const float *rs, const T *dy,
+                    T *dres, float *dgout, bool dres_in) -> cudaError_t {
+    float *part = lnbuf ? h->dg_partial2 : h->dg_partial;
+    if (have_cs[lnbuf]) CUDA_TRY(join(h->ev_cs[lnbuf]));
+    CUDA_TRY(launch_layernorm_bwd<T>(x, g, mu, rs, dy, dres, part, dgout, M, C, st, acc, dres_in,
+                                     !sd));
+    if (sd) {
+      CUDA_TRY(fork());
+      CUDA_TRY(launch_ln_colsum(part, M, C, dgout, acc, h->side));
+      CUDA_TRY(mark(h->ev_cs[lnbuf]));
+      have_cs[lnbuf] = true;
+    }
+    lnbuf ^= 1;
+    return cudaSuccess;
+  };
   bool have_wte = false;
   for (int r0 = 0; r0 < M; r0 += h->chunk_rows) {
     const int R = M - r0 < h->chunk_rows ? M - r0 : h->chunk_rows;
@@ -407,8 +427,8 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
   }
   T *dx = (T *)h->dx;  // the residual-stream gradient starts here (nothing to add to)
   TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes - (double)M * C * es,
-        launch_layernorm_bwd<T>((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf, dx,
-                                h->dg_partial, G + h->off_lnf, M, C, st, acc, false)); nl += 2;
+        ln_bwd((T *)h->x_final, W + h->off_lnf, h->muf, h->rsf, (T *)h->dyf, dx, G + h->off_lnf,
+               false)); nl += 2;
   bool have_wfc = false, have_wqkv = false;
   for (int l = h->L - 1; l >= 0; --l) {
     Acts &A = h->acts[l];
@@ -436,8 +456,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(gemm(h, d));
     CUDA_TRY(join(h->ev_wmp));  // dx is rewritten: dWmp has read it
     TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
-          launch_layernorm_bwd<T>((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx,
-                                  h->dg_partial, G + P.ln2, M, C, st, acc)); nl += 2;
+          ln_bwd((T *)A.x_mid, W + P.ln2, A.mu2, A.rs2, (T *)h->dc, dx, G + P.ln2, true)); nl += 2;
     // attention: x_mid = x_in + attn(a) Wap^T
     CUDA_TRY(fork());
     d = gdesc(C, C, M, dx, C, 0, A.o, C, 0);
@@ -462,8 +481,7 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(gemm(h, d));
     CUDA_TRY(join(h->ev_wap));  // dx is rewritten: dWap has read it
     TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
-          launch_layernorm_bwd<T>((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx,
-                                  h->dg_partial, G + P.ln1, M, C, st, acc)); nl += 2;
+          ln_bwd((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx, G + P.ln1, true)); nl += 2;
   }
   // every weight gradient is complete before anything reads the gradients, or the next phase
   // rewrites the activations the side stream reads (and a captured graph rejoins here)
@@ -711,6 +729,7 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   if (use_dst) need((void **)&h->dst, dst_bytes);
   else h->dst = nullptr;
   need((void **)&h->dg_partial, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
+  need((void **)&h->dg_partial2, (size_t)layernorm_bwd_blocks((int)M) * C * 4);
   need((void **)&h->gn_partials, (size_t)grad_norm_blocks() * 8);
   need((void **)&h->splitk, h->splitk_elems * 4);
   need((void **)&h->splitk2, h->splitk_elems * 4);
@@ -755,8 +774,8 @@ gpt_handle *gpt_create(const gpt_config *cfg, int *status) {
   // the weight-gradient stream and its events; without them everything runs on one stream
   h->side = nullptr;
   if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess) {
-    cudaEvent_t *evs[7] = {&h->ev_fork, &h->ev_wmp, &h->ev_wfc, &h->ev_wap, &h->ev_wqkv,
-                           &h->ev_wte, &h->ev_side_done};
+    cudaEvent_t *evs[9] = {&h->ev_fork, &h->ev_wmp, &h->ev_wfc, &h->ev_wap, &h->ev_wqkv,
+                           &h->ev_wte, &h->ev_side_done, &h->ev_cs[0], &h->ev_cs[1]};
     bool ok = true;
     for (auto *ev : evs) ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
     if (!ok) {
@@ -779,7 +798,7 @@ void gpt_destroy(gpt_handle *h) {
   for (auto ev : h->ev) cudaEventDestroy(ev);
   if (h->side) {
     for (auto ev : {h->ev_fork, h->ev_wmp, h->ev_wfc, h->ev_wap, h->ev_wqkv, h->ev_wte,
-                    h->ev_side_done})
+                    h->ev_side_done, h->ev_cs[0], h->ev_cs[1]})
       cudaEventDestroy(ev);
     cudaStreamDestroy(h->side);
   }
