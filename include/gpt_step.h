@@ -97,7 +97,12 @@ size_t gpt_num_params(const gpt_handle *h);
  * lnf.g [C]. Returns the number of tensors (6*n_layer + 3), or a negative code. */
 int gpt_param_layout(const gpt_handle *h, gpt_tensor_desc *out, int cap);
 
-/* All device work of later calls is enqueued on this cudaStream_t (NULL = legacy default). */
+/* All device work of later calls is ordered on this cudaStream_t (NULL = legacy default).
+ * Inside a training call, the backward's weight-gradient GEMMs and LayerNorm dgamma sums
+ * run on a second stream that the handle owns. That stream forks from this one and joins
+ * back into it, through events, before the call's last kernels. So work the caller enqueues
+ * on this stream after the call sees every result, and a graph captured on this stream
+ * holds both branches. */
 int gpt_set_stream(gpt_handle *h, void *cuda_stream);
 
 /* Forward pass only. params: device fp32 [num_params], read only. tokens, targets: int32
