@@ -483,16 +483,18 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     TIMED(h, GPT_KSTAT_LN_BWD, ln_bwd_bytes,
           ln_bwd((T *)A.x_in, W + P.ln1, A.mu1, A.rs1, (T *)h->dc, dx, G + P.ln1, true)); nl += 2;
   }
+  // the embedding backward adds into the wte gradient after the last dwte
+  if (have_wte) CUDA_TRY(join(h->ev_wte));
+  EmbedBwdWs ew{h->emb_ws};
+  TIMED(h, GPT_KSTAT_EMBED_BWD, (double)M * C * es + 4.0 * C * h->maxT * (acc ? 2 : 1) + 8.0 * M,
+        launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C, h->Vp,
+                            ew, st, acc)); nl += embed_bwd_launches(h->Vp);
   // every weight gradient is complete before anything reads the gradients, or the next phase
   // rewrites the activations the side stream reads (and a captured graph rejoins here)
   if (sd) {
     CUDA_TRY(mark(h->ev_side_done));
     CUDA_TRY(join(h->ev_side_done));
   }
-  EmbedBwdWs ew{h->emb_ws};
-  TIMED(h, GPT_KSTAT_EMBED_BWD, (double)M * C * es + 4.0 * C * h->maxT * (acc ? 2 : 1) + 8.0 * M,
-        launch_embed_bwd<T>(h->tok, dx, G + h->off_wte, G + h->off_wpe, M, Tlen, h->maxT, C, h->Vp,
-                            ew, st, acc)); nl += embed_bwd_launches(h->Vp);
   if (phase == PH_FIRST || phase == PH_MIDDLE) return cudaSuccess;  // update after the last
   // ---------------- clip + AdamW ----------------
   TIMED(h, GPT_KSTAT_GRAD_NORM, 4.0 * h->nparams,
