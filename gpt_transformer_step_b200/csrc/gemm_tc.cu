@@ -8,9 +8,9 @@
 // data-gradient GEMMs of the backward pass need no transposed copies.
 //
 // Structure: persistent CTAs (one per SM), 10 warps.
-//   warp 0      TMA producer: fills a ring of shared-memory stages (A 128x64, B 256x64 or,
-//               for CTA pairs, this CTA's 128x64 half of B)
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K = 16 per stage
+//   warp 0      TMA producer: fills a ring of shared-memory stages (A 128x128, B 256x128 or,
+//               for CTA pairs, this CTA's 128x128 half of B), K as two 64-element chunks
+//   warp 1      TMEM allocator and MMA issuer (one thread): 8 MMAs of K = 16 per stage
 //               (128x256 per CTA, or 256x256 per CTA pair with cta_group::2);
 //               tcgen05.commit frees the stage; a second commit marks the accumulator full
 //   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (one row per thread, two warps
@@ -32,7 +32,9 @@ namespace {
 using namespace tc;
 
 constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int KC = BK / 64;            // 128-byte swizzle chunks per stage along K
+constexpr int A_BYTES = BM * BK * 2;   // 32 KB
+constexpr int A_CHUNK = BM * 64 * 2;   // 16 KB: one chunk of A (K-major: 64 k; MN-major: 64 m)
 constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
@@ -54,6 +56,9 @@ struct TcParams {
   int batch;       // independent products (batched GEMM); units = tiles * splits * batch
   int n_fast;      // 1: units walk the N tiles of one M tile first (see unit_coords)
   int a_mn, b_mn;  // 1 = MN-major
+  // 1: the operand's map views its contiguous dimension as 64-element chunks, so one TMA
+  // load brings a stage's whole operand tile (32 KB per CTA); 0: one load per chunk
+  int a_wide, b_wide;
   uint32_t idesc;
   Epi epi;
   float *partial;
@@ -186,12 +191,15 @@ __device__ __forceinline__ void ce_stats_chunk(const TcParams &P, int row, int c
 template <int CG>
 struct TcCfg {
   static constexpr int B_ROWS = BN / CG;                 // rows of B each CTA loads
-  static constexpr int B_CTA_BYTES = B_ROWS * BK * 2;    // 32 KB / 16 KB
-  static constexpr int STAGE = A_BYTES + B_CTA_BYTES;    // 48 KB / 32 KB
-  // Pairs: six 32 KB stages and 4 KB of epilogue staging per warp (two bf16 chunk slots, or
-  // one for two outputs / fp32) measured faster than five stages with 8 KB: the deeper ring
-  // covers more TMA latency, and the epilogue's smaller slot count costs less than that.
-  static constexpr int NSTAGE = CG == 1 ? 4 : 6;
+  static constexpr int B_CTA_BYTES = B_ROWS * BK * 2;    // 64 KB / 32 KB
+  static constexpr int B_CHUNK = B_ROWS * 64 * 2;        // one 64-element chunk of B
+  static constexpr int STAGE = A_BYTES + B_CTA_BYTES;    // 96 KB / 64 KB
+  // 192 KB of stages in flight, 4 KB of epilogue staging per warp (two bf16 chunk slots, or
+  // one for two outputs / fp32). A stage's operands arrive in one 32 KB TMA load each: a
+  // producer thread's loads complete at a rate set per load more than per byte, so 128-wide
+  // K stages (one load per operand) feed the MMAs faster than 64-wide ones (one 16 KB load
+  // per operand).
+  static constexpr int NSTAGE = CG == 1 ? 2 : 3;
   static constexpr int WARP_STAGE = 4096;  // epilogue staging per warp
   static constexpr int SMEM = NSTAGE * STAGE + EPI_WARPS * WARP_STAGE + 1024 + 256;
   static_assert(SMEM <= 232448, "GEMM shared memory");
@@ -249,6 +257,24 @@ __device__ __forceinline__ void tma_load_pair(void *dst, const CUtensorMap *map,
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+// The same with a 4D map (an operand whose contiguous dimension is viewed as 64-element chunks).
+template <int CG>
+__device__ __forceinline__ void tma_load_pair4(void *dst, const CUtensorMap *map,
+                                               uint32_t mbar_cluster, int c0, int c1, int c2,
+                                               int c3) {
+  if (CG == 2)
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+  else
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
 template <int CG>
@@ -423,19 +449,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t fb = smem_u32(&full_bar[stage]);
           const uint32_t fbl = CG == 2 ? mapa_shared(fb, 0) : fb;  // the leader's barrier
           if (rank == 0) mbar_expect_tx_addr(fb, Cf::STAGE * CG);
+          // smem layout of an operand tile: its 64-element chunks one after the other, each
+          // 128-byte swizzled (K-major: [k chunk][row][64 k]; MN-major: [mn chunk][k][64 mn])
           const int k0 = kb * BK;
-          if (!P.a_mn) {
-            tma_load_pair<CG>(sA, &tmA, fbl, k0, m0, bz);
+          if (P.a_wide) {
+            if (!P.a_mn) tma_load_pair4<CG>(sA, &tmA, fbl, 0, m0, k0 / 64, bz);
+            else tma_load_pair4<CG>(sA, &tmA, fbl, 0, k0, m0 / 64, bz);
           } else {
-            tma_load_pair<CG>(sA, &tmA, fbl, m0, k0, bz);
-            tma_load_pair<CG>(sA + A_BYTES / 2, &tmA, fbl, m0 + 64, k0, bz);
+#pragma unroll
+            for (int j = 0; j < KC; ++j) {
+              if (!P.a_mn) tma_load_pair<CG>(sA + j * A_CHUNK, &tmA, fbl, k0 + 64 * j, m0, bz);
+              else tma_load_pair<CG>(sA + j * A_CHUNK, &tmA, fbl, m0 + 64 * j, k0, bz);
+            }
           }
-          if (!P.b_mn) {
-            tma_load_pair<CG>(sB, &tmB, fbl, k0, n0, bz);
+          if (P.b_wide) {
+            if (!P.b_mn) tma_load_pair4<CG>(sB, &tmB, fbl, 0, n0, k0 / 64, bz);
+            else tma_load_pair4<CG>(sB, &tmB, fbl, 0, k0, n0 / 64, bz);
+          } else if (!P.b_mn) {
+#pragma unroll
+            for (int j = 0; j < KC; ++j)
+              tma_load_pair<CG>(sB + j * Cf::B_CHUNK, &tmB, fbl, k0 + 64 * j, n0, bz);
           } else {
 #pragma unroll
             for (int j = 0; j < Cf::B_ROWS / 64; ++j)
-              tma_load_pair<CG>(sB + j * 8192, &tmB, fbl, n0 + 64 * j, k0, bz);
+              tma_load_pair<CG>(sB + j * (BK * 128), &tmB, fbl, n0 + 64 * j, k0, bz);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -461,10 +498,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t phase = 0;
       bool ok = true;
       int i = 0;
-      const uint32_t a_step = P.a_mn ? 2048u : 32u;
-      const uint32_t b_step = P.b_mn ? 2048u : 32u;
-      const uint32_t a_lbo = P.a_mn ? 8192u : 16u;
-      const uint32_t b_lbo = P.b_mn ? 8192u : 16u;
+      // byte offset of MMA k-step k (16 k) in an operand tile: K-major, chunk k / 4 and 32 B
+      // per step inside it; MN-major, 16 k rows of 128 B per step. MN-major chunks (64 m or n)
+      // are BK rows of 128 B apart (the descriptor's leading byte offset).
+      const uint32_t a_lbo = P.a_mn ? (uint32_t)(BK * 128) : 16u;
+      const uint32_t b_lbo = P.b_mn ? (uint32_t)(BK * 128) : 16u;
       for (int u = unit0; u < P.units && ok; u += ustride, ++i) {
         const int z = (u / (P.num_mt * P.num_nt)) % P.splits;
         const int kb0 = z * P.kblocks_per_split;
@@ -480,10 +518,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t sA = smem_u32(smem + stage * Cf::STAGE);
           const uint64_t ad0 = sdesc(sA, a_lbo, 1024u), bd0 = sdesc(sA + A_BYTES, b_lbo, 1024u);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_issue<CG>(d_tmem, ad0 + (uint64_t)((k * a_step) >> 4),
-                           bd0 + (uint64_t)((k * b_step) >> 4), P.idesc,
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t ao = P.a_mn ? (uint32_t)k * 2048u
+                                       : (uint32_t)(k >> 2) * A_CHUNK + (uint32_t)(k & 3) * 32u;
+            const uint32_t bo = P.b_mn ? (uint32_t)k * 2048u
+                                       : (uint32_t)(k >> 2) * Cf::B_CHUNK + (uint32_t)(k & 3) * 32u;
+            umma_issue<CG>(d_tmem, ad0 + (uint64_t)(ao >> 4), bd0 + (uint64_t)(bo >> 4), P.idesc,
                            (kb > kb0 || k > 0) ? 1u : 0u);
+          }
           umma_commit_pair<CG>(&empty_bar[stage]);
           if (++stage == NS) { stage = 0; phase ^= 1u; }
         }
@@ -675,6 +717,24 @@ bool make_map(CUtensorMap *m, const void *base, long inner, long outer, long ld,
   return r == CUDA_SUCCESS;
 }
 
+// The same operand viewed as [batch][inner / 64][outer][64] (inner % 64 == 0): box
+// {64, box_outer, box_chunks, 1} brings box_chunks 64-element chunks of box_outer rows,
+// one chunk after the other in shared memory.
+bool make_map_chunked(CUtensorMap *m, const void *base, long inner, long outer, long ld,
+                      int box_outer, int box_chunks, long batch = 1, long bstride = 0) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || inner % 64 != 0) return false;
+  if (batch <= 1) { batch = 1; bstride = ld * outer; }
+  cuuint64_t dims[4] = {64u, (cuuint64_t)outer, (cuuint64_t)(inner / 64), (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)ld * 2, 128u, (cuuint64_t)bstride * 2};
+  cuuint32_t box[4] = {64u, (cuuint32_t)box_outer, (cuuint32_t)box_chunks, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, (void *)base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int EPI, int CG>
 cudaError_t launch_kind(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &o,
                         const CUtensorMap &o2, const TcParams &P, int grid, cudaStream_t st) {
@@ -792,7 +852,7 @@ void tc_gemm_plan(const GemmDesc &d, size_t capacity, int sms, int *cta_group, i
     S = 1;
     if ((f32out || elementwise) && capacity > 0) {
       // automatic: the CTA group and K split with the smallest estimated time, in units of
-      // one k-block of one CTA tile (~0.4 us as measured): the wave-quantised main loop, CTA
+      // one 128-wide k-block of one CTA tile (~0.8 us): the wave-quantised main loop, CTA
       // pairs credited with their smaller shared-memory traffic, plus for a split the ordered
       // reduce, which reads the s fp32 partials and writes the result (~6 TB/s), and its
       // launch (the partial stores themselves overlap the main loop)
@@ -801,11 +861,11 @@ void tc_gemm_plan(const GemmDesc &d, size_t capacity, int sms, int *cta_group, i
         const long tiles = (long)((d.M + cg * BM - 1) / (cg * BM)) * nt * nbatch;
         const long slots = sms / cg;
         for (int s = 1; s <= 16; ++s) {
-          if (s > 1 && (kblocks / s < 4 || (size_t)s * d.M * d.N > capacity)) break;
+          if (s > 1 && (kblocks / s < 2 || (size_t)s * d.M * d.N > capacity)) break;
           const long units = tiles * s;
           const long waves = (units + slots - 1) / slots;
           double est = (double)waves * (double)((kblocks + s - 1) / s) * (cg == 2 ? 0.93 : 1.0);
-          if (s > 1) est += ((s + 1.0) * d.M * d.N * 4.0 / 6.0e12 + 3e-6) / 0.4e-6;
+          if (s > 1) est += ((s + 1.0) * d.M * d.N * 4.0 / 6.0e12 + 3e-6) / 0.8e-6;
           if (est < best) { best = est; CG = cg; S = s; }
         }
       }
@@ -856,10 +916,25 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   if (!P.err) return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
   const int b_rows = BN / CG;
-  bool ok = P.a_mn ? make_map(&ma, d.A, d.M, d.K, d.lda, 64, P.batch, d.a_bstride)
-                   : make_map(&ma, d.A, d.K, d.M, d.lda, BM, P.batch, d.a_bstride);
-  ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, 64, P.batch, d.b_bstride)
-                     : make_map(&mb, d.B, d.K, d.N, d.ldb, b_rows, P.batch, d.b_bstride));
+  // one load per operand and stage when the contiguous dimension is whole 64-element chunks
+  // (a chunk past the end is then out of bounds and zero-filled, never part of the next row)
+  P.a_wide = ((P.a_mn ? d.M : d.K) % 64 == 0) ? 1 : 0;
+  P.b_wide = ((P.b_mn ? d.N : d.K) % 64 == 0) ? 1 : 0;
+  bool ok;
+  if (P.a_wide)
+    ok = P.a_mn ? make_map_chunked(&ma, d.A, d.M, d.K, d.lda, BK, BM / 64, P.batch, d.a_bstride)
+                : make_map_chunked(&ma, d.A, d.K, d.M, d.lda, BM, KC, P.batch, d.a_bstride);
+  else
+    ok = P.a_mn ? make_map(&ma, d.A, d.M, d.K, d.lda, BK, P.batch, d.a_bstride)
+                : make_map(&ma, d.A, d.K, d.M, d.lda, BM, P.batch, d.a_bstride);
+  if (P.b_wide)
+    ok = ok && (P.b_mn ? make_map_chunked(&mb, d.B, d.N, d.K, d.ldb, BK, b_rows / 64, P.batch,
+                                          d.b_bstride)
+                       : make_map_chunked(&mb, d.B, d.K, d.N, d.ldb, b_rows, KC, P.batch,
+                                          d.b_bstride));
+  else
+    ok = ok && (P.b_mn ? make_map(&mb, d.B, d.N, d.K, d.ldb, BK, P.batch, d.b_bstride)
+                       : make_map(&mb, d.B, d.K, d.N, d.ldb, b_rows, P.batch, d.b_bstride));
   if (!ok) return cudaErrorInvalidValue;
   // output maps of the TMA-store epilogue (rows and columns past M, N are clipped by TMA)
   CUtensorMap mo, mo2;

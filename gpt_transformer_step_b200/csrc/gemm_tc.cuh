@@ -4,7 +4,7 @@
 
 constexpr int TC_BM = 128;  // rows per CTA tile (TMEM lanes)
 constexpr int TC_BN = 256;  // columns per CTA tile (TMEM fp32 columns)
-constexpr int TC_BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int TC_BK = 128;  // K per pipeline stage (two 64-element, 128-byte swizzle chunks of bf16)
 constexpr int TC_CE_TILE = TC_BN / 2;  // column width of one cross-entropy statistics partial
 
 struct TcGemm;

@@ -33,8 +33,8 @@ def test_weight_gradients_split_k_on_pairs(gb):
     for m, n in [(4 * C, C), (3 * C, C), (C, C), (C, 4 * C)]:
         cg, sk = _plan(gb, m, n, M, "f32_store")
         assert cg == 2 and 2 <= sk <= 16, (m, n, cg, sk)
-        # a split of s needs s*M*N floats of scratch and at least 4 k-blocks per range
-        assert sk * m * n <= CAP_124M and M // 64 // sk >= 4
+        # a split of s needs s*M*N floats of scratch and at least 2 k-blocks (128 wide) per range
+        assert sk * m * n <= CAP_124M and M // 128 // sk >= 2
 
 
 def test_no_scratch_means_no_split(gb):
@@ -52,7 +52,7 @@ def test_splits_leave_no_empty_k_range(gb):
     for k in (64, 100, 520, 777 // 8 * 8, 4000, 16384, 50304):
         for m, n in [(300, 200), (768, 768), (2304, 768)]:
             _, sk = _plan(gb, m, n, k, "f32_store")
-            kb = math.ceil(k / 64)
+            kb = math.ceil(k / 128)
             per = math.ceil(kb / sk)
             assert 1 <= sk <= max(1, kb) and per * (sk - 1) < kb, (m, n, k, sk)
 
