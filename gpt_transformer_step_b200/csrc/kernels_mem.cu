@@ -424,34 +424,51 @@ constexpr int EW = 64;  // sorted entries per window
 
 // Window w covers sorted entries [w*EW, (w+1)*EW). Runs of one id that lie wholly inside the
 // window are added to dwte here; a run that starts before the window goes to slot 0, a run
-// that continues past it (and did not start before) to slot 1, for the merge kernel. Threads
-// own 16-byte column vectors; the entries of a run are summed in sorted (position) order.
+// that continues past it (and did not start before) to slot 1, for the merge kernel. The
+// block's warps take the window's runs in turn (run r to warp r mod 4), so short runs do not
+// wait on one another; a lane owns 16-byte column vectors, and the entries of a run are summed
+// in sorted (position) order.
 template <typename T>
 __global__ void __launch_bounds__(128) embed_seg_kernel(const int *__restrict__ sid,
                                                         const int *__restrict__ spos,
                                                         const T *__restrict__ dx,
                                                         float *__restrict__ dwte,
                                                         float *__restrict__ partial, int M, int C) {
+  static_assert(EW == 64, "a window is two 32-entry ballots");
   constexpr int VN = Vec<T>::N;
   const int w = blockIdx.x;
   const int e0 = w * EW, e1 = min(M, e0 + EW);
+  const int n = e1 - e0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int s_id[EW], s_pos[EW];
-  if (threadIdx.x < EW && e0 + (int)threadIdx.x < M) {
+  __shared__ unsigned s_start[2];  // bit t: entry t starts a run
+  if (threadIdx.x < EW && (int)threadIdx.x < n) {
     s_id[threadIdx.x] = sid[e0 + threadIdx.x];
     s_pos[threadIdx.x] = spos[e0 + threadIdx.x];
   }
   __syncthreads();
+  if (warp < 2) {
+    const int t = warp * 32 + lane;
+    const bool st = t < n && (t == 0 || s_id[t] != s_id[t - 1]);
+    const unsigned b = __ballot_sync(0xffffffffu, st);
+    if (lane == 0) s_start[warp] = b;
+  }
+  __syncthreads();
+  const unsigned long long starts =
+      (unsigned long long)s_start[0] | ((unsigned long long)s_start[1] << 32);
   const int id_before = e0 > 0 ? sid[e0 - 1] : -1;
   const int id_after = e1 < M ? sid[e1] : -1;
   const int nvec = C / VN;
-  int s = e0;
-  while (s < e1) {
-    const int id = s_id[s - e0];
-    int e = s + 1;
-    while (e < e1 && s_id[e - e0] == id) ++e;
-    const bool before = (s == e0) && (id == id_before);
-    const bool after = (e == e1) && (id == id_after);
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+  unsigned long long rest = starts;
+  for (int r = 0; rest != 0ull; ++r) {
+    const int s = __ffsll((long long)rest) - 1;  // this run: entries [s, e)
+    rest &= rest - 1ull;
+    const int e = rest ? __ffsll((long long)rest) - 1 : n;
+    if ((r & 3) != warp) continue;
+    const int id = s_id[s];
+    const bool before = (s == 0) && (id == id_before);
+    const bool after = (e == n) && (id == id_after);
+    for (int v = lane; v < nvec; v += 32) {
       const int c = v * VN;
       float acc[VN];
 #pragma unroll
@@ -460,7 +477,7 @@ __global__ void __launch_bounds__(128) embed_seg_kernel(const int *__restrict__ 
       for (; k0 + 4 <= e; k0 += 4) {  // four rows in flight, added in order
         float a[4][VN];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) load_vec<T>(dx + (long)s_pos[k0 + u - e0] * C + c, a[u]);
+        for (int u = 0; u < 4; ++u) load_vec<T>(dx + (long)s_pos[k0 + u] * C + c, a[u]);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -468,7 +485,7 @@ __global__ void __launch_bounds__(128) embed_seg_kernel(const int *__restrict__ 
       }
       for (; k0 < e; ++k0) {
         float a[VN];
-        load_vec<T>(dx + (long)s_pos[k0 - e0] * C + c, a);
+        load_vec<T>(dx + (long)s_pos[k0] * C + c, a);
 #pragma unroll
         for (int k = 0; k < VN; ++k) acc[k] += a[k];
       }
@@ -476,15 +493,14 @@ __global__ void __launch_bounds__(128) embed_seg_kernel(const int *__restrict__ 
                                        : partial + ((long)w * 2 + (before ? 0 : 1)) * C + c;
 #pragma unroll
       for (int k = 0; k < VN; k += 4) {
-        float4 r = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+        float4 q = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
         if (!before && !after) {
           const float4 o = *reinterpret_cast<const float4 *>(dst + k);
-          r.x += o.x; r.y += o.y; r.z += o.z; r.w += o.w;
+          q.x += o.x; q.y += o.y; q.z += o.z; q.w += o.w;
         }
-        *reinterpret_cast<float4 *>(dst + k) = r;
+        *reinterpret_cast<float4 *>(dst + k) = q;
       }
     }
-    s = e;
   }
 }
 
