@@ -1300,7 +1300,7 @@ cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B,
 cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
                                     const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
                                     int C, int H, int window, unsigned *err, cudaStream_t st,
-                                    bf16 *dst) {
+                                    bf16 *dst, bool d_ready) {
   CUDA_TRY(set_attrs());
   CUtensorMap mq, md, mo, mdq, mdkv;
   if (!map_rows(&mq, qkv, 3L * C, (long)B * T, 3L * C) ||
@@ -1324,10 +1324,12 @@ cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *
         !map_rows(&mk, qkv, 3L * C, (long)B * T, 3L * C, 64) ||
         !map_btc(&mdq64, dqkv, 3L * C, T, B, 3L * C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-    const long rows = (long)B * T;
-    const int pb = (int)((rows + 7) / 8 < 148 * 16 ? (rows + 7) / 8 : 148 * 16);
-    attn_bwd_prep_d<<<pb, 256, 0, st>>>(o, dout, Dbuf, B, T, C, H);
-    CUDA_TRY(cudaGetLastError());
+    if (!d_ready) {  // D = rowsum(dO * O), unless the producer of dO wrote it alongside
+      const long rows = (long)B * T;
+      const int pb = (int)((rows + 7) / 8 < 148 * 16 ? (rows + 7) / 8 : 148 * 16);
+      attn_bwd_prep_d<<<pb, 256, 0, st>>>(o, dout, Dbuf, B, T, C, H);
+      CUDA_TRY(cudaGetLastError());
+    }
     attn_bwd_dkv_tc<DKV_STAGES_DS, true><<<grid, BWD_THREADS, dkv_smem(DKV_STAGES_DS, true), st>>>(
         mq, md, mdkv, mst, p);
     CUDA_TRY(cudaGetLastError());

@@ -112,6 +112,9 @@ enum EpiKind {
   EPI_DGELU_RECOMP,   // out[m][n] = acc * gelu'(aux[m][n]) ; out2[m][n] = gelu(aux[m][n]),
                       // aux = the pre-activation the forward kept
   EPI_AXPBY,          // out[m][n] = alpha * acc + beta * aux[m][n]        (activation type)
+  // attention backward: dO and, per row and 64-column head, D = rowsum(dO * O)
+  EPI_STORE_DOT,      // out[m][n] = acc ; outf[(b * N/64 + n/64) * dot_T + t] = sum over the
+                      // head's 64 columns of bf16(acc) * aux[m][n], for row m = b * dot_T + t
 };
 
 struct Epi {
@@ -131,6 +134,7 @@ struct Epi {
   const DevScalars *sc;  // inv_M
   float alpha, beta;     // EPI_AXPBY
   long aux_bstride;      // batched GEMMs: elements between the aux matrices of two batches
+  int dot_T;             // EPI_STORE_DOT: rows per sequence
 };
 
 struct GemmDesc {

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(256) splitk_reduce4_kernel(GemmDesc d, int vec
 template <typename T>
 cudaError_t launch_gemm_simt(const GemmDesc &d, cudaStream_t st) {
   if (d.M <= 0 || d.N <= 0) return cudaSuccess;
+  if (d.epi.kind == EPI_STORE_DOT) return cudaErrorInvalidValue;  // tensor-core path only
   const int S = d.split_k > 1 ? d.split_k : 1;
   dim3 grid((d.N + BN - 1) / BN, (d.M + BM - 1) / BM, S);
   gemm_simt_kernel<T><<<grid, 256, 0, st>>>(d);

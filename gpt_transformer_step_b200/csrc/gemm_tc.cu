@@ -42,11 +42,12 @@ constexpr int TMEM_COLS = 512;
 
 enum TcEpi {
   TE_STORE = 0, TE_STORE_GELU, TE_RESID, TE_DGELU, TE_F32_STORE, TE_F32_ACCUM, TE_CE_STATS,
-  TE_CE_DS, TE_PARTIAL, TE_STORE_PRE_GELU, TE_DGELU_RECOMP, TE_AXPBY
+  TE_CE_DS, TE_PARTIAL, TE_STORE_PRE_GELU, TE_DGELU_RECOMP, TE_AXPBY, TE_STORE_DOT
 };
 // epilogues that read an auxiliary bf16 input of the output's shape
 __host__ __device__ constexpr bool epi_has_aux(int e) {
-  return e == TE_RESID || e == TE_DGELU || e == TE_DGELU_RECOMP || e == TE_AXPBY;
+  return e == TE_RESID || e == TE_DGELU || e == TE_DGELU_RECOMP || e == TE_AXPBY ||
+         e == TE_STORE_DOT;
 }
 
 struct TcParams {
@@ -568,6 +569,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0);
       float ce_max = -INFINITY, ce_sum = 0.f;
+      float dot_part = 0.f;  // TE_STORE_DOT: the first half of a head's dot
       const int ncols = min(BN, P.N - nt * BN) - c0;
       // the accumulator load of chunk c + 1 (and its auxiliary input) is in flight during
       // chunk c's math and store
@@ -591,6 +593,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         float v2[32];
         epi_math<EPI>(P, col0, er, aux, v, v2);
+        if (EPI == TE_STORE_DOT) {
+          // the head's dot of the stored (bf16) dO row with O, over its two 32-column chunks
+          float a[32];
+          unpack_bf16x32(aux, a);
+          float sdot = 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            sdot = fmaf(__bfloat162float(__float2bfloat16_rn(v[k])), a[k], sdot);
+          if ((col0 & 63) == 0) {
+            dot_part = sdot;
+          } else if (row < P.M) {
+            const int b = row / P.epi.dot_T, t = row - b * P.epi.dot_T;
+            P.epi.outf[((long)b * (P.N / 64) + col0 / 64) * P.epi.dot_T + t] = dot_part + sdot;
+          }
+        }
         if (epi_has_aux(EPI)) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) aux[q] = aux_nx[q];
@@ -780,6 +797,7 @@ cudaError_t launch_epi(int kind, bool split, const CUtensorMap &ma, const CUtens
     case EPI_STORE_PRE_GELU: return TC_L(TE_STORE_PRE_GELU);
     case EPI_DGELU_RECOMP: return TC_L(TE_DGELU_RECOMP);
     case EPI_AXPBY: return TC_L(TE_AXPBY);
+    case EPI_STORE_DOT: return TC_L(TE_STORE_DOT);
     default: return cudaErrorInvalidValue;
   }
 #undef TC_L
@@ -827,6 +845,9 @@ bool tc_gemm_supported(const GemmDesc &d) {
     case EPI_AXPBY:
       return (e.ldo & 7) == 0 && (e.ld_aux & 7) == 0 && (e.aux_bstride & 7) == 0 &&
              aligned16(e.out) && aligned16(e.aux);
+    case EPI_STORE_DOT:  // whole 64-column heads, one sequence length for the rows
+      return (e.ldo & 7) == 0 && (e.ld_aux & 7) == 0 && aligned16(e.out) && aligned16(e.aux) &&
+             e.outf && e.dot_T > 0 && d.M % e.dot_T == 0 && d.N % 64 == 0 && d.split_k == 1;
     case EPI_F32_STORE:
     case EPI_F32_ACCUM:
       return (e.ldf & 3) == 0 && aligned16(e.outf);
@@ -946,6 +967,7 @@ cudaError_t tc_gemm_launch(TcGemm *t, GemmDesc &d, cudaStream_t st, int *launche
   } else {
     switch (e0.kind) {
       case EPI_STORE: case EPI_RESID: case EPI_DGELU: case EPI_CE_DS: case EPI_AXPBY:
+      case EPI_STORE_DOT:
         ok = make_out_map(&mo, e0.out, false, d.N, d.M, e0.ldo, P.batch, d.out_bstride);
         break;
       case EPI_STORE_GELU: case EPI_STORE_PRE_GELU: case EPI_DGELU_RECOMP:

@@ -84,14 +84,15 @@ cudaError_t launch_attention_bwd(const T *qkv, const T *o, const T *dout, const 
 // Attention on the tensor cores (head_dim 64, bf16): forward, and backward. Backward with
 // dst == NULL: a dQ pass that also writes D = rowsum(dO o O), then the dK/dV pass. With dst
 // (B*H*T*T bf16 scratch): D, then the dK/dV pass also writing dS^T to dst, then dQ = dS K
-// from dst on the tensor cores (no second pass over the scores). err: device error word.
+// from dst on the tensor cores (no second pass over the scores); d_ready: Dbuf already holds
+// D (the GEMM that produced dO wrote it), only with dst. err: device error word.
 bool attention_tc_supported(int C, int H);
 cudaError_t launch_attention_fwd_tc(const bf16 *qkv, bf16 *o, float *lse, int B, int T, int C,
                                     int H, int window, unsigned *err, cudaStream_t st);
 cudaError_t launch_attention_bwd_tc(const bf16 *qkv, const bf16 *o, const bf16 *dout,
                                     const float *lse, float *Dbuf, bf16 *dqkv, int B, int T,
                                     int C, int H, int window, unsigned *err, cudaStream_t st,
-                                    bf16 *dst = nullptr);
+                                    bf16 *dst = nullptr, bool d_ready = false);
 
 // The same backward with its D scratch in a file-scope device array (no allocation); rejects
 // B*H*T > attention_bwd_noalloc_max_rows() with cudaErrorInvalidValue.

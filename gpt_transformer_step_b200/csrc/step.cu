@@ -268,12 +268,17 @@ cudaError_t attention_bwd(gpt_handle *h, const T *qkv, const T *o, const T *dout
   return launch_attention_bwd<T>(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
                                  h->stream);
 }
+// The attention backward of the bf16 step takes D = rowsum(dO * O) from the epilogue of the
+// GEMM that forms dO (EPI_STORE_DOT) when it runs the stored-dS form on the tensor cores.
+bool fused_d(const gpt_handle *h, int Tlen) {
+  return h->use_bf16 && h->tc && attention_tc_supported(h->C, h->H) && attn_dst(h, Tlen);
+}
 template <>
 cudaError_t attention_bwd<bf16>(gpt_handle *h, const bf16 *qkv, const bf16 *o, const bf16 *dout,
                                 const float *lse, bf16 *dqkv, int B, int Tlen, int w) {
   if (attention_tc_supported(h->C, h->H))
     return launch_attention_bwd_tc(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
-                                   &h->sc->err, h->stream, attn_dst(h, Tlen));
+                                   &h->sc->err, h->stream, attn_dst(h, Tlen), fused_d(h, Tlen));
   return launch_attention_bwd<bf16>(qkv, o, dout, lse, h->Dbuf, dqkv, B, Tlen, h->C, h->H, w,
                                     h->stream);
 }
@@ -465,11 +470,15 @@ cudaError_t enqueue(gpt_handle *h, const float *params, float *grads, float *ada
     CUDA_TRY(mark(h->ev_wap));
     d = gdesc(M, C, C, dx, C, 1, W + P.wap, C, 0);
     d.epi.kind = EPI_STORE; d.epi.out = h->dout; d.epi.ldo = C;
+    if (fused_d(h, Tlen)) {  // D = rowsum(dO * O) per head, for the attention backward
+      d.epi.kind = EPI_STORE_DOT; d.epi.aux = A.o; d.epi.ld_aux = C; d.epi.outf = h->Dbuf;
+      d.epi.dot_T = Tlen; d.split_k = 1;
+    }
     CUDA_TRY(gemm(h, d));
     if (have_wqkv) CUDA_TRY(join(h->ev_wqkv));  // dqkv is rewritten: the last dWqkv has read it
     TIMED(h, GPT_KSTAT_ATTN_BWD, attn_flops(h->windows[l], 8.0),
           attention_bwd<T>(h, (T *)A.qkv, (T *)A.o, (T *)h->dout, A.lse, (T *)h->dqkv, B, Tlen,
-                           h->windows[l])); nl += (h->use_bf16 && attn_dst(h, Tlen)) ? 3 : 2;
+                           h->windows[l])); nl += (h->use_bf16 && attn_dst(h, Tlen) && !fused_d(h, Tlen)) ? 3 : 2;
     CUDA_TRY(fork());
     d = gdesc(3 * C, C, M, h->dqkv, 3 * C, 0, A.a, C, 0);
     d.epi.kind = wgrad; d.epi.outf = G + P.wqkv; d.epi.ldf = C;
