@@ -381,7 +381,7 @@ def run_ours(args, wl, rank, world, local_rank):
                                      "dram__bytes_write.sum)",
                      "flops": "algorithmic: 2MNK of the block GEMMs and the lm_head forward, "
                               "dX and dwte; the logits recompute is timed but not counted",
-                     "peak_kind": f"{pk_kind} burst bf16 (the step is ~19 ms, not a seconds-long "
+                     "peak_kind": f"{pk_kind} burst bf16 (the step is ~17 ms, not a seconds-long "
                                   f"loop); sustained {peak_s} beside it",
                      "launches_timed": n_l,
                      "gemm_ms_per_step": gemm_ms / n_inst,
