@@ -34,7 +34,7 @@ using namespace tc;
 constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK;
 constexpr int KC = BK / 64;            // 128-byte swizzle chunks per stage along K
 constexpr int A_BYTES = BM * BK * 2;   // 32 KB
-constexpr int A_CHUNK = BM * 64 * 2;   // 16 KB: one chunk of A (K-major: 64 k; MN-major: 64 m)
+constexpr int A_CHUNK = BM * 64 * 2;   // 16 KB: one 64-k chunk of a K-major A tile
 constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
@@ -456,12 +456,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (P.a_wide) {
             if (!P.a_mn) tma_load_pair4<CG>(sA, &tmA, fbl, 0, m0, k0 / 64, bz);
             else tma_load_pair4<CG>(sA, &tmA, fbl, 0, k0, m0 / 64, bz);
+          } else if (!P.a_mn) {
+#pragma unroll
+            for (int j = 0; j < KC; ++j)
+              tma_load_pair<CG>(sA + j * A_CHUNK, &tmA, fbl, k0 + 64 * j, m0, bz);
           } else {
 #pragma unroll
-            for (int j = 0; j < KC; ++j) {
-              if (!P.a_mn) tma_load_pair<CG>(sA + j * A_CHUNK, &tmA, fbl, k0 + 64 * j, m0, bz);
-              else tma_load_pair<CG>(sA + j * A_CHUNK, &tmA, fbl, m0 + 64 * j, k0, bz);
-            }
+            for (int j = 0; j < BM / 64; ++j)  // MN-major chunks: 64 m by BK k rows of 128 B
+              tma_load_pair<CG>(sA + j * (BK * 128), &tmA, fbl, m0 + 64 * j, k0, bz);
           }
           if (P.b_wide) {
             if (!P.b_mn) tma_load_pair4<CG>(sB, &tmB, fbl, 0, n0, k0 / 64, bz);
