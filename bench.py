@@ -38,6 +38,8 @@ METRIC = "train tokens/s (GPT-2 step, MFU from 6N+attn FLOPs)"
 # chunks (kernel_bench cases, profiles/gemm_shapes_gpt2_124m_ncu.md), averaged with the launch
 # counts of one step (148 launches; 148.7 MB algorithmic per launch on the same basis). The
 # split-K reduce kernels and the lm_head statistics / recompute launches are not in the mean.
+# In the step, the attention-projection dgrad GEMM also reads the attention output (25 MB) for
+# the D epilogue; its capture is the plain-store form, so the step's mean is ~2 MB higher.
 GEMM_DRAM_BYTES_PER_LAUNCH: dict = {"gpt2_124m_bf16": 136.6e6}
 GEMM_ALG_BYTES_PER_LAUNCH: dict = {"gpt2_124m_bf16": 148.7e6}
 
